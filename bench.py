@@ -1,0 +1,466 @@
+#!/usr/bin/env python
+"""Benchmark: batched ISD verify-and-propose step on B200.
+
+One step = attention over the paged KV cache (with the KV append) + LM head +
+row statistics + p/q accept / residual draw / proposals, for a batch of B
+requests, through the C ABI of libisd.so.  Default workload: Qwen3-8B shapes,
+B=32, N=4 (Q=7), prefixes U[512, 8192] in 16-token pages, vocab 151936, bf16,
+constructed per-position acceptance 0.9.
+
+Prints one JSON line (rank 0).  `--impl reference` times the CPU oracle
+instead (host cores, bounded samples of the same workload).
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "ISD steps/s and accepted tokens/s at B=32,N=4 (Qwen3-8B shapes); % HBM roofline"
+FALLBACK_HBM_GBS = 6650.0
+FALLBACK_BF16_TFLOPS = 1590.0
+
+
+def parse_args():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=2000)
+    ap.add_argument("--warmup", type=int, default=20)
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--config", default="qwen3_8b_b32_n4")
+    ap.add_argument("--e2e-steps", type=int, default=200)
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--cpu-budget-s", type=float, default=20.0)
+    return ap.parse_args()
+
+
+# ---------------------------------------------------------------------------
+def measured_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            j = json.load(f)
+        return float(j["hbm_gbs"]), float(j["bf16_tflops"]), float(
+            j.get("bf16_tflops_sustained", j["bf16_tflops"])), "measured"
+    return FALLBACK_HBM_GBS, FALLBACK_BF16_TFLOPS, 1400.0, "fallback"
+
+
+class ClockSampler:
+    """nvidia-smi clocks / throttle reasons sampled during the timed region."""
+
+    FIELDS = ("index,pci.bus_id,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, bus_id: str | None):
+        self.bus_id = bus_id
+        self.proc = None
+        self.lines = []
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
+                 "-lms", "100"], stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+            self.thread = threading.Thread(target=self._read, daemon=True)
+            self.thread.start()
+        except (OSError, FileNotFoundError):
+            self.proc = None
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.lines.append(line.strip())
+
+    def stop(self):
+        if not self.proc:
+            return None
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+        self.thread.join(timeout=2)
+        rows = [l.split(", ") for l in self.lines if l]
+        if self.bus_id:
+            mine = [r for r in rows if len(r) > 1 and self.bus_id.lower() in r[1].lower()]
+            rows = mine or rows
+        if not rows:
+            return None
+        idx0 = rows[0][0]
+        rows = [r for r in rows if r[0] == idx0 and len(r) >= 10]
+        sm = [float(r[2]) for r in rows if r[2].replace(".", "").isdigit()]
+        mx = [float(r[3]) for r in rows if r[3].replace(".", "").isdigit()]
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({names[i] for r in rows for i in range(4) if r[6 + i].strip() == "Active"})
+        return {"sm_mhz": statistics.median(sm) if sm else None,
+                "sm_max_mhz": max(mx) if mx else None, "reasons": reasons, "samples": len(rows)}
+
+
+def profile_traffic(kernel_file: str):
+    """dram bytes per launch of the LM-head kernel from the committed ncu summary,
+    if the kernel source is unchanged since the counters were taken."""
+    p = os.path.join(ROOT, "profiles", "lm_head_traffic.json")
+    src = os.path.join(ROOT, "speculative_verification_isd_b200", "csrc", kernel_file)
+    if not (os.path.exists(p) and os.path.exists(src)):
+        return None
+    with open(p) as f:
+        j = json.load(f)
+    h = hashlib.sha256(open(src, "rb").read()).hexdigest()[:16]
+    if j.get("source_sha256_16") != h:
+        return None
+    return j.get("dram_bytes_per_launch_full")
+
+
+# ---------------------------------------------------------------------------
+# CPU oracle sampling (used by the cpu_baseline leg and by --impl reference)
+# ---------------------------------------------------------------------------
+class OracleSampler:
+    """Host copies of the workload and timed oracle runs on bounded pieces.
+
+    A full step is estimated as B x (one request's attention) + (V / Vs) x
+    (the LM head of every row over a Vs-entry vocabulary slice) + B x (one
+    request's acceptance), each piece timed with the oracle as it stands.
+    """
+
+    def __init__(self, wl, cfg):
+        import numpy as np
+        from oracle import isd_oracle as O
+        from speculative_verification_isd_b200.workload import request_slice
+        self.O, self.np, self.cfg = O, np, cfg
+        host = wl.host_view()
+        self.slices = [request_slice(host, cfg, b) for b in range(min(cfg.B, 4))]
+        self.W = wl.W.contiguous().view(__import__("torch").int16).cpu().numpy().view(np.uint16)
+        self.hidden = wl.hidden.contiguous().view(__import__("torch").int16).cpu().numpy().view(np.uint16)
+        self.logits0 = wl.logits[: cfg.Q].cpu().numpy().reshape(1, cfg.Q, cfg.V)
+        self.prev0 = wl.prev_logits[: cfg.Q].cpu().numpy().reshape(1, cfg.Q, cfg.V)
+        self.host = host
+        self.threads = self._threads()
+
+    @staticmethod
+    def _threads():
+        try:
+            from threadpoolctl import threadpool_info
+            n = [i.get("num_threads", 1) for i in threadpool_info() if i.get("user_api") == "blas"]
+            return max(n) if n else 1
+        except Exception:
+            return os.cpu_count() or 1
+
+    def time_attention(self, k):
+        s = self.slices[k % len(self.slices)]
+        t = time.perf_counter()
+        self.O.attention(s["q"], s["k_new"], s["v_new"], s["k_pool"], s["v_pool"], s["page_table"],
+                         s["kv_len"], s["n_clean"], self.cfg.N, self.cfg.page_size,
+                         self.cfg.D ** -0.5)
+        return time.perf_counter() - t
+
+    def time_lm_head(self, k, vs):
+        v0 = (k * vs) % max(1, self.cfg.V - vs + 1)
+        t = time.perf_counter()
+        self.O.lm_head(self.hidden, self.W[v0:v0 + vs])
+        return time.perf_counter() - t
+
+    def time_accept(self):
+        h = self.host
+        t = time.perf_counter()
+        self.O.accept(self.logits0, self.prev0, h["n_clean"][:1], h["clean_tok"][:1],
+                      h["kv_len"][:1], h["uniforms"][:1], self.cfg.N)
+        return time.perf_counter() - t
+
+    def estimate_step_seconds(self, k, vs):
+        cfg = self.cfg
+        ta, tl, tc = self.time_attention(k), self.time_lm_head(k, vs), self.time_accept()
+        return cfg.B * ta + (cfg.V / vs) * tl + cfg.B * tc, ta + tl + tc
+
+
+def cpu_baseline(wl, cfg, budget_s):
+    sampler = OracleSampler(wl, cfg)
+    vs = 8192
+    ests, spent, k = [], 0.0, 0
+    while spent < budget_s and k < 50:
+        est, used = sampler.estimate_step_seconds(k, vs)
+        ests.append(est)
+        spent += used
+        k += 1
+    est = statistics.median(ests)
+    return {"value": 1.0 / est, "unit": "ISD steps/s", "cores": sampler.threads, "kind": "oracle",
+            "sample": (f"{k} samples, each: 1 request's attention, the LM head of all {cfg.M} rows "
+                       f"over a {vs}-entry vocabulary slice, 1 request's acceptance; full step "
+                       f"extrapolated as {cfg.B} x attention + {cfg.V}/{vs} x LM-head slice + "
+                       f"{cfg.B} x acceptance ({spent:.1f} s of CPU work)")}
+
+
+# ---------------------------------------------------------------------------
+def setup_dist(args):
+    import torch
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1:
+        import datetime
+        import torch.distributed as dist
+        torch.cuda.set_device(local)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=torch.device("cuda", local))
+    else:
+        torch.cuda.set_device(0)
+    return world, rank, local
+
+
+def allreduce_max(x: float, world: int) -> float:
+    if world == 1:
+        return x
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([x], dtype=torch.float64, device="cuda")
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def allreduce_sum(x: float, world: int) -> float:
+    if world == 1:
+        return x
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([x], dtype=torch.float64, device="cuda")
+    dist.all_reduce(t, op=dist.ReduceOp.SUM)
+    return float(t.item())
+
+
+def barrier(world):
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+
+
+def run_reference(args):
+    """--impl reference: the CPU oracle, timed on host cores (rank 0 only)."""
+    import torch
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return 0
+    from speculative_verification_isd_b200 import build as B
+    B.build()
+    from speculative_verification_isd_b200 import inputs as I
+    from speculative_verification_isd_b200 import isd
+    from speculative_verification_isd_b200.workload import DeviceWorkload
+    cfg = I.CONFIGS[args.config]
+    torch.cuda.set_device(0)
+    wl = DeviceWorkload(isd, cfg, seed=0)  # inputs only; the timed work is the oracle's
+    wl.step()
+    torch.cuda.synchronize()
+    sampler = OracleSampler(wl, cfg)
+    total_budget = 150.0
+    per_step = total_budget / max(1, args.steps + args.warmup)
+    # vocabulary slice sized to the per-step budget (at least 256 entries)
+    t0 = time.perf_counter()
+    sampler.time_lm_head(0, 1024)
+    t_1k = max(1e-4, time.perf_counter() - t0)
+    vs = int(max(256, min(cfg.V, 1024 * max(0.05, per_step * 0.6) / t_1k)))
+    for k in range(args.warmup):
+        sampler.estimate_step_seconds(k, vs)
+    ests = []
+    tstart = time.perf_counter()
+    for k in range(args.steps):
+        ests.append(sampler.estimate_step_seconds(k, vs)[0])
+        if time.perf_counter() - tstart > total_budget:
+            break
+    est = statistics.median(ests)
+    value = 1.0 / est
+    line = {"impl": "reference", "metric": METRIC, "value": value, "unit": "ISD steps/s",
+            "n_gpus": world, "steps": len(ests), "warmup": args.warmup, "ms_per_step": est * 1e3,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+            "data": "synthetic",
+            "config": {"workload": cfg.name, "B": cfg.B, "N": cfg.N, "Q": cfg.Q, "V": cfg.V,
+                       "hidden": cfg.H, "heads": f"{cfg.Hq}q/{cfg.Hkv}kv x {cfg.D}",
+                       "prefix": f"U[{cfg.prefix_lo},{cfg.prefix_hi}]",
+                       "page_size": cfg.page_size},
+            "cpu_baseline": {"value": value, "unit": "ISD steps/s", "cores": sampler.threads,
+                             "kind": "oracle",
+                             "sample": (f"per step: 1 request's attention, LM head of all "
+                                        f"{cfg.M} rows over a {vs}-entry vocabulary slice, 1 "
+                                        f"request's acceptance; extrapolated to the full step")},
+            "e2e": {"value": value, "unit": "ISD steps/s", "h2d_bytes_per_step": 0,
+                    "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+def main():
+    args = parse_args()
+    if args.impl == "reference":
+        return run_reference(args)
+    import numpy as np
+    import torch
+    world, rank, local = setup_dist(args)
+    from speculative_verification_isd_b200 import build as B
+    if rank == 0:
+        B.build()
+    barrier(world)
+    from speculative_verification_isd_b200 import inputs as I
+    from speculative_verification_isd_b200 import isd
+    from speculative_verification_isd_b200.workload import DeviceWorkload
+    cfg = I.CONFIGS[args.config]
+    hbm, tf_burst, tf_sus, peak_src = measured_peaks()
+    # weak scaling: every rank runs its own batch of B requests (requests are
+    # independent), so there is no collective on the data path
+    wl = DeviceWorkload(isd, cfg, seed=rank, n_uniform_steps=max(64, args.warmup + 1))
+    d = wl.dims
+    K, W = args.steps, args.warmup
+    stream = torch.cuda.current_stream()
+    acc_hist = torch.zeros(K, cfg.B, dtype=torch.int32, device="cuda")
+
+    def run_step(k, acc_out=None):
+        wl.set_uniforms(k)
+        if acc_out is not None:
+            wl.accept_len = acc_out
+        wl.step()
+
+    for k in range(W):
+        run_step(k)
+    torch.cuda.synchronize()
+    bus = None
+    try:
+        bus = torch.cuda.get_device_properties(torch.cuda.current_device()).pci_bus_id
+    except Exception:
+        bus = None
+    clocks = ClockSampler(bus)
+    clocks.start()
+    time.sleep(0.3)
+    # ---------------- timed region: K steps through isd_step
+    barrier(world)
+    torch.cuda.synchronize()
+    ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    ev0.record(stream)
+    for k in range(K):
+        run_step(k, acc_hist[k])
+    ev1.record(stream)
+    torch.cuda.synchronize()
+    barrier(world)
+    clk = clocks.stop()
+    t_ms = allreduce_max(ev0.elapsed_time(ev1), world)
+    wl.accept_len = torch.empty(cfg.B, dtype=torch.int32, device="cuda")
+    accepted = allreduce_sum(float(acc_hist.sum().item()), world)
+    steps_total = K * world
+    value = steps_total / (t_ms / 1e3)
+    tok_s = accepted / (t_ms / 1e3)
+    mean_acc = accepted / (steps_total * cfg.B)
+    flags = int(wl.err.item())
+
+    # ---------------- stage breakdown (same work, stage by stage, events between)
+    KS = min(K, 300)
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(5)] for _ in range(KS)]
+    for k in range(KS):
+        wl.set_uniforms(k)
+        e = evs[k]
+        e[0].record(stream)
+        isd.attention(d, wl.q, wl.k_new, wl.v_new, wl.k_pool, wl.v_pool, wl.page_table, wl.kv_len,
+                      wl.n_clean, wl.hidden, wl.ws, wl.err)
+        e[1].record(stream)
+        isd.lm_head(d, wl.hidden, wl.W, wl.logits, None, wl.ws, wl.lora_A, wl.lora_B, wl.err)
+        e[2].record(stream)
+        isd.row_stats(d, wl.logits, d.M, wl.row_stats, wl.ws)
+        e[3].record(stream)
+        isd.accept(d, wl.logits, wl.row_stats, wl.prev_logits, wl.prev_row_stats, wl.n_clean,
+                   wl.clean_tok, wl.kv_len, wl.uniforms, wl.accept_len, wl.out_tok,
+                   wl.next_n_clean, wl.next_clean_tok, wl.next_kv_len, wl.ws, wl.ratio, wl.err)
+        e[4].record(stream)
+    torch.cuda.synchronize()
+    stage = np.array([[evs[k][i].elapsed_time(evs[k][i + 1]) for i in range(4)]
+                      for k in range(KS)])
+    st_ms = stage.mean(axis=0)
+    t_attn, t_lm, t_stats, t_acc = [float(x) for x in st_ms]
+
+    # ---------------- e2e: public API with host buffers, copies inside the timed region
+    host = {}
+    for name in ("q", "k_new", "v_new"):
+        t = getattr(wl, name)
+        host[name] = torch.empty(t.shape, dtype=t.dtype, pin_memory=True).copy_(t)
+    for name in ("kv_len", "n_clean", "clean_tok", "page_table"):
+        t = getattr(wl, name)
+        host[name] = torch.empty(t.shape, dtype=t.dtype, pin_memory=True).copy_(t)
+    host["uniforms"] = torch.empty(wl.uniforms_all.shape, dtype=torch.float32,
+                                   pin_memory=True).copy_(wl.uniforms_all)
+    outs = ("accept_len", "out_tok", "next_n_clean", "next_clean_tok", "next_kv_len")
+    host_out = {n: torch.empty(getattr(wl, n).shape, dtype=torch.int32, pin_memory=True)
+                for n in outs}
+    h2d = sum(host[n].numel() * host[n].element_size() for n in host if n != "uniforms") + \
+        host["uniforms"][0].numel() * 4
+    d2h = sum(v.numel() * 4 for v in host_out.values())
+    KE = min(args.e2e_steps, K)
+    barrier(world)
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for k in range(KE):
+        for n in ("q", "k_new", "v_new", "kv_len", "n_clean", "clean_tok", "page_table"):
+            getattr(wl, n).copy_(host[n], non_blocking=True)
+        wl.uniforms = wl.uniforms_all[0]
+        wl.uniforms.copy_(host["uniforms"][k % host["uniforms"].shape[0]], non_blocking=True)
+        wl.step()
+        for n in outs:
+            host_out[n].copy_(getattr(wl, n), non_blocking=True)
+        stream.synchronize()  # the caller needs this step's result before the next one
+    e1.record(stream)
+    torch.cuda.synchronize()
+    barrier(world)
+    e2e_ms = allreduce_max(e0.elapsed_time(e1), world)
+    e2e_value = KE * world / (e2e_ms / 1e3)
+
+    # ---------------- roofline of the dominant kernel (LM head)
+    lm_bytes = float(cfg.V) * cfg.H * 2 + float(cfg.M) * cfg.H * 2 + float(cfg.M) * cfg.V * 4
+    lm_flops = 2.0 * cfg.M * cfg.H * cfg.V
+    achieved = lm_bytes / (t_lm / 1e3) / 1e9
+    kv_bytes = float(np.sum(wl.kv_len_h.astype(np.float64))) * cfg.Hkv * cfg.D * 4
+    step_bytes = lm_bytes + kv_bytes + float(cfg.M) * (cfg.H + 2 * cfg.Hkv * cfg.D) * 2 \
+        + float(cfg.M) * cfg.H * 2
+    step_ms = t_ms / K
+    line = {
+        "metric": METRIC, "value": value, "unit": "ISD steps/s", "n_gpus": world, "steps": K,
+        "warmup": W, "ms_per_step": step_ms, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+        "accepted_tokens_per_s": tok_s, "mean_accept_len": mean_acc,
+        "config": {"workload": cfg.name, "B": cfg.B, "N": cfg.N, "Q": cfg.Q, "V": cfg.V,
+                   "hidden": cfg.H, "heads": f"{cfg.Hq}q/{cfg.Hkv}kv x {cfg.D}",
+                   "prefix": f"U[{cfg.prefix_lo},{cfg.prefix_hi}]", "page_size": cfg.page_size,
+                   "accept_rate": cfg.accept_rate, "global_batch": cfg.B * world,
+                   "parallelism": f"dp{world} (independent batches)",
+                   "l2": "no flush; every step streams >1.8 GB (LM head 1.245 GB + KV cache) > 126 MB L2"},
+        "roofline": {"bound": "hbm", "kernel": "lm_head_kernel", "achieved": achieved,
+                     "peak": hbm, "unit": "GB/s", "frac": achieved / hbm,
+                     "traffic": profile_traffic("lm_head.cu"),
+                     "bytes_per_launch": lm_bytes, "ms_per_launch": t_lm,
+                     "tensor_tflops": lm_flops / (t_lm / 1e3) / 1e12,
+                     "tensor_frac_of_sustained": lm_flops / (t_lm / 1e3) / 1e12 / tf_sus,
+                     "peak_source": peak_src},
+        "step_roofline": {"algorithmic_bytes": step_bytes,
+                          "achieved_gbs": step_bytes / (step_ms / 1e3) / 1e9,
+                          "frac": step_bytes / (step_ms / 1e3) / 1e9 / hbm,
+                          "stage_ms": {"attention": t_attn, "lm_head": t_lm, "row_stats": t_stats,
+                                       "accept": t_acc}},
+        "e2e": {"value": e2e_value, "unit": "ISD steps/s", "h2d_bytes_per_step": int(h2d),
+                "d2h_bytes_per_step": int(d2h), "steps": KE},
+        "gpu_launches": K * (4 + (3 if cfg.lora_rank else 0)),
+        "clocks": clk, "err_flags": flags,
+    }
+    if world == 1 and rank == 0 and not args.no_cpu_baseline:
+        line["cpu_baseline"] = cpu_baseline(wl, cfg, args.cpu_budget_s)
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        import torch.distributed as dist
+        dist.destroy_process_group()
+    return 0
+
+
+if __name__ == "__main__":
+    sys.exit(main())

@@ -1,0 +1,194 @@
+/*
+ * isd.h -- C ABI of the batched ISD (Introspective Strided Decoding)
+ * verify-and-propose step for I-DLM, sm_100a (B200).
+ *
+ * The operation is the one the I-DLM pages describe:
+ *   [PRJ] I-DLM project page, Traditional-Chinese text (news.myit.tw/news/ml1xco)
+ *   [EXP] "I-DLM：扩散模型如何用“自省一致性”追上自回归模型质量" (blog.hypho.cn)
+ *   [ENG] "自省扩散语言模型的 token 生成机制与工程实践" (blog.hotdry.top)
+ * One forward over a block of Q = 2N-1 query slots per request verifies the
+ * previous stride's N proposals with the p/q criterion min(1, p(x)/q(x)) and
+ * proposes the next N tokens ([EXP §Introspective Strided Decoding（ISD）],
+ * [ENG §从质量差距到自省机制, §Token 生成的核心参数与验收机制]).
+ *
+ * Conventions for every entry point:
+ *  - All tensor pointers are DEVICE pointers, owned by the caller, row-major
+ *    and densely packed in the layouts stated below.  bf16 tensors are passed
+ *    as uint16_t bit patterns.  Nothing is allocated and nothing synchronises:
+ *    work is enqueued on `stream` (a cudaStream_t; NULL = legacy default).
+ *  - `ws` is caller-owned device scratch of at least isd_workspace_bytes(d)
+ *    bytes, 256-byte aligned, with no initial contents required (each call
+ *    clears the counters it keeps there on its own stream).  Two calls that
+ *    share one workspace must not overlap on the GPU.
+ *  - Host-side validation returns a negative isd_status and enqueues nothing.
+ *    Data-dependent faults found on the device never trap: they OR a bit into
+ *    *err_flag (a device int32 the caller zeroes and reads when it wants) and
+ *    the offending request or row is skipped.
+ *  - Inputs are never modified, except the KV-pool rows at positions
+ *    >= kv_len[b] that the step itself appends; a step can be re-issued on the
+ *    same buffers and gives bit-identical results (fixed reduction orders, no
+ *    floating-point atomics).
+ *
+ * Slot layout of the block (Q = 2N-1 rows per request, request-major):
+ *   rows 0..N-1 are CLEAN slots: the first c = n_clean[b] hold the tokens
+ *   t_1..t_c at positions kv_len..kv_len+c-1, the rest are inactive;
+ *   rows N..2N-2 are MASK slots at positions kv_len+c .. kv_len+c+N-2.
+ *   By the logit shift ([EXP §三项关键训练创新]) the hidden state of a slot
+ *   predicts the token one position later, so t_1 is always accepted
+ *   ([PRJ], geometric acceptance paragraph).
+ */
+#ifndef ISD_H_
+#define ISD_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef int32_t isd_status;
+#define ISD_OK                     0
+#define ISD_ERR_INVALID_ARG       (-1)  /* null pointer, bad dims or mode */
+#define ISD_ERR_UNSUPPORTED_SHAPE (-2)  /* valid but not built: see each call */
+#define ISD_ERR_WORKSPACE         (-3)  /* ws too small or misaligned */
+#define ISD_ERR_CUDA              (-4)  /* a CUDA launch or driver call failed */
+
+/* Bits OR-ed into *err_flag by the kernels (never a trap). */
+#define ISD_FLAG_PAGE_OOB      1  /* a page id outside [0, num_pages) */
+#define ISD_FLAG_TOKEN_OOB     2  /* a clean token outside [0, V) */
+#define ISD_FLAG_NCLEAN_RANGE  4  /* n_clean outside [1, N] */
+#define ISD_FLAG_CAPACITY      8  /* kv_len + block exceeds the request's page capacity */
+#define ISD_FLAG_WAIT_TIMEOUT 16  /* a bounded on-chip wait gave up (LM-head pipeline) */
+
+#define ISD_PROPOSE_ARGMAX 0      /* argmax proposals ([ENG §服务部署与 SGLang 集成]) */
+#define ISD_PROPOSE_SAMPLE 1      /* inverse-CDF draws with the u_prop uniforms */
+
+typedef struct {
+    int32_t B;                  /* requests in the batch */
+    int32_t N;                  /* stride; the block has Q = 2N-1 slots */
+    int32_t Hq, Hkv, D;         /* query heads, KV heads (Hq % Hkv == 0), head dim */
+    int32_t V;                  /* vocabulary size */
+    int32_t page_size;          /* tokens per KV page (P) */
+    int32_t num_pages;          /* pages in each of k_pool / v_pool */
+    int32_t max_pages_per_req;  /* columns of page_table */
+    int32_t lora_rank;          /* 0 = no R-ISD adapter, else the rank r */
+    int32_t proposal_mode;      /* ISD_PROPOSE_ARGMAX or ISD_PROPOSE_SAMPLE */
+    float sm_scale;             /* attention logit scale, usually 1/sqrt(D) */
+} isd_dims;
+
+/* Per logits row: max, sum_i exp(z_i - max), argmax (ties -> lowest index). */
+typedef struct {
+    float max;
+    float sumexp;
+    int32_t argmax;
+    int32_t reserved;
+} isd_row_stat;
+
+/* Bytes of scratch needed by any entry point for these dims (isd_step's
+ * need is the largest).  Returns 0 for invalid dims. */
+size_t isd_workspace_bytes(const isd_dims* d);
+
+/* Static, human-readable name of a status code. */
+const char* isd_status_string(isd_status s);
+
+/* Detail of the last failing call on this host thread ("" if none). */
+const char* isd_last_error(void);
+
+/*
+ * isd_attention -- KV append + strict-causal GQA attention over the paged
+ * cache plus the block ([EXP §三项关键训练创新, 严格因果掩码]; paged KV cache
+ * per [EXP §推理：复用 AR 推理栈]).
+ *   q      [B, Q, Hq, D]  bf16   query vectors of the block slots
+ *   k_new  [B, Q, Hkv, D] bf16   keys of the block slots
+ *   v_new  [B, Q, Hkv, D] bf16   values of the block slots
+ *   k_pool, v_pool [num_pages, page_size, Hkv, D] bf16, in/out: the active
+ *          slots' K/V rows are written at their positions (page
+ *          page_table[b][pos / P], row pos % P)
+ *   page_table [B, max_pages_per_req] int32; kv_len [B] int32 (cached
+ *          prefix length); n_clean [B] int32 (c in [1, N])
+ *   out    [B*Q, Hq*D] bf16: for each active slot s and head h, the softmax
+ *          (sm_scale q.k) weighted sum of v over keys at positions <= pos_s,
+ *          query head h reading KV head h / (Hq/Hkv); inactive slots -> 0.
+ * Supported: D in {64, 128}; (Hq/Hkv)*Q <= 128.
+ */
+isd_status isd_attention(const isd_dims* d, const uint16_t* q, const uint16_t* k_new,
+                         const uint16_t* v_new, uint16_t* k_pool, uint16_t* v_pool,
+                         const int32_t* page_table, const int32_t* kv_len,
+                         const int32_t* n_clean, uint16_t* out, void* ws, size_t ws_bytes,
+                         int32_t* err_flag, void* stream);
+
+/*
+ * isd_lm_head -- (optional R-ISD gated LoRA on MASK rows) + LM head + row
+ * statistics.  [EXP §ISD 核心逻辑伪代码] maps every slot to a vocabulary
+ * distribution; [ENG §Token 生成的核心参数与验收机制] and [PRJ] (R-ISD) apply
+ * the rank-r gated adapter at MASK positions only.
+ *   hidden [B*Q, H] bf16 (H = Hq*D)
+ *   W      [V, H] bf16
+ *   lora_A [H, r] bf16, lora_B [r, H] bf16 (both NULL iff lora_rank == 0):
+ *          MASK rows use h' = bf16(h + bf16(h A) B); clean rows use h.
+ *   logits [B*Q, V] fp32 = h' . W^T (fp32 accumulation on tensor cores)
+ *   row_stats [B*Q] isd_row_stat, or NULL to skip the statistics.
+ * Supported: H % 64 == 0, B*Q <= 512, V >= 1.
+ */
+isd_status isd_lm_head(const isd_dims* d, const uint16_t* hidden, const uint16_t* W,
+                       const uint16_t* lora_A, const uint16_t* lora_B, float* logits,
+                       isd_row_stat* row_stats, void* ws, size_t ws_bytes, int32_t* err_flag,
+                       void* stream);
+
+/* isd_row_stats -- row statistics of `rows` fp32 logits rows of length V. */
+isd_status isd_row_stats(const isd_dims* d, const float* logits, int32_t rows,
+                         isd_row_stat* row_stats, void* ws, size_t ws_bytes, void* stream);
+
+/*
+ * isd_accept -- p/q verification, residual draw, next-stride proposals and
+ * state update ([EXP §Introspective Strided Decoding（ISD）];
+ * [ENG §从质量差距到自省机制]).  For request b with c = n_clean[b]:
+ *   for j = 2..c: x = t_j, p = softmax(logits row (b, j-2)), q = softmax
+ *   (prev_logits row (b, N+j-2)); accept iff u_acc[j-2] < p(x)/q(x); the
+ *   first rejection stops.  On a rejection at j the replacement is drawn by
+ *   inverse CDF from max(0, p - q) with u_res (argmax p if that mass is 0);
+ *   otherwise the next proposals are x'_1 from row (b, c-1) and x'_{m+2} from
+ *   row (b, N+m) (argmax, or inverse CDF with u_prop in sample mode).
+ *   logits, prev_logits [B, Q, V] fp32 (this and the previous step's)
+ *   row_stats, prev_row_stats [B*Q] isd_row_stat of those logits
+ *   n_clean [B], clean_tok [B, N], kv_len [B] int32
+ *   uniforms [B, 2N] fp32 in [0,1): u_acc[0..N-2], u_res[N-1], u_prop[N..2N-1]
+ * Outputs (int32):
+ *   accept_len [B] = A = 1 + accepted proposals = tokens emitted this step
+ *   out_tok [B, N]: t_2..t_A then the replacement (or x'_1); -1 padded
+ *   next_n_clean [B] (1 after a rejection, else N); next_clean_tok [B, N]
+ *   (-1 padded); next_kv_len [B] = kv_len + A
+ *   ratio [B, max(N-1,1)] fp32 or NULL: p/q of each tested proposal, -1 if
+ *   not tested.
+ */
+isd_status isd_accept(const isd_dims* d, const float* logits, const isd_row_stat* row_stats,
+                      const float* prev_logits, const isd_row_stat* prev_row_stats,
+                      const int32_t* n_clean, const int32_t* clean_tok, const int32_t* kv_len,
+                      const float* uniforms, int32_t* accept_len, int32_t* out_tok,
+                      int32_t* next_n_clean, int32_t* next_clean_tok, int32_t* next_kv_len,
+                      float* ratio, void* ws, size_t ws_bytes, int32_t* err_flag, void* stream);
+
+/*
+ * isd_step -- the whole step: isd_attention, then isd_lm_head (with row
+ * statistics), then isd_accept, enqueued back to back on `stream`.
+ * `hidden` [B*Q, H] bf16 receives the attention output if non-NULL (else it
+ * stays in ws).  `logits` and `row_stats` are outputs of this step and become
+ * the caller's prev_logits / prev_row_stats for the next one.
+ */
+isd_status isd_step(const isd_dims* d, const uint16_t* q, const uint16_t* k_new,
+                    const uint16_t* v_new, uint16_t* k_pool, uint16_t* v_pool,
+                    const int32_t* page_table, const int32_t* kv_len, const int32_t* n_clean,
+                    const int32_t* clean_tok, const uint16_t* W, const uint16_t* lora_A,
+                    const uint16_t* lora_B, const float* prev_logits,
+                    const isd_row_stat* prev_row_stats, const float* uniforms,
+                    uint16_t* hidden, float* logits, isd_row_stat* row_stats,
+                    int32_t* accept_len, int32_t* out_tok, int32_t* next_n_clean,
+                    int32_t* next_clean_tok, int32_t* next_kv_len, float* ratio, void* ws,
+                    size_t ws_bytes, int32_t* err_flag, void* stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* ISD_H_ */

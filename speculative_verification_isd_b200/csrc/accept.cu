@@ -1,0 +1,413 @@
+// Row statistics (a5) and the fused p/q accept / residual draw / proposal /
+// state-update kernel (a6-a9) of the ISD step.
+//
+// Verification follows the p/q criterion min(1, p(x)/q(x)) of the I-DLM pages
+// ("I-DLM：扩散模型如何用“自省一致性”追上自回归模型质量", section
+// "Introspective Strided Decoding（ISD）"; "自省扩散语言模型的 token 生成机制与
+// 工程实践", section "从质量差距到自省机制"): p is the anchor distribution of the
+// clean slot one position earlier (logit shift), q the proposal distribution
+// of the MASK slot that proposed the token in the previous step.  Proposals
+// are argmax ("服务部署与 SGLang 集成": argmax proposal strategy) unless sample
+// mode is selected.  A rejection draws its replacement from max(0, p - q), the
+// rule under which the pages' "lossless" claim holds.
+//
+// All reductions run in a fixed order (no floating-point atomics), so a
+// repeated call is bit-identical.  Cross-CTA combination uses the
+// last-block-done ticket: every CTA publishes its partial, fences, and the
+// CTA that draws the last ticket combines; nothing spins.
+#include "common.cuh"
+#include "plan.h"
+
+namespace isd {
+
+// ---------------------------------------------------------------------------
+// a5: per-row max, sum exp(z - max), argmax (ties -> lowest index)
+// ---------------------------------------------------------------------------
+template <int THREADS>
+__global__ void __launch_bounds__(THREADS)
+row_stats_kernel(const float* __restrict__ logits, int V, int n_chunks, int chunk_len,
+                 float4* __restrict__ part, int* __restrict__ ticket,
+                 isd_row_stat* __restrict__ out) {
+    const int row = blockIdx.y;
+    const int ch = blockIdx.x;
+    const int beg = ch * chunk_len;
+    const int end = min(V, beg + chunk_len);
+    const float* z = logits + (size_t)row * V;
+    RowStat st = rowstat_empty();
+    if ((V & 3) == 0) {
+        for (int i = beg + 4 * threadIdx.x; i < end; i += 4 * THREADS) {
+            const float4 v = ld_stream_f4(z + i);
+            rowstat_push(st, v.x, i);
+            rowstat_push(st, v.y, i + 1);
+            rowstat_push(st, v.z, i + 2);
+            rowstat_push(st, v.w, i + 3);
+        }
+    } else {
+        for (int i = beg + threadIdx.x; i < end; i += THREADS) rowstat_push(st, __ldg(z + i), i);
+    }
+    st = rowstat_block_reduce<THREADS>(st);
+    if (threadIdx.x != 0) return;
+    if (n_chunks == 1) {
+        out[row] = isd_row_stat{st.m, st.s, st.idx, 0};
+        return;
+    }
+    part[(size_t)row * n_chunks + ch] = make_float4(st.m, st.s, __int_as_float(st.idx), 0.f);
+    __threadfence();
+    const int t = atomicAdd(&ticket[row], 1);
+    if (t != n_chunks - 1) return;
+    __threadfence();
+    RowStat acc = rowstat_empty();
+    for (int k = 0; k < n_chunks; ++k) {
+        const float4 p = __ldcg(&part[(size_t)row * n_chunks + k]);
+        acc = rowstat_merge(acc, RowStat{p.x, p.y, __float_as_int(p.z)});
+    }
+    out[row] = isd_row_stat{acc.m, acc.s, acc.idx, 0};
+    ticket[row] = 0;
+}
+
+// ---------------------------------------------------------------------------
+// a6-a9
+// ---------------------------------------------------------------------------
+struct AcceptArgs {
+    int B, N, V, mode;
+    const float* logits;
+    const isd_row_stat* stats;
+    const float* prev_logits;
+    const isd_row_stat* prev_stats;
+    const int32_t* n_clean;
+    const int32_t* clean_tok;
+    const int32_t* kv_len;
+    const float* uniforms;
+    int32_t* accept_len;
+    int32_t* out_tok;
+    int32_t* next_n_clean;
+    int32_t* next_clean_tok;
+    int32_t* next_kv_len;
+    float* ratio;
+    float* part;     // [B][N+1][n_chunks] chunk totals
+    int* ticket;     // [B]
+    int n_chunks;
+    int32_t* err_flag;
+};
+
+// Weight of vocabulary entry i for "row" r of a sweep.
+//   residual (r = 0 of a rejecting request): max(0, p_i - q_i)
+//   sample-mode proposal rows: exp(z_i - max) of that row
+struct SweepRow {
+    const float* zp;
+    const float* zq;  // null for proposal rows
+    float mp, inv_sp, mq, inv_sq;
+};
+
+ISD_DEVINL float sweep_weight(const SweepRow& r, int i) {
+    const float a = __expf(__ldg(r.zp + i) - r.mp);
+    if (!r.zq) return a;
+    const float p = a * r.inv_sp;
+    const float q = __expf(__ldg(r.zq + i) - r.mq) * r.inv_sq;
+    return fmaxf(p - q, 0.f);
+}
+
+constexpr int kSeg = kAcceptChunk / kAcceptThreads;  // contiguous entries per thread
+
+// Exclusive block scan of one float per thread (fixed order); returns the
+// exclusive prefix and writes the block total to *total.
+ISD_DEVINL float block_exclusive_scan(float v, float* total) {
+    __shared__ float warp_tot[kAcceptThreads / 32];
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    float incl = v;
+#pragma unroll
+    for (int off = 1; off < 32; off <<= 1) {
+        const float n = __shfl_up_sync(0xffffffffu, incl, off);
+        if (lane >= off) incl += n;
+    }
+    if (lane == 31) warp_tot[warp] = incl;
+    __syncthreads();
+    float base = 0.f, tot = 0.f;
+#pragma unroll
+    for (int w = 0; w < kAcceptThreads / 32; ++w) {
+        if (w < warp) base += warp_tot[w];
+        tot += warp_tot[w];
+    }
+    __syncthreads();
+    *total = tot;
+    return base + incl - v;
+}
+
+// Chunk [beg, end): per-thread contiguous segments; returns the chunk total
+// (identical bits every time it is recomputed) and, if target >= 0, the first
+// index whose prefix exceeds target (or -1).
+ISD_DEVINL float chunk_scan(const SweepRow& r, int beg, int end, float target, int* found) {
+    float w[kSeg];
+    float local = 0.f;
+    const int s0 = beg + threadIdx.x * kSeg;
+#pragma unroll
+    for (int k = 0; k < kSeg; ++k) {
+        const int i = s0 + k;
+        w[k] = (i < end) ? sweep_weight(r, i) : 0.f;
+        local += w[k];
+    }
+    float total;
+    const float excl = block_exclusive_scan(local, &total);
+    if (target >= 0.f) {
+        __shared__ int first;
+        if (threadIdx.x == 0) first = 0x7fffffff;
+        __syncthreads();
+        if (excl + local > target) atomicMin(&first, (int)threadIdx.x);
+        __syncthreads();
+        int idx = -1;
+        if ((int)threadIdx.x == first) {
+            float part = 0.f;
+            for (int k = 0; k < kSeg; ++k) {
+                part += w[k];
+                if (w[k] > 0.f && excl + part > target) {
+                    idx = s0 + k;
+                    break;
+                }
+            }
+        }
+        // last index with positive weight, for the rounding fallback
+        __shared__ int last_pos, hit;
+        if (threadIdx.x == 0) {
+            last_pos = -1;
+            hit = -1;
+        }
+        __syncthreads();
+        for (int k = kSeg - 1; k >= 0; --k)
+            if (w[k] > 0.f && s0 + k < end) {
+                atomicMax(&last_pos, s0 + k);
+                break;
+            }
+        if (idx >= 0) hit = idx;
+        __syncthreads();
+        *found = hit >= 0 ? hit : last_pos;
+        __syncthreads();
+    }
+    return total;
+}
+
+__global__ void __launch_bounds__(kAcceptThreads) accept_kernel(AcceptArgs a) {
+    const int b = blockIdx.y;
+    const int ch = blockIdx.x;
+    const int N = a.N, Q = 2 * N - 1, V = a.V;
+    const int rcols = N > 1 ? N - 1 : 1;
+    __shared__ int s_state;  // -1 invalid request, 0 no rejection, j = rejected proposal index
+    __shared__ int s_c;
+    __shared__ int s_last;
+    const float* ub = a.uniforms + (size_t)b * 2 * N;
+    if (threadIdx.x == 0) {
+        const int c = a.n_clean[b];
+        int state = 0;
+        if (c < 1 || c > N) {
+            raise_flag(a.err_flag, ISD_FLAG_NCLEAN_RANGE);
+            state = -1;
+        } else {
+            for (int j = 2; j <= c; ++j) {
+                const int x = a.clean_tok[(size_t)b * N + j - 1];
+                if (x < 0 || x >= V) {
+                    raise_flag(a.err_flag, ISD_FLAG_TOKEN_OOB);
+                    state = -1;
+                    break;
+                }
+                const size_t rp = (size_t)b * Q + (j - 2);
+                const size_t rq = (size_t)b * Q + (N + j - 2);
+                const isd_row_stat sp = a.stats[rp], sq = a.prev_stats[rq];
+                const float zp = a.logits[rp * V + x];
+                const float zq = a.prev_logits[rq * V + x];
+                // p(x)/q(x) = exp((zp - mp) - (zq - mq)) * Sq / Sp
+                const float r = expf((zp - sp.max) - (zq - sq.max)) * (sq.sumexp / sp.sumexp);
+                if (ch == 0 && a.ratio) a.ratio[(size_t)b * rcols + j - 2] = r;
+                if (!(ub[j - 2] < r)) {
+                    state = j;
+                    break;
+                }
+            }
+        }
+        if (ch == 0 && a.ratio && state >= 0) {
+            const int tested = state > 0 ? state - 1 : c - 1;
+            for (int k = tested; k < rcols; ++k) a.ratio[(size_t)b * rcols + k] = -1.f;
+        }
+        s_state = state;
+        s_c = c;
+    }
+    __syncthreads();
+    const int state = s_state, c = s_c;
+    const int* tok = a.clean_tok + (size_t)b * N;
+    if (state < 0) {  // invalid request: emit nothing, carry the state over
+        if (ch == 0 && threadIdx.x == 0) {
+            a.accept_len[b] = 0;
+            a.next_n_clean[b] = c;
+            a.next_kv_len[b] = a.kv_len[b];
+            for (int k = 0; k < N; ++k) {
+                a.out_tok[(size_t)b * N + k] = -1;
+                a.next_clean_tok[(size_t)b * N + k] = tok[k];
+            }
+            if (a.ratio)
+                for (int k = 0; k < rcols; ++k) a.ratio[(size_t)b * rcols + k] = -1.f;
+        }
+        return;
+    }
+    const bool sweep = state > 0 || a.mode == ISD_PROPOSE_SAMPLE;
+    const int nrows = state > 0 ? 1 : N;
+    // Describe the rows to sweep (or the argmax rows).
+    auto row_of = [&](int k, SweepRow* r) {
+        if (state > 0) {
+            const size_t rp = (size_t)b * Q + (state - 2);
+            const size_t rq = (size_t)b * Q + (N + state - 2);
+            const isd_row_stat sp = a.stats[rp], sq = a.prev_stats[rq];
+            *r = SweepRow{a.logits + rp * V, a.prev_logits + rq * V, sp.max, 1.f / sp.sumexp,
+                          sq.max, 1.f / sq.sumexp};
+        } else {
+            const size_t rr = (size_t)b * Q + (k == 0 ? c - 1 : N + k - 1);
+            const isd_row_stat s = a.stats[rr];
+            *r = SweepRow{a.logits + rr * V, nullptr, s.max, 0.f, 0.f, 0.f};
+        }
+    };
+    int picked[16];  // N <= 16 (checked on the host)
+    if (sweep) {
+        const int beg = ch * kAcceptChunk, end = min(V, beg + kAcceptChunk);
+        float* part = a.part + (size_t)b * (N + 1) * a.n_chunks;
+        for (int k = 0; k < nrows; ++k) {
+            SweepRow r;
+            row_of(k, &r);
+            int dummy;
+            const float tot = chunk_scan(r, beg, end, -1.f, &dummy);
+            if (threadIdx.x == 0) part[(size_t)k * a.n_chunks + ch] = tot;
+        }
+        __threadfence();
+        __syncthreads();
+        if (threadIdx.x == 0) s_last = (atomicAdd(&a.ticket[b], 1) == a.n_chunks - 1);
+        __syncthreads();
+        if (!s_last) return;
+        __threadfence();
+        for (int k = 0; k < nrows; ++k) {
+            SweepRow r;
+            row_of(k, &r);
+            const float u = state > 0 ? ub[N - 1] : ub[N + k];
+            // totals in chunk order
+            __shared__ float s_target;
+            __shared__ int s_chunk;
+            if (threadIdx.x == 0) {
+                float total = 0.f;
+                for (int q = 0; q < a.n_chunks; ++q) total += __ldcg(&part[(size_t)k * a.n_chunks + q]);
+                const float target = u * total;
+                float cum = 0.f;
+                int hit = -1, lastpos = -1;
+                float local = 0.f;
+                for (int q = 0; q < a.n_chunks; ++q) {
+                    const float t = __ldcg(&part[(size_t)k * a.n_chunks + q]);
+                    if (t > 0.f) lastpos = q;
+                    if (hit < 0 && cum + t > target) {
+                        hit = q;
+                        local = target - cum;
+                    }
+                    cum += t;
+                }
+                if (total <= 0.f) {
+                    s_chunk = -2;  // no mass: residual falls back to argmax p
+                } else if (hit < 0) {
+                    s_chunk = lastpos;
+                    local = 3.0e38f;  // take the last positive entry of that chunk
+                } else {
+                    s_chunk = hit;
+                }
+                s_target = fmaxf(local, 0.f);
+            }
+            __syncthreads();
+            const int q = s_chunk;
+            const float tgt = s_target;
+            __syncthreads();
+            int y;
+            if (q == -2) {  // argmax of the anchor (or proposal) row
+                const size_t fr = state > 0 ? (size_t)b * Q + (state - 2)
+                                            : (size_t)b * Q + (k == 0 ? c - 1 : N + k - 1);
+                y = a.stats[fr].argmax;
+            } else {
+                const int beg2 = q * kAcceptChunk, end2 = min(V, beg2 + kAcceptChunk);
+                chunk_scan(r, beg2, end2, tgt, &y);
+            }
+            if (threadIdx.x == 0) picked[k] = y;
+        }
+        if (threadIdx.x == 0) a.ticket[b] = 0;
+    } else {
+        if (ch != 0) return;
+        if (threadIdx.x == 0) {
+            picked[0] = a.stats[(size_t)b * Q + c - 1].argmax;
+            for (int m = 0; m + 1 < N; ++m) picked[m + 1] = a.stats[(size_t)b * Q + N + m].argmax;
+        }
+    }
+    if (threadIdx.x != 0) return;
+    // a9: emitted tokens and next state
+    int32_t* ot = a.out_tok + (size_t)b * N;
+    int32_t* nt = a.next_clean_tok + (size_t)b * N;
+    int A;
+    if (state > 0) {
+        A = state - 1;
+        for (int k = 0; k < A - 1; ++k) ot[k] = tok[k + 1];
+        ot[A - 1] = picked[0];
+        for (int k = A; k < N; ++k) ot[k] = -1;
+        nt[0] = picked[0];
+        for (int k = 1; k < N; ++k) nt[k] = -1;
+        a.next_n_clean[b] = 1;
+    } else {
+        A = c;
+        for (int k = 0; k < c - 1; ++k) ot[k] = tok[k + 1];
+        ot[c - 1] = picked[0];
+        for (int k = c; k < N; ++k) ot[k] = -1;
+        for (int k = 0; k < N; ++k) nt[k] = picked[k];
+        a.next_n_clean[b] = N;
+    }
+    a.accept_len[b] = A;
+    a.next_kv_len[b] = a.kv_len[b] + A;
+}
+
+// ---------------------------------------------------------------------------
+// launchers
+// ---------------------------------------------------------------------------
+cudaError_t launch_row_stats(const Plan& p, const float* logits, int rows, int V,
+                             isd_row_stat* out, void* ws, cudaStream_t st) {
+    char* w = static_cast<char*>(ws);
+    dim3 grid(p.stats_chunks, rows);
+    row_stats_kernel<kStatsThreads><<<grid, kStatsThreads, 0, st>>>(
+        logits, V, p.stats_chunks, p.stats_chunk_len,
+        reinterpret_cast<float4*>(w + p.off_stats_part),
+        reinterpret_cast<int*>(w + p.off_stats_ticket), out);
+    return cudaGetLastError();
+}
+
+cudaError_t launch_accept(const Plan& p, const isd_dims* d, const float* logits,
+                          const isd_row_stat* stats, const float* prev_logits,
+                          const isd_row_stat* prev_stats, const int32_t* n_clean,
+                          const int32_t* clean_tok, const int32_t* kv_len, const float* uniforms,
+                          int32_t* accept_len, int32_t* out_tok, int32_t* next_n_clean,
+                          int32_t* next_clean_tok, int32_t* next_kv_len, float* ratio, void* ws,
+                          int32_t* err_flag, cudaStream_t st) {
+    char* w = static_cast<char*>(ws);
+    AcceptArgs a;
+    a.B = d->B;
+    a.N = d->N;
+    a.V = d->V;
+    a.mode = d->proposal_mode;
+    a.logits = logits;
+    a.stats = stats;
+    a.prev_logits = prev_logits;
+    a.prev_stats = prev_stats;
+    a.n_clean = n_clean;
+    a.clean_tok = clean_tok;
+    a.kv_len = kv_len;
+    a.uniforms = uniforms;
+    a.accept_len = accept_len;
+    a.out_tok = out_tok;
+    a.next_n_clean = next_n_clean;
+    a.next_clean_tok = next_clean_tok;
+    a.next_kv_len = next_kv_len;
+    a.ratio = ratio;
+    a.part = reinterpret_cast<float*>(w + p.off_acc_part);
+    a.ticket = reinterpret_cast<int*>(w + p.off_acc_ticket);
+    a.n_chunks = p.acc_chunks;
+    a.err_flag = err_flag;
+    dim3 grid(p.acc_chunks, d->B);
+    accept_kernel<<<grid, kAcceptThreads, 0, st>>>(a);
+    return cudaGetLastError();
+}
+
+}  // namespace isd

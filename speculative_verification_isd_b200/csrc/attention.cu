@@ -1,0 +1,517 @@
+// KV append (a1) and strict-causal GQA attention over the paged cache (a2).
+//
+// Strict causal attention over clean and MASK slots alike is the first of the
+// training changes on "I-DLM：扩散模型如何用“自省一致性”追上自回归模型质量"
+// (section "三项关键训练创新", 严格因果掩码); the paged KV cache is the AR
+// serving structure the same page reuses (section "推理：复用 AR 推理栈").
+//
+// Design (B200, memory-bound: ~28 flop per KV byte):
+//  * one CTA per (request, KV head, split of the key range, row-group block);
+//    the grp*Q query rows that share a KV head (28 for Qwen3-8B at N=4) are
+//    processed together, so every KV byte is read from HBM once;
+//  * keys stream through a 3-stage cp.async pipeline in 64-key tiles gathered
+//    page by page (XOR-swizzled 16-byte chunks, conflict-free ldmatrix);
+//  * each warp owns 16 keys of a tile and all 32 rows of its row group:
+//    S = Q K^T and O += P V on mma.sync m16n8k16 (bf16 in, fp32 accumulate),
+//    online softmax in the log2 domain;
+//  * warps merge in a fixed order; splits of one (request, head) are merged
+//    by the CTA that draws the last ticket (no spinning, deterministic);
+//  * block keys are read from k_new/v_new directly, and the CTA of the last
+//    split writes them into the pages, so the append needs no ordering.
+#include "common.cuh"
+#include "plan.h"
+
+namespace isd {
+
+constexpr int kStages = 3;
+constexpr int kKT = kAttnKeyTile;
+
+struct AttnArgs {
+    int B, N, Q, Hq, Hkv, grp, rows, P, num_pages, max_pages, split, n_rgb;
+    float scale_log2;  // sm_scale * log2(e)
+    const __nv_bfloat16* q;
+    const __nv_bfloat16* k_new;
+    const __nv_bfloat16* v_new;
+    __nv_bfloat16* k_pool;
+    __nv_bfloat16* v_pool;
+    const int32_t* page_table;
+    const int32_t* kv_len;
+    const int32_t* n_clean;
+    __nv_bfloat16* out;
+    char* part;
+    size_t part_stride;
+    int max_splits;
+    int* ticket;
+    int32_t* err_flag;
+};
+
+// smem byte offset of 16-byte chunk `c` of row `r` (rows of D bf16)
+template <int D>
+ISD_DEVINL uint32_t swz(int r, int c) {
+    return (uint32_t)(r * D * 2 + ((c ^ (r & 7)) << 4));
+}
+
+// position of block slot s (-1 = inactive), c clean tokens
+ISD_DEVINL int slot_pos(int s, int kv, int c, int N) {
+    if (s < c) return kv + s;
+    if (s < N) return -1;
+    return kv + c + (s - N);
+}
+
+template <int D, int NRG>
+__global__ void __launch_bounds__(128 * NRG) attention_kernel(AttnArgs a) {
+    constexpr int THREADS = 128 * NRG;
+    constexpr int ROWS = 32 * NRG;
+    constexpr int CH = D / 8;  // 16-byte chunks per row
+    constexpr int NT = D / 8;  // n8 tiles of the output
+    extern __shared__ __align__(128) unsigned char smem[];
+    unsigned char* sQ = smem;
+    unsigned char* sK = smem + ROWS * D * 2;
+    unsigned char* sV = sK + kStages * kKT * D * 2;
+
+    const int sp = blockIdx.x;
+    const int g = blockIdx.y / a.n_rgb;
+    const int rgb = blockIdx.y % a.n_rgb;
+    const int b = blockIdx.z;
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    const int rg = warp >> 2;          // row group of this warp
+    const int kw = (warp & 3) * 16;    // this warp's keys within a tile
+
+    const int kv = a.kv_len[b];
+    const int c = a.n_clean[b];
+    const bool bad_c = (c < 1 || c > a.N);
+    const long long want = bad_c ? 0 : (long long)kv + c + a.N - 1;  // keys incl. the block
+    const bool over = kv < 0 || (want + a.P - 1) / a.P > a.max_pages;
+    // a request that cannot be served (bad n_clean, negative or over-capacity
+    // length) is one empty split: its rows are written as zeros
+    const int total = (bad_c || over) ? 0 : (int)want;
+    const int ns = total > 0 ? (total + a.split - 1) / a.split : 1;
+    if (sp >= ns) return;
+    if (tid == 0 && sp == 0 && rgb == 0) {
+        if (bad_c) raise_flag(a.err_flag, ISD_FLAG_NCLEAN_RANGE);
+        else if (over) raise_flag(a.err_flag, ISD_FLAG_CAPACITY);
+    }
+    const int kbeg = sp * a.split;
+    const int kend = min(total, kbeg + a.split);
+    const int32_t* ptab = a.page_table + (size_t)b * a.max_pages;
+    const size_t row_stride = (size_t)a.Hkv * D;  // elements between consecutive positions
+
+    // ---- a1: the last split's CTA appends the block's K/V rows to the pages
+    if (sp == ns - 1 && rgb == 0 && total > 0) {
+        const int nblk = c + a.N - 1;
+        for (int i = tid; i < nblk * CH; i += THREADS) {
+            const int r = i / CH, cc = i % CH;
+            const int t = kv + r;
+            const int slot = r < c ? r : a.N + (r - c);
+            const int page = ptab[t / a.P];
+            if (page < 0 || page >= a.num_pages) {
+                raise_flag(a.err_flag, ISD_FLAG_PAGE_OOB);
+                continue;
+            }
+            const size_t dst = ((size_t)page * a.P + t % a.P) * row_stride + (size_t)g * D + cc * 8;
+            const size_t src = (((size_t)b * a.Q + slot) * a.Hkv + g) * D + cc * 8;
+            *reinterpret_cast<uint4*>(a.k_pool + dst) = *reinterpret_cast<const uint4*>(a.k_new + src);
+            *reinterpret_cast<uint4*>(a.v_pool + dst) = *reinterpret_cast<const uint4*>(a.v_new + src);
+        }
+    }
+
+    // ---- query rows of this CTA -> smem (zero rows for padding / inactive)
+    const int row0 = rgb * ROWS;
+    for (int i = tid; i < ROWS * CH; i += THREADS) {
+        const int r = i / CH, cc = i % CH;
+        const int rr = row0 + r;
+        uint4 v = make_uint4(0, 0, 0, 0);
+        if (rr < a.rows) {
+            const int hh = rr / a.Q, s = rr % a.Q;
+            const int h = g * a.grp + hh;
+            v = *reinterpret_cast<const uint4*>(a.q + (((size_t)b * a.Q + s) * a.Hq + h) * D + cc * 8);
+        }
+        *reinterpret_cast<uint4*>(sQ + swz<D>(r, cc)) = v;
+    }
+
+    // positions of the 4 rows this thread holds in the S/O fragments
+    int rpos[4];
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+        const int r = rg * 32 + (i >> 1) * 16 + (i & 1) * 8 + (lane >> 2);
+        const int rr = row0 + r;
+        rpos[i] = (rr < a.rows && total > 0) ? slot_pos(rr % a.Q, kv, c, a.N) : -1;
+    }
+
+    // ---- tile loader: keys [k0, k0+64) of this (request, head)
+    auto load_tile = [&](int stage, int k0) {
+        unsigned char* dk = sK + stage * kKT * D * 2;
+        unsigned char* dv = sV + stage * kKT * D * 2;
+        for (int i = tid; i < kKT * CH; i += THREADS) {
+            const int key = i / CH, cc = i % CH;
+            const int t = k0 + key;
+            const __nv_bfloat16* srck = a.k_new;
+            const __nv_bfloat16* srcv = a.v_new;
+            int bytes = 0;
+            if (t < kend) {
+                size_t off;
+                if (t < kv) {
+                    const int page = ptab[t / a.P];
+                    if (page >= 0 && page < a.num_pages) {
+                        off = ((size_t)page * a.P + t % a.P) * row_stride + (size_t)g * D + cc * 8;
+                        srck = a.k_pool;
+                        srcv = a.v_pool;
+                        bytes = 16;
+                    } else {
+                        raise_flag(a.err_flag, ISD_FLAG_PAGE_OOB);
+                        off = 0;
+                    }
+                } else {
+                    const int r = t - kv;
+                    const int slot = r < c ? r : a.N + (r - c);
+                    off = (((size_t)b * a.Q + slot) * a.Hkv + g) * D + cc * 8;
+                    bytes = 16;
+                }
+                srck += off;
+                srcv += off;
+            }
+            cp_async16(smem_u32(dk + swz<D>(key, cc)), srck, bytes);
+            cp_async16(smem_u32(dv + swz<D>(key, cc)), srcv, bytes);
+        }
+    };
+
+    float o[2][NT][4];
+#pragma unroll
+    for (int mt = 0; mt < 2; ++mt)
+#pragma unroll
+        for (int nt = 0; nt < NT; ++nt)
+#pragma unroll
+            for (int e = 0; e < 4; ++e) o[mt][nt][e] = 0.f;
+    float m_run[4], l_run[4];
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+        m_run[i] = -INFINITY;
+        l_run[i] = 0.f;
+    }
+
+    const int n_tiles = (kend - kbeg + kKT - 1) / kKT;
+#pragma unroll
+    for (int s = 0; s < kStages - 1; ++s) {
+        if (s < n_tiles) load_tile(s, kbeg + s * kKT);
+        cp_async_commit();
+    }
+    const uint32_t q_base = smem_u32(sQ);
+    for (int it = 0; it < n_tiles; ++it) {
+        cp_async_wait<kStages - 2>();
+        __syncthreads();
+        {
+            const int nxt = it + kStages - 1;
+            if (nxt < n_tiles) load_tile(nxt % kStages, kbeg + nxt * kKT);
+            cp_async_commit();
+        }
+        const int stage = it % kStages;
+        const uint32_t k_base = smem_u32(sK + stage * kKT * D * 2);
+        const uint32_t v_base = smem_u32(sV + stage * kKT * D * 2);
+        const int k0 = kbeg + it * kKT + kw;  // first key of this warp
+        if (k0 >= kend) continue;             // warp has no keys in this tile
+
+        // S = Q K^T  (32 rows x 16 keys)
+        float s[2][2][4];
+#pragma unroll
+        for (int mt = 0; mt < 2; ++mt)
+#pragma unroll
+            for (int nt = 0; nt < 2; ++nt)
+#pragma unroll
+                for (int e = 0; e < 4; ++e) s[mt][nt][e] = 0.f;
+#pragma unroll
+        for (int kk = 0; kk < D / 16; ++kk) {
+            uint32_t kb[4];
+            {
+                const int j = lane >> 3;
+                const int key = kw + (j >> 1) * 8 + (lane & 7);
+                ldmatrix_x4(kb, k_base + swz<D>(key, kk * 2 + (j & 1)));
+            }
+#pragma unroll
+            for (int mt = 0; mt < 2; ++mt) {
+                uint32_t qa[4];
+                const int j = lane >> 3;
+                const int r = rg * 32 + mt * 16 + (j & 1) * 8 + (lane & 7);
+                ldmatrix_x4(qa, q_base + swz<D>(r, kk * 2 + (j >> 1)));
+                mma_bf16_16816(s[mt][0], qa, kb[0], kb[1]);
+                mma_bf16_16816(s[mt][1], qa, kb[2], kb[3]);
+            }
+        }
+        // mask + online softmax (log2 domain)
+        float alpha[4];
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+            const int mt = i >> 1, hi = i & 1;
+            float mx = -INFINITY;
+#pragma unroll
+            for (int nt = 0; nt < 2; ++nt)
+#pragma unroll
+                for (int e = 0; e < 2; ++e) {
+                    const int key = k0 + nt * 8 + (lane & 3) * 2 + e;
+                    float v = s[mt][nt][hi * 2 + e] * a.scale_log2;
+                    if (key >= kend || key > rpos[i]) v = -INFINITY;
+                    s[mt][nt][hi * 2 + e] = v;
+                    mx = fmaxf(mx, v);
+                }
+            mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 1));
+            mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 2));
+            const float m_new = fmaxf(m_run[i], mx);
+            const float m_use = (m_new == -INFINITY) ? 0.f : m_new;
+            alpha[i] = exp2f(m_run[i] - m_use);
+            float rs = 0.f;
+#pragma unroll
+            for (int nt = 0; nt < 2; ++nt)
+#pragma unroll
+                for (int e = 0; e < 2; ++e) {
+                    const float p = exp2f(s[mt][nt][hi * 2 + e] - m_use);
+                    s[mt][nt][hi * 2 + e] = p;
+                    rs += p;
+                }
+            rs += __shfl_xor_sync(0xffffffffu, rs, 1);
+            rs += __shfl_xor_sync(0xffffffffu, rs, 2);
+            l_run[i] = l_run[i] * alpha[i] + rs;
+            m_run[i] = m_new;
+        }
+#pragma unroll
+        for (int mt = 0; mt < 2; ++mt)
+#pragma unroll
+            for (int nt = 0; nt < NT; ++nt) {
+                o[mt][nt][0] *= alpha[mt * 2];
+                o[mt][nt][1] *= alpha[mt * 2];
+                o[mt][nt][2] *= alpha[mt * 2 + 1];
+                o[mt][nt][3] *= alpha[mt * 2 + 1];
+            }
+        // O += P V  (P: 32 x 16 keys as the A operand, straight from the S fragments)
+        uint32_t pa[2][4];
+#pragma unroll
+        for (int mt = 0; mt < 2; ++mt) {
+            pa[mt][0] = pack_bf16(s[mt][0][0], s[mt][0][1]);
+            pa[mt][1] = pack_bf16(s[mt][0][2], s[mt][0][3]);
+            pa[mt][2] = pack_bf16(s[mt][1][0], s[mt][1][1]);
+            pa[mt][3] = pack_bf16(s[mt][1][2], s[mt][1][3]);
+        }
+#pragma unroll
+        for (int dn = 0; dn < NT; dn += 2) {
+            uint32_t vb[4];
+            const int j = lane >> 3;
+            const int key = kw + (j & 1) * 8 + (lane & 7);
+            ldmatrix_x4_trans(vb, v_base + swz<D>(key, dn + (j >> 1)));
+#pragma unroll
+            for (int mt = 0; mt < 2; ++mt) {
+                mma_bf16_16816(o[mt][dn], pa[mt], vb[0], vb[1]);
+                mma_bf16_16816(o[mt][dn + 1], pa[mt], vb[2], vb[3]);
+            }
+        }
+    }
+    cp_async_wait<0>();
+    __syncthreads();
+
+    // ---- merge the 4 warps of each row group in a fixed order
+    float* red = reinterpret_cast<float*>(sK);   // pipeline buffers are free now
+    float* sm = red;                              // [warps][32] running max
+    float* sl = red + THREADS / 32 * 32;          // [warps][32] running sum
+    float* obuf = red + 2 * (THREADS / 32) * 32;  // [rg][2][NT*8][32]
+    const int wig = warp & 3;  // warp index within its row group
+    if ((lane & 3) == 0) {
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+            const int r = (i >> 1) * 16 + (i & 1) * 8 + (lane >> 2);
+            sm[warp * 32 + r] = m_run[i];
+            sl[warp * 32 + r] = l_run[i];
+        }
+    }
+    __syncthreads();
+    float m_fin[4], l_fin[4];
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+        const int r = (i >> 1) * 16 + (i & 1) * 8 + (lane >> 2);
+        float M = -INFINITY;
+#pragma unroll
+        for (int w = 0; w < 4; ++w) M = fmaxf(M, sm[(rg * 4 + w) * 32 + r]);
+        const float Mu = (M == -INFINITY) ? 0.f : M;
+        float L = 0.f;
+#pragma unroll
+        for (int w = 0; w < 4; ++w) {
+            const int ww = (rg * 4 + w) * 32 + r;
+            L += sl[ww] * exp2f(sm[ww] - Mu);
+        }
+        const float f = exp2f(m_run[i] - Mu);
+        m_fin[i] = M;
+        l_fin[i] = L;
+        const int mt = i >> 1, hi = i & 1;
+#pragma unroll
+        for (int nt = 0; nt < NT; ++nt) {
+            o[mt][nt][hi * 2] *= f;
+            o[mt][nt][hi * 2 + 1] *= f;
+        }
+    }
+    float* my_buf = obuf + (size_t)(rg * 2) * (2 * NT * 4) * 32;  // two buffers per row group
+    auto store_o = [&](float* buf) {
+#pragma unroll
+        for (int mt = 0; mt < 2; ++mt)
+#pragma unroll
+            for (int nt = 0; nt < NT; ++nt)
+#pragma unroll
+                for (int e = 0; e < 4; ++e) buf[((mt * NT + nt) * 4 + e) * 32 + lane] = o[mt][nt][e];
+    };
+    auto add_o = [&](const float* buf) {
+#pragma unroll
+        for (int mt = 0; mt < 2; ++mt)
+#pragma unroll
+            for (int nt = 0; nt < NT; ++nt)
+#pragma unroll
+                for (int e = 0; e < 4; ++e) o[mt][nt][e] += buf[((mt * NT + nt) * 4 + e) * 32 + lane];
+    };
+    const int buf_elems = 2 * NT * 4 * 32;
+    __syncthreads();
+    if (wig >= 2) store_o(my_buf + (wig - 2) * buf_elems);
+    __syncthreads();
+    if (wig < 2) add_o(my_buf + wig * buf_elems);
+    __syncthreads();
+    if (wig == 1) store_o(my_buf);
+    __syncthreads();
+    if (wig == 0) add_o(my_buf);
+
+    // ---- write: direct output (single split) or a partial + ticket combine
+    const size_t unit = ((size_t)b * a.Hkv + g) * a.n_rgb + rgb;
+    if (ns == 1) {
+        if (wig == 0) {
+#pragma unroll
+            for (int i = 0; i < 4; ++i) {
+                const int r = rg * 32 + (i >> 1) * 16 + (i & 1) * 8 + (lane >> 2);
+                const int rr = row0 + r;
+                if (rr >= a.rows) continue;
+                const int hh = rr / a.Q, s = rr % a.Q;
+                const int h = g * a.grp + hh;
+                const float inv = l_fin[i] > 0.f ? 1.f / l_fin[i] : 0.f;
+                __nv_bfloat16* dst = a.out + ((size_t)b * a.Q + s) * a.Hq * D + (size_t)h * D;
+                const int mt = i >> 1, hi = i & 1;
+#pragma unroll
+                for (int nt = 0; nt < NT; ++nt) {
+                    const int col = nt * 8 + (lane & 3) * 2;
+                    *reinterpret_cast<__nv_bfloat162*>(dst + col) = __floats2bfloat162_rn(
+                        o[mt][nt][hi * 2] * inv, o[mt][nt][hi * 2 + 1] * inv);
+                }
+            }
+        }
+        return;
+    }
+    // partial: m[ROWS], l[ROWS], O[ROWS][D] (fp32, O scaled to m)
+    char* pbase = a.part + (unit * a.max_splits + sp) * a.part_stride;
+    float* pm = reinterpret_cast<float*>(pbase);
+    float* pl = pm + ROWS;
+    float* po = pl + ROWS;
+    if (wig == 0) {
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+            const int r = rg * 32 + (i >> 1) * 16 + (i & 1) * 8 + (lane >> 2);
+            if ((lane & 3) == 0) {
+                pm[r] = m_fin[i];
+                pl[r] = l_fin[i];
+            }
+            const int mt = i >> 1, hi = i & 1;
+#pragma unroll
+            for (int nt = 0; nt < NT; ++nt) {
+                const int col = nt * 8 + (lane & 3) * 2;
+                *reinterpret_cast<float2*>(po + (size_t)r * D + col) =
+                    make_float2(o[mt][nt][hi * 2], o[mt][nt][hi * 2 + 1]);
+            }
+        }
+    }
+    __threadfence();
+    __syncthreads();
+    __shared__ int s_last;
+    if (tid == 0) s_last = (atomicAdd(&a.ticket[unit], 1) == ns - 1);
+    __syncthreads();
+    if (!s_last) return;
+    __threadfence();
+    // combine all splits in order 0..ns-1
+    const char* ubase = a.part + unit * a.max_splits * a.part_stride;
+    for (int i = tid; i < ROWS * (D / 2); i += THREADS) {
+        const int r = i / (D / 2), col = (i % (D / 2)) * 2;
+        const int rr = row0 + r;
+        if (rr >= a.rows) continue;
+        float M = -INFINITY;
+        for (int k = 0; k < ns; ++k)
+            M = fmaxf(M, __ldcg(reinterpret_cast<const float*>(ubase + k * a.part_stride) + r));
+        const float Mu = (M == -INFINITY) ? 0.f : M;
+        float L = 0.f, o0 = 0.f, o1 = 0.f;
+        for (int k = 0; k < ns; ++k) {
+            const float* km = reinterpret_cast<const float*>(ubase + k * a.part_stride);
+            const float f = exp2f(__ldcg(km + r) - Mu);
+            L += __ldcg(km + ROWS + r) * f;
+            const float2 ov = __ldcg(reinterpret_cast<const float2*>(km + 2 * ROWS + (size_t)r * D + col));
+            o0 += ov.x * f;
+            o1 += ov.y * f;
+        }
+        const float inv = L > 0.f ? 1.f / L : 0.f;
+        const int hh = rr / a.Q, s = rr % a.Q;
+        const int h = g * a.grp + hh;
+        __nv_bfloat16* dst = a.out + ((size_t)b * a.Q + s) * a.Hq * D + (size_t)h * D + col;
+        *reinterpret_cast<__nv_bfloat162*>(dst) = __floats2bfloat162_rn(o0 * inv, o1 * inv);
+    }
+    if (tid == 0) a.ticket[unit] = 0;
+}
+
+template <int D, int NRG>
+static size_t attn_smem_bytes() {
+    return (size_t)32 * NRG * D * 2 + (size_t)2 * kStages * kKT * D * 2;
+}
+
+template <int D, int NRG>
+static cudaError_t launch_attention_t(const AttnArgs& a, dim3 grid, cudaStream_t st) {
+    const size_t smem = attn_smem_bytes<D, NRG>();
+    static bool configured = false;  // per-process attribute, set once
+    if (!configured) {
+        cudaError_t e = cudaFuncSetAttribute(attention_kernel<D, NRG>,
+                                             cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+        if (e != cudaSuccess) return e;
+        configured = true;
+    }
+    attention_kernel<D, NRG><<<grid, 128 * NRG, smem, st>>>(a);
+    return cudaGetLastError();
+}
+
+cudaError_t launch_attention(const Plan& p, const isd_dims* d, const uint16_t* q,
+                             const uint16_t* k_new, const uint16_t* v_new, uint16_t* k_pool,
+                             uint16_t* v_pool, const int32_t* page_table, const int32_t* kv_len,
+                             const int32_t* n_clean, uint16_t* out, void* ws, int32_t* err_flag,
+                             cudaStream_t st) {
+    char* w = static_cast<char*>(ws);
+    AttnArgs a;
+    a.B = d->B;
+    a.N = d->N;
+    a.Q = p.Q;
+    a.Hq = d->Hq;
+    a.Hkv = d->Hkv;
+    a.grp = p.grp;
+    a.rows = p.rows;
+    a.P = d->page_size;
+    a.num_pages = d->num_pages;
+    a.max_pages = d->max_pages_per_req;
+    a.split = p.attn_split;
+    a.n_rgb = p.attn_rgb;
+    a.scale_log2 = d->sm_scale * 1.4426950408889634f;
+    a.q = reinterpret_cast<const __nv_bfloat16*>(q);
+    a.k_new = reinterpret_cast<const __nv_bfloat16*>(k_new);
+    a.v_new = reinterpret_cast<const __nv_bfloat16*>(v_new);
+    a.k_pool = reinterpret_cast<__nv_bfloat16*>(k_pool);
+    a.v_pool = reinterpret_cast<__nv_bfloat16*>(v_pool);
+    a.page_table = page_table;
+    a.kv_len = kv_len;
+    a.n_clean = n_clean;
+    a.out = reinterpret_cast<__nv_bfloat16*>(out);
+    a.part = w + p.off_attn_part;
+    a.part_stride = p.attn_part_stride;
+    a.max_splits = p.attn_max_splits;
+    a.ticket = reinterpret_cast<int*>(w + p.off_attn_ticket);
+    a.err_flag = err_flag;
+    dim3 grid(p.attn_max_splits, d->Hkv * p.attn_rgb, d->B);
+    if (d->D == 128) {
+        return p.attn_nrg == 1 ? launch_attention_t<128, 1>(a, grid, st)
+                               : launch_attention_t<128, 2>(a, grid, st);
+    }
+    return p.attn_nrg == 1 ? launch_attention_t<64, 1>(a, grid, st)
+                           : launch_attention_t<64, 2>(a, grid, st);
+}
+
+}  // namespace isd

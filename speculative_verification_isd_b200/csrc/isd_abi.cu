@@ -1,0 +1,249 @@
+// C-ABI entry points of libisd.so (declared in include/isd.h): host-side
+// validation, workspace checks and the launch sequence of one ISD step.  No
+// entry point allocates, synchronises or reads device data on the host, so a
+// whole step can be captured into a CUDA graph.
+#include <cuda_runtime.h>
+#include <stdint.h>
+#include <stdio.h>
+
+#include "common.cuh"
+#include "plan.h"
+
+namespace isd {
+cudaError_t launch_attention(const Plan& p, const isd_dims* d, const uint16_t* q,
+                             const uint16_t* k_new, const uint16_t* v_new, uint16_t* k_pool,
+                             uint16_t* v_pool, const int32_t* page_table, const int32_t* kv_len,
+                             const int32_t* n_clean, uint16_t* out, void* ws, int32_t* err_flag,
+                             cudaStream_t st);
+cudaError_t launch_lm_head(const uint16_t* hidden, const uint16_t* W, int Mh, int H, int V,
+                           float* logits, int32_t* err_flag, cudaStream_t st);
+cudaError_t launch_lora(const Plan& p, const isd_dims* d, const uint16_t* hidden,
+                        const uint16_t* lora_A, const uint16_t* lora_B, uint16_t* hidden_out,
+                        void* ws, cudaStream_t st);
+cudaError_t launch_row_stats(const Plan& p, const float* logits, int rows, int V,
+                             isd_row_stat* out, void* ws, cudaStream_t st);
+cudaError_t launch_accept(const Plan& p, const isd_dims* d, const float* logits,
+                          const isd_row_stat* stats, const float* prev_logits,
+                          const isd_row_stat* prev_stats, const int32_t* n_clean,
+                          const int32_t* clean_tok, const int32_t* kv_len, const float* uniforms,
+                          int32_t* accept_len, int32_t* out_tok, int32_t* next_n_clean,
+                          int32_t* next_clean_tok, int32_t* next_kv_len, float* ratio, void* ws,
+                          int32_t* err_flag, cudaStream_t st);
+}  // namespace isd
+
+using isd::Plan;
+
+namespace {
+
+thread_local char g_last_error[256] = "";
+
+isd_status cuda_fail(cudaError_t e) {
+    snprintf(g_last_error, sizeof(g_last_error), "%s: %s", cudaGetErrorName(e),
+             cudaGetErrorString(e));
+    return ISD_ERR_CUDA;
+}
+
+isd_status check_ws(const Plan& p, void* ws, size_t ws_bytes) {
+    if (!ws || ws_bytes < p.total || (reinterpret_cast<uintptr_t>(ws) & 255)) {
+        snprintf(g_last_error, sizeof(g_last_error), "workspace: need %zu bytes, 256-aligned",
+                 p.total);
+        return ISD_ERR_WORKSPACE;
+    }
+    return ISD_OK;
+}
+
+isd_status invalid(const char* what) {
+    snprintf(g_last_error, sizeof(g_last_error), "invalid argument: %s", what);
+    return ISD_ERR_INVALID_ARG;
+}
+
+isd_status unsupported(const char* what) {
+    snprintf(g_last_error, sizeof(g_last_error), "unsupported shape: %s", what);
+    return ISD_ERR_UNSUPPORTED_SHAPE;
+}
+
+isd_status plan_or_fail(const isd_dims* d, Plan* p) {
+    if (!isd::make_plan(d, p)) return invalid("dims");
+    return ISD_OK;
+}
+
+isd_status check_attention_shape(const isd_dims* d, const Plan& p) {
+    if (d->D != 64 && d->D != 128) return unsupported("head dim must be 64 or 128");
+    if (p.rows > 128) return unsupported("(Hq/Hkv)*(2N-1) must be <= 128");
+    return ISD_OK;
+}
+
+isd_status check_lm_shape(const isd_dims* d, const Plan& p, const void* A, const void* Bm) {
+    if (p.H % 64) return unsupported("hidden size must be a multiple of 64");
+    if (p.M > 512) return unsupported("B*(2N-1) must be <= 512");
+    if (d->lora_rank) {
+        if (!A || !Bm) return invalid("lora_A/lora_B required when lora_rank > 0");
+        if (d->lora_rank % 32 || d->lora_rank > 256)
+            return unsupported("lora rank must be a multiple of 32, <= 256");
+    } else if (A || Bm) {
+        return invalid("lora_A/lora_B given with lora_rank == 0");
+    }
+    return ISD_OK;
+}
+
+isd_status check_accept_shape(const isd_dims* d) {
+    if (d->N > 16) return unsupported("stride N must be <= 16");
+    return ISD_OK;
+}
+
+#define ISD_TRY(x)                        \
+    do {                                  \
+        isd_status s_ = (x);              \
+        if (s_ != ISD_OK) return s_;      \
+    } while (0)
+#define ISD_CUDA(x)                         \
+    do {                                    \
+        cudaError_t e_ = (x);               \
+        if (e_ != cudaSuccess) return cuda_fail(e_); \
+    } while (0)
+
+isd_status do_attention(const isd_dims* d, const Plan& p, const uint16_t* q,
+                        const uint16_t* k_new, const uint16_t* v_new, uint16_t* k_pool,
+                        uint16_t* v_pool, const int32_t* page_table, const int32_t* kv_len,
+                        const int32_t* n_clean, uint16_t* out, void* ws, int32_t* err_flag,
+                        cudaStream_t st) {
+    if (!q || !k_new || !v_new || !k_pool || !v_pool || !page_table || !kv_len || !n_clean || !out)
+        return invalid("null attention pointer");
+    ISD_TRY(check_attention_shape(d, p));
+    ISD_CUDA(cudaMemsetAsync(static_cast<char*>(ws) + p.off_attn_ticket, 0,
+                             (size_t)d->B * d->Hkv * p.attn_rgb * 4, st));
+    ISD_CUDA(isd::launch_attention(p, d, q, k_new, v_new, k_pool, v_pool, page_table, kv_len,
+                                   n_clean, out, ws, err_flag, st));
+    return ISD_OK;
+}
+
+isd_status do_lm_head(const isd_dims* d, const Plan& p, const uint16_t* hidden, const uint16_t* W,
+                      const uint16_t* lora_A, const uint16_t* lora_B, float* logits,
+                      isd_row_stat* row_stats, void* ws, int32_t* err_flag, cudaStream_t st) {
+    if (!hidden || !W || !logits) return invalid("null lm-head pointer");
+    ISD_TRY(check_lm_shape(d, p, lora_A, lora_B));
+    const uint16_t* h = hidden;
+    if (d->lora_rank) {
+        uint16_t* hl = reinterpret_cast<uint16_t*>(static_cast<char*>(ws) + p.off_hidden_lora);
+        ISD_CUDA(isd::launch_lora(p, d, hidden, lora_A, lora_B, hl, ws, st));
+        h = hl;
+    }
+    ISD_CUDA(isd::launch_lm_head(h, W, p.M, p.H, d->V, logits, err_flag, st));
+    if (row_stats) {
+        ISD_CUDA(cudaMemsetAsync(static_cast<char*>(ws) + p.off_stats_ticket, 0, (size_t)p.M * 4, st));
+        ISD_CUDA(isd::launch_row_stats(p, logits, p.M, d->V, row_stats, ws, st));
+    }
+    return ISD_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+size_t isd_workspace_bytes(const isd_dims* d) {
+    Plan p;
+    if (!isd::make_plan(d, &p)) return 0;
+    return p.total;
+}
+
+const char* isd_status_string(isd_status s) {
+    switch (s) {
+        case ISD_OK: return "ISD_OK";
+        case ISD_ERR_INVALID_ARG: return "ISD_ERR_INVALID_ARG";
+        case ISD_ERR_UNSUPPORTED_SHAPE: return "ISD_ERR_UNSUPPORTED_SHAPE";
+        case ISD_ERR_WORKSPACE: return "ISD_ERR_WORKSPACE";
+        case ISD_ERR_CUDA: return "ISD_ERR_CUDA";
+        default: return "ISD_ERR_UNKNOWN";
+    }
+}
+
+const char* isd_last_error(void) { return g_last_error; }
+
+isd_status isd_attention(const isd_dims* d, const uint16_t* q, const uint16_t* k_new,
+                         const uint16_t* v_new, uint16_t* k_pool, uint16_t* v_pool,
+                         const int32_t* page_table, const int32_t* kv_len,
+                         const int32_t* n_clean, uint16_t* out, void* ws, size_t ws_bytes,
+                         int32_t* err_flag, void* stream) {
+    Plan p;
+    ISD_TRY(plan_or_fail(d, &p));
+    ISD_TRY(check_ws(p, ws, ws_bytes));
+    return do_attention(d, p, q, k_new, v_new, k_pool, v_pool, page_table, kv_len, n_clean, out,
+                        ws, err_flag, static_cast<cudaStream_t>(stream));
+}
+
+isd_status isd_lm_head(const isd_dims* d, const uint16_t* hidden, const uint16_t* W,
+                       const uint16_t* lora_A, const uint16_t* lora_B, float* logits,
+                       isd_row_stat* row_stats, void* ws, size_t ws_bytes, int32_t* err_flag,
+                       void* stream) {
+    Plan p;
+    ISD_TRY(plan_or_fail(d, &p));
+    ISD_TRY(check_ws(p, ws, ws_bytes));
+    return do_lm_head(d, p, hidden, W, lora_A, lora_B, logits, row_stats, ws, err_flag,
+                      static_cast<cudaStream_t>(stream));
+}
+
+isd_status isd_row_stats(const isd_dims* d, const float* logits, int32_t rows,
+                         isd_row_stat* row_stats, void* ws, size_t ws_bytes, void* stream) {
+    Plan p;
+    ISD_TRY(plan_or_fail(d, &p));
+    ISD_TRY(check_ws(p, ws, ws_bytes));
+    if (!logits || !row_stats) return invalid("null row-stats pointer");
+    if (rows < 0 || rows > p.M) return invalid("rows must be in [0, B*(2N-1)]");
+    if (rows == 0) return ISD_OK;
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    ISD_CUDA(cudaMemsetAsync(static_cast<char*>(ws) + p.off_stats_ticket, 0, (size_t)p.M * 4, st));
+    ISD_CUDA(isd::launch_row_stats(p, logits, rows, d->V, row_stats, ws, st));
+    return ISD_OK;
+}
+
+isd_status isd_accept(const isd_dims* d, const float* logits, const isd_row_stat* row_stats,
+                      const float* prev_logits, const isd_row_stat* prev_row_stats,
+                      const int32_t* n_clean, const int32_t* clean_tok, const int32_t* kv_len,
+                      const float* uniforms, int32_t* accept_len, int32_t* out_tok,
+                      int32_t* next_n_clean, int32_t* next_clean_tok, int32_t* next_kv_len,
+                      float* ratio, void* ws, size_t ws_bytes, int32_t* err_flag, void* stream) {
+    Plan p;
+    ISD_TRY(plan_or_fail(d, &p));
+    ISD_TRY(check_ws(p, ws, ws_bytes));
+    ISD_TRY(check_accept_shape(d));
+    if (!logits || !row_stats || !prev_logits || !prev_row_stats || !n_clean || !clean_tok ||
+        !kv_len || !uniforms || !accept_len || !out_tok || !next_n_clean || !next_clean_tok ||
+        !next_kv_len)
+        return invalid("null accept pointer");
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    ISD_CUDA(cudaMemsetAsync(static_cast<char*>(ws) + p.off_acc_ticket, 0, (size_t)d->B * 4, st));
+    ISD_CUDA(isd::launch_accept(p, d, logits, row_stats, prev_logits, prev_row_stats, n_clean,
+                                clean_tok, kv_len, uniforms, accept_len, out_tok, next_n_clean,
+                                next_clean_tok, next_kv_len, ratio, ws, err_flag, st));
+    return ISD_OK;
+}
+
+isd_status isd_step(const isd_dims* d, const uint16_t* q, const uint16_t* k_new,
+                    const uint16_t* v_new, uint16_t* k_pool, uint16_t* v_pool,
+                    const int32_t* page_table, const int32_t* kv_len, const int32_t* n_clean,
+                    const int32_t* clean_tok, const uint16_t* W, const uint16_t* lora_A,
+                    const uint16_t* lora_B, const float* prev_logits,
+                    const isd_row_stat* prev_row_stats, const float* uniforms, uint16_t* hidden,
+                    float* logits, isd_row_stat* row_stats, int32_t* accept_len,
+                    int32_t* out_tok, int32_t* next_n_clean, int32_t* next_clean_tok,
+                    int32_t* next_kv_len, float* ratio, void* ws, size_t ws_bytes,
+                    int32_t* err_flag, void* stream) {
+    Plan p;
+    ISD_TRY(plan_or_fail(d, &p));
+    ISD_TRY(check_ws(p, ws, ws_bytes));
+    ISD_TRY(check_attention_shape(d, p));
+    ISD_TRY(check_lm_shape(d, p, lora_A, lora_B));
+    ISD_TRY(check_accept_shape(d));
+    if (!row_stats || !logits) return invalid("null logits/row_stats");
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    uint16_t* h = hidden ? hidden
+                         : reinterpret_cast<uint16_t*>(static_cast<char*>(ws) + p.off_hidden);
+    ISD_TRY(do_attention(d, p, q, k_new, v_new, k_pool, v_pool, page_table, kv_len, n_clean, h,
+                         ws, err_flag, st));
+    ISD_TRY(do_lm_head(d, p, h, W, lora_A, lora_B, logits, row_stats, ws, err_flag, st));
+    return isd_accept(d, logits, row_stats, prev_logits, prev_row_stats, n_clean, clean_tok,
+                      kv_len, uniforms, accept_len, out_tok, next_n_clean, next_clean_tok,
+                      next_kv_len, ratio, ws, ws_bytes, err_flag, stream);
+}
+
+}  // extern "C"

@@ -1,0 +1,107 @@
+// Launch plan and workspace layout of one ISD step, derived from the dims
+// alone (no device data is read on the host, so every call is capturable).
+#pragma once
+
+#include <stddef.h>
+#include <stdint.h>
+
+#include "../../include/isd.h"
+
+namespace isd {
+
+constexpr int kAttnKeyTile = 64;      // keys per pipeline stage
+constexpr int kAttnRowsPerGroup = 32; // query rows handled by one 4-warp group
+constexpr int kStatsThreads = 256;
+constexpr int kAcceptThreads = 256;
+constexpr int kAcceptChunk = 4096;    // vocabulary entries per accept CTA
+constexpr int kNumSMs = 148;
+
+struct Plan {
+    // derived dims
+    int Q, H, M, grp, rows;  // rows = grp * Q query rows per (request, kv head)
+    // attention
+    int attn_nrg;            // 4-warp row groups per CTA (1 or 2)
+    int attn_rgb;            // row-group blocks per (request, kv head)
+    int attn_split;          // keys per split (multiple of kAttnKeyTile)
+    int attn_max_splits;     // splits for the longest possible request
+    size_t attn_part_stride; // bytes of one split's partial
+    // statistics / accept
+    int stats_chunks, stats_chunk_len;
+    int acc_chunks;
+    // R-ISD LoRA
+    int lora_rows, lora_ksplit;
+    // workspace offsets (bytes)
+    size_t off_attn_part, off_attn_ticket, off_hidden, off_hidden_lora, off_lora_t,
+        off_stats_part, off_stats_ticket, off_acc_part, off_acc_ticket, off_lora_part, total;
+};
+
+inline size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
+
+// Returns false if the dims are invalid.
+inline bool make_plan(const isd_dims* d, Plan* p) {
+    if (!d || d->B < 1 || d->N < 1 || d->Hq < 1 || d->Hkv < 1 || d->D < 1 || d->V < 1 ||
+        d->page_size < 1 || d->num_pages < 1 || d->max_pages_per_req < 1 || d->lora_rank < 0 ||
+        d->Hq % d->Hkv != 0 ||
+        (d->proposal_mode != ISD_PROPOSE_ARGMAX && d->proposal_mode != ISD_PROPOSE_SAMPLE))
+        return false;
+    p->Q = 2 * d->N - 1;
+    p->H = d->Hq * d->D;
+    p->M = d->B * p->Q;
+    p->grp = d->Hq / d->Hkv;
+    p->rows = p->grp * p->Q;
+    p->attn_nrg = p->rows > kAttnRowsPerGroup ? 2 : 1;
+    const int rows_per_cta = kAttnRowsPerGroup * p->attn_nrg;
+    p->attn_rgb = (p->rows + rows_per_cta - 1) / rows_per_cta;
+    const long long max_ctx = (long long)d->max_pages_per_req * d->page_size;
+    // Aim for about 3 waves of 2 CTAs per SM over the expected keys (half
+    // the longest context per request on average).
+    long long est = (long long)d->B * d->Hkv * p->attn_rgb * (max_ctx / 2 + 1);
+    long long split = est / (kNumSMs * 2 * 3);
+    if (split < 256) split = 256;
+    if (split > 8192) split = 8192;
+    split = (split + kAttnKeyTile - 1) / kAttnKeyTile * kAttnKeyTile;
+    p->attn_split = (int)split;
+    p->attn_max_splits = (int)((max_ctx + split - 1) / split);
+    if (p->attn_max_splits < 1) p->attn_max_splits = 1;
+    p->attn_part_stride = align_up((size_t)rows_per_cta * d->D * 4 + (size_t)rows_per_cta * 8, 256);
+    // row statistics: enough CTAs to fill the GPU, chunks of >= 2048 entries
+    int target = (kNumSMs * 8 + p->M - 1) / p->M;
+    int max_chunks = (d->V + 2047) / 2048;
+    p->stats_chunks = target < 1 ? 1 : (target > max_chunks ? max_chunks : target);
+    if (p->stats_chunks < 1) p->stats_chunks = 1;
+    p->stats_chunk_len = (int)align_up((size_t)((d->V + p->stats_chunks - 1) / p->stats_chunks), 4);
+    p->acc_chunks = (d->V + kAcceptChunk - 1) / kAcceptChunk;
+    p->lora_rows = d->B * (d->N - 1);
+    p->lora_ksplit = 1;
+    if (d->lora_rank > 0) {
+        // split the long K = H reduction of h.A so that about 100 CTAs work on it
+        const int tiles = ((p->lora_rows + 63) / 64) * ((d->lora_rank + 63) / 64);
+        int ks = (100 + tiles - 1) / tiles;
+        const int kiters = p->H / 32;
+        if (ks > kiters) ks = kiters;
+        if (ks < 1) ks = 1;
+        p->lora_ksplit = ks;
+    }
+    // workspace
+    size_t off = 0;
+    auto take = [&](size_t bytes) {
+        size_t o = off;
+        off = align_up(off + bytes, 256);
+        return o;
+    };
+    const size_t n_units = (size_t)d->B * d->Hkv * p->attn_rgb;
+    p->off_attn_part = take(n_units * p->attn_max_splits * p->attn_part_stride);
+    p->off_attn_ticket = take(n_units * 4);
+    p->off_hidden = take((size_t)p->M * p->H * 2);
+    p->off_hidden_lora = take(d->lora_rank ? (size_t)p->M * p->H * 2 : 0);
+    p->off_lora_t = take(d->lora_rank ? (size_t)p->M * d->lora_rank * 2 : 0);
+    p->off_stats_part = take((size_t)p->M * p->stats_chunks * 16);
+    p->off_stats_ticket = take((size_t)p->M * 4);
+    p->off_acc_part = take((size_t)d->B * (d->N + 1) * p->acc_chunks * 4);
+    p->off_acc_ticket = take((size_t)d->B * 4);
+    p->off_lora_part = take(d->lora_rank ? (size_t)p->lora_ksplit * p->lora_rows * d->lora_rank * 4 : 0);
+    p->total = off;
+    return true;
+}
+
+}  // namespace isd

@@ -1,0 +1,238 @@
+"""Python binding of libisd.so (include/isd.h): argument marshalling only.
+
+Every function takes torch CUDA tensors, checks dtype / shape / contiguity,
+and passes raw device pointers plus the current CUDA stream to the C ABI.
+All arithmetic of the ISD step runs in the library's kernels; there is no
+fallback.  Importing this module raises ImportError when libisd.so has not
+been built (``python -m speculative_verification_isd_b200.build``).
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+from typing import Optional
+
+import torch
+
+_PKG = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_PKG, "libisd.so")
+
+if not os.path.exists(LIB_PATH):
+    raise ImportError(f"libisd.so not found at {LIB_PATH}: build it with "
+                      "`python -m speculative_verification_isd_b200.build`")
+_lib = ctypes.CDLL(LIB_PATH)
+
+ISD_OK = 0
+ISD_ERR_INVALID_ARG = -1
+ISD_ERR_UNSUPPORTED_SHAPE = -2
+ISD_ERR_WORKSPACE = -3
+ISD_ERR_CUDA = -4
+FLAG_PAGE_OOB = 1
+FLAG_TOKEN_OOB = 2
+FLAG_NCLEAN_RANGE = 4
+FLAG_CAPACITY = 8
+FLAG_WAIT_TIMEOUT = 16
+PROPOSE_ARGMAX = 0
+PROPOSE_SAMPLE = 1
+
+EXPORTED = ("isd_workspace_bytes", "isd_status_string", "isd_last_error", "isd_attention",
+            "isd_lm_head", "isd_row_stats", "isd_accept", "isd_step")
+
+
+class Dims(ctypes.Structure):
+    _fields_ = [("B", ctypes.c_int32), ("N", ctypes.c_int32), ("Hq", ctypes.c_int32),
+                ("Hkv", ctypes.c_int32), ("D", ctypes.c_int32), ("V", ctypes.c_int32),
+                ("page_size", ctypes.c_int32), ("num_pages", ctypes.c_int32),
+                ("max_pages_per_req", ctypes.c_int32), ("lora_rank", ctypes.c_int32),
+                ("proposal_mode", ctypes.c_int32), ("sm_scale", ctypes.c_float)]
+
+    @property
+    def Q(self):
+        return 2 * self.N - 1
+
+    @property
+    def H(self):
+        return self.Hq * self.D
+
+    @property
+    def M(self):
+        return self.B * self.Q
+
+
+ROW_STAT_FIELDS = 4  # isd_row_stat = {float max, float sumexp, int32 argmax, int32 reserved}
+
+_vp = ctypes.c_void_p
+_sz = ctypes.c_size_t
+_i32 = ctypes.c_int32
+_dims_p = ctypes.POINTER(Dims)
+
+_lib.isd_workspace_bytes.argtypes = [_dims_p]
+_lib.isd_workspace_bytes.restype = _sz
+_lib.isd_status_string.argtypes = [_i32]
+_lib.isd_status_string.restype = ctypes.c_char_p
+_lib.isd_last_error.argtypes = []
+_lib.isd_last_error.restype = ctypes.c_char_p
+_lib.isd_attention.argtypes = [_dims_p] + [_vp] * 10 + [_sz, _vp, _vp]
+_lib.isd_attention.restype = _i32
+_lib.isd_lm_head.argtypes = [_dims_p] + [_vp] * 7 + [_sz, _vp, _vp]
+_lib.isd_lm_head.restype = _i32
+_lib.isd_row_stats.argtypes = [_dims_p, _vp, _i32, _vp, _vp, _sz, _vp]
+_lib.isd_row_stats.restype = _i32
+_lib.isd_accept.argtypes = [_dims_p] + [_vp] * 16 + [_sz, _vp, _vp]
+_lib.isd_accept.restype = _i32
+_lib.isd_step.argtypes = [_dims_p] + [_vp] * 25 + [_sz, _vp, _vp]
+_lib.isd_step.restype = _i32
+
+
+class IsdError(RuntimeError):
+    def __init__(self, status: int):
+        self.status = status
+        name = _lib.isd_status_string(status).decode()
+        detail = _lib.isd_last_error().decode()
+        super().__init__(f"{name}: {detail}")
+
+
+def library() -> ctypes.CDLL:
+    return _lib
+
+
+def make_dims(B, N, Hq, Hkv, D, V, page_size, num_pages, max_pages_per_req, lora_rank=0,
+              proposal_mode=PROPOSE_ARGMAX, sm_scale=None) -> Dims:
+    if sm_scale is None:
+        sm_scale = D ** -0.5
+    return Dims(B, N, Hq, Hkv, D, V, page_size, num_pages, max_pages_per_req, lora_rank,
+                proposal_mode, float(sm_scale))
+
+
+def workspace_bytes(d: Dims) -> int:
+    return int(_lib.isd_workspace_bytes(ctypes.byref(d)))
+
+
+def alloc_workspace(d: Dims, device="cuda") -> torch.Tensor:
+    n = workspace_bytes(d)
+    if n == 0:
+        raise IsdError(ISD_ERR_INVALID_ARG)
+    return torch.empty(n, dtype=torch.uint8, device=device)
+
+
+def _ptr(t: Optional[torch.Tensor], dtype=None, numel=None, name="tensor"):
+    if t is None:
+        return None
+    if not t.is_cuda:
+        raise ValueError(f"{name} must be a CUDA tensor")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+    if dtype is not None and t.dtype not in (dtype if isinstance(dtype, tuple) else (dtype,)):
+        raise ValueError(f"{name} has dtype {t.dtype}, expected {dtype}")
+    if numel is not None and t.numel() != numel:
+        raise ValueError(f"{name} has {t.numel()} elements, expected {numel}")
+    return t.data_ptr()
+
+
+_BF16 = (torch.bfloat16, torch.int16, torch.uint16)
+
+
+def _stream(stream) -> int:
+    if stream is None:
+        return torch.cuda.current_stream().cuda_stream
+    return stream.cuda_stream if hasattr(stream, "cuda_stream") else int(stream)
+
+
+def _check(status: int):
+    if status != ISD_OK:
+        raise IsdError(status)
+
+
+def attention(d: Dims, q, k_new, v_new, k_pool, v_pool, page_table, kv_len, n_clean, out, ws,
+              err_flag=None, stream=None):
+    kvrow = d.page_size * d.Hkv * d.D
+    _check(_lib.isd_attention(
+        ctypes.byref(d), _ptr(q, _BF16, d.M * d.Hq * d.D, "q"),
+        _ptr(k_new, _BF16, d.M * d.Hkv * d.D, "k_new"),
+        _ptr(v_new, _BF16, d.M * d.Hkv * d.D, "v_new"),
+        _ptr(k_pool, _BF16, d.num_pages * kvrow, "k_pool"),
+        _ptr(v_pool, _BF16, d.num_pages * kvrow, "v_pool"),
+        _ptr(page_table, torch.int32, d.B * d.max_pages_per_req, "page_table"),
+        _ptr(kv_len, torch.int32, d.B, "kv_len"), _ptr(n_clean, torch.int32, d.B, "n_clean"),
+        _ptr(out, _BF16, d.M * d.H, "out"), _ptr(ws, torch.uint8, None, "ws"), ws.numel(),
+        _ptr(err_flag, torch.int32, 1, "err_flag"), _stream(stream)))
+
+
+def lm_head(d: Dims, hidden, W, logits, row_stats, ws, lora_A=None, lora_B=None, err_flag=None,
+            stream=None):
+    _check(_lib.isd_lm_head(
+        ctypes.byref(d), _ptr(hidden, _BF16, d.M * d.H, "hidden"),
+        _ptr(W, _BF16, d.V * d.H, "W"),
+        _ptr(lora_A, _BF16, d.H * d.lora_rank, "lora_A"),
+        _ptr(lora_B, _BF16, d.lora_rank * d.H, "lora_B"),
+        _ptr(logits, torch.float32, d.M * d.V, "logits"),
+        _ptr(row_stats, (torch.int32, torch.float32), d.M * ROW_STAT_FIELDS, "row_stats"),
+        _ptr(ws, torch.uint8, None, "ws"), ws.numel(),
+        _ptr(err_flag, torch.int32, 1, "err_flag"), _stream(stream)))
+
+
+def row_stats(d: Dims, logits, rows: int, out, ws, stream=None):
+    _check(_lib.isd_row_stats(
+        ctypes.byref(d), _ptr(logits, torch.float32, None, "logits"), int(rows),
+        _ptr(out, (torch.int32, torch.float32), None, "row_stats"),
+        _ptr(ws, torch.uint8, None, "ws"), ws.numel(), _stream(stream)))
+
+
+def accept(d: Dims, logits, row_stats, prev_logits, prev_row_stats, n_clean, clean_tok, kv_len,
+           uniforms, accept_len, out_tok, next_n_clean, next_clean_tok, next_kv_len, ws,
+           ratio=None, err_flag=None, stream=None):
+    B, N = d.B, d.N
+    _check(_lib.isd_accept(
+        ctypes.byref(d), _ptr(logits, torch.float32, d.M * d.V, "logits"),
+        _ptr(row_stats, (torch.int32, torch.float32), d.M * ROW_STAT_FIELDS, "row_stats"),
+        _ptr(prev_logits, torch.float32, d.M * d.V, "prev_logits"),
+        _ptr(prev_row_stats, (torch.int32, torch.float32), d.M * ROW_STAT_FIELDS, "prev_row_stats"),
+        _ptr(n_clean, torch.int32, B, "n_clean"), _ptr(clean_tok, torch.int32, B * N, "clean_tok"),
+        _ptr(kv_len, torch.int32, B, "kv_len"), _ptr(uniforms, torch.float32, B * 2 * N, "uniforms"),
+        _ptr(accept_len, torch.int32, B, "accept_len"), _ptr(out_tok, torch.int32, B * N, "out_tok"),
+        _ptr(next_n_clean, torch.int32, B, "next_n_clean"),
+        _ptr(next_clean_tok, torch.int32, B * N, "next_clean_tok"),
+        _ptr(next_kv_len, torch.int32, B, "next_kv_len"),
+        _ptr(ratio, torch.float32, B * max(N - 1, 1), "ratio"),
+        _ptr(ws, torch.uint8, None, "ws"), ws.numel(),
+        _ptr(err_flag, torch.int32, 1, "err_flag"), _stream(stream)))
+
+
+def step(d: Dims, q, k_new, v_new, k_pool, v_pool, page_table, kv_len, n_clean, clean_tok, W,
+         prev_logits, prev_row_stats, uniforms, logits, row_stats, accept_len, out_tok,
+         next_n_clean, next_clean_tok, next_kv_len, ws, hidden=None, ratio=None, lora_A=None,
+         lora_B=None, err_flag=None, stream=None):
+    B, N = d.B, d.N
+    kvrow = d.page_size * d.Hkv * d.D
+    _check(_lib.isd_step(
+        ctypes.byref(d), _ptr(q, _BF16, d.M * d.Hq * d.D, "q"),
+        _ptr(k_new, _BF16, d.M * d.Hkv * d.D, "k_new"),
+        _ptr(v_new, _BF16, d.M * d.Hkv * d.D, "v_new"),
+        _ptr(k_pool, _BF16, d.num_pages * kvrow, "k_pool"),
+        _ptr(v_pool, _BF16, d.num_pages * kvrow, "v_pool"),
+        _ptr(page_table, torch.int32, d.B * d.max_pages_per_req, "page_table"),
+        _ptr(kv_len, torch.int32, B, "kv_len"), _ptr(n_clean, torch.int32, B, "n_clean"),
+        _ptr(clean_tok, torch.int32, B * N, "clean_tok"), _ptr(W, _BF16, d.V * d.H, "W"),
+        _ptr(lora_A, _BF16, d.H * d.lora_rank, "lora_A"),
+        _ptr(lora_B, _BF16, d.lora_rank * d.H, "lora_B"),
+        _ptr(prev_logits, torch.float32, d.M * d.V, "prev_logits"),
+        _ptr(prev_row_stats, (torch.int32, torch.float32), d.M * ROW_STAT_FIELDS, "prev_row_stats"),
+        _ptr(uniforms, torch.float32, B * 2 * N, "uniforms"),
+        _ptr(hidden, _BF16, d.M * d.H, "hidden"),
+        _ptr(logits, torch.float32, d.M * d.V, "logits"),
+        _ptr(row_stats, (torch.int32, torch.float32), d.M * ROW_STAT_FIELDS, "row_stats"),
+        _ptr(accept_len, torch.int32, B, "accept_len"), _ptr(out_tok, torch.int32, B * N, "out_tok"),
+        _ptr(next_n_clean, torch.int32, B, "next_n_clean"),
+        _ptr(next_clean_tok, torch.int32, B * N, "next_clean_tok"),
+        _ptr(next_kv_len, torch.int32, B, "next_kv_len"),
+        _ptr(ratio, torch.float32, B * max(N - 1, 1), "ratio"),
+        _ptr(ws, torch.uint8, None, "ws"), ws.numel(),
+        _ptr(err_flag, torch.int32, 1, "err_flag"), _stream(stream)))
+
+
+def row_stats_view(rs: torch.Tensor):
+    """(max, sumexp, argmax) views of an isd_row_stat buffer stored as int32 [M, 4]."""
+    r = rs.view(-1, ROW_STAT_FIELDS)
+    f = r.view(torch.float32) if r.dtype == torch.int32 else r
+    i = r if r.dtype == torch.int32 else r.view(torch.int32)
+    return f[:, 0], f[:, 1], i[:, 2]

@@ -1,0 +1,171 @@
+"""Full-size synthetic ISD workloads resident on the GPU.
+
+Used by the benchmark, the smoke run and the full-size parity test.  It only
+prepares inputs: the structural ones (prefix lengths, page tables, tokens,
+uniforms) come from ``inputs``; the large tensors (KV pool, LM head, block
+activations, LoRA) are drawn N(0, std) with a seeded CUDA generator and stored
+as bf16.  All step arithmetic runs in libisd.so.
+
+Constructed acceptance: for a target rate a, the previous step's MASK rows
+are set so that p(x)/q(x) = a exactly for every proposal x.  This needs this
+step's anchor rows p, so one untimed step is run first; then q = p except
+at x, whose logit is raised by log((1 - P) / (a - P)), P = p(x).
+"""
+from __future__ import annotations
+
+import math
+from typing import Dict, Optional
+
+import numpy as np
+import torch
+
+from . import inputs as I
+
+
+def _randn_bf16(shape, std: float, gen: torch.Generator) -> torch.Tensor:
+    out = torch.empty(shape, dtype=torch.bfloat16, device="cuda")
+    flat = out.view(-1)
+    chunk = 1 << 26
+    tmp = torch.empty(min(chunk, flat.numel()), dtype=torch.float32, device="cuda")
+    for s in range(0, flat.numel(), chunk):
+        n = min(chunk, flat.numel() - s)
+        t = tmp[:n]
+        t.normal_(0.0, std, generator=gen)
+        flat[s:s + n].copy_(t)
+    return out
+
+
+class DeviceWorkload:
+    """Device buffers of one ISD step at a given config, ready to run."""
+
+    def __init__(self, isd, cfg: I.IsdConfig, seed: int = 0, n_uniform_steps: int = 64,
+                 accept_rate: Optional[float] = "cfg", n_clean: str = "full"):
+        self.isd = isd
+        self.cfg = cfg
+        self.seed = seed
+        a = cfg.accept_rate if accept_rate == "cfg" else accept_rate
+        self.accept_rate = a
+        B, N, Q = cfg.B, cfg.N, cfg.Q
+        kv_len = I.prefix_lengths(cfg, seed)
+        table, num_pages = I.page_layout(cfg, kv_len, seed)
+        rng = np.random.default_rng([seed, 31])
+        if n_clean == "full":
+            nc = np.full(B, N, np.int32)
+        else:
+            nc = rng.integers(1, N + 1, B).astype(np.int32)
+        tok = rng.integers(0, cfg.V, size=(B, N)).astype(np.int32)
+        self.kv_len_h, self.page_table_h, self.n_clean_h, self.clean_tok_h = kv_len, table, nc, tok
+        self.uniforms_h = np.stack([I.step_uniforms(seed, k, B, N) for k in range(n_uniform_steps)])
+        gen = torch.Generator(device="cuda")
+        gen.manual_seed(seed)
+        self.dims = isd.make_dims(B, N, cfg.Hq, cfg.Hkv, cfg.D, cfg.V, cfg.page_size, num_pages,
+                                  table.shape[1], cfg.lora_rank, 0)
+        d = self.dims
+        self.q = _randn_bf16((B, Q, cfg.Hq, cfg.D), cfg.qkv_std, gen)
+        self.k_new = _randn_bf16((B, Q, cfg.Hkv, cfg.D), cfg.qkv_std, gen)
+        self.v_new = _randn_bf16((B, Q, cfg.Hkv, cfg.D), cfg.qkv_std, gen)
+        self.k_pool = _randn_bf16((num_pages, cfg.page_size, cfg.Hkv, cfg.D), cfg.kv_std, gen)
+        self.v_pool = _randn_bf16((num_pages, cfg.page_size, cfg.Hkv, cfg.D), cfg.kv_std, gen)
+        self.W = _randn_bf16((cfg.V, cfg.H), cfg.w_std, gen)
+        self.lora_A = _randn_bf16((cfg.H, cfg.lora_rank), cfg.lora_std, gen) if cfg.lora_rank else None
+        self.lora_B = _randn_bf16((cfg.lora_rank, cfg.H), cfg.lora_std, gen) if cfg.lora_rank else None
+        dev = lambda x: torch.from_numpy(np.ascontiguousarray(x)).cuda()
+        self.page_table = dev(table)
+        self.kv_len = dev(kv_len)
+        self.n_clean = dev(nc)
+        self.clean_tok = dev(tok)
+        self.uniforms_all = dev(self.uniforms_h)
+        self.uniforms = self.uniforms_all[0]
+        self.ws = isd.alloc_workspace(d)
+        self.err = torch.zeros(1, dtype=torch.int32, device="cuda")
+        M, V = d.M, d.V
+        self.hidden = torch.empty(M, d.H, dtype=torch.bfloat16, device="cuda")
+        self.logits = torch.empty(M, V, dtype=torch.float32, device="cuda")
+        self.row_stats = torch.empty(M, 4, dtype=torch.int32, device="cuda")
+        self.prev_logits = torch.zeros(M, V, dtype=torch.float32, device="cuda")
+        self.prev_row_stats = torch.empty(M, 4, dtype=torch.int32, device="cuda")
+        self.accept_len = torch.empty(B, dtype=torch.int32, device="cuda")
+        self.out_tok = torch.empty(B, N, dtype=torch.int32, device="cuda")
+        self.next_n_clean = torch.empty(B, dtype=torch.int32, device="cuda")
+        self.next_clean_tok = torch.empty(B, N, dtype=torch.int32, device="cuda")
+        self.next_kv_len = torch.empty(B, dtype=torch.int32, device="cuda")
+        self.ratio = torch.empty(B, max(N - 1, 1), dtype=torch.float32, device="cuda")
+        isd.row_stats(d, self.prev_logits, M, self.prev_row_stats, self.ws)
+        self._prepare_prev()
+
+    # ------------------------------------------------------------------
+    def _prepare_prev(self):
+        """Previous step's logits: random rows, with constructed MASK rows."""
+        cfg, d = self.cfg, self.dims
+        B, N, Q, V = cfg.B, cfg.N, cfg.Q, cfg.V
+        gen = torch.Generator(device="cuda")
+        gen.manual_seed(self.seed + 1)
+        prev = torch.empty(B, Q, V, dtype=torch.float32, device="cuda")
+        prev.normal_(0.0, 1.0, generator=gen)
+        if self.accept_rate is not None:
+            self.step()  # untimed: this step's anchor rows p
+            torch.cuda.synchronize()
+            cur = self.logits.view(B, Q, V)
+            a = float(self.accept_rate)
+            for j in range(2, N + 1):
+                x = self.clean_tok[:, j - 1].long()
+                prow = cur[:, j - 2].double()
+                lse = torch.logsumexp(prow, dim=-1)
+                zx = prow.gather(1, x[:, None])[:, 0]
+                P = torch.exp(zx - lse)
+                if torch.any(P >= a):
+                    raise ValueError("constructed acceptance needs p(x) < a")
+                delta = torch.log((1.0 - P) / (a - P))
+                qrow = cur[:, j - 2].clone()
+                qrow.scatter_(1, x[:, None], (zx + delta).float()[:, None])
+                prev[:, N + j - 2] = qrow
+        self.prev_logits.copy_(prev.view(d.M, V))
+        self.isd.row_stats(d, self.prev_logits, d.M, self.prev_row_stats, self.ws)
+        torch.cuda.synchronize()
+
+    def set_uniforms(self, k: int):
+        self.uniforms = self.uniforms_all[k % self.uniforms_all.shape[0]]
+
+    def step(self, stream=None):
+        self.isd.step(self.dims, self.q, self.k_new, self.v_new, self.k_pool, self.v_pool,
+                      self.page_table, self.kv_len, self.n_clean, self.clean_tok, self.W,
+                      self.prev_logits, self.prev_row_stats, self.uniforms, self.logits,
+                      self.row_stats, self.accept_len, self.out_tok, self.next_n_clean,
+                      self.next_clean_tok, self.next_kv_len, self.ws, hidden=self.hidden,
+                      ratio=self.ratio, lora_A=self.lora_A, lora_B=self.lora_B,
+                      err_flag=self.err, stream=stream)
+
+    def outputs(self) -> Dict[str, np.ndarray]:
+        torch.cuda.synchronize()
+        return dict(accept_len=self.accept_len.cpu().numpy(), out_tok=self.out_tok.cpu().numpy(),
+                    next_n_clean=self.next_n_clean.cpu().numpy(),
+                    next_clean_tok=self.next_clean_tok.cpu().numpy(),
+                    next_kv_len=self.next_kv_len.cpu().numpy(), ratio=self.ratio.cpu().numpy())
+
+    def host_view(self) -> Dict[str, np.ndarray]:
+        """Small inputs of the current step on the host (for oracle checks)."""
+        u = self.uniforms.cpu().numpy()
+        return dict(kv_len=self.kv_len_h, n_clean=self.n_clean_h, clean_tok=self.clean_tok_h,
+                    page_table=self.page_table_h, uniforms=u, _wl=self)
+
+
+def _bf16_host(t: torch.Tensor) -> np.ndarray:
+    return t.contiguous().view(torch.int16).cpu().numpy().view(np.uint16)
+
+
+def request_slice(host: Dict, cfg: I.IsdConfig, b: int) -> Dict[str, np.ndarray]:
+    """Single-request copy of the step's inputs (its own pages renumbered 0..)."""
+    wl = host["_wl"]
+    pages = host["page_table"][b]
+    pages = pages[pages >= 0]
+    idx = torch.from_numpy(pages.astype(np.int64)).cuda()
+    return dict(
+        q=_bf16_host(wl.q[b:b + 1]), k_new=_bf16_host(wl.k_new[b:b + 1]),
+        v_new=_bf16_host(wl.v_new[b:b + 1]),
+        k_pool=_bf16_host(wl.k_pool.index_select(0, idx)),
+        v_pool=_bf16_host(wl.v_pool.index_select(0, idx)),
+        page_table=np.arange(len(pages), dtype=np.int32)[None, :],
+        kv_len=host["kv_len"][b:b + 1], n_clean=host["n_clean"][b:b + 1])
+
+
+__all__ = ["DeviceWorkload", "request_slice"]

@@ -1,0 +1,96 @@
+"""C-ABI checks that need no GPU: the library loads, exports every entry
+point include/isd.h declares, sizes workspaces, and rejects bad arguments on
+the host before touching the device."""
+import ctypes
+import os
+import re
+
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+@pytest.fixture(scope="module")
+def isd():
+    from speculative_verification_isd_b200 import build as B
+    B.build()
+    from speculative_verification_isd_b200 import isd as lib
+    return lib
+
+
+def declared_functions():
+    text = open(os.path.join(ROOT, "include", "isd.h")).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return sorted(set(re.findall(r"\b(isd_[a-z_]+)\s*\(", text)))
+
+
+def test_every_declared_symbol_is_exported(isd):
+    names = declared_functions()
+    assert "isd_step" in names and "isd_accept" in names
+    lib = ctypes.CDLL(isd.LIB_PATH)
+    for n in names:
+        assert hasattr(lib, n), n
+    assert set(isd.EXPORTED) == set(names)
+
+
+def test_status_strings(isd):
+    lib = isd.library()
+    assert lib.isd_status_string(0) == b"ISD_OK"
+    assert lib.isd_status_string(-3) == b"ISD_ERR_WORKSPACE"
+    assert lib.isd_status_string(7) == b"ISD_ERR_UNKNOWN"
+
+
+def test_workspace_sizes(isd):
+    from speculative_verification_isd_b200 import inputs as I
+    for name, cfg in I.CONFIGS.items():
+        d = isd.make_dims(cfg.B, cfg.N, cfg.Hq, cfg.Hkv, cfg.D, cfg.V, cfg.page_size, 100,
+                          cfg.max_pages_per_req(), cfg.lora_rank)
+        n = isd.workspace_bytes(d)
+        assert n > 0 and n % 256 == 0, name
+        assert n >= cfg.M * cfg.H * 2
+    bad = isd.make_dims(2, 2, 4, 3, 64, 10, 16, 10, 4)   # Hq % Hkv != 0
+    assert isd.workspace_bytes(bad) == 0
+    bad = isd.make_dims(2, 0, 4, 1, 64, 10, 16, 10, 4)   # N = 0
+    assert isd.workspace_bytes(bad) == 0
+
+
+def test_host_validation_rejects_before_launch(isd):
+    lib = isd.library()
+    d = isd.make_dims(2, 2, 4, 1, 64, 512, 16, 10, 4)
+    need = isd.workspace_bytes(d)
+    fake = ctypes.c_void_p(1 << 20)   # never dereferenced: validation fails first
+    p = [fake] * 10
+    # missing workspace
+    st = lib.isd_attention(ctypes.byref(d), *p, 0, None, None)
+    assert st == isd.ISD_ERR_WORKSPACE
+    # misaligned workspace
+    st = lib.isd_attention(ctypes.byref(d), *p[:9], ctypes.c_void_p((1 << 20) + 8), need, None,
+                           None)
+    assert st == isd.ISD_ERR_WORKSPACE
+    # null tensor pointer
+    st = lib.isd_attention(ctypes.byref(d), None, *p[1:], need, None, None)
+    assert st == isd.ISD_ERR_INVALID_ARG
+    # unsupported head dim
+    d2 = isd.make_dims(2, 2, 4, 1, 96, 512, 16, 10, 4)
+    st = lib.isd_attention(ctypes.byref(d2), *p, isd.workspace_bytes(d2), None, None)
+    assert st == isd.ISD_ERR_UNSUPPORTED_SHAPE
+    # hidden size not a multiple of 64 for the tensor-core LM head
+    d3 = isd.make_dims(2, 2, 1, 1, 32, 512, 16, 10, 4)
+    st = lib.isd_lm_head(ctypes.byref(d3), fake, fake, None, None, fake, fake, fake,
+                         isd.workspace_bytes(d3), None, None)
+    assert st == isd.ISD_ERR_UNSUPPORTED_SHAPE
+    # LoRA pointers without a rank
+    st = lib.isd_lm_head(ctypes.byref(d), fake, fake, fake, fake, fake, fake, fake, need, None,
+                         None)
+    assert st == isd.ISD_ERR_INVALID_ARG
+    # bad proposal mode
+    d4 = isd.make_dims(2, 2, 4, 1, 64, 512, 16, 10, 4, proposal_mode=5)
+    assert isd.workspace_bytes(d4) == 0
+    assert b"invalid" in lib.isd_last_error() or b"unsupported" in lib.isd_last_error()
+
+
+def test_binding_checks_tensors_on_host(isd):
+    import torch
+    d = isd.make_dims(2, 2, 4, 1, 64, 512, 16, 10, 4)
+    with pytest.raises(ValueError):
+        isd._ptr(torch.zeros(4), torch.float32, 4, "cpu tensor")

@@ -1,0 +1,447 @@
+"""GPU parity: the CUDA path (through the C ABI) against the CPU oracle.
+
+Layered, so that a difference is charged to the stage that made it: every
+stage is compared with the oracle on the GPU's own input to that stage.
+Tolerances are the ones the method's acceptance spec states:
+  * attention outputs within 2e-2 absolute (bf16), KV pool bit-exact;
+  * logits within 1e-4 * sum_k |h_k w_k| + 1e-6 (fp32 re-association);
+  * row max bit-exact, argmax bit-exact (ties to the lowest index),
+    sum-exp and p/q ratios within 1e-5 relative;
+  * token ids, accept lengths and next state bit-exact, except requests whose
+    decision is within 1e-5 of the uniform that decides it (counted).
+"""
+import math
+
+import numpy as np
+import pytest
+import torch
+
+from oracle import isd_oracle as O
+from speculative_verification_isd_b200 import inputs as I
+
+from gpu_util import StepBuffers, bf16_host, f32_dev, i32_dev, row_stats_host
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module")
+def isd():
+    from speculative_verification_isd_b200 import isd as lib
+    return lib
+
+
+NEAR = 1e-5
+
+
+def near_threshold(b, logits, prev, tok, u, c, N, mode, ores):
+    """Does the oracle's decision for request b sit within NEAR of a boundary?"""
+    for j in range(2, c + 1):
+        r = ores["ratio"][b, j - 2]
+        if abs(float(u[b, j - 2]) - r) < NEAR:
+            return True
+        if not (float(u[b, j - 2]) < r):
+            break
+    rej = int(ores["rejected_at"][b])
+    rows = []
+    if rej > 0:
+        w = O.residual_distribution(logits[b, rej - 2], prev[b, N + rej - 2])
+        rows.append((w, float(u[b, N - 1])))
+    elif mode == O.PROPOSE_SAMPLE:
+        rows.append((O.softmax(logits[b, c - 1]), float(u[b, N])))
+        for m in range(N - 1):
+            rows.append((O.softmax(logits[b, N + m]), float(u[b, N + 1 + m])))
+    for w, uu in rows:
+        cum = np.cumsum(w)
+        tot = cum[-1]
+        if tot > 0 and np.min(np.abs(cum - uu * tot)) < NEAR * tot:
+            return True
+    return False
+
+
+def compare_accept(gpu, ores, logits, prev, inp, N, mode):
+    """Assert bit-exact outputs except near-threshold requests; return their count."""
+    B = logits.shape[0]
+    near = 0
+    for b in range(B):
+        c = int(inp["n_clean"][b])
+        if near_threshold(b, logits, prev, inp["clean_tok"], inp["uniforms"], c, N, mode, ores):
+            near += 1
+            continue
+        for key in ("accept_len", "next_n_clean", "next_kv_len"):
+            assert gpu[key][b] == ores[key][b], (key, b, gpu[key][b], ores[key][b])
+        assert np.array_equal(gpu["out_tok"][b], ores["out_tok"][b]), b
+        assert np.array_equal(gpu["next_clean_tok"][b], ores["next_clean_tok"][b]), b
+        # ratios of the tested proposals
+        for j in range(2, int(ores["accept_len"][b]) + 2):
+            if j - 2 >= ores["ratio"].shape[1] or ores["ratio"][b, j - 2] < 0:
+                break
+            assert gpu["ratio"][b, j - 2] == pytest.approx(ores["ratio"][b, j - 2], rel=NEAR)
+    return near
+
+
+def check_attention(sb, inp, cfg):
+    torch.cuda.synchronize()
+    out_o, kp_o, vp_o = O.attention(inp["q"], inp["k_new"], inp["v_new"], inp["k_pool"],
+                                    inp["v_pool"], inp["page_table"], inp["kv_len"],
+                                    inp["n_clean"], cfg.N, cfg.page_size, cfg.D ** -0.5)
+    got = O.bf16_to_f64(bf16_host(sb.hidden))
+    ref = O.bf16_to_f64(out_o)
+    err = np.abs(got - ref)
+    assert err.max() <= 2e-2, err.max()
+    assert err.mean() <= 3e-3, err.mean()
+    # inactive slots are exactly zero
+    for b in range(cfg.B):
+        for s in range(int(inp["n_clean"][b]), cfg.N):
+            assert np.all(got.reshape(cfg.B, cfg.Q, -1)[b, s] == 0.0)
+    assert np.array_equal(bf16_host(sb.k_pool), kp_o)
+    assert np.array_equal(bf16_host(sb.v_pool), vp_o)
+    return bf16_host(sb.hidden)
+
+
+def check_logits(sb, hidden_gpu, inp, cfg, rows=None):
+    """GPU logits against the oracle LM head on the GPU's own hidden."""
+    torch.cuda.synchronize()
+    h_in = hidden_gpu
+    if cfg.lora_rank:
+        h_in = O.gated_lora(hidden_gpu, inp["lora_A"], inp["lora_B"], cfg.B, cfg.N)
+    z_o = O.lm_head(h_in, inp["W"])
+    absdot = np.abs(O.bf16_to_f64(h_in)) @ np.abs(O.bf16_to_f64(inp["W"])).T
+    z_g = sb.logits.cpu().numpy()
+    bound = 1e-4 * absdot + 1e-6
+    if cfg.lora_rank:
+        # the adapter's intermediate bf16 roundings may differ by one ulp;
+        # allow the effect of one bf16 ulp of h' per product
+        bound = bound + absdot * 2.0 ** -8
+    assert np.all(np.abs(z_g - z_o) <= bound), np.max(np.abs(z_g - z_o) - bound)
+    return z_g
+
+
+def check_row_stats(sb, z_g):
+    m_g, s_g, a_g = row_stats_host(sb.row_stats)
+    m_o, s_o, a_o = O.row_stats_all(z_g)
+    assert np.array_equal(m_g, m_o.astype(np.float32).astype(np.float64))
+    assert np.array_equal(a_g, a_o)
+    assert np.all(np.abs(s_g - s_o) <= NEAR * s_o)
+
+
+PARITY_CONFIGS = ["tiny", "ragged_small", "ragged_lora", "qwen_medium"]
+
+
+@pytest.mark.parametrize("name", PARITY_CONFIGS)
+@pytest.mark.parametrize("n_clean", ["full", "mixed"])
+def test_staged_parity(isd, name, n_clean):
+    cfg = I.CONFIGS[name]
+    inp = I.make_step_inputs(cfg, seed=3, n_clean=n_clean)
+    sb = StepBuffers(isd, cfg, inp)
+    prev = I.random_logits(cfg.B, cfg.Q, cfg.V, seed=5, scale=2.0)
+    sb.set_prev_logits(prev)
+    sb.attention()
+    hid = check_attention(sb, inp, cfg)
+    sb.lm_head()
+    z_g = check_logits(sb, hid, inp, cfg)
+    check_row_stats(sb, z_g)
+    sb.accept()
+    gpu = sb.outputs()
+    logits = z_g.reshape(cfg.B, cfg.Q, cfg.V)
+    ores = O.accept(logits, prev, inp["n_clean"], inp["clean_tok"], inp["kv_len"],
+                    inp["uniforms"], cfg.N)
+    near = compare_accept(gpu, ores, logits, prev, inp, cfg.N, O.PROPOSE_ARGMAX)
+    assert near <= max(1, cfg.B // 10)
+    assert int(sb.err.item()) == 0
+
+
+@pytest.mark.parametrize("name", ["tiny", "ragged_small", "qwen_medium"])
+def test_whole_step_matches_stages(isd, name):
+    """isd_step gives bit-identical results to the three stage calls."""
+    cfg = I.CONFIGS[name]
+    inp = I.make_step_inputs(cfg, seed=4, n_clean="mixed")
+    prev = I.random_logits(cfg.B, cfg.Q, cfg.V, seed=6, scale=2.0)
+    a = StepBuffers(isd, cfg, inp)
+    a.set_prev_logits(prev)
+    a.attention()
+    a.lm_head()
+    a.accept()
+    oa = a.outputs()
+    b = StepBuffers(isd, cfg, inp)
+    b.set_prev_logits(prev)
+    b.step()
+    ob = b.outputs()
+    for k in oa:
+        assert np.array_equal(oa[k], ob[k]), k
+    assert torch.equal(a.logits, b.logits)
+    assert torch.equal(a.hidden, b.hidden)
+    # determinism: the same step again is bit-identical
+    b.step()
+    oc = b.outputs()
+    for k in ob:
+        assert np.array_equal(ob[k], oc[k]), k
+
+
+@pytest.mark.parametrize("mode", [O.PROPOSE_ARGMAX, O.PROPOSE_SAMPLE])
+@pytest.mark.parametrize("V,N,B", [(16, 2, 400), (1000, 4, 64), (9000, 3, 40), (151936, 4, 8)])
+def test_accept_on_random_logits(isd, mode, V, N, B):
+    """Accept kernel alone on wide-spread random logits: many rejections,
+    residual draws and (sample mode) inverse-CDF proposals."""
+    cfg = I.IsdConfig("acc", B=B, N=N, Hq=1, Hkv=1, D=64, V=V, page_size=16, prefix_lo=0,
+                      prefix_hi=100)
+    Q = 2 * N - 1
+    rng = np.random.default_rng(V + N)
+    logits = I.random_logits(B, Q, V, seed=V, scale=1.5)
+    prev = I.random_logits(B, Q, V, seed=V + 1, scale=1.5)
+    nc = rng.integers(1, N + 1, B).astype(np.int32)
+    tok = rng.integers(0, V, (B, N)).astype(np.int32)
+    # make some proposals likely under q so that both outcomes occur
+    for b in range(B):
+        for j in range(2, N + 1):
+            if rng.random() < 0.5:
+                prev[b, N + j - 2, tok[b, j - 1]] += 4.0
+    kv = rng.integers(0, 5000, B).astype(np.int32)
+    u = I.step_uniforms(9, 0, B, N)
+    d = isd.make_dims(B, N, 1, 1, 64, V, 16, 1, 1, 0, mode)
+    ws = isd.alloc_workspace(d)
+    zl, zp = f32_dev(logits.reshape(B * Q, V)), f32_dev(prev.reshape(B * Q, V))
+    rs = torch.empty(B * Q, 4, dtype=torch.int32, device="cuda")
+    prs = torch.empty_like(rs)
+    isd.row_stats(d, zl, B * Q, rs, ws)
+    isd.row_stats(d, zp, B * Q, prs, ws)
+    outs = dict(accept_len=torch.empty(B, dtype=torch.int32, device="cuda"),
+                out_tok=torch.empty(B, N, dtype=torch.int32, device="cuda"),
+                next_n_clean=torch.empty(B, dtype=torch.int32, device="cuda"),
+                next_clean_tok=torch.empty(B, N, dtype=torch.int32, device="cuda"),
+                next_kv_len=torch.empty(B, dtype=torch.int32, device="cuda"),
+                ratio=torch.empty(B, max(N - 1, 1), dtype=torch.float32, device="cuda"))
+    err = torch.zeros(1, dtype=torch.int32, device="cuda")
+    isd.accept(d, zl, rs, zp, prs, i32_dev(nc), i32_dev(tok), i32_dev(kv), f32_dev(u),
+               outs["accept_len"], outs["out_tok"], outs["next_n_clean"], outs["next_clean_tok"],
+               outs["next_kv_len"], ws, ratio=outs["ratio"], err_flag=err)
+    torch.cuda.synchronize()
+    gpu = {k: v.cpu().numpy() for k, v in outs.items()}
+    ores = O.accept(logits, prev, nc, tok, kv, u, N, mode)
+    inp = dict(n_clean=nc, clean_tok=tok, uniforms=u)
+    near = compare_accept(gpu, ores, logits, prev, inp, N, mode)
+    assert near <= max(2, B // 50)
+    assert (ores["rejected_at"] > 0).sum() > 0 or N == 1
+    assert int(err.item()) == 0
+    # row stats of both inputs
+    m_g, s_g, a_g = row_stats_host(rs)
+    m_o, s_o, a_o = O.row_stats_all(logits)
+    assert np.array_equal(a_g, a_o) and np.all(np.abs(s_g - s_o) <= NEAR * s_o)
+
+
+def test_identical_rows_accept_everything_gpu(isd):
+    B, N, V = 32, 4, 5000
+    Q = 2 * N - 1
+    logits = I.random_logits(B, Q, V, seed=1)
+    prev = I.random_logits(B, Q, V, seed=2)
+    for j in range(2, N + 1):
+        prev[:, N + j - 2] = logits[:, j - 2]
+    d = isd.make_dims(B, N, 1, 1, 64, V, 16, 1, 1, 0, 0)
+    ws = isd.alloc_workspace(d)
+    zl, zp = f32_dev(logits.reshape(B * Q, V)), f32_dev(prev.reshape(B * Q, V))
+    rs = torch.empty(B * Q, 4, dtype=torch.int32, device="cuda")
+    prs = torch.empty_like(rs)
+    isd.row_stats(d, zl, B * Q, rs, ws)
+    isd.row_stats(d, zp, B * Q, prs, ws)
+    tok = np.random.default_rng(0).integers(0, V, (B, N)).astype(np.int32)
+    u = np.full((B, 2 * N), np.nextafter(np.float32(1), np.float32(0)), np.float32)
+    al = torch.empty(B, dtype=torch.int32, device="cuda")
+    ot = torch.empty(B, N, dtype=torch.int32, device="cuda")
+    nn_ = torch.empty(B, dtype=torch.int32, device="cuda")
+    nt = torch.empty(B, N, dtype=torch.int32, device="cuda")
+    nk = torch.empty(B, dtype=torch.int32, device="cuda")
+    ra = torch.empty(B, N - 1, dtype=torch.float32, device="cuda")
+    isd.accept(d, zl, rs, zp, prs, i32_dev(np.full(B, N)), i32_dev(tok), i32_dev(np.zeros(B)),
+               f32_dev(u), al, ot, nn_, nt, nk, ws, ratio=ra)
+    torch.cuda.synchronize()
+    assert torch.all(al == N)
+    assert torch.all(ra == 1.0)
+
+
+def test_stride_one_and_empty_prefix(isd):
+    """N = 1 (plain greedy AR decoding) with some empty prefixes."""
+    cfg = I.IsdConfig("n1", B=4, N=1, Hq=8, Hkv=2, D=128, V=777, page_size=16, prefix_lo=0,
+                      prefix_hi=50, fixed_prefix=(0, 1, 16, 50), w_std=0.3, qkv_std=0.5,
+                      kv_std=1.0)
+    inp = I.make_step_inputs(cfg, seed=8, n_clean="one")
+    sb = StepBuffers(isd, cfg, inp)
+    sb.set_prev_logits(np.zeros((cfg.B, 1, cfg.V), np.float32))
+    sb.step()
+    hid = check_attention(sb, inp, cfg)
+    z = check_logits(sb, hid, inp, cfg)
+    gpu = sb.outputs()
+    assert np.array_equal(gpu["out_tok"][:, 0], z.reshape(cfg.B, cfg.V).argmax(-1))
+    assert np.array_equal(gpu["next_kv_len"], inp["kv_len"] + 1)
+
+
+def test_bad_page_and_bad_nclean_raise_flags(isd):
+    cfg = I.CONFIGS["ragged_small"]
+    inp = I.make_step_inputs(cfg, seed=2)
+    inp["page_table"] = inp["page_table"].copy()
+    inp["page_table"][1, 0] = 10 ** 6          # out of the pool: flagged, not read
+    inp["n_clean"] = inp["n_clean"].copy()
+    inp["n_clean"][2] = cfg.N + 1              # out of range: request skipped
+    sb = StepBuffers(isd, cfg, inp)
+    sb.set_prev_logits(I.random_logits(cfg.B, cfg.Q, cfg.V, seed=1))
+    sb.step()
+    gpu = sb.outputs()
+    flags = int(sb.err.item())
+    assert flags & isd.FLAG_PAGE_OOB
+    assert flags & isd.FLAG_NCLEAN_RANGE
+    assert gpu["accept_len"][2] == 0 and gpu["next_kv_len"][2] == inp["kv_len"][2]
+    assert np.all(np.isfinite(sb.logits.cpu().numpy()))
+
+
+def test_poisoned_unused_pages_do_not_leak(isd):
+    """NaN in every pool row that no request may read leaves outputs finite."""
+    cfg = I.CONFIGS["ragged_small"]
+    inp = I.make_step_inputs(cfg, seed=12)
+    P = cfg.page_size
+    readable = np.zeros(inp["k_pool"].shape[:2], bool)
+    for b in range(cfg.B):
+        for t in range(int(inp["kv_len"][b]) + int(inp["n_clean"][b]) + cfg.N - 1):
+            readable[inp["page_table"][b, t // P], t % P] = True
+    nan = np.uint16(0x7FC0)
+    inp["k_pool"][~readable] = nan
+    inp["v_pool"][~readable] = nan
+    sb = StepBuffers(isd, cfg, inp)
+    sb.set_prev_logits(I.random_logits(cfg.B, cfg.Q, cfg.V, seed=1))
+    sb.attention()
+    hid = check_attention(sb, inp, cfg)
+    assert np.all(np.isfinite(O.bf16_to_f64(hid)))
+
+
+def test_tiny_closed_loop_1000_steps(isd):
+    """Tiny config, 1000 consecutive steps: the GPU drives the loop; at every
+    step the oracle recomputes the step from the same state and the two must
+    agree (KV pool bit-exact, logits within tolerance, decisions exact except
+    counted near-threshold cases)."""
+    base = I.CONFIGS["tiny"]
+    steps = 1000
+    cfg = I.IsdConfig("tiny_loop", B=base.B, N=base.N, Hq=base.Hq, Hkv=base.Hkv, D=base.D,
+                      V=base.V, page_size=base.page_size, prefix_lo=base.prefix_lo,
+                      prefix_hi=base.prefix_hi + steps * base.N + 4, fixed_prefix=None)
+    kv0 = np.array(base.fixed_prefix, np.int32)
+    inp = I.make_step_inputs(base, seed=0, n_clean="one")
+    tables = I.make_embedding_tables(base, seed=0)
+    # a pool large enough for the whole run
+    P = cfg.page_size
+    max_pages = (int(kv0.max()) + steps * cfg.N + cfg.Q + P - 1) // P
+    num_pages = cfg.B * max_pages
+    rng = np.random.default_rng(0)
+    perm = rng.permutation(num_pages).astype(np.int32)
+    table = perm.reshape(cfg.B, max_pages)
+    pool_k = np.zeros((num_pages, P, cfg.Hkv, cfg.D), np.uint16)
+    pool_v = np.zeros_like(pool_k)
+    for b in range(cfg.B):   # copy the seeded prefix into the new pages
+        for t in range(int(kv0[b])):
+            src = inp["page_table"][b, t // P]
+            pool_k[table[b, t // P], t % P] = inp["k_pool"][src, t % P]
+            pool_v[table[b, t // P], t % P] = inp["v_pool"][src, t % P]
+    state = dict(kv_len=kv0.copy(), n_clean=np.ones(cfg.B, np.int32),
+                 clean_tok=np.array([[7, -1], [300, -1]], np.int32))
+    prev = np.zeros((cfg.B, cfg.Q, cfg.V), np.float32)
+    d = isd.make_dims(cfg.B, cfg.N, cfg.Hq, cfg.Hkv, cfg.D, cfg.V, P, num_pages, max_pages)
+    ws = isd.alloc_workspace(d)
+    from gpu_util import bf16_dev
+    kp, vp = bf16_dev(pool_k), bf16_dev(pool_v)
+    Wd = bf16_dev(inp["W"])
+    tab_d = i32_dev(table)
+    hid = torch.empty(d.M, d.H, dtype=torch.bfloat16, device="cuda")
+    logits = torch.empty(d.M, d.V, dtype=torch.float32, device="cuda")
+    rs = torch.empty(d.M, 4, dtype=torch.int32, device="cuda")
+    prev_d = torch.zeros(d.M, d.V, dtype=torch.float32, device="cuda")
+    prs = torch.empty(d.M, 4, dtype=torch.int32, device="cuda")
+    isd.row_stats(d, prev_d, d.M, prs, ws)
+    outs = [torch.empty(cfg.B, dtype=torch.int32, device="cuda"),
+            torch.empty(cfg.B, cfg.N, dtype=torch.int32, device="cuda"),
+            torch.empty(cfg.B, dtype=torch.int32, device="cuda"),
+            torch.empty(cfg.B, cfg.N, dtype=torch.int32, device="cuda"),
+            torch.empty(cfg.B, dtype=torch.int32, device="cuda")]
+    ratio = torch.empty(cfg.B, cfg.N - 1, dtype=torch.float32, device="cuda")
+    err = torch.zeros(1, dtype=torch.int32, device="cuda")
+    near_total, emitted = 0, 0
+    for k in range(steps):
+        q, kn, vn = I.embed_block(tables, state["clean_tok"], state["n_clean"], cfg.N, cfg.V)
+        u = I.step_uniforms(0, k, cfg.B, cfg.N)
+        isd.step(d, bf16_dev(q), bf16_dev(kn), bf16_dev(vn), kp, vp, tab_d,
+                 i32_dev(state["kv_len"]), i32_dev(state["n_clean"]),
+                 i32_dev(state["clean_tok"]), Wd, prev_d, prs, f32_dev(u), logits, rs, *outs,
+                 ws, hidden=hid, ratio=ratio, err_flag=err)
+        torch.cuda.synchronize()
+        # oracle on the same state
+        o_hid, pool_k, pool_v = O.attention(q, kn, vn, pool_k, pool_v, table, state["kv_len"],
+                                            state["n_clean"], cfg.N, P, cfg.D ** -0.5)
+        g_hid = bf16_host(hid)
+        assert np.abs(O.bf16_to_f64(g_hid) - O.bf16_to_f64(o_hid)).max() <= 2e-2
+        if k % 50 == 0 or k == steps - 1:
+            assert np.array_equal(bf16_host(kp), pool_k)
+            assert np.array_equal(bf16_host(vp), pool_v)
+        z_g = logits.cpu().numpy()
+        z_o = O.lm_head(g_hid, inp["W"])
+        absdot = np.abs(O.bf16_to_f64(g_hid)) @ np.abs(O.bf16_to_f64(inp["W"])).T
+        assert np.all(np.abs(z_g - z_o) <= 1e-4 * absdot + 1e-6)
+        L = z_g.reshape(cfg.B, cfg.Q, cfg.V)
+        ores = O.accept(L, prev, state["n_clean"], state["clean_tok"], state["kv_len"], u, cfg.N)
+        gpu = dict(accept_len=outs[0].cpu().numpy(), out_tok=outs[1].cpu().numpy(),
+                   next_n_clean=outs[2].cpu().numpy(), next_clean_tok=outs[3].cpu().numpy(),
+                   next_kv_len=outs[4].cpu().numpy(), ratio=ratio.cpu().numpy())
+        near_total += compare_accept(gpu, ores, L, prev, dict(state, uniforms=u), cfg.N,
+                                     O.PROPOSE_ARGMAX)
+        emitted += int(gpu["accept_len"].sum())
+        # advance with the GPU's state (the loop is driven by the CUDA path)
+        state = dict(kv_len=gpu["next_kv_len"], n_clean=gpu["next_n_clean"],
+                     clean_tok=gpu["next_clean_tok"])
+        prev = L.copy()
+        prev_d.copy_(logits)
+        prs.copy_(rs)
+    assert int(err.item()) == 0
+    assert near_total <= 10
+    assert emitted >= steps * cfg.B
+
+
+@pytest.mark.slow
+def test_full_size_b32_n4_sampled(isd):
+    """Qwen3-8B shapes, B=32, N=4 (the benchmark workload and launch
+    configuration): sampled attention rows, sampled logits, row statistics of
+    sampled rows, and the full accept decision checked against the oracle."""
+    from speculative_verification_isd_b200 import workload as Wk
+    cfg = I.CONFIGS["qwen3_8b_b32_n4"]
+    wl = Wk.DeviceWorkload(isd, cfg, seed=0)
+    wl.step()
+    torch.cuda.synchronize()
+    rng = np.random.default_rng(0)
+    # attention: a few (request, slot, head) rows
+    host = wl.host_view()
+    for b in rng.choice(cfg.B, 3, replace=False):
+        sub = Wk.request_slice(host, cfg, int(b))
+        out_o, _, _ = O.attention(sub["q"], sub["k_new"], sub["v_new"], sub["k_pool"],
+                                  sub["v_pool"], sub["page_table"], sub["kv_len"],
+                                  sub["n_clean"], cfg.N, cfg.page_size, cfg.D ** -0.5)
+        got = O.bf16_to_f64(bf16_host(wl.hidden[b * cfg.Q:(b + 1) * cfg.Q]))
+        assert np.abs(got - O.bf16_to_f64(out_o)).max() <= 2e-2
+    # logits: sampled entries, one float64 dot product each
+    hid = bf16_host(wl.hidden)
+    z = wl.logits
+    for _ in range(64):
+        m = int(rng.integers(0, cfg.M))
+        v = int(rng.integers(0, cfg.V))
+        w_row = bf16_host(wl.W[v:v + 1])[0]
+        ref = O.lm_head_entry(hid[m], w_row)
+        absdot = float(np.abs(O.bf16_to_f64(hid[m])) @ np.abs(O.bf16_to_f64(w_row)))
+        assert abs(float(z[m, v].item()) - ref) <= 1e-4 * absdot + 1e-6
+    # row statistics of a few rows and the complete accept step on GPU logits
+    zg = z.cpu().numpy().reshape(cfg.B, cfg.Q, cfg.V)
+    m_g, s_g, a_g = row_stats_host(wl.row_stats)
+    for r in rng.choice(cfg.M, 8, replace=False):
+        m_o, s_o, a_o = O.row_stats(zg.reshape(cfg.M, -1)[r])
+        assert m_g[r] == m_o and a_g[r] == a_o and abs(s_g[r] - s_o) <= NEAR * s_o
+    prev = wl.prev_logits.cpu().numpy().reshape(cfg.B, cfg.Q, cfg.V)
+    ores = O.accept(zg, prev, host["n_clean"], host["clean_tok"], host["kv_len"],
+                    host["uniforms"], cfg.N)
+    gpu = wl.outputs()
+    near = compare_accept(gpu, ores, zg, prev, host, cfg.N, O.PROPOSE_ARGMAX)
+    assert near <= 2
+    # the constructed acceptance rate holds on every tested proposal
+    r = ores["ratio"][ores["ratio"] >= 0]
+    assert np.all(np.abs(r - cfg.accept_rate) < 1e-4)
+    assert int(wl.err.item()) == 0
