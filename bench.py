@@ -91,7 +91,8 @@ class ClockSampler:
         self.thread.join(timeout=2)
         rows = [l.split(", ") for l in self.lines if l]
         if self.bus_id:
-            mine = [r for r in rows if len(r) > 1 and self.bus_id.lower() in r[1].lower()]
+            mine = [r for r in rows if len(r) > 1 and r[1].strip().lower().endswith(
+                self.bus_id.lower()[-10:])]
             rows = mine or rows
         if not rows:
             return None
@@ -330,7 +331,8 @@ def main():
     torch.cuda.synchronize()
     bus = None
     try:
-        bus = torch.cuda.get_device_properties(torch.cuda.current_device()).pci_bus_id
+        pr = torch.cuda.get_device_properties(torch.cuda.current_device())
+        bus = "%08X:%02X:00.0" % (int(getattr(pr, "pci_domain_id", 0)), int(pr.pci_bus_id))
     except Exception:
         bus = None
     clocks = ClockSampler(bus)

@@ -91,20 +91,27 @@ struct AcceptArgs {
 };
 
 // Weight of vocabulary entry i for "row" r of a sweep.
-//   residual (r = 0 of a rejecting request): max(0, p_i - q_i)
-//   sample-mode proposal rows: exp(z_i - max) of that row
+//   sample-mode proposal rows: exp(z_i - max) of that row;
+//   residual of a rejecting request: max(0, p_i - q_i), evaluated as
+//     q_i * expm1(log p_i - log q_i),
+//     log p_i - log q_i = (zp_i - zq_i) + [(mq - mp) + log(Sq / Sp)].
+//   A plain difference of the two probabilities cancels catastrophically
+//   when p and q nearly agree (both ~1/V, difference ~1e-6 of that); in this
+//   form entries with equal logits get exactly equal log-ratios, so the
+//   weights keep their shape and only the row constant carries rounding.
 struct SweepRow {
     const float* zp;
     const float* zq;  // null for proposal rows
-    float mp, inv_sp, mq, inv_sq;
+    float mp, mq, inv_sq, k;  // k = (mq - mp) + log(Sq / Sp)
 };
 
 ISD_DEVINL float sweep_weight(const SweepRow& r, int i) {
-    const float a = __expf(__ldg(r.zp + i) - r.mp);
-    if (!r.zq) return a;
-    const float p = a * r.inv_sp;
-    const float q = __expf(__ldg(r.zq + i) - r.mq) * r.inv_sq;
-    return fmaxf(p - q, 0.f);
+    const float zp = __ldg(r.zp + i);
+    if (!r.zq) return __expf(zp - r.mp);
+    const float zq = __ldg(r.zq + i);
+    const float d = (zp - zq) + r.k;
+    if (!(d > 0.f)) return 0.f;
+    return __expf(zq - r.mq) * r.inv_sq * expm1f(d);
 }
 
 constexpr int kSeg = kAcceptChunk / kAcceptThreads;  // contiguous entries per thread
@@ -254,8 +261,8 @@ __global__ void __launch_bounds__(kAcceptThreads) accept_kernel(AcceptArgs a) {
             const size_t rp = (size_t)b * Q + (state - 2);
             const size_t rq = (size_t)b * Q + (N + state - 2);
             const isd_row_stat sp = a.stats[rp], sq = a.prev_stats[rq];
-            *r = SweepRow{a.logits + rp * V, a.prev_logits + rq * V, sp.max, 1.f / sp.sumexp,
-                          sq.max, 1.f / sq.sumexp};
+            *r = SweepRow{a.logits + rp * V, a.prev_logits + rq * V, sp.max, sq.max,
+                          1.f / sq.sumexp, (sq.max - sp.max) + logf(sq.sumexp / sp.sumexp)};
         } else {
             const size_t rr = (size_t)b * Q + (k == 0 ? c - 1 : N + k - 1);
             const isd_row_stat s = a.stats[rr];

@@ -460,12 +460,15 @@ static size_t attn_smem_bytes() {
 template <int D, int NRG>
 static cudaError_t launch_attention_t(const AttnArgs& a, dim3 grid, cudaStream_t st) {
     const size_t smem = attn_smem_bytes<D, NRG>();
-    static bool configured = false;  // per-process attribute, set once
-    if (!configured) {
+    static unsigned long long configured = 0;  // bit per device: attribute set
+    int dev = 0;
+    cudaGetDevice(&dev);
+    if (dev < 0 || dev >= 64) return cudaErrorInvalidDevice;
+    if (!(configured >> dev & 1ull)) {
         cudaError_t e = cudaFuncSetAttribute(attention_kernel<D, NRG>,
                                              cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
         if (e != cudaSuccess) return e;
-        configured = true;
+        configured |= 1ull << dev;
     }
     attention_kernel<D, NRG><<<grid, 128 * NRG, smem, st>>>(a);
     return cudaGetLastError();

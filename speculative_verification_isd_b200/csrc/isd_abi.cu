@@ -9,7 +9,14 @@
 #include "common.cuh"
 #include "plan.h"
 
+namespace {
+thread_local char g_last_error[256] = "";
+thread_local char g_detail[160] = "";
+}  // namespace
+
 namespace isd {
+// Host-side context for the next CUDA failure report (this thread).
+void set_error_detail(const char* msg) { snprintf(g_detail, sizeof(g_detail), "%s", msg); }
 cudaError_t launch_attention(const Plan& p, const isd_dims* d, const uint16_t* q,
                              const uint16_t* k_new, const uint16_t* v_new, uint16_t* k_pool,
                              uint16_t* v_pool, const int32_t* page_table, const int32_t* kv_len,
@@ -35,11 +42,10 @@ using isd::Plan;
 
 namespace {
 
-thread_local char g_last_error[256] = "";
-
 isd_status cuda_fail(cudaError_t e) {
-    snprintf(g_last_error, sizeof(g_last_error), "%s: %s", cudaGetErrorName(e),
-             cudaGetErrorString(e));
+    snprintf(g_last_error, sizeof(g_last_error), "%s: %s%s%s", cudaGetErrorName(e),
+             cudaGetErrorString(e), g_detail[0] ? " -- " : "", g_detail);
+    g_detail[0] = 0;
     return ISD_ERR_CUDA;
 }
 

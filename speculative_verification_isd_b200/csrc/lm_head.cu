@@ -35,6 +35,7 @@ namespace isd {
 struct LmArgs {
     int V, Mh, H;
     int BN, NB, n_acc, stages, n_tiles;
+    int w_rows, h_rows0, h_rows1;  // TMA box heights (never taller than the tensor)
     uint32_t tmem_cols;
     float* logits;
     int32_t* err_flag;
@@ -44,8 +45,8 @@ constexpr uint64_t kWaitLimitNs = 2000000000ull;
 constexpr int kLmThreads = 192;
 
 __global__ void __launch_bounds__(kLmThreads, 1)
-lm_head_kernel(const __grid_constant__ CUtensorMap tmap_w, const __grid_constant__ CUtensorMap tmap_h,
-               LmArgs a) {
+lm_head_kernel(const __grid_constant__ CUtensorMap tmap_w, const __grid_constant__ CUtensorMap tmap_h0,
+               const __grid_constant__ CUtensorMap tmap_h1, LmArgs a) {
     using namespace sm100;
     extern __shared__ unsigned char smem_raw[];
     unsigned char* smem = reinterpret_cast<unsigned char*>(
@@ -76,7 +77,8 @@ lm_head_kernel(const __grid_constant__ CUtensorMap tmap_w, const __grid_constant
         never = 0;
         fence_mbar_init();
         prefetch_tmap(&tmap_w);
-        prefetch_tmap(&tmap_h);
+        prefetch_tmap(&tmap_h0);
+        if (a.NB > 1) prefetch_tmap(&tmap_h1);
     }
     if (warp == 1) {
         tmem_alloc(tmem_holder, a.tmem_cols);
@@ -100,6 +102,9 @@ lm_head_kernel(const __grid_constant__ CUtensorMap tmap_w, const __grid_constant
             const uint64_t pol_h = policy_evict_last();
             uint32_t armed = 0, parity_bits = 0;
             int it = 0;
+            // rows of a box beyond the tensor are not delivered (and not used:
+            // their accumulator columns / vocabulary rows are never stored)
+            const uint32_t tx = (uint32_t)(a.w_rows + a.h_rows0 + a.h_rows1) * 128u;
             bool ok = true;
             for (int tile = blockIdx.x; ok && tile < a.n_tiles; tile += gridDim.x) {
                 for (int kb = 0; kb < kblocks; ++kb, ++it) {
@@ -112,11 +117,11 @@ lm_head_kernel(const __grid_constant__ CUtensorMap tmap_w, const __grid_constant
                     }
                     unsigned char* sa = smem + (size_t)s * stage_bytes;
                     unsigned char* sb = sa + 16384;
-                    mbar_arrive_expect_tx(&full[s], (uint32_t)stage_bytes);
+                    mbar_arrive_expect_tx(&full[s], tx);
                     tma_load_2d(sa, &tmap_w, &full[s], kb * 64, tile * 128, pol_w);
-                    for (int nb = 0; nb < a.NB; ++nb)
-                        tma_load_2d(sb + nb * a.BN * 128, &tmap_h, &full[s], kb * 64, nb * a.BN,
-                                    pol_h);
+                    tma_load_2d(sb, &tmap_h0, &full[s], kb * 64, 0, pol_h);
+                    if (a.NB > 1)
+                        tma_load_2d(sb + a.BN * 128, &tmap_h1, &full[s], kb * 64, a.BN, pol_h);
                     armed |= 1u << s;
                     parity_bits = (parity_bits & ~(1u << s)) | ((round & 1) << s);
                 }
@@ -265,7 +270,7 @@ struct LmShape {
     size_t smem;
 };
 
-bool lm_head_shape(int Mh, LmShape* s) {
+bool lm_head_shape(int Mh, int smem_limit, LmShape* s) {
     if (Mh < 1 || Mh > 512) return false;
     if (Mh <= 256) {
         s->NB = 1;
@@ -281,7 +286,7 @@ bool lm_head_shape(int Mh, LmShape* s) {
     while ((int)alloc < need) alloc <<= 1;
     s->tmem_cols = alloc;
     const int stage_bytes = 16384 + cols * 128;
-    const int budget = 227 * 1024 - 1024 - 256;
+    const int budget = smem_limit - 1024 - 256;  // alignment slack + barriers
     s->stages = budget / stage_bytes;
     if (s->stages > 8) s->stages = 8;
     if (s->stages < 2) return false;
@@ -296,25 +301,59 @@ static int num_sms_of_current_device() {
     return n > 0 ? n : 148;
 }
 
+void set_error_detail(const char* msg);
+
 cudaError_t launch_lm_head(const uint16_t* hidden, const uint16_t* W, int Mh, int H, int V,
                            float* logits, int32_t* err_flag, cudaStream_t st) {
-    LmShape sh;
-    if (!lm_head_shape(Mh, &sh)) return cudaErrorInvalidValue;
-    CUtensorMap tw, th;
-    if (!encode_bf16_2d(&tw, W, (uint64_t)V, (uint64_t)H, 128)) return cudaErrorInvalidValue;
-    if (!encode_bf16_2d(&th, hidden, (uint64_t)Mh, (uint64_t)H, (uint32_t)sh.BN))
-        return cudaErrorInvalidValue;
-    static int configured_devices = 0;  // bit per device: smem attribute set
+    // dynamic shared memory available to this kernel on the current device
+    static int smem_limit_dev[64];
     int dev = 0;
     cudaGetDevice(&dev);
-    if (!(configured_devices >> dev & 1)) {
-        cudaError_t e = cudaFuncSetAttribute(lm_head_kernel,
-                                             cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                             227 * 1024);
-        if (e != cudaSuccess) return e;
-        configured_devices |= 1 << dev;
+    if (dev < 0 || dev >= 64) return cudaErrorInvalidDevice;
+    if (!smem_limit_dev[dev]) {
+        int optin = 0;
+        cudaDeviceGetAttribute(&optin, cudaDevAttrMaxSharedMemoryPerBlockOptin, dev);
+        cudaFuncAttributes fa;
+        if (cudaFuncGetAttributes(&fa, lm_head_kernel) != cudaSuccess) {
+            set_error_detail("lm_head: kernel attributes unavailable");
+            return cudaErrorInvalidValue;
+        }
+        const int limit = optin - (int)fa.sharedSizeBytes;
+        if (cudaFuncSetAttribute(lm_head_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 limit) != cudaSuccess) {
+            set_error_detail("lm_head: shared-memory attribute rejected");
+            return cudaErrorInvalidValue;
+        }
+        smem_limit_dev[dev] = limit;
+    }
+    LmShape sh;
+    if (!lm_head_shape(Mh, smem_limit_dev[dev], &sh)) {
+        set_error_detail("lm_head: no tile shape for these rows");
+        return cudaErrorInvalidValue;
+    }
+    if (!get_encode_fn()) {
+        set_error_detail("lm_head: cuTensorMapEncodeTiled entry point not found");
+        return cudaErrorInvalidValue;
     }
     LmArgs a;
+    a.w_rows = V < 128 ? V : 128;
+    a.h_rows0 = Mh < sh.BN ? Mh : sh.BN;
+    a.h_rows1 = sh.NB > 1 ? Mh - sh.BN : 0;
+    CUtensorMap tw, th0, th1;
+    if (!encode_bf16_2d(&tw, W, (uint64_t)V, (uint64_t)H, (uint32_t)a.w_rows)) {
+        set_error_detail("lm_head: tensor map of W rejected");
+        return cudaErrorInvalidValue;
+    }
+    if (!encode_bf16_2d(&th0, hidden, (uint64_t)Mh, (uint64_t)H, (uint32_t)a.h_rows0)) {
+        set_error_detail("lm_head: tensor map of hidden rejected");
+        return cudaErrorInvalidValue;
+    }
+    th1 = th0;
+    if (sh.NB > 1 &&
+        !encode_bf16_2d(&th1, hidden, (uint64_t)Mh, (uint64_t)H, (uint32_t)a.h_rows1)) {
+        set_error_detail("lm_head: tensor map of hidden (second block) rejected");
+        return cudaErrorInvalidValue;
+    }
     a.V = V;
     a.Mh = Mh;
     a.H = H;
@@ -328,8 +367,10 @@ cudaError_t launch_lm_head(const uint16_t* hidden, const uint16_t* W, int Mh, in
     a.err_flag = err_flag;
     int grid = num_sms_of_current_device();
     if (grid > a.n_tiles) grid = a.n_tiles;
-    lm_head_kernel<<<grid, kLmThreads, sh.smem, st>>>(tw, th, a);
-    return cudaGetLastError();
+    lm_head_kernel<<<grid, kLmThreads, sh.smem, st>>>(tw, th0, th1, a);
+    cudaError_t e = cudaGetLastError();
+    if (e != cudaSuccess) set_error_detail("lm_head: launch failed");
+    return e;
 }
 
 }  // namespace isd

@@ -78,7 +78,7 @@ _lib.isd_lm_head.argtypes = [_dims_p] + [_vp] * 7 + [_sz, _vp, _vp]
 _lib.isd_lm_head.restype = _i32
 _lib.isd_row_stats.argtypes = [_dims_p, _vp, _i32, _vp, _vp, _sz, _vp]
 _lib.isd_row_stats.restype = _i32
-_lib.isd_accept.argtypes = [_dims_p] + [_vp] * 16 + [_sz, _vp, _vp]
+_lib.isd_accept.argtypes = [_dims_p] + [_vp] * 15 + [_sz, _vp, _vp]
 _lib.isd_accept.restype = _i32
 _lib.isd_step.argtypes = [_dims_p] + [_vp] * 25 + [_sz, _vp, _vp]
 _lib.isd_step.restype = _i32

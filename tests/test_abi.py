@@ -94,3 +94,23 @@ def test_binding_checks_tensors_on_host(isd):
     d = isd.make_dims(2, 2, 4, 1, 64, 512, 16, 10, 4)
     with pytest.raises(ValueError):
         isd._ptr(torch.zeros(4), torch.float32, 4, "cpu tensor")
+
+
+def test_binding_prototypes_match_header(isd):
+    """Every ctypes prototype has the header's parameter count and kinds."""
+    text = open(os.path.join(ROOT, "include", "isd.h")).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    lib = isd.library()
+    for name in declared_functions():
+        m = re.search(r"\b" + name + r"\s*\(([^)]*)\)\s*;", text, flags=re.S)
+        assert m, name
+        params = [p.strip() for p in m.group(1).split(",") if p.strip() and p.strip() != "void"]
+        argtypes = getattr(lib, name).argtypes
+        assert len(argtypes) == len(params), (name, len(argtypes), len(params))
+        for p, a in zip(params, argtypes):
+            if "*" in p:
+                assert a in (ctypes.c_void_p, ctypes.c_char_p) or hasattr(a, "_type_"), (name, p)
+            elif p.startswith("size_t"):
+                assert a is ctypes.c_size_t, (name, p)
+            else:
+                assert a is ctypes.c_int32, (name, p)

@@ -33,46 +33,68 @@ def isd():
 NEAR = 1e-5
 
 
-def near_threshold(b, logits, prev, tok, u, c, N, mode, ores):
-    """Does the oracle's decision for request b sit within NEAR of a boundary?"""
+def ratio_near(b, c, u, ores):
+    """Is an accept decision of request b within NEAR of its uniform?"""
     for j in range(2, c + 1):
         r = ores["ratio"][b, j - 2]
         if abs(float(u[b, j - 2]) - r) < NEAR:
             return True
         if not (float(u[b, j - 2]) < r):
             break
-    rej = int(ores["rejected_at"][b])
-    rows = []
-    if rej > 0:
-        w = O.residual_distribution(logits[b, rej - 2], prev[b, N + rej - 2])
-        rows.append((w, float(u[b, N - 1])))
-    elif mode == O.PROPOSE_SAMPLE:
-        rows.append((O.softmax(logits[b, c - 1]), float(u[b, N])))
-        for m in range(N - 1):
-            rows.append((O.softmax(logits[b, N + m]), float(u[b, N + 1 + m])))
-    for w, uu in rows:
-        cum = np.cumsum(w)
-        tot = cum[-1]
-        if tot > 0 and np.min(np.abs(cum - uu * tot)) < NEAR * tot:
-            return True
     return False
 
 
+def draw_explained(w, u, y):
+    """Is bucket y within NEAR * sum(w) of the oracle's inverse-CDF target?"""
+    cum = np.cumsum(np.asarray(w, dtype=np.float64))
+    tot = cum[-1]
+    if not (0 <= y < len(w)) or w[y] <= 0 or tot <= 0:
+        return False
+    t = float(u) * tot
+    lo = cum[y - 1] if y > 0 else 0.0
+    dist = max(0.0, lo - t, t - cum[y])
+    return dist <= NEAR * tot
+
+
 def compare_accept(gpu, ores, logits, prev, inp, N, mode):
-    """Assert bit-exact outputs except near-threshold requests; return their count."""
+    """Decisions, lengths and states bit-exact; every differing token must be an
+    inverse-CDF draw whose GPU pick lies within NEAR * sum(w) of the oracle's
+    target.  Returns the number of requests excused (near-threshold ratio or
+    a rounding-explained draw)."""
     B = logits.shape[0]
+    u = inp["uniforms"]
     near = 0
     for b in range(B):
         c = int(inp["n_clean"][b])
-        if near_threshold(b, logits, prev, inp["clean_tok"], inp["uniforms"], c, N, mode, ores):
+        if ratio_near(b, c, u, ores):
             near += 1
             continue
         for key in ("accept_len", "next_n_clean", "next_kv_len"):
             assert gpu[key][b] == ores[key][b], (key, b, gpu[key][b], ores[key][b])
-        assert np.array_equal(gpu["out_tok"][b], ores["out_tok"][b]), b
-        assert np.array_equal(gpu["next_clean_tok"][b], ores["next_clean_tok"][b]), b
+        A = int(ores["accept_len"][b])
+        # draws of this request: (position in out_tok / next_clean_tok, weights, uniform)
+        draws = {}
+        rej = int(ores["rejected_at"][b])
+        if rej > 0:
+            draws[("out", A - 1)] = (O.residual_distribution(logits[b, rej - 2], prev[b, N + rej - 2]),
+                                     u[b, N - 1])
+            draws[("next", 0)] = draws[("out", A - 1)]
+        elif mode == O.PROPOSE_SAMPLE:
+            rows = [c - 1] + [N + m for m in range(N - 1)]
+            for k, r in enumerate(rows):
+                draws[("next", k)] = (O.softmax(logits[b, r]), u[b, N + k])
+            draws[("out", A - 1)] = draws[("next", 0)]
+        excused = False
+        for kind, key in (("out", "out_tok"), ("next", "next_clean_tok")):
+            g, o = gpu[key][b], ores[key][b]
+            for i in np.nonzero(g != o)[0]:
+                assert (kind, int(i)) in draws, (key, b, i, g, o)
+                w, uu = draws[(kind, int(i))]
+                assert draw_explained(w, uu, int(g[i])), (key, b, i, g[i], o[i])
+                excused = True
+        near += excused
         # ratios of the tested proposals
-        for j in range(2, int(ores["accept_len"][b]) + 2):
+        for j in range(2, A + 2):
             if j - 2 >= ores["ratio"].shape[1] or ores["ratio"][b, j - 2] < 0:
                 break
             assert gpu["ratio"][b, j - 2] == pytest.approx(ores["ratio"][b, j - 2], rel=NEAR)
@@ -219,7 +241,8 @@ def test_accept_on_random_logits(isd, mode, V, N, B):
     ores = O.accept(logits, prev, nc, tok, kv, u, N, mode)
     inp = dict(n_clean=nc, clean_tok=tok, uniforms=u)
     near = compare_accept(gpu, ores, logits, prev, inp, N, mode)
-    assert near <= max(2, B // 50)
+    print(f"requests excused by rounding near a threshold: {near} of {B}")
+    assert near <= max(2, B // 20)
     assert (ores["rejected_at"] > 0).sum() > 0 or N == 1
     assert int(err.item()) == 0
     # row stats of both inputs
