@@ -138,40 +138,64 @@ __global__ void __launch_bounds__(128 * NRG) attention_kernel(AttnArgs a) {
         rpos[i] = (rr < a.rows && total > 0) ? slot_pos(rr % a.Q, kv, c, a.N) : -1;
     }
 
-    // ---- tile loader: keys [k0, k0+64) of this (request, head)
-    auto load_tile = [&](int stage, int k0) {
-        unsigned char* dk = sK + stage * kKT * D * 2;
-        unsigned char* dv = sV + stage * kKT * D * 2;
-        for (int i = tid; i < kKT * CH; i += THREADS) {
-            const int key = i / CH, cc = i % CH;
-            const int t = k0 + key;
-            const __nv_bfloat16* srck = a.k_new;
-            const __nv_bfloat16* srcv = a.v_new;
-            int bytes = 0;
-            if (t < kend) {
-                size_t off;
-                if (t < kv) {
-                    const int page = ptab[t / a.P];
-                    if (page >= 0 && page < a.num_pages) {
-                        off = ((size_t)page * a.P + t % a.P) * row_stride + (size_t)g * D + cc * 8;
-                        srck = a.k_pool;
-                        srcv = a.v_pool;
-                        bytes = 16;
-                    } else {
-                        raise_flag(a.err_flag, ISD_FLAG_PAGE_OOB);
-                        off = 0;
-                    }
-                } else {
-                    const int r = t - kv;
-                    const int slot = r < c ? r : a.N + (r - c);
-                    off = (((size_t)b * a.Q + slot) * a.Hkv + g) * D + cc * 8;
-                    bytes = 16;
-                }
-                srck += off;
-                srcv += off;
+    // ---- key -> cache-row table of this split (one page lookup per key):
+    //   >= 0      : pool row page*P + t%P (prefix keys)
+    //   -(slot+1) : the block's own slot `slot` in k_new / v_new
+    //   kNoKey    : nothing to load (bad page id); the chunk is zero-filled
+    constexpr int kNoKey = INT_MIN;
+    int* s_rows = reinterpret_cast<int*>(sV + kStages * kKT * D * 2);
+    const int nkeys = kend - kbeg;
+    for (int k = tid; k < nkeys; k += THREADS) {
+        const int t = kbeg + k;
+        int row;
+        if (t < kv) {
+            const int page = ptab[t / a.P];
+            if (page >= 0 && page < a.num_pages) {
+                row = page * a.P + t % a.P;
+            } else {
+                raise_flag(a.err_flag, ISD_FLAG_PAGE_OOB);
+                row = kNoKey;
             }
-            cp_async16(smem_u32(dk + swz<D>(key, cc)), srck, bytes);
-            cp_async16(smem_u32(dv + swz<D>(key, cc)), srcv, bytes);
+        } else {
+            const int r = t - kv;
+            row = -((r < c ? r : a.N + (r - c)) + 1);
+        }
+        s_rows[k] = row;
+    }
+    __syncthreads();
+
+    // ---- tile loader: each thread always copies chunk `cc` of keys
+    //      kr0 + j*KPP, so its swizzled smem offset is a per-thread constant
+    constexpr int KPP = THREADS / CH;  // keys per pass (a multiple of 8)
+    constexpr int PASSES = kKT / KPP;
+    static_assert(KPP % 8 == 0, "constant swizzle needs 8-key passes");
+    const int cc = tid % CH, kr0 = tid / CH;
+    const size_t pool_col = (size_t)g * D + cc * 8;
+    const __nv_bfloat16* knew_b = a.k_new + ((size_t)b * a.Q * a.Hkv + g) * D + cc * 8;
+    const __nv_bfloat16* vnew_b = a.v_new + ((size_t)b * a.Q * a.Hkv + g) * D + cc * 8;
+    const size_t slot_stride = (size_t)a.Hkv * D;
+    const uint32_t dst0 = (uint32_t)(kr0 * D * 2 + ((cc ^ (kr0 & 7)) << 4));
+    auto load_tile = [&](int stage, int tile) {
+        const uint32_t dk = smem_u32(sK + stage * kKT * D * 2) + dst0;
+        const uint32_t dv = smem_u32(sV + stage * kKT * D * 2) + dst0;
+#pragma unroll
+        for (int j = 0; j < PASSES; ++j) {
+            const int k = tile * kKT + kr0 + j * KPP;
+            const int row = k < nkeys ? s_rows[k] : kNoKey;
+            const __nv_bfloat16* sk = a.k_new;
+            const __nv_bfloat16* sv = a.v_new;
+            int bytes = 16;
+            if (row >= 0) {
+                sk = a.k_pool + (size_t)row * row_stride + pool_col;
+                sv = a.v_pool + (size_t)row * row_stride + pool_col;
+            } else if (row != kNoKey) {
+                sk = knew_b + (size_t)(-row - 1) * slot_stride;
+                sv = vnew_b + (size_t)(-row - 1) * slot_stride;
+            } else {
+                bytes = 0;
+            }
+            cp_async16(dk + j * KPP * D * 2, sk, bytes);
+            cp_async16(dv + j * KPP * D * 2, sv, bytes);
         }
     };
 
@@ -182,26 +206,36 @@ __global__ void __launch_bounds__(128 * NRG) attention_kernel(AttnArgs a) {
         for (int nt = 0; nt < NT; ++nt)
 #pragma unroll
             for (int e = 0; e < 4; ++e) o[mt][nt][e] = 0.f;
+    // running reference max (log2 domain) and running sum of each row
     float m_run[4], l_run[4];
 #pragma unroll
     for (int i = 0; i < 4; ++i) {
         m_run[i] = -INFINITY;
         l_run[i] = 0.f;
     }
+    // Keys below mask_from are cached prefix keys of a live split: visible to
+    // every active row, so their tiles need no masking.
+    const int mask_from = min(kv, kend);
+    // The reference max only moves when a row's max exceeds it by more than
+    // 2^8: probabilities are then at most 256 (exact in fp32, same relative
+    // precision in bf16) and the O rescale is skipped almost always.  The
+    // result is independent of the reference after the final normalisation.
+    constexpr float kRescaleThreshold = 8.f;
 
-    const int n_tiles = (kend - kbeg + kKT - 1) / kKT;
+    const int n_tiles = (nkeys + kKT - 1) / kKT;
 #pragma unroll
     for (int s = 0; s < kStages - 1; ++s) {
-        if (s < n_tiles) load_tile(s, kbeg + s * kKT);
+        if (s < n_tiles) load_tile(s, s);
         cp_async_commit();
     }
     const uint32_t q_base = smem_u32(sQ);
+    const int l7 = lane & 7;
     for (int it = 0; it < n_tiles; ++it) {
         cp_async_wait<kStages - 2>();
         __syncthreads();
         {
             const int nxt = it + kStages - 1;
-            if (nxt < n_tiles) load_tile(nxt % kStages, kbeg + nxt * kKT);
+            if (nxt < n_tiles) load_tile(nxt % kStages, nxt);
             cp_async_commit();
         }
         const int stage = it % kStages;
@@ -210,7 +244,8 @@ __global__ void __launch_bounds__(128 * NRG) attention_kernel(AttnArgs a) {
         const int k0 = kbeg + it * kKT + kw;  // first key of this warp
         if (k0 >= kend) continue;             // warp has no keys in this tile
 
-        // S = Q K^T  (32 rows x 16 keys)
+        // S = Q K^T  (32 rows x 16 keys); rows and keys of every ldmatrix
+        // start at multiples of 8, so the swizzle XOR is lane & 7
         float s[2][2][4];
 #pragma unroll
         for (int mt = 0; mt < 2; ++mt)
@@ -218,68 +253,77 @@ __global__ void __launch_bounds__(128 * NRG) attention_kernel(AttnArgs a) {
             for (int nt = 0; nt < 2; ++nt)
 #pragma unroll
                 for (int e = 0; e < 4; ++e) s[mt][nt][e] = 0.f;
+        const int j8 = lane >> 3;
+        const uint32_t k_row = k_base + (uint32_t)((kw + (j8 >> 1) * 8 + l7) * D * 2);
+        const uint32_t q_row0 = q_base + (uint32_t)((rg * 32 + (j8 & 1) * 8 + l7) * D * 2);
 #pragma unroll
         for (int kk = 0; kk < D / 16; ++kk) {
             uint32_t kb[4];
-            {
-                const int j = lane >> 3;
-                const int key = kw + (j >> 1) * 8 + (lane & 7);
-                ldmatrix_x4(kb, k_base + swz<D>(key, kk * 2 + (j & 1)));
-            }
+            ldmatrix_x4(kb, k_row + (uint32_t)(((kk * 2 + (j8 & 1)) ^ l7) << 4));
 #pragma unroll
             for (int mt = 0; mt < 2; ++mt) {
                 uint32_t qa[4];
-                const int j = lane >> 3;
-                const int r = rg * 32 + mt * 16 + (j & 1) * 8 + (lane & 7);
-                ldmatrix_x4(qa, q_base + swz<D>(r, kk * 2 + (j >> 1)));
+                ldmatrix_x4(qa, q_row0 + (uint32_t)(mt * 16 * D * 2) +
+                                    (uint32_t)(((kk * 2 + (j8 >> 1)) ^ l7) << 4));
                 mma_bf16_16816(s[mt][0], qa, kb[0], kb[1]);
                 mma_bf16_16816(s[mt][1], qa, kb[2], kb[3]);
             }
         }
-        // mask + online softmax (log2 domain)
+        // mask (boundary tiles only) + online softmax in the log2 domain
+        if (k0 + 16 > mask_from) {
+#pragma unroll
+            for (int i = 0; i < 4; ++i) {
+                const int mt = i >> 1, hi = i & 1;
+#pragma unroll
+                for (int nt = 0; nt < 2; ++nt)
+#pragma unroll
+                    for (int e = 0; e < 2; ++e) {
+                        const int key = k0 + nt * 8 + (lane & 3) * 2 + e;
+                        if (key >= kend || key > rpos[i]) s[mt][nt][hi * 2 + e] = -INFINITY;
+                    }
+            }
+        }
         float alpha[4];
+        bool moved = false;
 #pragma unroll
         for (int i = 0; i < 4; ++i) {
             const int mt = i >> 1, hi = i & 1;
-            float mx = -INFINITY;
-#pragma unroll
-            for (int nt = 0; nt < 2; ++nt)
-#pragma unroll
-                for (int e = 0; e < 2; ++e) {
-                    const int key = k0 + nt * 8 + (lane & 3) * 2 + e;
-                    float v = s[mt][nt][hi * 2 + e] * a.scale_log2;
-                    if (key >= kend || key > rpos[i]) v = -INFINITY;
-                    s[mt][nt][hi * 2 + e] = v;
-                    mx = fmaxf(mx, v);
-                }
+            float mx = fmaxf(fmaxf(s[mt][0][hi * 2], s[mt][0][hi * 2 + 1]),
+                             fmaxf(s[mt][1][hi * 2], s[mt][1][hi * 2 + 1]));
             mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 1));
             mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 2));
-            const float m_new = fmaxf(m_run[i], mx);
-            const float m_use = (m_new == -INFINITY) ? 0.f : m_new;
-            alpha[i] = exp2f(m_run[i] - m_use);
+            mx *= a.scale_log2;
+            alpha[i] = 1.f;
+            if (mx > m_run[i] + kRescaleThreshold || (m_run[i] == -INFINITY && mx > -INFINITY)) {
+                alpha[i] = exp2f(m_run[i] - mx);
+                m_run[i] = mx;
+                moved = true;
+            }
+            const float m_use = (m_run[i] == -INFINITY) ? 0.f : m_run[i];
             float rs = 0.f;
 #pragma unroll
             for (int nt = 0; nt < 2; ++nt)
 #pragma unroll
                 for (int e = 0; e < 2; ++e) {
-                    const float p = exp2f(s[mt][nt][hi * 2 + e] - m_use);
+                    const float p = exp2f(fmaf(s[mt][nt][hi * 2 + e], a.scale_log2, -m_use));
                     s[mt][nt][hi * 2 + e] = p;
                     rs += p;
                 }
             rs += __shfl_xor_sync(0xffffffffu, rs, 1);
             rs += __shfl_xor_sync(0xffffffffu, rs, 2);
             l_run[i] = l_run[i] * alpha[i] + rs;
-            m_run[i] = m_new;
         }
+        if (__any_sync(0xffffffffu, moved)) {
 #pragma unroll
-        for (int mt = 0; mt < 2; ++mt)
+            for (int mt = 0; mt < 2; ++mt)
 #pragma unroll
-            for (int nt = 0; nt < NT; ++nt) {
-                o[mt][nt][0] *= alpha[mt * 2];
-                o[mt][nt][1] *= alpha[mt * 2];
-                o[mt][nt][2] *= alpha[mt * 2 + 1];
-                o[mt][nt][3] *= alpha[mt * 2 + 1];
-            }
+                for (int nt = 0; nt < NT; ++nt) {
+                    o[mt][nt][0] *= alpha[mt * 2];
+                    o[mt][nt][1] *= alpha[mt * 2];
+                    o[mt][nt][2] *= alpha[mt * 2 + 1];
+                    o[mt][nt][3] *= alpha[mt * 2 + 1];
+                }
+        }
         // O += P V  (P: 32 x 16 keys as the A operand, straight from the S fragments)
         uint32_t pa[2][4];
 #pragma unroll
@@ -289,12 +333,11 @@ __global__ void __launch_bounds__(128 * NRG) attention_kernel(AttnArgs a) {
             pa[mt][2] = pack_bf16(s[mt][1][0], s[mt][1][1]);
             pa[mt][3] = pack_bf16(s[mt][1][2], s[mt][1][3]);
         }
+        const uint32_t v_row = v_base + (uint32_t)((kw + (j8 & 1) * 8 + l7) * D * 2);
 #pragma unroll
         for (int dn = 0; dn < NT; dn += 2) {
             uint32_t vb[4];
-            const int j = lane >> 3;
-            const int key = kw + (j & 1) * 8 + (lane & 7);
-            ldmatrix_x4_trans(vb, v_base + swz<D>(key, dn + (j >> 1)));
+            ldmatrix_x4_trans(vb, v_row + (uint32_t)(((dn + (j8 >> 1)) ^ l7) << 4));
 #pragma unroll
             for (int mt = 0; mt < 2; ++mt) {
                 mma_bf16_16816(o[mt][dn], pa[mt], vb[0], vb[1]);
@@ -311,6 +354,14 @@ __global__ void __launch_bounds__(128 * NRG) attention_kernel(AttnArgs a) {
     float* sl = red + THREADS / 32 * 32;          // [warps][32] running sum
     float* obuf = red + 2 * (THREADS / 32) * 32;  // [rg][2][NT*8][32]
     const int wig = warp & 3;  // warp index within its row group
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+        // inactive / padding rows were not masked in prefix tiles: drop them
+        if (rpos[i] < 0) {
+            m_run[i] = -INFINITY;
+            l_run[i] = 0.f;
+        }
+    }
     if ((lane & 3) == 0) {
 #pragma unroll
         for (int i = 0; i < 4; ++i) {
@@ -324,6 +375,7 @@ __global__ void __launch_bounds__(128 * NRG) attention_kernel(AttnArgs a) {
 #pragma unroll
     for (int i = 0; i < 4; ++i) {
         const int r = (i >> 1) * 16 + (i & 1) * 8 + (lane >> 2);
+
         float M = -INFINITY;
 #pragma unroll
         for (int w = 0; w < 4; ++w) M = fmaxf(M, sm[(rg * 4 + w) * 32 + r]);
@@ -453,24 +505,25 @@ __global__ void __launch_bounds__(128 * NRG) attention_kernel(AttnArgs a) {
 }
 
 template <int D, int NRG>
-static size_t attn_smem_bytes() {
-    return (size_t)32 * NRG * D * 2 + (size_t)2 * kStages * kKT * D * 2;
+static size_t attn_smem_bytes(int split) {
+    // Q rows + K/V pipeline stages + the split's key -> row table
+    return (size_t)32 * NRG * D * 2 + (size_t)2 * kStages * kKT * D * 2 + (size_t)split * 4;
 }
 
 template <int D, int NRG>
 static cudaError_t launch_attention_t(const AttnArgs& a, dim3 grid, cudaStream_t st) {
-    const size_t smem = attn_smem_bytes<D, NRG>();
     static unsigned long long configured = 0;  // bit per device: attribute set
     int dev = 0;
     cudaGetDevice(&dev);
     if (dev < 0 || dev >= 64) return cudaErrorInvalidDevice;
     if (!(configured >> dev & 1ull)) {
         cudaError_t e = cudaFuncSetAttribute(attention_kernel<D, NRG>,
-                                             cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+                                             cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                             (int)attn_smem_bytes<D, NRG>(kAttnMaxSplit));
         if (e != cudaSuccess) return e;
         configured |= 1ull << dev;
     }
-    attention_kernel<D, NRG><<<grid, 128 * NRG, smem, st>>>(a);
+    attention_kernel<D, NRG><<<grid, 128 * NRG, attn_smem_bytes<D, NRG>(a.split), st>>>(a);
     return cudaGetLastError();
 }
 

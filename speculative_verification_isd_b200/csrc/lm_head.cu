@@ -89,6 +89,10 @@ lm_head_kernel(const __grid_constant__ CUtensorMap tmap_w, const __grid_constant
     tc_fence_after();
     const uint32_t tmem_base = *tmem_holder;
     const int kblocks = a.H / 64;
+    // Every CTA streams its own rows of W but all of them read the same
+    // hidden tile; starting each CTA's K loop at a different block spreads
+    // those reads over the L2 slices instead of hitting one slice from 148 SMs.
+    const int kb0 = (int)(blockIdx.x % (unsigned)kblocks);
 
     auto give_up = [&]() {
         *abort_flag = 1;
@@ -107,7 +111,8 @@ lm_head_kernel(const __grid_constant__ CUtensorMap tmap_w, const __grid_constant
             const uint32_t tx = (uint32_t)(a.w_rows + a.h_rows0 + a.h_rows1) * 128u;
             bool ok = true;
             for (int tile = blockIdx.x; ok && tile < a.n_tiles; tile += gridDim.x) {
-                for (int kb = 0; kb < kblocks; ++kb, ++it) {
+                for (int j = 0; j < kblocks; ++j, ++it) {
+                    const int kb = (j + kb0) % kblocks;
                     const int s = it % a.stages;
                     const uint32_t round = (uint32_t)(it / a.stages);
                     if (!mbar_wait_bounded(&empty[s], (round & 1) ^ 1, abort_flag, kWaitLimitNs)) {
@@ -147,7 +152,7 @@ lm_head_kernel(const __grid_constant__ CUtensorMap tmap_w, const __grid_constant
                 }
                 tc_fence_after();
                 const uint32_t d0 = tmem_base + (uint32_t)(acc * a.NB * a.BN);
-                for (int kb = 0; kb < kblocks; ++kb, ++it) {
+                for (int j = 0; j < kblocks; ++j, ++it) {
                     const int s = it % a.stages;
                     const uint32_t round = (uint32_t)(it / a.stages);
                     if (!mbar_wait_bounded(&full[s], round & 1, abort_flag, kWaitLimitNs)) {
@@ -163,7 +168,7 @@ lm_head_kernel(const __grid_constant__ CUtensorMap tmap_w, const __grid_constant
                         const uint64_t adesc = smem_desc_sw128(sa + k * 32);
                         for (int nb = 0; nb < a.NB; ++nb) {
                             const uint64_t bdesc = smem_desc_sw128(sb + nb * a.BN * 128 + k * 32);
-                            mma_f16_ss(d0 + nb * a.BN, adesc, bdesc, idesc, (kb | k) != 0);
+                            mma_f16_ss(d0 + nb * a.BN, adesc, bdesc, idesc, (j | k) != 0);
                         }
                     }
                     mma_commit(&empty[s]);

@@ -11,6 +11,7 @@ namespace isd {
 
 constexpr int kAttnKeyTile = 64;      // keys per pipeline stage
 constexpr int kAttnRowsPerGroup = 32; // query rows handled by one 4-warp group
+constexpr int kAttnMaxSplit = 2048;   // keys per split at most (bounds the key table)
 constexpr int kStatsThreads = 256;
 constexpr int kAcceptThreads = 256;
 constexpr int kAcceptChunk = 4096;    // vocabulary entries per accept CTA
@@ -58,7 +59,7 @@ inline bool make_plan(const isd_dims* d, Plan* p) {
     long long est = (long long)d->B * d->Hkv * p->attn_rgb * (max_ctx / 2 + 1);
     long long split = est / (kNumSMs * 2 * 3);
     if (split < 256) split = 256;
-    if (split > 8192) split = 8192;
+    if (split > kAttnMaxSplit) split = kAttnMaxSplit;
     split = (split + kAttnKeyTile - 1) / kAttnKeyTile * kAttnKeyTile;
     p->attn_split = (int)split;
     p->attn_max_splits = (int)((max_ctx + split - 1) / split);
