@@ -34,7 +34,8 @@ namespace isd {
 
 struct LmArgs {
     int V, Mh, H;
-    int BN, NB, n_acc, stages, n_tiles;
+    int BN, n_acc, n_tiles;
+    int w_stages, h_stages;        // depth of the W ring and of the hidden ring (w > h)
     int w_rows, h_rows0, h_rows1;  // TMA box heights (never taller than the tensor)
     uint32_t tmem_cols;
     float* logits;
@@ -42,8 +43,27 @@ struct LmArgs {
 };
 
 constexpr uint64_t kWaitLimitNs = 2000000000ull;
-constexpr int kLmThreads = 192;
+constexpr int kLmThreads = 224;  // W producer, MMA, 4 epilogue warps, hidden producer
+constexpr int kWStageBytes = 128 * 128;  // 128 vocabulary rows x 64 bf16
 
+// Fast path of a bounded wait: one try_wait, then the bounded loop.
+ISD_DEVINL bool lm_wait(uint64_t* bar, uint32_t parity, volatile int* abort) {
+    return sm100::mbar_try_wait(bar, parity) ||
+           sm100::mbar_wait_bounded(bar, parity, abort, kWaitLimitNs);
+}
+
+// Synchronisation (per k-block `it`, W slot ws = it % w_stages, hidden slot
+// hs = it % h_stages):
+//   full[ws]  : 2 arrivals (both producers, with their TMA byte counts); the
+//               MMA thread waits on it alone;
+//   empty[ws] : one tcgen05.commit per k-block.  The W producer reuses slot ws
+//               after it; the hidden producer reuses slot hs after the commit
+//               of k-block it - h_stages, which it reads from the same W-ring
+//               barrier (w_stages > h_stages keeps the phases unambiguous).
+// The MMA thread's loop is kept to one wait, the MMAs and one commit: the
+// tensor pipe queues only a couple of MMAs, so any extra work there would
+// become a bubble.
+template <int NB>
 __global__ void __launch_bounds__(kLmThreads, 1)
 lm_head_kernel(const __grid_constant__ CUtensorMap tmap_w, const __grid_constant__ CUtensorMap tmap_h0,
                const __grid_constant__ CUtensorMap tmap_h1, LmArgs a) {
@@ -51,11 +71,12 @@ lm_head_kernel(const __grid_constant__ CUtensorMap tmap_w, const __grid_constant
     extern __shared__ unsigned char smem_raw[];
     unsigned char* smem = reinterpret_cast<unsigned char*>(
         (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-    const int b_bytes = a.NB * a.BN * 128;
-    const int stage_bytes = 16384 + b_bytes;
-    uint64_t* full = reinterpret_cast<uint64_t*>(smem + (size_t)a.stages * stage_bytes);
-    uint64_t* empty = full + a.stages;
-    uint64_t* tfull = empty + a.stages;
+    const int h_bytes = NB * a.BN * 128;  // one hidden stage (K = 64)
+    unsigned char* wring = smem;
+    unsigned char* hring = smem + (size_t)a.w_stages * kWStageBytes;
+    uint64_t* full = reinterpret_cast<uint64_t*>(hring + (size_t)a.h_stages * h_bytes);
+    uint64_t* empty = full + a.w_stages;
+    uint64_t* tfull = empty + a.w_stages;
     uint64_t* tempty = tfull + 2;
     uint64_t* drain = tempty + 2;
     uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(drain + 1);
@@ -64,8 +85,8 @@ lm_head_kernel(const __grid_constant__ CUtensorMap tmap_w, const __grid_constant
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     if (threadIdx.x == 0) {
-        for (int s = 0; s < a.stages; ++s) {
-            mbar_init(&full[s], 1);
+        for (int s = 0; s < a.w_stages; ++s) {
+            mbar_init(&full[s], 2);
             mbar_init(&empty[s], 1);
         }
         for (int i = 0; i < 2; ++i) {
@@ -78,7 +99,7 @@ lm_head_kernel(const __grid_constant__ CUtensorMap tmap_w, const __grid_constant
         fence_mbar_init();
         prefetch_tmap(&tmap_w);
         prefetch_tmap(&tmap_h0);
-        if (a.NB > 1) prefetch_tmap(&tmap_h1);
+        if (NB > 1) prefetch_tmap(&tmap_h1);
     }
     if (warp == 1) {
         tmem_alloc(tmem_holder, a.tmem_cols);
@@ -89,89 +110,98 @@ lm_head_kernel(const __grid_constant__ CUtensorMap tmap_w, const __grid_constant
     tc_fence_after();
     const uint32_t tmem_base = *tmem_holder;
     const int kblocks = a.H / 64;
-    // Every CTA streams its own rows of W but all of them read the same
-    // hidden tile; starting each CTA's K loop at a different block spreads
-    // those reads over the L2 slices instead of hitting one slice from 148 SMs.
+    // Each CTA starts its K loop at a different block so that the 148 CTAs
+    // read different hidden slices at any moment.
     const int kb0 = (int)(blockIdx.x % (unsigned)kblocks);
+    int n_my_tiles = 0;
+    for (int t = blockIdx.x; t < a.n_tiles; t += gridDim.x) ++n_my_tiles;
+    const int total_kb = n_my_tiles * kblocks;
 
     auto give_up = [&]() {
         *abort_flag = 1;
         raise_flag(a.err_flag, ISD_FLAG_WAIT_TIMEOUT);
     };
 
-    if (warp == 0) {
+    if (warp == 0 || warp == 6) {
         if (lane == 0) {
-            // ---------------- TMA producer
-            const uint64_t pol_w = policy_evict_first();
-            const uint64_t pol_h = policy_evict_last();
-            uint32_t armed = 0, parity_bits = 0;
-            int it = 0;
-            // rows of a box beyond the tensor are not delivered (and not used:
-            // their accumulator columns / vocabulary rows are never stored)
-            const uint32_t tx = (uint32_t)(a.w_rows + a.h_rows0 + a.h_rows1) * 128u;
-            bool ok = true;
-            for (int tile = blockIdx.x; ok && tile < a.n_tiles; tile += gridDim.x) {
-                for (int j = 0; j < kblocks; ++j, ++it) {
-                    const int kb = (j + kb0) % kblocks;
-                    const int s = it % a.stages;
-                    const uint32_t round = (uint32_t)(it / a.stages);
-                    if (!mbar_wait_bounded(&empty[s], (round & 1) ^ 1, abort_flag, kWaitLimitNs)) {
-                        give_up();
-                        ok = false;
-                        break;
-                    }
-                    unsigned char* sa = smem + (size_t)s * stage_bytes;
-                    unsigned char* sb = sa + 16384;
-                    mbar_arrive_expect_tx(&full[s], tx);
-                    tma_load_2d(sa, &tmap_w, &full[s], kb * 64, tile * 128, pol_w);
-                    tma_load_2d(sb, &tmap_h0, &full[s], kb * 64, 0, pol_h);
-                    if (a.NB > 1)
-                        tma_load_2d(sb + a.BN * 128, &tmap_h1, &full[s], kb * 64, a.BN, pol_h);
-                    armed |= 1u << s;
-                    parity_bits = (parity_bits & ~(1u << s)) | ((round & 1) << s);
+            // ---------------- TMA producers: warp 0 streams W from HBM through
+            // the deep ring; warp 6 feeds the L2-resident hidden tiles
+            const bool is_w = (warp == 0);
+            const uint64_t pol = is_w ? policy_evict_first() : policy_evict_last();
+            const uint32_t tx = is_w ? (uint32_t)a.w_rows * 128u
+                                     : (uint32_t)(a.h_rows0 + a.h_rows1) * 128u;
+            int ws = 0, hs = 0, kb = kb0, tile = blockIdx.x, jt = 0;
+            uint32_t wph = 0;
+            // hidden producer: the k-block that last used its slot, as a W slot/phase
+            int pws = 0;
+            uint32_t pwph = 0;
+            for (int it = 0; it < total_kb; ++it) {
+                bool ok;
+                if (is_w) {
+                    ok = lm_wait(&empty[ws], wph ^ 1, abort_flag);
+                } else if (it >= a.h_stages) {
+                    ok = lm_wait(&empty[pws], pwph, abort_flag);
+                    if (++pws == a.w_stages) { pws = 0; pwph ^= 1; }
+                } else {
+                    ok = true;
                 }
+                if (!ok) {
+                    give_up();
+                    break;
+                }
+                mbar_arrive_expect_tx(&full[ws], tx);
+                if (is_w) {
+                    tma_load_2d(wring + (size_t)ws * kWStageBytes, &tmap_w, &full[ws], kb * 64,
+                                tile * 128, pol);
+                } else {
+                    unsigned char* sb = hring + (size_t)hs * h_bytes;
+                    tma_load_2d(sb, &tmap_h0, &full[ws], kb * 64, 0, pol);
+                    if (NB > 1) tma_load_2d(sb + a.BN * 128, &tmap_h1, &full[ws], kb * 64, a.BN, pol);
+                }
+                if (++ws == a.w_stages) { ws = 0; wph ^= 1; }
+                if (++hs == a.h_stages) hs = 0;
+                if (++kb == kblocks) kb = 0;
+                if (++jt == kblocks) { jt = 0; tile += gridDim.x; }
             }
-            // no TMA write may land after this CTA leaves: wait for every
-            // stage's last armed phase
-            for (int s = 0; s < a.stages; ++s)
-                if (armed >> s & 1)
-                    mbar_wait_bounded(&full[s], parity_bits >> s & 1, &never, kWaitLimitNs);
         }
     } else if (warp == 1) {
         if (lane == 0) {
             // ---------------- MMA issuer
             const uint32_t idesc = idesc_bf16_f32(128, a.BN);
-            int it = 0, lt = 0;
+            const uint64_t adesc0 = smem_desc_sw128(smem_u32(wring));
+            const uint64_t bdesc0 = smem_desc_sw128(smem_u32(hring));
+            const uint64_t astep = kWStageBytes >> 4, bstep = (uint64_t)(h_bytes >> 4);
+            int ws = 0, hs = 0;
+            uint32_t wph = 0;
             bool ok = true;
-            for (int tile = blockIdx.x; ok && tile < a.n_tiles; tile += gridDim.x, ++lt) {
+            for (int lt = 0; ok && lt < n_my_tiles; ++lt) {
                 const int acc = lt % a.n_acc;
                 const uint32_t use = (uint32_t)(lt / a.n_acc);
-                if (!mbar_wait_bounded(&tempty[acc], (use & 1) ^ 1, abort_flag, kWaitLimitNs)) {
+                if (!lm_wait(&tempty[acc], (use & 1) ^ 1, abort_flag)) {
                     give_up();
                     break;
                 }
                 tc_fence_after();
-                const uint32_t d0 = tmem_base + (uint32_t)(acc * a.NB * a.BN);
-                for (int j = 0; j < kblocks; ++j, ++it) {
-                    const int s = it % a.stages;
-                    const uint32_t round = (uint32_t)(it / a.stages);
-                    if (!mbar_wait_bounded(&full[s], round & 1, abort_flag, kWaitLimitNs)) {
+                const uint32_t d0 = tmem_base + (uint32_t)(acc * NB * a.BN);
+                for (int j = 0; j < kblocks; ++j) {
+                    if (!lm_wait(&full[ws], wph, abort_flag)) {
                         give_up();
                         ok = false;
                         break;
                     }
                     tc_fence_after();
-                    const uint32_t sa = smem_u32(smem + (size_t)s * stage_bytes);
-                    const uint32_t sb = sa + 16384;
+                    const uint64_t ad = adesc0 + (uint64_t)ws * astep;
+                    const uint64_t bd = bdesc0 + (uint64_t)hs * bstep;
 #pragma unroll
                     for (int k = 0; k < 4; ++k) {
-                        const uint64_t adesc = smem_desc_sw128(sa + k * 32);
-                        for (int nb = 0; nb < a.NB; ++nb) {
-                            const uint64_t bdesc = smem_desc_sw128(sb + nb * a.BN * 128 + k * 32);
-                            mma_f16_ss(d0 + nb * a.BN, adesc, bdesc, idesc, (j | k) != 0);
-                        }
+#pragma unroll
+                        for (int nb = 0; nb < NB; ++nb)
+                            mma_f16_ss(d0 + nb * a.BN, ad + 2 * k,
+                                       bd + (uint64_t)(nb * a.BN * 8) + 2 * k, idesc, (j | k) != 0);
                     }
-                    mma_commit(&empty[s]);
+                    mma_commit(&empty[ws]);
+                    if (++ws == a.w_stages) { ws = 0; wph ^= 1; }
+                    if (++hs == a.h_stages) hs = 0;
                 }
                 if (ok) mma_commit(&tfull[acc]);
             }
@@ -188,7 +218,7 @@ lm_head_kernel(const __grid_constant__ CUtensorMap tmap_w, const __grid_constant
             const uint32_t use = (uint32_t)(lt / a.n_acc);
             int ok = 1;
             if (lane == 0) {
-                ok = mbar_wait_bounded(&tfull[acc], use & 1, abort_flag, kWaitLimitNs);
+                ok = lm_wait(&tfull[acc], use & 1, abort_flag);
                 if (!ok) give_up();
             }
             ok = __shfl_sync(0xffffffffu, ok, 0);
@@ -197,8 +227,9 @@ lm_head_kernel(const __grid_constant__ CUtensorMap tmap_w, const __grid_constant
             const int v = tile * 128 + quarter * 32 + lane;
             const bool v_ok = v < a.V;
             const uint32_t taddr =
-                tmem_base + ((uint32_t)(quarter * 32) << 16) + (uint32_t)(acc * a.NB * a.BN);
-            for (int nb = 0; nb < a.NB; ++nb) {
+                tmem_base + ((uint32_t)(quarter * 32) << 16) + (uint32_t)(acc * NB * a.BN);
+#pragma unroll
+            for (int nb = 0; nb < NB; ++nb) {
                 for (int j0 = 0; j0 < a.BN; j0 += 32) {
                     uint32_t r[32];
                     // BN is a multiple of 16: the tail is one 16-column load,
@@ -270,7 +301,7 @@ static bool encode_bf16_2d(CUtensorMap* m, const void* ptr, uint64_t rows, uint6
 }
 
 struct LmShape {
-    int BN, NB, n_acc, stages;
+    int BN, NB, n_acc, w_stages, h_stages;
     uint32_t tmem_cols;
     size_t smem;
 };
@@ -290,12 +321,20 @@ bool lm_head_shape(int Mh, int smem_limit, LmShape* s) {
     uint32_t alloc = 32;
     while ((int)alloc < need) alloc <<= 1;
     s->tmem_cols = alloc;
-    const int stage_bytes = 16384 + cols * 128;
-    const int budget = smem_limit - 1024 - 256;  // alignment slack + barriers
-    s->stages = budget / stage_bytes;
-    if (s->stages > 8) s->stages = 8;
-    if (s->stages < 2) return false;
-    s->smem = (size_t)s->stages * stage_bytes + 1024 + 256;
+    const int h_bytes = cols * 128;
+    const int budget = smem_limit - 1024 - 512;  // alignment slack + barriers
+    // hidden tiles are L2 hits: 3 stages; the rest of the budget deepens the
+    // W ring (HBM latency under load is several microseconds)
+    s->h_stages = 3;
+    s->w_stages = (budget - s->h_stages * h_bytes) / kWStageBytes;
+    if (s->w_stages > 16) s->w_stages = 16;
+    if (s->w_stages < 4) {
+        s->h_stages = 2;
+        s->w_stages = (budget - s->h_stages * h_bytes) / kWStageBytes;
+        if (s->w_stages > 16) s->w_stages = 16;
+    }
+    if (s->w_stages <= s->h_stages) return false;
+    s->smem = (size_t)s->w_stages * kWStageBytes + (size_t)s->h_stages * h_bytes + 1024 + 512;
     return true;
 }
 
@@ -318,13 +357,18 @@ cudaError_t launch_lm_head(const uint16_t* hidden, const uint16_t* W, int Mh, in
     if (!smem_limit_dev[dev]) {
         int optin = 0;
         cudaDeviceGetAttribute(&optin, cudaDevAttrMaxSharedMemoryPerBlockOptin, dev);
-        cudaFuncAttributes fa;
-        if (cudaFuncGetAttributes(&fa, lm_head_kernel) != cudaSuccess) {
+        cudaFuncAttributes fa1, fa2;
+        if (cudaFuncGetAttributes(&fa1, lm_head_kernel<1>) != cudaSuccess ||
+            cudaFuncGetAttributes(&fa2, lm_head_kernel<2>) != cudaSuccess) {
             set_error_detail("lm_head: kernel attributes unavailable");
             return cudaErrorInvalidValue;
         }
-        const int limit = optin - (int)fa.sharedSizeBytes;
-        if (cudaFuncSetAttribute(lm_head_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+        const size_t stat = fa1.sharedSizeBytes > fa2.sharedSizeBytes ? fa1.sharedSizeBytes
+                                                                       : fa2.sharedSizeBytes;
+        const int limit = optin - (int)stat;
+        if (cudaFuncSetAttribute(lm_head_kernel<1>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 limit) != cudaSuccess ||
+            cudaFuncSetAttribute(lm_head_kernel<2>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                  limit) != cudaSuccess) {
             set_error_detail("lm_head: shared-memory attribute rejected");
             return cudaErrorInvalidValue;
@@ -363,16 +407,19 @@ cudaError_t launch_lm_head(const uint16_t* hidden, const uint16_t* W, int Mh, in
     a.Mh = Mh;
     a.H = H;
     a.BN = sh.BN;
-    a.NB = sh.NB;
     a.n_acc = sh.n_acc;
-    a.stages = sh.stages;
+    a.w_stages = sh.w_stages;
+    a.h_stages = sh.h_stages;
     a.n_tiles = (V + 127) / 128;
     a.tmem_cols = sh.tmem_cols;
     a.logits = logits;
     a.err_flag = err_flag;
     int grid = num_sms_of_current_device();
     if (grid > a.n_tiles) grid = a.n_tiles;
-    lm_head_kernel<<<grid, kLmThreads, sh.smem, st>>>(tw, th0, th1, a);
+    if (sh.NB == 1)
+        lm_head_kernel<1><<<grid, kLmThreads, sh.smem, st>>>(tw, th0, th1, a);
+    else
+        lm_head_kernel<2><<<grid, kLmThreads, sh.smem, st>>>(tw, th0, th1, a);
     cudaError_t e = cudaGetLastError();
     if (e != cudaSuccess) set_error_detail("lm_head: launch failed");
     return e;
