@@ -187,6 +187,36 @@ isd_status isd_step(const isd_dims* d, const uint16_t* q, const uint16_t* k_new,
                     int32_t* next_clean_tok, int32_t* next_kv_len, float* ratio, void* ws,
                     size_t ws_bytes, int32_t* err_flag, void* stream);
 
+/*
+ * isd_attention_noalloc -- isd_attention for callers that cannot provide a
+ * workspace.  The paper has no counterpart: this is a deployment convenience.
+ *
+ * Some callers cannot allocate device memory for us: a serving engine that
+ * gave all free device memory to its KV-cache pool at start-up, or code that
+ * must not call the CUDA allocator (cudaMalloc/cudaFree can synchronise the
+ * device).  This call takes the same inputs and outputs as isd_attention, but
+ * its scratch (the split-KV partial results and counters) lives in a fixed
+ * array inside the library of ISD_NOALLOC_SCRATCH_BYTES bytes, which every
+ * GPU that loads the library keeps until the process exits.  It allocates
+ * nothing and calls no allocating routine.
+ *  - Dims whose scratch need exceeds ISD_NOALLOC_SCRATCH_BYTES are rejected
+ *    with ISD_ERR_WORKSPACE (isd_last_error() states both sizes).  The need
+ *    grows with B * Hkv * (longest context); B=32, 8 KV heads and 8 K
+ *    contexts fit.
+ *  - The first call on each device (made with that device current) looks up
+ *    the array's device address; make that first call before any stream
+ *    capture.
+ *  - All calls on a device share the array: calls that overlap on the GPU
+ *    (e.g. on two unordered streams) race on it.  Each call clears the
+ *    counters it needs on its own stream.
+ */
+#define ISD_NOALLOC_SCRATCH_BYTES (32u * 1024u * 1024u)
+isd_status isd_attention_noalloc(const isd_dims* d, const uint16_t* q, const uint16_t* k_new,
+                                 const uint16_t* v_new, uint16_t* k_pool, uint16_t* v_pool,
+                                 const int32_t* page_table, const int32_t* kv_len,
+                                 const int32_t* n_clean, uint16_t* out, int32_t* err_flag,
+                                 void* stream);
+
 #ifdef __cplusplus
 }
 #endif

@@ -1,0 +1,108 @@
+// isd_attention_noalloc: the attention step (KV append + paged GQA attention)
+// for callers that cannot give the library a workspace.
+//
+// Who needs it: a serving engine that hands all free device memory to its KV
+// cache pool when it starts (so nothing is left to allocate per step), and
+// code that must not call the CUDA allocator at all, for instance because
+// cudaMalloc/cudaFree may synchronise the device in the middle of a pipelined
+// decode loop.  Such callers still pass every input and output buffer; only
+// the scratch that the split-KV attention needs (per-split partial results
+// and the last-CTA counters) comes from a fixed array inside the library.
+//
+// That array is a file-scope __device__ array of kNoAllocScratchBytes bytes.
+// Every GPU that loads the library keeps it for the life of the process.  All
+// calls on a device share it: two calls that overlap on the GPU (different
+// streams, no ordering between them) race on it.  Its counters are cleared on
+// the caller's stream at every call; the partial results need no clearing.
+//
+// Host code cannot use the array's name as a device address, so the first
+// call on each device (with that device current) looks the address up with
+// cudaGetSymbolAddress and keeps it; make that first call before any stream
+// capture.
+#include <cuda_runtime.h>
+#include <stdint.h>
+#include <stdio.h>
+
+#include "common.cuh"
+#include "plan.h"
+
+#define ISD_NOALLOC_MAX_DEVICES 64
+
+namespace {
+
+constexpr size_t kNoAllocScratchBytes = (size_t)ISD_NOALLOC_SCRATCH_BYTES;
+
+static __device__ __align__(256) unsigned char g_attn_scratch[kNoAllocScratchBytes];
+
+void* g_scratch_ptr[ISD_NOALLOC_MAX_DEVICES];  // per device, filled on first use
+
+}  // namespace
+
+namespace isd {
+cudaError_t launch_attention(const Plan& p, const isd_dims* d, const uint16_t* q,
+                             const uint16_t* k_new, const uint16_t* v_new, uint16_t* k_pool,
+                             uint16_t* v_pool, const int32_t* page_table, const int32_t* kv_len,
+                             const int32_t* n_clean, uint16_t* out, void* ws, int32_t* err_flag,
+                             cudaStream_t st);
+void set_last_error(const char* msg);
+}  // namespace isd
+
+extern "C" isd_status isd_attention_noalloc(const isd_dims* d, const uint16_t* q,
+                                            const uint16_t* k_new, const uint16_t* v_new,
+                                            uint16_t* k_pool, uint16_t* v_pool,
+                                            const int32_t* page_table, const int32_t* kv_len,
+                                            const int32_t* n_clean, uint16_t* out,
+                                            int32_t* err_flag, void* stream) {
+    isd::Plan p;
+    if (!isd::make_plan(d, &p)) {
+        isd::set_last_error("isd_attention_noalloc: invalid dims");
+        return ISD_ERR_INVALID_ARG;
+    }
+    if (!q || !k_new || !v_new || !k_pool || !v_pool || !page_table || !kv_len || !n_clean ||
+        !out) {
+        isd::set_last_error("isd_attention_noalloc: null pointer");
+        return ISD_ERR_INVALID_ARG;
+    }
+    if ((d->D != 64 && d->D != 128) || p.rows > 128) {
+        isd::set_last_error("isd_attention_noalloc: unsupported head dim or block rows");
+        return ISD_ERR_UNSUPPORTED_SHAPE;
+    }
+    // The attention uses the workspace from offset 0 up to the end of its
+    // counters (off_hidden): that much must fit in the built-in array.
+    const size_t need = p.off_hidden;
+    if (need > kNoAllocScratchBytes) {
+        char msg[160];
+        snprintf(msg, sizeof(msg),
+                 "isd_attention_noalloc: needs %zu bytes of scratch, more than the built-in %zu",
+                 need, kNoAllocScratchBytes);
+        isd::set_last_error(msg);
+        return ISD_ERR_WORKSPACE;
+    }
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= ISD_NOALLOC_MAX_DEVICES) {
+        isd::set_last_error("isd_attention_noalloc: no usable current device");
+        return ISD_ERR_CUDA;
+    }
+    if (!g_scratch_ptr[dev]) {
+        void* ptr = nullptr;
+        const cudaError_t e = cudaGetSymbolAddress(&ptr, g_attn_scratch);
+        if (e != cudaSuccess || !ptr) {
+            isd::set_last_error("isd_attention_noalloc: device address of the scratch array");
+            return ISD_ERR_CUDA;
+        }
+        g_scratch_ptr[dev] = ptr;
+    }
+    char* ws = static_cast<char*>(g_scratch_ptr[dev]);
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    if (cudaMemsetAsync(ws + p.off_attn_ticket, 0, (size_t)d->B * d->Hkv * p.attn_rgb * 4, st) !=
+        cudaSuccess) {
+        isd::set_last_error("isd_attention_noalloc: clearing the counters");
+        return ISD_ERR_CUDA;
+    }
+    if (isd::launch_attention(p, d, q, k_new, v_new, k_pool, v_pool, page_table, kv_len, n_clean,
+                              out, ws, err_flag, st) != cudaSuccess) {
+        isd::set_last_error("isd_attention_noalloc: launch failed");
+        return ISD_ERR_CUDA;
+    }
+    return ISD_OK;
+}

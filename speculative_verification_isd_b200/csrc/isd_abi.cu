@@ -17,6 +17,8 @@ thread_local char g_detail[160] = "";
 namespace isd {
 // Host-side context for the next CUDA failure report (this thread).
 void set_error_detail(const char* msg) { snprintf(g_detail, sizeof(g_detail), "%s", msg); }
+// The message isd_last_error() returns (this thread).
+void set_last_error(const char* msg) { snprintf(g_last_error, sizeof(g_last_error), "%s", msg); }
 cudaError_t launch_attention(const Plan& p, const isd_dims* d, const uint16_t* q,
                              const uint16_t* k_new, const uint16_t* v_new, uint16_t* k_pool,
                              uint16_t* v_pool, const int32_t* page_table, const int32_t* kv_len,

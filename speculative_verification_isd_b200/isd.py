@@ -36,7 +36,8 @@ PROPOSE_ARGMAX = 0
 PROPOSE_SAMPLE = 1
 
 EXPORTED = ("isd_workspace_bytes", "isd_status_string", "isd_last_error", "isd_attention",
-            "isd_lm_head", "isd_row_stats", "isd_accept", "isd_step")
+            "isd_lm_head", "isd_row_stats", "isd_accept", "isd_step", "isd_attention_noalloc")
+NOALLOC_SCRATCH_BYTES = 32 * 1024 * 1024  # ISD_NOALLOC_SCRATCH_BYTES in include/isd.h
 
 
 class Dims(ctypes.Structure):
@@ -82,6 +83,8 @@ _lib.isd_accept.argtypes = [_dims_p] + [_vp] * 15 + [_sz, _vp, _vp]
 _lib.isd_accept.restype = _i32
 _lib.isd_step.argtypes = [_dims_p] + [_vp] * 25 + [_sz, _vp, _vp]
 _lib.isd_step.restype = _i32
+_lib.isd_attention_noalloc.argtypes = [_dims_p] + [_vp] * 9 + [_vp, _vp]
+_lib.isd_attention_noalloc.restype = _i32
 
 
 class IsdError(RuntimeError):
@@ -156,6 +159,23 @@ def attention(d: Dims, q, k_new, v_new, k_pool, v_pool, page_table, kv_len, n_cl
         _ptr(kv_len, torch.int32, d.B, "kv_len"), _ptr(n_clean, torch.int32, d.B, "n_clean"),
         _ptr(out, _BF16, d.M * d.H, "out"), _ptr(ws, torch.uint8, None, "ws"), ws.numel(),
         _ptr(err_flag, torch.int32, 1, "err_flag"), _stream(stream)))
+
+
+def attention_noalloc(d: Dims, q, k_new, v_new, k_pool, v_pool, page_table, kv_len, n_clean, out,
+                      err_flag=None, stream=None):
+    """isd_attention without a workspace argument, for callers that cannot
+    allocate device memory (scratch comes from a fixed array in the library)."""
+    kvrow = d.page_size * d.Hkv * d.D
+    _check(_lib.isd_attention_noalloc(
+        ctypes.byref(d), _ptr(q, _BF16, d.M * d.Hq * d.D, "q"),
+        _ptr(k_new, _BF16, d.M * d.Hkv * d.D, "k_new"),
+        _ptr(v_new, _BF16, d.M * d.Hkv * d.D, "v_new"),
+        _ptr(k_pool, _BF16, d.num_pages * kvrow, "k_pool"),
+        _ptr(v_pool, _BF16, d.num_pages * kvrow, "v_pool"),
+        _ptr(page_table, torch.int32, d.B * d.max_pages_per_req, "page_table"),
+        _ptr(kv_len, torch.int32, d.B, "kv_len"), _ptr(n_clean, torch.int32, d.B, "n_clean"),
+        _ptr(out, _BF16, d.M * d.H, "out"), _ptr(err_flag, torch.int32, 1, "err_flag"),
+        _stream(stream)))
 
 
 def lm_head(d: Dims, hidden, W, logits, row_stats, ws, lora_A=None, lora_B=None, err_flag=None,
