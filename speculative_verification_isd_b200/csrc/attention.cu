@@ -6,14 +6,18 @@
 // serving structure the same page reuses (section "推理：复用 AR 推理栈").
 //
 // Design (B200, memory-bound: ~28 flop per KV byte):
-//  * one CTA per (request, KV head, split of the key range, row-group block);
-//    the grp*Q query rows that share a KV head (28 for Qwen3-8B at N=4) are
+//  * one CTA per (request, KV head, split of the key range, row block); the
+//    grp*Q query rows that share a KV head (28 for Qwen3-8B at N=4) are
 //    processed together, so every KV byte is read from HBM once;
 //  * keys stream through a 3-stage cp.async pipeline in 64-key tiles gathered
-//    page by page (XOR-swizzled 16-byte chunks, conflict-free ldmatrix);
-//  * each warp owns 16 keys of a tile and all 32 rows of its row group:
-//    S = Q K^T and O += P V on mma.sync m16n8k16 (bf16 in, fp32 accumulate),
-//    online softmax in the log2 domain;
+//    page by page; a per-split key -> cache-row table (one page lookup per
+//    key) keeps the per-tile address work to a load and a multiply-add;
+//  * warps are arranged as (16-row group) x (16 keys of the tile): every warp
+//    owns 16 query rows, so its output accumulator is 64 registers and two
+//    CTAs of 8 warps fit on an SM (the kernel is latency-bound: warps hide
+//    each other's mma.sync dependency chains);
+//  * S = Q K^T and O += P V on mma.sync m16n8k16 (bf16 in, fp32 accumulate),
+//    online softmax in the log2 domain with a lazily moved reference maximum;
 //  * warps merge in a fixed order; splits of one (request, head) are merged
 //    by the CTA that draws the last ticket (no spinning, deterministic);
 //  * block keys are read from k_new/v_new directly, and the CTA of the last
@@ -58,12 +62,12 @@ ISD_DEVINL int slot_pos(int s, int kv, int c, int N) {
     return kv + c + (s - N);
 }
 
-template <int D, int NRG>
-__global__ void __launch_bounds__(128 * NRG) attention_kernel(AttnArgs a) {
-    constexpr int THREADS = 128 * NRG;
-    constexpr int ROWS = 32 * NRG;
-    constexpr int CH = D / 8;  // 16-byte chunks per row
-    constexpr int NT = D / 8;  // n8 tiles of the output
+template <int D, int RG>
+__global__ void __launch_bounds__(128 * RG, (RG <= 2 ? 2 : 1)) attention_kernel(AttnArgs a) {
+    constexpr int THREADS = 128 * RG;
+    constexpr int ROWS = 16 * RG;  // query rows of this CTA
+    constexpr int CH = D / 8;      // 16-byte chunks per row
+    constexpr int NT = D / 8;      // n8 tiles of the output
     extern __shared__ __align__(128) unsigned char smem[];
     unsigned char* sQ = smem;
     unsigned char* sK = smem + ROWS * D * 2;
@@ -74,7 +78,7 @@ __global__ void __launch_bounds__(128 * NRG) attention_kernel(AttnArgs a) {
     const int rgb = blockIdx.y % a.n_rgb;
     const int b = blockIdx.z;
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-    const int rg = warp >> 2;          // row group of this warp
+    const int rg = warp >> 2;          // 16-row group of this warp
     const int kw = (warp & 3) * 16;    // this warp's keys within a tile
 
     const int kv = a.kv_len[b];
@@ -115,7 +119,7 @@ __global__ void __launch_bounds__(128 * NRG) attention_kernel(AttnArgs a) {
         }
     }
 
-    // ---- query rows of this CTA -> smem (zero rows for padding / inactive)
+    // ---- query rows of this CTA -> smem (zero rows for padding)
     const int row0 = rgb * ROWS;
     for (int i = tid; i < ROWS * CH; i += THREADS) {
         const int r = i / CH, cc = i % CH;
@@ -129,12 +133,11 @@ __global__ void __launch_bounds__(128 * NRG) attention_kernel(AttnArgs a) {
         *reinterpret_cast<uint4*>(sQ + swz<D>(r, cc)) = v;
     }
 
-    // positions of the 4 rows this thread holds in the S/O fragments
-    int rpos[4];
+    // positions of the 2 rows this thread holds in the S/O fragments
+    int rpos[2];
 #pragma unroll
-    for (int i = 0; i < 4; ++i) {
-        const int r = rg * 32 + (i >> 1) * 16 + (i & 1) * 8 + (lane >> 2);
-        const int rr = row0 + r;
+    for (int i = 0; i < 2; ++i) {
+        const int rr = row0 + rg * 16 + i * 8 + (lane >> 2);
         rpos[i] = (rr < a.rows && total > 0) ? slot_pos(rr % a.Q, kv, c, a.N) : -1;
     }
 
@@ -168,7 +171,7 @@ __global__ void __launch_bounds__(128 * NRG) attention_kernel(AttnArgs a) {
     //      kr0 + j*KPP, so its swizzled smem offset is a per-thread constant
     constexpr int KPP = THREADS / CH;  // keys per pass (a multiple of 8)
     constexpr int PASSES = kKT / KPP;
-    static_assert(KPP % 8 == 0, "constant swizzle needs 8-key passes");
+    static_assert(KPP % 8 == 0 && kKT % KPP == 0, "constant swizzle needs 8-key passes");
     const int cc = tid % CH, kr0 = tid / CH;
     const size_t pool_col = (size_t)g * D + cc * 8;
     const __nv_bfloat16* knew_b = a.k_new + ((size_t)b * a.Q * a.Hkv + g) * D + cc * 8;
@@ -199,20 +202,13 @@ __global__ void __launch_bounds__(128 * NRG) attention_kernel(AttnArgs a) {
         }
     };
 
-    float o[2][NT][4];
+    float o[NT][4];
 #pragma unroll
-    for (int mt = 0; mt < 2; ++mt)
+    for (int nt = 0; nt < NT; ++nt)
 #pragma unroll
-        for (int nt = 0; nt < NT; ++nt)
-#pragma unroll
-            for (int e = 0; e < 4; ++e) o[mt][nt][e] = 0.f;
+        for (int e = 0; e < 4; ++e) o[nt][e] = 0.f;
     // running reference max (log2 domain) and running sum of each row
-    float m_run[4], l_run[4];
-#pragma unroll
-    for (int i = 0; i < 4; ++i) {
-        m_run[i] = -INFINITY;
-        l_run[i] = 0.f;
-    }
+    float m_run[2] = {-INFINITY, -INFINITY}, l_run[2] = {0.f, 0.f};
     // Keys below mask_from are cached prefix keys of a live split: visible to
     // every active row, so their tiles need no masking.
     const int mask_from = min(kv, kend);
@@ -228,8 +224,8 @@ __global__ void __launch_bounds__(128 * NRG) attention_kernel(AttnArgs a) {
         if (s < n_tiles) load_tile(s, s);
         cp_async_commit();
     }
-    const uint32_t q_base = smem_u32(sQ);
-    const int l7 = lane & 7;
+    const int l7 = lane & 7, j8 = lane >> 3;
+    const uint32_t q_row = smem_u32(sQ) + (uint32_t)((rg * 16 + (j8 & 1) * 8 + l7) * D * 2);
     for (int it = 0; it < n_tiles; ++it) {
         cp_async_wait<kStages - 2>();
         __syncthreads();
@@ -244,52 +240,39 @@ __global__ void __launch_bounds__(128 * NRG) attention_kernel(AttnArgs a) {
         const int k0 = kbeg + it * kKT + kw;  // first key of this warp
         if (k0 >= kend) continue;             // warp has no keys in this tile
 
-        // S = Q K^T  (32 rows x 16 keys); rows and keys of every ldmatrix
+        // S = Q K^T  (16 rows x 16 keys); rows and keys of every ldmatrix
         // start at multiples of 8, so the swizzle XOR is lane & 7
-        float s[2][2][4];
+        float s[2][4];
 #pragma unroll
-        for (int mt = 0; mt < 2; ++mt)
+        for (int nt = 0; nt < 2; ++nt)
 #pragma unroll
-            for (int nt = 0; nt < 2; ++nt)
-#pragma unroll
-                for (int e = 0; e < 4; ++e) s[mt][nt][e] = 0.f;
-        const int j8 = lane >> 3;
+            for (int e = 0; e < 4; ++e) s[nt][e] = 0.f;
         const uint32_t k_row = k_base + (uint32_t)((kw + (j8 >> 1) * 8 + l7) * D * 2);
-        const uint32_t q_row0 = q_base + (uint32_t)((rg * 32 + (j8 & 1) * 8 + l7) * D * 2);
 #pragma unroll
         for (int kk = 0; kk < D / 16; ++kk) {
-            uint32_t kb[4];
+            uint32_t kb[4], qa[4];
             ldmatrix_x4(kb, k_row + (uint32_t)(((kk * 2 + (j8 & 1)) ^ l7) << 4));
-#pragma unroll
-            for (int mt = 0; mt < 2; ++mt) {
-                uint32_t qa[4];
-                ldmatrix_x4(qa, q_row0 + (uint32_t)(mt * 16 * D * 2) +
-                                    (uint32_t)(((kk * 2 + (j8 >> 1)) ^ l7) << 4));
-                mma_bf16_16816(s[mt][0], qa, kb[0], kb[1]);
-                mma_bf16_16816(s[mt][1], qa, kb[2], kb[3]);
-            }
+            ldmatrix_x4(qa, q_row + (uint32_t)(((kk * 2 + (j8 >> 1)) ^ l7) << 4));
+            mma_bf16_16816(s[0], qa, kb[0], kb[1]);
+            mma_bf16_16816(s[1], qa, kb[2], kb[3]);
         }
         // mask (boundary tiles only) + online softmax in the log2 domain
         if (k0 + 16 > mask_from) {
 #pragma unroll
-            for (int i = 0; i < 4; ++i) {
-                const int mt = i >> 1, hi = i & 1;
+            for (int i = 0; i < 2; ++i)
 #pragma unroll
                 for (int nt = 0; nt < 2; ++nt)
 #pragma unroll
                     for (int e = 0; e < 2; ++e) {
                         const int key = k0 + nt * 8 + (lane & 3) * 2 + e;
-                        if (key >= kend || key > rpos[i]) s[mt][nt][hi * 2 + e] = -INFINITY;
+                        if (key >= kend || key > rpos[i]) s[nt][i * 2 + e] = -INFINITY;
                     }
-            }
         }
-        float alpha[4];
+        float alpha[2];
         bool moved = false;
 #pragma unroll
-        for (int i = 0; i < 4; ++i) {
-            const int mt = i >> 1, hi = i & 1;
-            float mx = fmaxf(fmaxf(s[mt][0][hi * 2], s[mt][0][hi * 2 + 1]),
-                             fmaxf(s[mt][1][hi * 2], s[mt][1][hi * 2 + 1]));
+        for (int i = 0; i < 2; ++i) {
+            float mx = fmaxf(fmaxf(s[0][i * 2], s[0][i * 2 + 1]), fmaxf(s[1][i * 2], s[1][i * 2 + 1]));
             mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 1));
             mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 2));
             mx *= a.scale_log2;
@@ -305,8 +288,8 @@ __global__ void __launch_bounds__(128 * NRG) attention_kernel(AttnArgs a) {
             for (int nt = 0; nt < 2; ++nt)
 #pragma unroll
                 for (int e = 0; e < 2; ++e) {
-                    const float p = exp2f(fmaf(s[mt][nt][hi * 2 + e], a.scale_log2, -m_use));
-                    s[mt][nt][hi * 2 + e] = p;
+                    const float p = exp2f(fmaf(s[nt][i * 2 + e], a.scale_log2, -m_use));
+                    s[nt][i * 2 + e] = p;
                     rs += p;
                 }
             rs += __shfl_xor_sync(0xffffffffu, rs, 1);
@@ -315,34 +298,26 @@ __global__ void __launch_bounds__(128 * NRG) attention_kernel(AttnArgs a) {
         }
         if (__any_sync(0xffffffffu, moved)) {
 #pragma unroll
-            for (int mt = 0; mt < 2; ++mt)
-#pragma unroll
-                for (int nt = 0; nt < NT; ++nt) {
-                    o[mt][nt][0] *= alpha[mt * 2];
-                    o[mt][nt][1] *= alpha[mt * 2];
-                    o[mt][nt][2] *= alpha[mt * 2 + 1];
-                    o[mt][nt][3] *= alpha[mt * 2 + 1];
-                }
+            for (int nt = 0; nt < NT; ++nt) {
+                o[nt][0] *= alpha[0];
+                o[nt][1] *= alpha[0];
+                o[nt][2] *= alpha[1];
+                o[nt][3] *= alpha[1];
+            }
         }
-        // O += P V  (P: 32 x 16 keys as the A operand, straight from the S fragments)
-        uint32_t pa[2][4];
-#pragma unroll
-        for (int mt = 0; mt < 2; ++mt) {
-            pa[mt][0] = pack_bf16(s[mt][0][0], s[mt][0][1]);
-            pa[mt][1] = pack_bf16(s[mt][0][2], s[mt][0][3]);
-            pa[mt][2] = pack_bf16(s[mt][1][0], s[mt][1][1]);
-            pa[mt][3] = pack_bf16(s[mt][1][2], s[mt][1][3]);
-        }
+        // O += P V  (P: 16 rows x 16 keys as the A operand, from the S fragments)
+        uint32_t pa[4];
+        pa[0] = pack_bf16(s[0][0], s[0][1]);
+        pa[1] = pack_bf16(s[0][2], s[0][3]);
+        pa[2] = pack_bf16(s[1][0], s[1][1]);
+        pa[3] = pack_bf16(s[1][2], s[1][3]);
         const uint32_t v_row = v_base + (uint32_t)((kw + (j8 & 1) * 8 + l7) * D * 2);
 #pragma unroll
         for (int dn = 0; dn < NT; dn += 2) {
             uint32_t vb[4];
             ldmatrix_x4_trans(vb, v_row + (uint32_t)(((dn + (j8 >> 1)) ^ l7) << 4));
-#pragma unroll
-            for (int mt = 0; mt < 2; ++mt) {
-                mma_bf16_16816(o[mt][dn], pa[mt], vb[0], vb[1]);
-                mma_bf16_16816(o[mt][dn + 1], pa[mt], vb[2], vb[3]);
-            }
+            mma_bf16_16816(o[dn], pa, vb[0], vb[1]);
+            mma_bf16_16816(o[dn + 1], pa, vb[2], vb[3]);
         }
     }
     cp_async_wait<0>();
@@ -350,12 +325,12 @@ __global__ void __launch_bounds__(128 * NRG) attention_kernel(AttnArgs a) {
 
     // ---- merge the 4 warps of each row group in a fixed order
     float* red = reinterpret_cast<float*>(sK);   // pipeline buffers are free now
-    float* sm = red;                              // [warps][32] running max
-    float* sl = red + THREADS / 32 * 32;          // [warps][32] running sum
-    float* obuf = red + 2 * (THREADS / 32) * 32;  // [rg][2][NT*8][32]
+    float* sm = red;                              // [warps][16] running max
+    float* sl = red + THREADS / 32 * 16;          // [warps][16] running sum
+    float* obuf = red + 2 * (THREADS / 32) * 16;  // [rg][2][NT*4][32]
     const int wig = warp & 3;  // warp index within its row group
 #pragma unroll
-    for (int i = 0; i < 4; ++i) {
+    for (int i = 0; i < 2; ++i) {
         // inactive / padding rows were not masked in prefix tiles: drop them
         if (rpos[i] < 0) {
             m_run[i] = -INFINITY;
@@ -364,56 +339,50 @@ __global__ void __launch_bounds__(128 * NRG) attention_kernel(AttnArgs a) {
     }
     if ((lane & 3) == 0) {
 #pragma unroll
-        for (int i = 0; i < 4; ++i) {
-            const int r = (i >> 1) * 16 + (i & 1) * 8 + (lane >> 2);
-            sm[warp * 32 + r] = m_run[i];
-            sl[warp * 32 + r] = l_run[i];
+        for (int i = 0; i < 2; ++i) {
+            const int r = i * 8 + (lane >> 2);
+            sm[warp * 16 + r] = m_run[i];
+            sl[warp * 16 + r] = l_run[i];
         }
     }
     __syncthreads();
-    float m_fin[4], l_fin[4];
+    float m_fin[2], l_fin[2];
 #pragma unroll
-    for (int i = 0; i < 4; ++i) {
-        const int r = (i >> 1) * 16 + (i & 1) * 8 + (lane >> 2);
-
+    for (int i = 0; i < 2; ++i) {
+        const int r = i * 8 + (lane >> 2);
         float M = -INFINITY;
 #pragma unroll
-        for (int w = 0; w < 4; ++w) M = fmaxf(M, sm[(rg * 4 + w) * 32 + r]);
+        for (int w = 0; w < 4; ++w) M = fmaxf(M, sm[(rg * 4 + w) * 16 + r]);
         const float Mu = (M == -INFINITY) ? 0.f : M;
         float L = 0.f;
 #pragma unroll
         for (int w = 0; w < 4; ++w) {
-            const int ww = (rg * 4 + w) * 32 + r;
+            const int ww = (rg * 4 + w) * 16 + r;
             L += sl[ww] * exp2f(sm[ww] - Mu);
         }
         const float f = exp2f(m_run[i] - Mu);
         m_fin[i] = M;
         l_fin[i] = L;
-        const int mt = i >> 1, hi = i & 1;
 #pragma unroll
         for (int nt = 0; nt < NT; ++nt) {
-            o[mt][nt][hi * 2] *= f;
-            o[mt][nt][hi * 2 + 1] *= f;
+            o[nt][i * 2] *= f;
+            o[nt][i * 2 + 1] *= f;
         }
     }
-    float* my_buf = obuf + (size_t)(rg * 2) * (2 * NT * 4) * 32;  // two buffers per row group
+    constexpr int buf_elems = NT * 4 * 32;
+    float* my_buf = obuf + (size_t)(rg * 2) * buf_elems;  // two buffers per row group
     auto store_o = [&](float* buf) {
 #pragma unroll
-        for (int mt = 0; mt < 2; ++mt)
+        for (int nt = 0; nt < NT; ++nt)
 #pragma unroll
-            for (int nt = 0; nt < NT; ++nt)
-#pragma unroll
-                for (int e = 0; e < 4; ++e) buf[((mt * NT + nt) * 4 + e) * 32 + lane] = o[mt][nt][e];
+            for (int e = 0; e < 4; ++e) buf[(nt * 4 + e) * 32 + lane] = o[nt][e];
     };
     auto add_o = [&](const float* buf) {
 #pragma unroll
-        for (int mt = 0; mt < 2; ++mt)
+        for (int nt = 0; nt < NT; ++nt)
 #pragma unroll
-            for (int nt = 0; nt < NT; ++nt)
-#pragma unroll
-                for (int e = 0; e < 4; ++e) o[mt][nt][e] += buf[((mt * NT + nt) * 4 + e) * 32 + lane];
+            for (int e = 0; e < 4; ++e) o[nt][e] += buf[(nt * 4 + e) * 32 + lane];
     };
-    const int buf_elems = 2 * NT * 4 * 32;
     __syncthreads();
     if (wig >= 2) store_o(my_buf + (wig - 2) * buf_elems);
     __syncthreads();
@@ -428,20 +397,18 @@ __global__ void __launch_bounds__(128 * NRG) attention_kernel(AttnArgs a) {
     if (ns == 1) {
         if (wig == 0) {
 #pragma unroll
-            for (int i = 0; i < 4; ++i) {
-                const int r = rg * 32 + (i >> 1) * 16 + (i & 1) * 8 + (lane >> 2);
-                const int rr = row0 + r;
+            for (int i = 0; i < 2; ++i) {
+                const int rr = row0 + rg * 16 + i * 8 + (lane >> 2);
                 if (rr >= a.rows) continue;
                 const int hh = rr / a.Q, s = rr % a.Q;
                 const int h = g * a.grp + hh;
                 const float inv = l_fin[i] > 0.f ? 1.f / l_fin[i] : 0.f;
                 __nv_bfloat16* dst = a.out + ((size_t)b * a.Q + s) * a.Hq * D + (size_t)h * D;
-                const int mt = i >> 1, hi = i & 1;
 #pragma unroll
                 for (int nt = 0; nt < NT; ++nt) {
                     const int col = nt * 8 + (lane & 3) * 2;
-                    *reinterpret_cast<__nv_bfloat162*>(dst + col) = __floats2bfloat162_rn(
-                        o[mt][nt][hi * 2] * inv, o[mt][nt][hi * 2 + 1] * inv);
+                    *reinterpret_cast<__nv_bfloat162*>(dst + col) =
+                        __floats2bfloat162_rn(o[nt][i * 2] * inv, o[nt][i * 2 + 1] * inv);
                 }
             }
         }
@@ -454,18 +421,17 @@ __global__ void __launch_bounds__(128 * NRG) attention_kernel(AttnArgs a) {
     float* po = pl + ROWS;
     if (wig == 0) {
 #pragma unroll
-        for (int i = 0; i < 4; ++i) {
-            const int r = rg * 32 + (i >> 1) * 16 + (i & 1) * 8 + (lane >> 2);
+        for (int i = 0; i < 2; ++i) {
+            const int r = rg * 16 + i * 8 + (lane >> 2);
             if ((lane & 3) == 0) {
                 pm[r] = m_fin[i];
                 pl[r] = l_fin[i];
             }
-            const int mt = i >> 1, hi = i & 1;
 #pragma unroll
             for (int nt = 0; nt < NT; ++nt) {
                 const int col = nt * 8 + (lane & 3) * 2;
                 *reinterpret_cast<float2*>(po + (size_t)r * D + col) =
-                    make_float2(o[mt][nt][hi * 2], o[mt][nt][hi * 2 + 1]);
+                    make_float2(o[nt][i * 2], o[nt][i * 2 + 1]);
             }
         }
     }
@@ -504,27 +470,34 @@ __global__ void __launch_bounds__(128 * NRG) attention_kernel(AttnArgs a) {
     if (tid == 0) a.ticket[unit] = 0;
 }
 
-template <int D, int NRG>
+template <int D, int RG>
 static size_t attn_smem_bytes(int split) {
     // Q rows + K/V pipeline stages + the split's key -> row table
-    return (size_t)32 * NRG * D * 2 + (size_t)2 * kStages * kKT * D * 2 + (size_t)split * 4;
+    return (size_t)16 * RG * D * 2 + (size_t)2 * kStages * kKT * D * 2 + (size_t)split * 4;
 }
 
-template <int D, int NRG>
+template <int D, int RG>
 static cudaError_t launch_attention_t(const AttnArgs& a, dim3 grid, cudaStream_t st) {
     static unsigned long long configured = 0;  // bit per device: attribute set
     int dev = 0;
     cudaGetDevice(&dev);
     if (dev < 0 || dev >= 64) return cudaErrorInvalidDevice;
     if (!(configured >> dev & 1ull)) {
-        cudaError_t e = cudaFuncSetAttribute(attention_kernel<D, NRG>,
+        cudaError_t e = cudaFuncSetAttribute(attention_kernel<D, RG>,
                                              cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                             (int)attn_smem_bytes<D, NRG>(kAttnMaxSplit));
+                                             (int)attn_smem_bytes<D, RG>(kAttnMaxSplit));
         if (e != cudaSuccess) return e;
         configured |= 1ull << dev;
     }
-    attention_kernel<D, NRG><<<grid, 128 * NRG, attn_smem_bytes<D, NRG>(a.split), st>>>(a);
+    attention_kernel<D, RG><<<grid, 128 * RG, attn_smem_bytes<D, RG>(a.split), st>>>(a);
     return cudaGetLastError();
+}
+
+template <int D>
+static cudaError_t launch_attention_d(int rg, const AttnArgs& a, dim3 grid, cudaStream_t st) {
+    if (rg == 1) return launch_attention_t<D, 1>(a, grid, st);
+    if (rg == 2) return launch_attention_t<D, 2>(a, grid, st);
+    return launch_attention_t<D, 4>(a, grid, st);
 }
 
 cudaError_t launch_attention(const Plan& p, const isd_dims* d, const uint16_t* q,
@@ -562,12 +535,8 @@ cudaError_t launch_attention(const Plan& p, const isd_dims* d, const uint16_t* q
     a.ticket = reinterpret_cast<int*>(w + p.off_attn_ticket);
     a.err_flag = err_flag;
     dim3 grid(p.attn_max_splits, d->Hkv * p.attn_rgb, d->B);
-    if (d->D == 128) {
-        return p.attn_nrg == 1 ? launch_attention_t<128, 1>(a, grid, st)
-                               : launch_attention_t<128, 2>(a, grid, st);
-    }
-    return p.attn_nrg == 1 ? launch_attention_t<64, 1>(a, grid, st)
-                           : launch_attention_t<64, 2>(a, grid, st);
+    if (d->D == 128) return launch_attention_d<128>(p.attn_rg, a, grid, st);
+    return launch_attention_d<64>(p.attn_rg, a, grid, st);
 }
 
 }  // namespace isd

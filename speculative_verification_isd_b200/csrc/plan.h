@@ -10,7 +10,7 @@
 namespace isd {
 
 constexpr int kAttnKeyTile = 64;      // keys per pipeline stage
-constexpr int kAttnRowsPerGroup = 32; // query rows handled by one 4-warp group
+constexpr int kAttnRowsPerGroup = 16; // query rows handled by one 4-warp group
 constexpr int kAttnMaxSplit = 2048;   // keys per split at most (bounds the key table)
 constexpr int kStatsThreads = 256;
 constexpr int kAcceptThreads = 256;
@@ -21,7 +21,7 @@ struct Plan {
     // derived dims
     int Q, H, M, grp, rows;  // rows = grp * Q query rows per (request, kv head)
     // attention
-    int attn_nrg;            // 4-warp row groups per CTA (1 or 2)
+    int attn_rg;             // 16-row warp groups per CTA (1, 2 or 4)
     int attn_rgb;            // row-group blocks per (request, kv head)
     int attn_split;          // keys per split (multiple of kAttnKeyTile)
     int attn_max_splits;     // splits for the longest possible request
@@ -50,8 +50,8 @@ inline bool make_plan(const isd_dims* d, Plan* p) {
     p->M = d->B * p->Q;
     p->grp = d->Hq / d->Hkv;
     p->rows = p->grp * p->Q;
-    p->attn_nrg = p->rows > kAttnRowsPerGroup ? 2 : 1;
-    const int rows_per_cta = kAttnRowsPerGroup * p->attn_nrg;
+    p->attn_rg = p->rows <= 16 ? 1 : (p->rows <= 32 ? 2 : 4);
+    const int rows_per_cta = kAttnRowsPerGroup * p->attn_rg;
     p->attn_rgb = (p->rows + rows_per_cta - 1) / rows_per_cta;
     const long long max_ctx = (long long)d->max_pages_per_req * d->page_size;
     // Aim for about 3 waves of 2 CTAs per SM over the expected keys (half
