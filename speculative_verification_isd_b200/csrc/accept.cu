@@ -65,6 +65,23 @@ row_stats_kernel(const float* __restrict__ logits, int V, int n_chunks, int chun
     ticket[row] = 0;
 }
 
+// Row statistics from the LM head's per-(vocabulary tile, warp) partials:
+// part[row][k], k = 0..n_parts-1, merged in a fixed order.
+template <int THREADS>
+__global__ void __launch_bounds__(THREADS)
+row_stats_finalize_kernel(const float4* __restrict__ part, int n_parts,
+                          isd_row_stat* __restrict__ out) {
+    const int row = blockIdx.x;
+    const float4* pr = part + (size_t)row * n_parts;
+    RowStat st = rowstat_empty();
+    for (int k = threadIdx.x; k < n_parts; k += THREADS) {
+        const float4 p = __ldcs(pr + k);
+        st = rowstat_merge(st, RowStat{p.x, p.y, __float_as_int(p.z)});
+    }
+    st = rowstat_block_reduce<THREADS>(st);
+    if (threadIdx.x == 0) out[row] = isd_row_stat{st.m, st.s, st.idx, 0};
+}
+
 // ---------------------------------------------------------------------------
 // a6-a9
 // ---------------------------------------------------------------------------
@@ -378,6 +395,12 @@ cudaError_t launch_row_stats(const Plan& p, const float* logits, int rows, int V
         logits, V, p.stats_chunks, p.stats_chunk_len,
         reinterpret_cast<float4*>(w + p.off_stats_part),
         reinterpret_cast<int*>(w + p.off_stats_ticket), out);
+    return cudaGetLastError();
+}
+
+cudaError_t launch_row_stats_finalize(const float4* part, int n_parts, int rows,
+                                      isd_row_stat* out, cudaStream_t st) {
+    row_stats_finalize_kernel<kStatsThreads><<<rows, kStatsThreads, 0, st>>>(part, n_parts, out);
     return cudaGetLastError();
 }
 

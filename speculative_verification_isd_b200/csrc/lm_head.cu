@@ -39,8 +39,12 @@ struct LmArgs {
     int w_rows, h_rows0, h_rows1;  // TMA box heights (never taller than the tensor)
     uint32_t tmem_cols;
     float* logits;
+    float4* stats_part;  // [Mh][n_tiles * 4] partial row statistics, or null
     int32_t* err_flag;
 };
+
+constexpr int kEpiPitch = 33;  // floats per row of an epilogue transposition buffer
+constexpr int kEpiSmemBytes = 4 * 32 * kEpiPitch * 4;
 
 constexpr uint64_t kWaitLimitNs = 2000000000ull;
 constexpr int kLmThreads = 224;  // W producer, MMA, 4 epilogue warps, hidden producer
@@ -74,7 +78,9 @@ lm_head_kernel(const __grid_constant__ CUtensorMap tmap_w, const __grid_constant
     const int h_bytes = NB * a.BN * 128;  // one hidden stage (K = 64)
     unsigned char* wring = smem;
     unsigned char* hring = smem + (size_t)a.w_stages * kWStageBytes;
-    uint64_t* full = reinterpret_cast<uint64_t*>(hring + (size_t)a.h_stages * h_bytes);
+    float* epi_buf = reinterpret_cast<float*>(hring + (size_t)a.h_stages * h_bytes);
+    uint64_t* full = reinterpret_cast<uint64_t*>(reinterpret_cast<unsigned char*>(epi_buf) +
+                                                 kEpiSmemBytes);
     uint64_t* empty = full + a.w_stages;
     uint64_t* tfull = empty + a.w_stages;
     uint64_t* tempty = tfull + 2;
@@ -226,8 +232,12 @@ lm_head_kernel(const __grid_constant__ CUtensorMap tmap_w, const __grid_constant
             tc_fence_after();
             const int v = tile * 128 + quarter * 32 + lane;
             const bool v_ok = v < a.V;
+            const int nvalid = a.V - (tile * 128 + quarter * 32);  // valid vocab rows of this warp
             const uint32_t taddr =
                 tmem_base + ((uint32_t)(quarter * 32) << 16) + (uint32_t)(acc * NB * a.BN);
+            float* tb = epi_buf + quarter * 32 * kEpiPitch;
+            float4* part = a.stats_part ? a.stats_part + (size_t)(tile * 4 + quarter) : nullptr;
+            const size_t part_pitch = (size_t)a.n_tiles * 4;
 #pragma unroll
             for (int nb = 0; nb < NB; ++nb) {
                 for (int j0 = 0; j0 < a.BN; j0 += 32) {
@@ -247,6 +257,35 @@ lm_head_kernel(const __grid_constant__ CUtensorMap tmap_w, const __grid_constant
                             if (j0 + k < a.BN && m < a.Mh)
                                 a.logits[(size_t)m * a.V + v] = __uint_as_float(r[k]);
                         }
+                    }
+                    if (part) {
+                        // Row statistics of this warp's 32 vocabulary entries:
+                        // transpose through shared memory so that lane k holds
+                        // logits row mbase + k, then max / sum-exp / argmax
+                        // (first index among equal maxima).
+#pragma unroll
+                        for (int k = 0; k < 32; ++k) tb[lane * kEpiPitch + k] = __uint_as_float(r[k]);
+                        __syncwarp();
+                        float x[32];
+                        float mx = -INFINITY;
+                        int arg = 0;
+#pragma unroll
+                        for (int i = 0; i < 32; ++i) {
+                            x[i] = tb[i * kEpiPitch + lane];
+                            if (i < nvalid && x[i] > mx) {
+                                mx = x[i];
+                                arg = i;
+                            }
+                        }
+                        float se = 0.f;
+#pragma unroll
+                        for (int i = 0; i < 32; ++i)
+                            if (i < nvalid) se += __expf(x[i] - mx);
+                        const int m = mbase + lane;
+                        if (j0 + lane < a.BN && m < a.Mh)
+                            part[(size_t)m * part_pitch] =
+                                make_float4(mx, se, __int_as_float(tile * 128 + quarter * 32 + arg), 0.f);
+                        __syncwarp();
                     }
                 }
             }
@@ -322,7 +361,7 @@ bool lm_head_shape(int Mh, int smem_limit, LmShape* s) {
     while ((int)alloc < need) alloc <<= 1;
     s->tmem_cols = alloc;
     const int h_bytes = cols * 128;
-    const int budget = smem_limit - 1024 - 512;  // alignment slack + barriers
+    const int budget = smem_limit - 1024 - 512 - kEpiSmemBytes;  // slack, barriers, epilogue
     // hidden tiles are L2 hits: 3 stages; the rest of the budget deepens the
     // W ring (HBM latency under load is several microseconds)
     s->h_stages = 3;
@@ -334,7 +373,8 @@ bool lm_head_shape(int Mh, int smem_limit, LmShape* s) {
         if (s->w_stages > 16) s->w_stages = 16;
     }
     if (s->w_stages <= s->h_stages) return false;
-    s->smem = (size_t)s->w_stages * kWStageBytes + (size_t)s->h_stages * h_bytes + 1024 + 512;
+    s->smem = (size_t)s->w_stages * kWStageBytes + (size_t)s->h_stages * h_bytes + kEpiSmemBytes +
+              1024 + 512;
     return true;
 }
 
@@ -348,7 +388,7 @@ static int num_sms_of_current_device() {
 void set_error_detail(const char* msg);
 
 cudaError_t launch_lm_head(const uint16_t* hidden, const uint16_t* W, int Mh, int H, int V,
-                           float* logits, int32_t* err_flag, cudaStream_t st) {
+                           float* logits, float4* stats_part, int32_t* err_flag, cudaStream_t st) {
     // dynamic shared memory available to this kernel on the current device
     static int smem_limit_dev[64];
     int dev = 0;
@@ -413,6 +453,7 @@ cudaError_t launch_lm_head(const uint16_t* hidden, const uint16_t* W, int Mh, in
     a.n_tiles = (V + 127) / 128;
     a.tmem_cols = sh.tmem_cols;
     a.logits = logits;
+    a.stats_part = stats_part;
     a.err_flag = err_flag;
     int grid = num_sms_of_current_device();
     if (grid > a.n_tiles) grid = a.n_tiles;

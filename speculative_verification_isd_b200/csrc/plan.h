@@ -31,9 +31,12 @@ struct Plan {
     int acc_chunks;
     // R-ISD LoRA
     int lora_rows, lora_ksplit;
+    // LM-head row-statistics partials: one per (128-entry vocabulary tile, warp)
+    int lm_stat_parts;
     // workspace offsets (bytes)
     size_t off_attn_part, off_attn_ticket, off_hidden, off_hidden_lora, off_lora_t,
-        off_stats_part, off_stats_ticket, off_acc_part, off_acc_ticket, off_lora_part, total;
+        off_stats_part, off_stats_ticket, off_acc_part, off_acc_ticket, off_lora_part,
+        off_lm_stats, total;
 };
 
 inline size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
@@ -101,6 +104,8 @@ inline bool make_plan(const isd_dims* d, Plan* p) {
     p->off_acc_part = take((size_t)d->B * (d->N + 1) * p->acc_chunks * 4);
     p->off_acc_ticket = take((size_t)d->B * 4);
     p->off_lora_part = take(d->lora_rank ? (size_t)p->lora_ksplit * p->lora_rows * d->lora_rank * 4 : 0);
+    p->lm_stat_parts = ((d->V + 127) / 128) * 4;
+    p->off_lm_stats = take((size_t)p->M * p->lm_stat_parts * 16);
     p->total = off;
     return true;
 }
