@@ -215,46 +215,57 @@ __global__ void __launch_bounds__(kAcceptThreads) accept_kernel(AcceptArgs a) {
     const int N = a.N, Q = 2 * N - 1, V = a.V;
     const int rcols = N > 1 ? N - 1 : 1;
     __shared__ int s_state;  // -1 invalid request, 0 no rejection, j = rejected proposal index
-    __shared__ int s_c;
-    __shared__ int s_last;
+    __shared__ int s_last, s_bad;
+    __shared__ float s_ratio[16];
     const float* ub = a.uniforms + (size_t)b * 2 * N;
-    if (threadIdx.x == 0) {
-        const int c = a.n_clean[b];
-        int state = 0;
-        if (c < 1 || c > N) {
-            raise_flag(a.err_flag, ISD_FLAG_NCLEAN_RANGE);
-            state = -1;
-        } else {
-            for (int j = 2; j <= c; ++j) {
-                const int x = a.clean_tok[(size_t)b * N + j - 1];
-                if (x < 0 || x >= V) {
-                    raise_flag(a.err_flag, ISD_FLAG_TOKEN_OOB);
-                    state = -1;
-                    break;
-                }
+    const int c_in = __ldg(&a.n_clean[b]);
+    const bool bad_c = (c_in < 1 || c_in > N);
+    if (threadIdx.x == 0) s_bad = 0;
+    __syncthreads();
+    // all p/q ratios of this request at once (one gather round, not a chain)
+    {
+        const int j = (int)threadIdx.x + 2;
+        if (!bad_c && j <= c_in) {
+            const int x = __ldg(&a.clean_tok[(size_t)b * N + j - 1]);
+            if (x < 0 || x >= V) {
+                s_bad = 1;
+            } else {
                 const size_t rp = (size_t)b * Q + (j - 2);
                 const size_t rq = (size_t)b * Q + (N + j - 2);
                 const isd_row_stat sp = a.stats[rp], sq = a.prev_stats[rq];
                 const float zp = a.logits[rp * V + x];
                 const float zq = a.prev_logits[rq * V + x];
                 // p(x)/q(x) = exp((zp - mp) - (zq - mq)) * Sq / Sp
-                const float r = expf((zp - sp.max) - (zq - sq.max)) * (sq.sumexp / sp.sumexp);
-                if (ch == 0 && a.ratio) a.ratio[(size_t)b * rcols + j - 2] = r;
-                if (!(ub[j - 2] < r)) {
+                s_ratio[j - 2] = expf((zp - sp.max) - (zq - sq.max)) * (sq.sumexp / sp.sumexp);
+            }
+        }
+    }
+    __syncthreads();
+    if (threadIdx.x == 0) {
+        int state = 0;
+        if (bad_c) {
+            raise_flag(a.err_flag, ISD_FLAG_NCLEAN_RANGE);
+            state = -1;
+        } else if (s_bad) {
+            raise_flag(a.err_flag, ISD_FLAG_TOKEN_OOB);
+            state = -1;
+        } else {
+            // the first rejection stops the pass
+            for (int j = 2; j <= c_in; ++j)
+                if (!(ub[j - 2] < s_ratio[j - 2])) {
                     state = j;
                     break;
                 }
-            }
         }
         if (ch == 0 && a.ratio && state >= 0) {
-            const int tested = state > 0 ? state - 1 : c - 1;
-            for (int k = tested; k < rcols; ++k) a.ratio[(size_t)b * rcols + k] = -1.f;
+            const int tested = state > 0 ? state - 1 : c_in - 1;
+            for (int k = 0; k < rcols; ++k)
+                a.ratio[(size_t)b * rcols + k] = k < tested ? s_ratio[k] : -1.f;
         }
         s_state = state;
-        s_c = c;
     }
     __syncthreads();
-    const int state = s_state, c = s_c;
+    const int state = s_state, c = c_in;
     const int* tok = a.clean_tok + (size_t)b * N;
     if (state < 0) {  // invalid request: emit nothing, carry the state over
         if (ch == 0 && threadIdx.x == 0) {
@@ -307,35 +318,36 @@ __global__ void __launch_bounds__(kAcceptThreads) accept_kernel(AcceptArgs a) {
             SweepRow r;
             row_of(k, &r);
             const float u = state > 0 ? ub[N - 1] : ub[N + k];
-            // totals in chunk order
+            // chunk totals in chunk order, scanned by the whole block
             __shared__ float s_target;
-            __shared__ int s_chunk;
+            __shared__ int s_chunk, s_hit, s_lastpos;
+            const float tv = (int)threadIdx.x < a.n_chunks
+                                 ? __ldcg(&part[(size_t)k * a.n_chunks + threadIdx.x]) : 0.f;
+            float total;
+            const float excl = block_exclusive_scan(tv, &total);
+            const float target = u * total;
             if (threadIdx.x == 0) {
-                float total = 0.f;
-                for (int q = 0; q < a.n_chunks; ++q) total += __ldcg(&part[(size_t)k * a.n_chunks + q]);
-                const float target = u * total;
-                float cum = 0.f;
-                int hit = -1, lastpos = -1;
-                float local = 0.f;
-                for (int q = 0; q < a.n_chunks; ++q) {
-                    const float t = __ldcg(&part[(size_t)k * a.n_chunks + q]);
-                    if (t > 0.f) lastpos = q;
-                    if (hit < 0 && cum + t > target) {
-                        hit = q;
-                        local = target - cum;
-                    }
-                    cum += t;
-                }
-                if (total <= 0.f) {
-                    s_chunk = -2;  // no mass: residual falls back to argmax p
-                } else if (hit < 0) {
-                    s_chunk = lastpos;
-                    local = 3.0e38f;  // take the last positive entry of that chunk
-                } else {
-                    s_chunk = hit;
-                }
-                s_target = fmaxf(local, 0.f);
+                s_hit = 0x7fffffff;
+                s_lastpos = -1;
             }
+            __syncthreads();
+            if (tv > 0.f) atomicMax(&s_lastpos, (int)threadIdx.x);
+            if ((int)threadIdx.x < a.n_chunks && excl + tv > target) atomicMin(&s_hit, (int)threadIdx.x);
+            __syncthreads();
+            if (threadIdx.x == 0) {
+                if (!(total > 0.f)) {
+                    s_chunk = -2;  // no mass: residual falls back to argmax p
+                    s_target = 0.f;
+                } else if (s_hit == 0x7fffffff) {
+                    s_chunk = s_lastpos;
+                    s_target = 3.0e38f;  // take the last positive entry of that chunk
+                } else {
+                    s_chunk = s_hit;
+                }
+            }
+            __syncthreads();
+            if (s_chunk >= 0 && s_chunk == s_hit && (int)threadIdx.x == s_hit)
+                s_target = fmaxf(target - excl, 0.f);
             __syncthreads();
             const int q = s_chunk;
             const float tgt = s_target;
