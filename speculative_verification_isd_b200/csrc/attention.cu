@@ -500,11 +500,23 @@ static cudaError_t launch_attention_d(int rg, const AttnArgs& a, dim3 grid, cuda
     return launch_attention_t<D, 4>(a, grid, st);
 }
 
+cudaError_t launch_attention_tc(const Plan& p, const isd_dims* d, const uint16_t* q,
+                                const uint16_t* k_new, const uint16_t* v_new, uint16_t* k_pool,
+                                uint16_t* v_pool, const int32_t* page_table, const int32_t* kv_len,
+                                const int32_t* n_clean, uint16_t* out, void* ws, int32_t* err_flag,
+                                cudaStream_t st, bool* handled);
+
+// The tensor-core kernel (attention_tc.cu) where the shape fits it, else the
+// general mma.sync kernel above.
 cudaError_t launch_attention(const Plan& p, const isd_dims* d, const uint16_t* q,
                              const uint16_t* k_new, const uint16_t* v_new, uint16_t* k_pool,
                              uint16_t* v_pool, const int32_t* page_table, const int32_t* kv_len,
                              const int32_t* n_clean, uint16_t* out, void* ws, int32_t* err_flag,
                              cudaStream_t st) {
+    bool handled = false;
+    const cudaError_t te = launch_attention_tc(p, d, q, k_new, v_new, k_pool, v_pool, page_table,
+                                               kv_len, n_clean, out, ws, err_flag, st, &handled);
+    if (handled || te != cudaSuccess) return te;
     char* w = static_cast<char*>(ws);
     AttnArgs a;
     a.B = d->B;

@@ -1,0 +1,871 @@
+// Strict-causal GQA attention over the paged KV cache (a2) on the
+// 5th-generation tensor cores, with the KV append (a1) as a separate kernel.
+//
+// Same operation as attention.cu: every query slot of the block attends to
+// the cached prefix and to the block keys at or before its own position
+// (strict causal mask over clean and MASK slots, "I-DLM：扩散模型如何用“自省一致性”
+// 追上自回归模型质量", section "三项关键训练创新"; paged KV cache, section
+// "推理：复用 AR 推理栈").  Organised for sm_100a:
+//
+//  * kv_append_kernel first writes the block's K/V rows into their pages, so
+//    every key is then read from the pool by TMA: a 4-D tensor map (d, kv head,
+//    token in page, page) whose page coordinate comes from the page table; a
+//    page past the request (or a bad page id) is a box out of range and
+//    reads zeros;
+//  * the work is split tile-granularly ("stream-K"): the flattened sequence of
+//    (request, kv head, 128-key tile) is cut into G equal ranges, one per
+//    persistent CTA, so every SM streams the same number of KV bytes.  A
+//    (request, kv head) cut by a range boundary leaves a partial result per
+//    CTA; the CTA that draws the last ticket merges them in CTA order, so the
+//    result does not depend on timing;
+//  * per 128-key tile two tensor-core products, issued by one thread:
+//      S^T[128 keys, R rows] = K . Q^T         (M=128, N=R, K=128 d)
+//      O^T[128 d,   R rows] += V^T . P^T       (M=128, N=R, K=128 keys)
+//    with Q/K/V/P in 128-byte-swizzled shared memory and S, O in TMEM;
+//  * softmax warps own one key each per thread and 16 of the rows (R / 16
+//    groups of 4 warps); the
+//    per-row reference maximum moves only when a score exceeds it by more
+//    than 2^8 (then O^T is rescaled in TMEM), and P^T goes to shared memory
+//    as bf16 for the second product;
+//  * every wait is bounded (about 2 s): on time-out the CTA raises
+//    ISD_FLAG_WAIT_TIMEOUT, all roles leave their loops, in-flight copies and
+//    MMAs are drained and TMEM is released.
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+#include "common.cuh"
+#include "plan.h"
+#include "sm100.cuh"
+#include "tmap.h"
+
+namespace isd {
+
+void set_error_detail(const char* msg);
+
+namespace {
+
+constexpr int kTcKeys = 128;            // keys per tile (M of S^T)
+constexpr int kTcHalf = kTcKeys * 128;  // bytes of one 64-d half of a K or V tile
+constexpr uint64_t kTcWaitNs = 2000000000ull;
+
+struct TcArgs {
+    int B, N, Q, Hq, Hkv, grp, rows, P, num_pages, max_pages;
+    float scale_log2;
+    const int32_t* page_table;
+    const int32_t* kv_len;
+    const int32_t* n_clean;
+    __nv_bfloat16* out;
+    float* part;        // [gridDim.x][2][part_stride] partial results
+    int part_stride;    // floats per partial: R maxima, R sums, R x 128 O values
+    int* ticket;        // [B * Hkv], zero between calls
+    int32_t* err_flag;
+};
+
+ISD_DEVINL int tc_slot_pos(int s, int kv, int c, int N) {
+    if (s < c) return kv + s;
+    if (s < N) return -1;
+    return kv + c + (s - N);
+}
+
+// Keys of request b (prefix and active block rows); 0 for a request that
+// cannot be served (bad n_clean, negative or over-capacity length).
+ISD_DEVINL int tc_total_keys(const TcArgs& a, int b) {
+    const int kv = a.kv_len[b], c = a.n_clean[b];
+    if (c < 1 || c > a.N || kv < 0) return 0;
+    const long long t = (long long)kv + c + a.N - 1;
+    if ((t + a.P - 1) / a.P > a.max_pages) return 0;
+    return (int)t;
+}
+
+// a1: the block's K/V rows into their pages (16 bytes per thread and step);
+// a request that cannot be served gets zero attention output here.
+__global__ void kv_append_kernel(TcArgs a, const __nv_bfloat16* k_new, const __nv_bfloat16* v_new,
+                                 __nv_bfloat16* k_pool, __nv_bfloat16* v_pool) {
+    const int b = blockIdx.x;
+    const int kv = a.kv_len[b], c = a.n_clean[b];
+    const bool bad_c = (c < 1 || c > a.N);
+    const long long want = bad_c ? 0 : (long long)kv + c + a.N - 1;
+    const bool over = kv < 0 || (want + a.P - 1) / a.P > a.max_pages;
+    if (bad_c || over) {
+        if (threadIdx.x == 0) raise_flag(a.err_flag, bad_c ? ISD_FLAG_NCLEAN_RANGE : ISD_FLAG_CAPACITY);
+        uint4* o = reinterpret_cast<uint4*>(a.out + (size_t)b * a.Q * a.Hq * 128);
+        for (int i = threadIdx.x; i < a.Q * a.Hq * 16; i += blockDim.x) o[i] = make_uint4(0, 0, 0, 0);
+        return;
+    }
+    const int nblk = c + a.N - 1;
+    const int per_pos = a.Hkv * 16;  // 16-byte chunks of one position, all kv heads
+    for (int i = threadIdx.x; i < nblk * per_pos; i += blockDim.x) {
+        const int r = i / per_pos, rem = i % per_pos;
+        const int t = kv + r;
+        const int slot = r < c ? r : a.N + (r - c);
+        const int page = a.page_table[(size_t)b * a.max_pages + t / a.P];
+        if (page < 0 || page >= a.num_pages) {
+            raise_flag(a.err_flag, ISD_FLAG_PAGE_OOB);
+            continue;
+        }
+        const size_t dst = ((size_t)page * a.P + t % a.P) * a.Hkv * 128 + (size_t)rem * 8;
+        const size_t src = ((size_t)b * a.Q + slot) * a.Hkv * 128 + (size_t)rem * 8;
+        *reinterpret_cast<uint4*>(k_pool + dst) = *reinterpret_cast<const uint4*>(k_new + src);
+        *reinterpret_cast<uint4*>(v_pool + dst) = *reinterpret_cast<const uint4*>(v_new + src);
+    }
+}
+
+template <int STAGES>
+struct TcShared {
+    uint64_t kv_full[STAGES], kv_empty[STAGES];
+    uint64_t s_full[2], s_empty[2], p_full[2], p_empty[2];
+    uint64_t o_full, o_empty, q_full, q_empty, drain;
+    uint32_t tmem;
+    int abort_flag;
+    int never;
+};
+
+// Softmax warps: 4 per column group (one per TMEM lane quarter); each
+// column group covers 16 of the R query rows, so a thread holds 16 scores,
+// reference maxima and row sums, and for R >= 32 every SM sub-partition runs
+// two or more softmax warps that hide each other's latencies.
+template <int R>
+struct TcRoles {
+    static constexpr int RC = 16;               // rows per softmax thread
+    static constexpr int CG = R / RC;           // column groups
+    static constexpr int kSoft = 128 * CG;      // softmax threads
+    static constexpr int kThreads = 64 + kSoft; // + TMA warp + MMA warp
+};
+
+template <int R, int STAGES>
+constexpr size_t tc_smem_fixed() {
+    return (size_t)STAGES * 4 * kTcHalf    // K and V stages
+           + 2 * R * 128                   // Q (two 64-d halves)
+           + 2 * 2 * R * 128               // P^T, two buffers of two 64-key halves
+           + 4 * R * 4 * 2                 // per-warp row maxima and row sums
+           + R * 4                         // per-row causal key limit
+           + sizeof(TcShared<STAGES>);
+}
+
+// named barrier 1 over the NT softmax threads, OR of a predicate
+template <int NT>
+ISD_DEVINL bool group_or(bool v) {
+    uint32_t r;
+    asm volatile(
+        "{\n .reg .pred p, q;\n setp.ne.u32 p, %1, 0;\n bar.red.or.pred q, 1, %2, p;\n"
+        " selp.u32 %0, 1, 0, q;\n}\n"
+        : "=r"(r)
+        : "r"((uint32_t)v), "n"(NT)
+        : "memory");
+    return r != 0;
+}
+template <int NT>
+ISD_DEVINL void group_sync() { asm volatile("bar.sync 1, %0;\n" ::"n"(NT) : "memory"); }
+
+template <int C>
+ISD_DEVINL void tmem_load_cols(uint32_t taddr, uint32_t (&v)[C]) {
+#pragma unroll
+    for (int j = 0; j < C / 16; ++j) sm100::tmem_ld16(taddr + j * 16, v + j * 16);
+}
+template <int C>
+ISD_DEVINL void tmem_store_cols(uint32_t taddr, const uint32_t (&v)[C]) {
+#pragma unroll
+    for (int j = 0; j < C / 16; ++j) sm100::tmem_st16(taddr + j * 16, v + j * 16);
+}
+
+template <int R, int STAGES>
+__global__ void __launch_bounds__(TcRoles<R>::kThreads, 1)
+attention_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_v,
+                    const __grid_constant__ CUtensorMap tm_q, TcArgs a) {
+    using namespace sm100;
+    constexpr int RC = TcRoles<R>::RC, CG = TcRoles<R>::CG, kSoft = TcRoles<R>::kSoft;
+    constexpr int kThreads = TcRoles<R>::kThreads;
+    constexpr uint32_t kQBytes = 2 * R * 128;
+    constexpr uint32_t kPBytes = 2 * R * 128;
+    constexpr uint32_t kTmemCols = 4 * R <= 32 ? 32 : (4 * R <= 64 ? 64 : (4 * R <= 128 ? 128 : 256));
+    extern __shared__ unsigned char smem_raw[];
+    unsigned char* smem = reinterpret_cast<unsigned char*>(
+        (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    unsigned char* sK = smem;
+    unsigned char* sV = sK + STAGES * 2 * kTcHalf;
+    unsigned char* sQ = sV + STAGES * 2 * kTcHalf;
+    unsigned char* sP = sQ + kQBytes;
+    float* red_m = reinterpret_cast<float*>(sP + 2 * kPBytes);  // [4][R]
+    float* red_l = red_m + 4 * R;                                // [4][R]
+    int* lim = reinterpret_cast<int*>(red_l + 4 * R);            // [R]
+    TcShared<STAGES>* sh = reinterpret_cast<TcShared<STAGES>*>(lim + R);
+    int* prefix = reinterpret_cast<int*>(sh + 1);                // [B*Hkv + 1]
+
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int n_units = a.B * a.Hkv;
+
+    // ---- set-up
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < STAGES; ++s) {
+            mbar_init(&sh->kv_full[s], 1);
+            mbar_init(&sh->kv_empty[s], 1);
+        }
+        for (int i = 0; i < 2; ++i) {
+            mbar_init(&sh->s_full[i], 1);
+            mbar_init(&sh->s_empty[i], 4 * CG);
+            mbar_init(&sh->p_full[i], 4 * CG);
+            mbar_init(&sh->p_empty[i], 1);
+        }
+        mbar_init(&sh->o_full, 1);
+        mbar_init(&sh->o_empty, 4 * CG);
+        mbar_init(&sh->q_full, 1);
+        mbar_init(&sh->q_empty, 1);
+        mbar_init(&sh->drain, 1);
+        sh->abort_flag = 0;
+        sh->never = 0;
+        fence_mbar_init();
+        prefetch_tmap(&tm_k);
+        prefetch_tmap(&tm_v);
+        prefetch_tmap(&tm_q);
+    }
+    if (warp == 1) {
+        tmem_alloc(&sh->tmem, kTmemCols);
+        tmem_relinquish();
+    }
+    // Q rows past `rows` stay zero (no TMA box covers them)
+    for (int i = threadIdx.x; i < (int)(kQBytes / 16); i += kThreads)
+        reinterpret_cast<uint4*>(sQ)[i] = make_uint4(0, 0, 0, 0);
+    if (warp == 0) {
+        // prefix[u] = tiles of the units before u (unit u = request u / Hkv, kv head u % Hkv)
+        int run = 0;
+        for (int u0 = 0; u0 < n_units; u0 += 32) {
+            const int u = u0 + lane;
+            const int nt = u < n_units ? (tc_total_keys(a, u / a.Hkv) + kTcKeys - 1) / kTcKeys : 0;
+            int incl = nt;
+#pragma unroll
+            for (int off = 1; off < 32; off <<= 1) {
+                const int v = __shfl_up_sync(0xffffffffu, incl, off);
+                if (lane >= off) incl += v;
+            }
+            if (u < n_units) prefix[u] = run + incl - nt;
+            run += __shfl_sync(0xffffffffu, incl, 31);
+        }
+        if (lane == 0) prefix[n_units] = run;
+    }
+    asm volatile("fence.proxy.async.shared::cta;\n" ::: "memory");
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = sh->tmem;
+    const int T = prefix[n_units];
+    const int G = (int)gridDim.x < T ? (int)gridDim.x : T;  // every active CTA gets >= 1 tile
+    const bool active = (int)blockIdx.x < G;
+    const int my0 = active ? (int)((long long)T * blockIdx.x / G) : 0;
+    const int my1 = active ? (int)((long long)T * (blockIdx.x + 1) / G) : 0;
+    volatile int* abort_flag = &sh->abort_flag;
+
+    // unit holding `tile`: the largest u with prefix[u] <= tile
+    auto unit_of = [&](int tile) {
+        int lo = 0, hi = n_units;
+        while (hi - lo > 1) {
+            const int mid = (lo + hi) >> 1;
+            if (prefix[mid] <= tile) lo = mid; else hi = mid;
+        }
+        return lo;
+    };
+    auto give_up = [&]() {
+        *abort_flag = 1;
+        raise_flag(a.err_flag, ISD_FLAG_WAIT_TIMEOUT);
+    };
+
+    if (warp == 0) {
+        if (active) {
+            // ------------------------------------------------ TMA producer
+            // The whole warp walks the tiles: page ids come in chunks of 32
+            // (lane i holds one), the next chunk's load in flight while the
+            // current one is issued; lane 0 waits and issues the copies.
+            const uint64_t pol_kv = policy_evict_first();  // each K/V byte is read once
+            const uint64_t pol_q = policy_evict_last();
+            const int np = kTcKeys / a.P;  // pages per tile (<= 16)
+            int st = 0;
+            uint32_t ph = 0, q_use = 0, armed = 0, armed_par = 0;
+            bool ok = true;
+            for (int tile = my0; ok && tile < my1;) {
+                const int u = unit_of(tile);
+                const int us = prefix[u], ue = prefix[u + 1];
+                const int t0 = tile - us, t1 = min(ue, my1) - us;
+                const int b = u / a.Hkv, g = u % a.Hkv;
+                const int need_pages = (tc_total_keys(a, b) + a.P - 1) / a.P;
+                if (lane == 0) {
+                    ok = mbar_wait_bounded(&sh->q_empty, (q_use & 1) ^ 1, abort_flag, kTcWaitNs);
+                    if (!ok) {
+                        give_up();
+                    } else {
+                        mbar_arrive_expect_tx(&sh->q_full, (uint32_t)a.rows * 256u);
+                        tma_load_4d(sQ, &tm_q, &sh->q_full, 0, g * a.grp, 0, b, pol_q);
+                        tma_load_4d(sQ + R * 128, &tm_q, &sh->q_full, 64, g * a.grp, 0, b, pol_q);
+                    }
+                }
+                ok = __shfl_sync(0xffffffffu, ok, 0);
+                if (!ok) break;
+                ++q_use;
+                const int32_t* ptab = a.page_table + (size_t)b * a.max_pages;
+                const int tpc = 32 / np;  // tiles per chunk of page ids
+                // page id of page (first tile of the chunk) * np + lane; pages
+                // past the request (or bad ids) read as zeros
+                auto load_ids = [&](int tc0) {
+                    const int pidx = tc0 * np + lane;
+                    int id = -1;
+                    if (pidx < need_pages) {
+                        id = __ldg(ptab + pidx);
+                        if (id < 0 || id >= a.num_pages) {
+                            raise_flag(a.err_flag, ISD_FLAG_PAGE_OOB);
+                            id = -1;
+                        }
+                    }
+                    return id;
+                };
+                int ids = load_ids(t0), ids_next = load_ids(t0 + tpc);
+                for (int t = t0; t < t1; ++t) {
+                    const int j = (t - t0) % tpc;  // tile within the chunk
+                    if (j == 0 && t > t0) {
+                        ids = ids_next;
+                        ids_next = load_ids(t + tpc);
+                    }
+                    if (lane == 0) {
+                        ok = mbar_wait_bounded(&sh->kv_empty[st], ph ^ 1, abort_flag, kTcWaitNs);
+                        if (!ok) give_up();
+                        else mbar_arrive_expect_tx(&sh->kv_full[st], 4u * kTcHalf);
+                    }
+                    ok = __shfl_sync(0xffffffffu, ok, 0);
+                    if (!ok) break;
+                    unsigned char* k_dst = sK + st * 2 * kTcHalf;
+                    unsigned char* v_dst = sV + st * 2 * kTcHalf;
+                    for (int pg = 0; pg < np; ++pg) {
+                        const int page = __shfl_sync(0xffffffffu, ids, j * np + pg);
+                        if (lane == 0) {
+                            const int off = pg * a.P * 128;
+                            tma_load_4d(k_dst + off, &tm_k, &sh->kv_full[st], 0, g, 0, page, pol_kv);
+                            tma_load_4d(k_dst + kTcHalf + off, &tm_k, &sh->kv_full[st], 64, g, 0, page, pol_kv);
+                            tma_load_4d(v_dst + off, &tm_v, &sh->kv_full[st], 0, g, 0, page, pol_kv);
+                            tma_load_4d(v_dst + kTcHalf + off, &tm_v, &sh->kv_full[st], 64, g, 0, page, pol_kv);
+                        }
+                    }
+                    armed |= 1u << st;
+                    armed_par = (armed_par & ~(1u << st)) | (ph << st);
+                    if (++st == STAGES) {
+                        st = 0;
+                        ph ^= 1;
+                    }
+                }
+                tile = us + t1;
+            }
+            // drain: every armed copy has landed before the CTA may exit
+            if (lane == 0) {
+                for (int s = 0; s < STAGES; ++s)
+                    if (armed >> s & 1)
+                        mbar_wait_bounded(&sh->kv_full[s], armed_par >> s & 1, &sh->never, kTcWaitNs);
+                if (q_use) mbar_wait_bounded(&sh->q_full, (q_use - 1) & 1, &sh->never, kTcWaitNs);
+            }
+        }
+    } else if (warp == 1) {
+        if (lane == 0 && active) {
+            // ------------------------------------------------ MMA issuer
+            constexpr uint32_t idesc_s = idesc_bf16_f32(128, R);
+            constexpr uint32_t idesc_o = idesc_bf16_f32(128, R) | (1u << 15);  // A = V^T, MN-major
+            const uint64_t dq = smem_desc_sw128(smem_u32(sQ));
+            const uint64_t dk = smem_desc_sw128(smem_u32(sK));
+            const uint64_t dp = smem_desc_sw128(smem_u32(sP));
+            // V^T as an MN-major operand: the two 64-d blocks are kTcHalf apart
+            // (leading byte offset), 8-key groups 1024 bytes apart (stride byte offset)
+            const uint64_t dv = (smem_desc_sw128(smem_u32(sV)) & ~(0x3FFFull << 16)) |
+                                ((uint64_t)(kTcHalf >> 4) << 16);
+            const uint32_t tm_o = tmem + 2 * R;
+            // S products run ahead of the P.V products: S(t+1) is issued as
+            // soon as its K tile and S buffer are ready, PV(t) as soon as P(t)
+            // is, so a stage is released right after its PV completes
+            int s_tc = 0, s_st = 0;    // S products issued; stage of the next one
+            uint32_t s_ph = 0;
+            int pv_tc = 0, pv_st = 0;  // PV products issued; stage of the next one
+            uint32_t q_use = 0, o_use = 0;
+            bool ok = true;
+            auto wait = [&](uint64_t* bar, uint32_t par) {
+                if (mbar_try_wait(bar, par) || mbar_wait_bounded(bar, par, abort_flag, kTcWaitNs))
+                    return true;
+                give_up();
+                ok = false;
+                return false;
+            };
+            auto issue_s = [&]() {
+                const int buf = s_tc & 1;
+                tc_fence_after();
+                const uint32_t k_off = (uint32_t)(s_st * 2 * kTcHalf);
+#pragma unroll
+                for (int kk = 0; kk < 8; ++kk) {
+                    const uint64_t ad = dk + ((k_off + (kk >> 2) * kTcHalf + (kk & 3) * 32) >> 4);
+                    const uint64_t bd = dq + (((kk >> 2) * R * 128 + (kk & 3) * 32) >> 4);
+                    mma_f16_ss(tmem + buf * R, ad, bd, idesc_s, kk != 0);
+                }
+                mma_commit(&sh->s_full[buf]);
+                if (++s_st == STAGES) {
+                    s_st = 0;
+                    s_ph ^= 1;
+                }
+                ++s_tc;
+            };
+            auto s_inputs_ready = [&]() {
+                return mbar_test(&sh->kv_full[s_st], s_ph) &&
+                       mbar_test(&sh->s_empty[s_tc & 1], ((s_tc >> 1) & 1) ^ 1);
+            };
+            auto issue_s_blocking = [&]() {
+                if (!wait(&sh->kv_full[s_st], s_ph)) return false;
+                if (!wait(&sh->s_empty[s_tc & 1], ((s_tc >> 1) & 1) ^ 1)) return false;
+                issue_s();
+                return true;
+            };
+            for (int tile = my0; ok && tile < my1;) {
+                const int u = unit_of(tile);
+                const int us = prefix[u], ue = prefix[u + 1];
+                const int t0 = tile - us, t1 = min(ue, my1) - us;
+                const int end_tc = s_tc + (t1 - t0);  // tile numbers of this piece: [s_tc, end_tc)
+                if (!wait(&sh->q_full, q_use & 1)) break;
+                ++q_use;
+                if (!issue_s_blocking()) break;
+                bool q_done = false, first_pv = true;
+                while (ok && pv_tc < end_tc) {
+                    // wait for P(pv_tc); issue the next S meanwhile once it can go
+                    const uint64_t tstart = global_ns();
+                    for (uint32_t it = 0;; ++it) {
+                        if (s_tc < end_tc && s_inputs_ready()) issue_s();
+                        if (mbar_test(&sh->p_full[pv_tc & 1], (pv_tc >> 1) & 1)) break;
+                        if ((it & 255) == 255 && (*abort_flag || global_ns() - tstart > kTcWaitNs)) {
+                            give_up();
+                            ok = false;
+                            break;
+                        }
+                    }
+                    if (!ok) break;
+                    if (s_tc == end_tc && !q_done) {
+                        mma_commit(&sh->q_empty);  // every S product of this unit issued
+                        q_done = true;
+                    }
+                    if (first_pv && !wait(&sh->o_empty, (o_use & 1) ^ 1)) break;
+                    tc_fence_after();
+                    const uint32_t v_off = (uint32_t)(pv_st * 2 * kTcHalf);
+                    const uint32_t p_off = (uint32_t)((pv_tc & 1) * kPBytes);
+#pragma unroll
+                    for (int kk = 0; kk < kTcKeys / 16; ++kk) {
+                        const uint64_t ad = dv + ((v_off + kk * 2048) >> 4);
+                        const uint64_t bd = dp + ((p_off + (kk >> 2) * R * 128 + (kk & 3) * 32) >> 4);
+                        mma_f16_ss(tm_o, ad, bd, idesc_o, (first_pv && kk == 0) ? 0u : 1u);
+                    }
+                    mma_commit(&sh->kv_empty[pv_st]);
+                    mma_commit(&sh->p_empty[pv_tc & 1]);
+                    first_pv = false;
+                    if (++pv_st == STAGES) pv_st = 0;
+                    ++pv_tc;
+                    // the softmax continues with S(pv_tc): issue it now if it is still missing
+                    if (pv_tc < end_tc && s_tc == pv_tc && !issue_s_blocking()) break;
+                }
+                if (!ok) break;
+                if (!q_done) mma_commit(&sh->q_empty);
+                mma_commit(&sh->o_full);
+                ++o_use;
+                tile = us + t1;
+            }
+            mma_commit(&sh->drain);
+            mbar_wait_bounded(&sh->drain, 0, &sh->never, kTcWaitNs);
+        }
+    } else if (active) {
+        // ------------------------------------------------ softmax + epilogue
+        // thread = key kl of the tile (S^T lane) and rows r0 .. r0+RC-1;
+        // in the epilogue thread = output dimension d = kl of O^T
+        const int q4 = warp & 3;             // TMEM lane quarter of this warp
+        const int cg = (warp - 2) >> 2;      // column group
+        const int r0 = cg * RC;
+        const int kl = q4 * 32 + lane;
+        const int et = threadIdx.x - 64;     // 0 .. kSoft-1
+        const uint32_t tm_lane = tmem + ((uint32_t)(q4 * 32) << 16);
+        // this thread's P^T column: 64-key half, swizzled 16-byte chunk, element
+        const int kin = kl & 63;
+        unsigned char* p_col = sP + (kl >> 6) * R * 128 + (kin & 7) * 2;
+        const int p_chunk = kin >> 3;
+        // one thread waits, the group follows: every thread takes the same exit
+        auto group_wait = [&](uint64_t* bar, uint32_t par) -> bool {
+            bool fail = false;
+            if (et == 0) {
+                fail = !(mbar_try_wait(bar, par) || mbar_wait_bounded(bar, par, abort_flag, kTcWaitNs));
+                if (fail) give_up();
+            }
+            return !group_or<kSoft>(fail);
+        };
+        float m_ref[RC], l_part[RC];
+        int tc = 0, kst = 0;
+        uint32_t o_use = 0;
+        bool ok = true;
+        for (int tile = my0; ok && tile < my1;) {
+            const int u = unit_of(tile);
+            const int us = prefix[u], ue = prefix[u + 1];
+            const int t0 = tile - us, t1 = min(ue, my1) - us;
+            const int b = u / a.Hkv, g = u % a.Hkv;
+            const int kv = a.kv_len[b], c = a.n_clean[b];
+            const int total = tc_total_keys(a, b);
+            // last visible key of each row (rows are slot-major, then head in
+            // the group); read after the next group barrier
+            if (et < R) {
+                const int pos = et < a.rows ? tc_slot_pos(et / a.grp, kv, c, a.N) : -1;
+                lim[et] = min(pos, total - 1);
+            }
+#pragma unroll
+            for (int r = 0; r < RC; ++r) {
+                m_ref[r] = -INFINITY;
+                l_part[r] = 0.f;
+            }
+            for (int t = t0; t < t1; ++t) {
+                const int buf = tc & 1;
+                if (!group_wait(&sh->s_full[buf], (tc >> 1) & 1)) {
+                    ok = false;
+                    break;
+                }
+                tc_fence_after();
+                __syncwarp();
+                uint32_t sr[RC];
+                tmem_load_cols<RC>(tm_lane + buf * R + r0, sr);
+                tmem_ld_wait();
+                tc_fence_before();
+                __syncwarp();
+                if (lane == 0) mbar_arrive(&sh->s_empty[buf]);
+                float s[RC];
+#pragma unroll
+                for (int r = 0; r < RC; ++r) s[r] = __uint_as_float(sr[r]) * a.scale_log2;
+                const int key = t * kTcKeys + kl;  // key index within the request
+                if (key >= kv) {
+                    // block keys and the tail: the causal limit of each row
+#pragma unroll
+                    for (int r = 0; r < RC; ++r)
+                        if (key > lim[r0 + r]) s[r] = -INFINITY;
+                    if (key >= total && cg == 0) {
+                        // a V row past the request's keys may hold anything:
+                        // zero it so that 0 * V stays 0 in the second product
+                        uint4* vr = reinterpret_cast<uint4*>(sV + kst * 2 * kTcHalf + kl * 128);
+#pragma unroll
+                        for (int j = 0; j < 8; ++j) {
+                            vr[j] = make_uint4(0, 0, 0, 0);
+                            vr[j + kTcHalf / 16] = make_uint4(0, 0, 0, 0);
+                        }
+                    }
+                }
+                bool need = false;
+#pragma unroll
+                for (int r = 0; r < RC; ++r) need |= s[r] > m_ref[r] + 8.f;
+                if (group_or<kSoft>(need)) {
+                    // exact row maxima of this tile; move the references that it beats by > 2^8
+#pragma unroll
+                    for (int r = 0; r < RC; ++r) {
+                        float mx = s[r];
+#pragma unroll
+                        for (int off = 16; off > 0; off >>= 1)
+                            mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, off));
+                        if (lane == 0) red_m[(cg * 4 + q4) * RC + r] = mx;
+                    }
+                    group_sync<kSoft>();
+                    const float* rm = red_m + cg * 4 * RC;
+                    float alpha[RC];
+                    bool rescale = false;
+#pragma unroll
+                    for (int r = 0; r < RC; ++r) {
+                        const float mx = fmaxf(fmaxf(rm[r], rm[RC + r]), fmaxf(rm[2 * RC + r], rm[3 * RC + r]));
+                        alpha[r] = 1.f;
+                        if (mx > m_ref[r] + 8.f) {
+                            if (m_ref[r] != -INFINITY) {
+                                alpha[r] = exp2f(m_ref[r] - mx);
+                                rescale = true;
+                            }
+                            m_ref[r] = mx;
+                        }
+                        l_part[r] *= alpha[r];
+                    }
+                    // O^T (thread = d, column = row) is rescaled once the
+                    // previous tile's product is complete
+                    if (t > t0 && group_or<kSoft>(rescale)) {
+                        const int tp = tc - 1;
+                        if (!group_wait(&sh->p_empty[tp & 1], (tp >> 1) & 1)) {
+                            ok = false;
+                            break;
+                        }
+                        tc_fence_after();
+                        __syncwarp();
+                        if (rescale) {  // uniform within the warp (same rows)
+                            uint32_t ov[RC];
+                            tmem_load_cols<RC>(tm_lane + 2 * R + r0, ov);
+                            tmem_ld_wait();
+#pragma unroll
+                            for (int r = 0; r < RC; ++r)
+                                ov[r] = __float_as_uint(__uint_as_float(ov[r]) * alpha[r]);
+                            tmem_store_cols<RC>(tm_lane + 2 * R + r0, ov);
+                            tmem_st_wait();
+                        }
+                        tc_fence_before();
+                    }
+                }
+                // P^T[row][key] = 2^(s - m_ref) as bf16, 128-byte-swizzled rows
+                if (tc >= 2 && !group_wait(&sh->p_empty[buf], ((tc - 2) >> 1) & 1)) {
+                    ok = false;
+                    break;
+                }
+                unsigned char* pcol = p_col + buf * kPBytes + r0 * 128;
+#pragma unroll
+                for (int r = 0; r < RC; ++r) {
+                    const float m_use = m_ref[r] == -INFINITY ? 0.f : m_ref[r];
+                    const float p = exp2f(s[r] - m_use);
+                    l_part[r] += p;
+                    *reinterpret_cast<__nv_bfloat16*>(pcol + r * 128 + ((p_chunk ^ (r & 7)) << 4)) =
+                        __float2bfloat16_rn(p);
+                }
+                asm volatile("fence.proxy.async.shared::cta;\n" ::: "memory");
+                __syncwarp();
+                if (lane == 0) mbar_arrive(&sh->p_full[buf]);
+                ++tc;
+                if (++kst == STAGES) kst = 0;
+            }
+            if (!ok) break;
+
+            // ---- end of this CTA's piece of unit u: row sums, O^T, output
+#pragma unroll
+            for (int r = 0; r < RC; ++r) {
+                float v = l_part[r];
+#pragma unroll
+                for (int off = 16; off > 0; off >>= 1) v += __shfl_xor_sync(0xffffffffu, v, off);
+                if (lane == 0) red_l[(cg * 4 + q4) * RC + r] = v;
+            }
+            if (!group_wait(&sh->o_full, o_use & 1)) {  // also orders red_l
+                ok = false;
+                break;
+            }
+            ++o_use;
+            tc_fence_after();
+            __syncwarp();
+            uint32_t ov[RC];
+            tmem_load_cols<RC>(tm_lane + 2 * R + r0, ov);
+            tmem_ld_wait();
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&sh->o_empty);
+            const float* rl = red_l + cg * 4 * RC;
+            float lt[RC];
+#pragma unroll
+            for (int r = 0; r < RC; ++r) lt[r] = (rl[r] + rl[RC + r]) + (rl[2 * RC + r] + rl[3 * RC + r]);
+            const int d = kl;
+            // output rows are staged as bf16 [rows][128] in the P buffers (free
+            // until the next P write, which follows a group barrier) and then
+            // written with 16-byte stores
+            __nv_bfloat16* sO = reinterpret_cast<__nv_bfloat16*>(sP);
+            // CTAs whose ranges meet unit u: first .. last (all non-empty)
+            const long long TL = T;
+            const int first = (int)(((long long)(us + 1) * G + TL - 1) / TL) - 1;
+            const int last = (int)(((long long)ue * G + TL - 1) / TL) - 1;
+            const int npieces = last - first + 1;
+            bool write_out = true;
+            if (npieces == 1) {
+#pragma unroll
+                for (int r = 0; r < RC; ++r) {
+                    const bool live = lim[r0 + r] >= 0 && lt[r] > 0.f;  // active row with keys
+                    const float inv = live ? __frcp_rn(lt[r]) : 0.f;
+                    sO[(r0 + r) * 128 + d] = __float2bfloat16_rn(__uint_as_float(ov[r]) * inv);
+                }
+            } else {
+                // partial slot: 0 for the first unit of a CTA's range, 1 for its last
+                auto slot_of = [&](int cta) {
+                    return (cta > first || (long long)T * cta / G == us) ? 0 : 1;
+                };
+                auto part_of = [&](int cta) {
+                    return a.part + ((size_t)cta * 2 + slot_of(cta)) * a.part_stride;
+                };
+                float* pb = part_of(blockIdx.x);
+#pragma unroll
+                for (int r = 0; r < RC; ++r) pb[2 * R + (r0 + r) * 128 + d] = __uint_as_float(ov[r]);
+                if (kl == 0) {
+#pragma unroll
+                    for (int r = 0; r < RC; ++r) {
+                        pb[r0 + r] = m_ref[r];
+                        pb[R + r0 + r] = lt[r];
+                    }
+                }
+                __threadfence();
+                bool is_last = false;
+                group_sync<kSoft>();
+                if (et == 0) is_last = atomicAdd(&a.ticket[u], 1) == npieces - 1;
+                write_out = group_or<kSoft>(is_last);
+                if (write_out) {
+                    __threadfence();
+                    // online merge in CTA order, up to 4 partials at a time:
+                    // their maxima and sums go through shared memory, the O
+                    // values of this thread's rows are loaded in one batch
+                    float Mr[RC], Lr[RC], Or[RC];
+#pragma unroll
+                    for (int r = 0; r < RC; ++r) {
+                        Mr[r] = -INFINITY;
+                        Lr[r] = 0.f;
+                        Or[r] = 0.f;
+                    }
+                    for (int k0 = 0; k0 < npieces; k0 += 4) {
+                        const int kn = min(4, npieces - k0);
+                        group_sync<kSoft>();  // the previous chunk is consumed
+                        for (int i = et; i < kn * R; i += kSoft) {
+                            const float* pk = part_of(first + k0 + i / R);
+                            red_m[i] = __ldcg(pk + i % R);
+                            red_l[i] = __ldcg(pk + R + i % R);
+                        }
+                        group_sync<kSoft>();
+                        for (int k = 0; k < kn; ++k) {
+                            const float* pk = part_of(first + k0 + k);
+                            float okv[RC];
+#pragma unroll
+                            for (int r = 0; r < RC; ++r) okv[r] = __ldcg(pk + 2 * R + (size_t)(r0 + r) * 128 + d);
+#pragma unroll
+                            for (int r = 0; r < RC; ++r) {
+                                const float mk = red_m[k * R + r0 + r], lk = red_l[k * R + r0 + r];
+                                const float mn = fmaxf(Mr[r], mk);
+                                const float mu = mn == -INFINITY ? 0.f : mn;
+                                const float fa = exp2f(Mr[r] - mu), fb = exp2f(mk - mu);
+                                Lr[r] = Lr[r] * fa + lk * fb;
+                                Or[r] = Or[r] * fa + okv[r] * fb;
+                                Mr[r] = mn;
+                            }
+                        }
+                    }
+#pragma unroll
+                    for (int r = 0; r < RC; ++r) {
+                        const bool live = lim[r0 + r] >= 0 && Lr[r] > 0.f;
+                        const float inv = live ? __frcp_rn(Lr[r]) : 0.f;
+                        sO[(r0 + r) * 128 + d] = __float2bfloat16_rn(Or[r] * inv);
+                    }
+                    if (et == 0) a.ticket[u] = 0;
+                }
+            }
+            if (write_out) {
+                group_sync<kSoft>();
+                for (int i = et; i < a.rows * 16; i += kSoft) {
+                    const int r = i >> 4, ch = i & 15;
+                    const int slot = r / a.grp, hh = r - slot * a.grp;
+                    const uint4 v = *reinterpret_cast<const uint4*>(sO + r * 128 + ch * 8);
+                    *reinterpret_cast<uint4*>(a.out + ((size_t)b * a.Q + slot) * a.Hq * 128 +
+                                              (size_t)(g * a.grp + hh) * 128 + ch * 8) = v;
+                }
+            }
+            // lim and the staged rows are rewritten only after the next group barrier
+            group_sync<kSoft>();
+            tile = us + t1;
+        }
+    }
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 1) {
+        __syncwarp();
+        tc_fence_after();
+        tmem_dealloc(tmem, kTmemCols);
+    }
+}
+
+bool encode_bf16_4d(CUtensorMap* m, const void* ptr, const uint64_t dims[4],
+                    const uint64_t strides_bytes[3], const uint32_t box[4]) {
+    EncodeTiledFn fn = get_encode_fn();
+    if (!fn) return false;
+    cuuint64_t gd[4] = {dims[0], dims[1], dims[2], dims[3]};
+    cuuint64_t gs[3] = {strides_bytes[0], strides_bytes[1], strides_bytes[2]};
+    cuuint32_t bx[4] = {box[0], box[1], box[2], box[3]};
+    cuuint32_t es[4] = {1, 1, 1, 1};
+    return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, const_cast<void*>(ptr), gd, gs, bx, es,
+              CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+              CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+template <int R, int STAGES>
+cudaError_t launch_tc(const TcArgs& a, const CUtensorMap& tk, const CUtensorMap& tv,
+                      const CUtensorMap& tq, size_t smem, cudaStream_t st) {
+    static unsigned long long configured = 0;  // bit per device
+    int dev = 0;
+    cudaGetDevice(&dev);
+    if (dev < 0 || dev >= 64) return cudaErrorInvalidDevice;
+    if (!(configured >> dev & 1ull)) {
+        int optin = 0;
+        cudaDeviceGetAttribute(&optin, cudaDevAttrMaxSharedMemoryPerBlockOptin, dev);
+        const cudaError_t e = cudaFuncSetAttribute(attention_tc_kernel<R, STAGES>,
+                                                   cudaFuncAttributeMaxDynamicSharedMemorySize, optin);
+        if (e != cudaSuccess) return e;
+        configured |= 1ull << dev;
+    }
+    attention_tc_kernel<R, STAGES><<<kNumSMs, TcRoles<R>::kThreads, smem, st>>>(tk, tv, tq, a);
+    return cudaGetLastError();
+}
+
+}  // namespace
+
+// Tensor-core attention for D = 128, block rows per kv head <= 64 and pages
+// of 8..128 tokens dividing 128.  Sets *handled = false (and launches
+// nothing) when the shape or the device does not fit; the caller then uses
+// the general kernel.
+cudaError_t launch_attention_tc(const Plan& p, const isd_dims* d, const uint16_t* q,
+                                const uint16_t* k_new, const uint16_t* v_new, uint16_t* k_pool,
+                                uint16_t* v_pool, const int32_t* page_table, const int32_t* kv_len,
+                                const int32_t* n_clean, uint16_t* out, void* ws, int32_t* err_flag,
+                                cudaStream_t st, bool* handled) {
+    *handled = false;
+    const int R = p.attn_tc_rows;
+    if (R == 0) return cudaSuccess;
+    int dev = 0, optin = 0;
+    cudaGetDevice(&dev);
+    cudaDeviceGetAttribute(&optin, cudaDevAttrMaxSharedMemoryPerBlockOptin, dev);
+    const size_t extra = 1024 + (size_t)(d->B * d->Hkv + 1) * 4;  // alignment slack + tile prefix
+    int stages = 0;
+    size_t smem = 0;
+    for (int s = 3; s >= 2 && !stages; --s) {
+        size_t f = 0;
+        if (R == 16) f = s == 3 ? tc_smem_fixed<16, 3>() : tc_smem_fixed<16, 2>();
+        if (R == 32) f = s == 3 ? tc_smem_fixed<32, 3>() : tc_smem_fixed<32, 2>();
+        if (R == 64) f = s == 3 ? tc_smem_fixed<64, 3>() : tc_smem_fixed<64, 2>();
+        if (f + extra <= (size_t)optin) {
+            stages = s;
+            smem = f + extra;
+        }
+    }
+    if (!stages || !get_encode_fn()) return cudaSuccess;
+    const int Q = p.Q, P = d->page_size, Hkv = d->Hkv, Hq = d->Hq;
+    CUtensorMap tk, tv, tq;
+    {
+        const uint64_t dims[4] = {128, (uint64_t)Hkv, (uint64_t)P, (uint64_t)d->num_pages};
+        const uint64_t strides[3] = {256, (uint64_t)Hkv * 256, (uint64_t)P * Hkv * 256};
+        const uint32_t box[4] = {64, 1, (uint32_t)P, 1};
+        if (!encode_bf16_4d(&tk, k_pool, dims, strides, box) ||
+            !encode_bf16_4d(&tv, v_pool, dims, strides, box))
+            return cudaSuccess;
+    }
+    {
+        const uint64_t dims[4] = {128, (uint64_t)Hq, (uint64_t)Q, (uint64_t)d->B};
+        const uint64_t strides[3] = {256, (uint64_t)Hq * 256, (uint64_t)Q * Hq * 256};
+        const uint32_t box[4] = {64, (uint32_t)p.grp, (uint32_t)Q, 1};
+        if (!encode_bf16_4d(&tq, q, dims, strides, box)) return cudaSuccess;
+    }
+    *handled = true;
+    TcArgs a;
+    a.B = d->B;
+    a.N = d->N;
+    a.Q = Q;
+    a.Hq = Hq;
+    a.Hkv = Hkv;
+    a.grp = p.grp;
+    a.rows = p.rows;
+    a.P = P;
+    a.num_pages = d->num_pages;
+    a.max_pages = d->max_pages_per_req;
+    a.scale_log2 = d->sm_scale * 1.4426950408889634f;
+    a.page_table = page_table;
+    a.kv_len = kv_len;
+    a.n_clean = n_clean;
+    a.out = reinterpret_cast<__nv_bfloat16*>(out);
+    a.part = reinterpret_cast<float*>(static_cast<char*>(ws) + p.off_attn_part);
+    a.part_stride = p.attn_tc_part_stride;
+    a.ticket = reinterpret_cast<int*>(static_cast<char*>(ws) + p.off_attn_ticket);
+    a.err_flag = err_flag;
+    kv_append_kernel<<<d->B, 256, 0, st>>>(a, reinterpret_cast<const __nv_bfloat16*>(k_new),
+                                           reinterpret_cast<const __nv_bfloat16*>(v_new),
+                                           reinterpret_cast<__nv_bfloat16*>(k_pool),
+                                           reinterpret_cast<__nv_bfloat16*>(v_pool));
+    cudaError_t e = cudaGetLastError();
+    if (e != cudaSuccess) return e;
+    if (R == 16) return stages == 3 ? launch_tc<16, 3>(a, tk, tv, tq, smem, st) : launch_tc<16, 2>(a, tk, tv, tq, smem, st);
+    if (R == 32) return stages == 3 ? launch_tc<32, 3>(a, tk, tv, tq, smem, st) : launch_tc<32, 2>(a, tk, tv, tq, smem, st);
+    return stages == 3 ? launch_tc<64, 3>(a, tk, tv, tq, smem, st) : launch_tc<64, 2>(a, tk, tv, tq, smem, st);
+}
+
+}  // namespace isd

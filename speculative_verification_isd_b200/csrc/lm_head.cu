@@ -29,6 +29,7 @@
 #include "common.cuh"
 #include "plan.h"
 #include "sm100.cuh"
+#include "tmap.h"
 
 namespace isd {
 
@@ -305,25 +306,6 @@ lm_head_kernel(const __grid_constant__ CUtensorMap tmap_w, const __grid_constant
 // ---------------------------------------------------------------------------
 // host side
 // ---------------------------------------------------------------------------
-typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
-                                  const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
-                                  const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
-                                  CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
-
-static EncodeTiledFn get_encode_fn() {
-    static EncodeTiledFn fn = nullptr;
-    if (!fn) {
-        void* p = nullptr;
-        cudaDriverEntryPointQueryResult q;
-        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) !=
-                cudaSuccess ||
-            q != cudaDriverEntryPointSuccess)
-            return nullptr;
-        fn = reinterpret_cast<EncodeTiledFn>(p);
-    }
-    return fn;
-}
-
 // 2-D bf16 [rows, cols] row-major tensor, box = 64 columns x box_rows rows, 128B swizzle.
 static bool encode_bf16_2d(CUtensorMap* m, const void* ptr, uint64_t rows, uint64_t cols,
                            uint32_t box_rows) {

@@ -26,6 +26,10 @@ struct Plan {
     int attn_split;          // keys per split (multiple of kAttnKeyTile)
     int attn_max_splits;     // splits for the longest possible request
     size_t attn_part_stride; // bytes of one split's partial
+    // tensor-core attention (D = 128, pages dividing 128 keys, <= 64 rows):
+    // rows padded to the MMA N (16, 32 or 64), 0 when the shape does not fit
+    int attn_tc_rows;
+    int attn_tc_part_stride; // floats of one partial (per CTA and slot)
     // statistics / accept
     int stats_chunks, stats_chunk_len;
     int acc_chunks;
@@ -68,6 +72,12 @@ inline bool make_plan(const isd_dims* d, Plan* p) {
     p->attn_max_splits = (int)((max_ctx + split - 1) / split);
     if (p->attn_max_splits < 1) p->attn_max_splits = 1;
     p->attn_part_stride = align_up((size_t)rows_per_cta * d->D * 4 + (size_t)rows_per_cta * 8, 256);
+    const int P = d->page_size;
+    const bool tc_pages = P == 8 || P == 16 || P == 32 || P == 64 || P == 128;
+    p->attn_tc_rows = 0;
+    if (d->D == 128 && tc_pages && p->rows <= 64)
+        p->attn_tc_rows = p->rows <= 16 ? 16 : (p->rows <= 32 ? 32 : 64);
+    p->attn_tc_part_stride = 2 * p->attn_tc_rows + 128 * p->attn_tc_rows;
     // row statistics: enough CTAs to fill the GPU, chunks of >= 2048 entries
     int target = (kNumSMs * 8 + p->M - 1) / p->M;
     int max_chunks = (d->V + 2047) / 2048;
@@ -94,7 +104,12 @@ inline bool make_plan(const isd_dims* d, Plan* p) {
         return o;
     };
     const size_t n_units = (size_t)d->B * d->Hkv * p->attn_rgb;
-    p->off_attn_part = take(n_units * p->attn_max_splits * p->attn_part_stride);
+    // split partials of the general kernel, or two partials per persistent
+    // CTA of the tensor-core kernel: whichever is larger
+    size_t part_bytes = n_units * p->attn_max_splits * p->attn_part_stride;
+    const size_t tc_bytes = (size_t)kNumSMs * 2 * p->attn_tc_part_stride * 4;
+    if (tc_bytes > part_bytes) part_bytes = tc_bytes;
+    p->off_attn_part = take(part_bytes);
     p->off_attn_ticket = take(n_units * 4);
     p->off_hidden = take((size_t)p->M * p->H * 2);
     p->off_hidden_lora = take(d->lora_rank ? (size_t)p->M * p->H * 2 : 0);
