@@ -45,6 +45,10 @@ void set_error_detail(const char* msg);
 namespace {
 
 constexpr int kTcKeys = 128;            // keys per tile (M of S^T)
+// A (request, kv head) also costs an epilogue: the partition counts it as
+// this many extra tiles, so CTAs whose ranges hold many short requests get
+// fewer tiles.
+constexpr int kTcUnitCost = 4;
 constexpr int kTcHalf = kTcKeys * 128;  // bytes of one 64-d half of a K or V tile
 constexpr uint64_t kTcWaitNs = 2000000000ull;
 
@@ -113,11 +117,17 @@ __global__ void kv_append_kernel(TcArgs a, const __nv_bfloat16* k_new, const __n
 template <int STAGES>
 struct TcShared {
     uint64_t kv_full[STAGES], kv_empty[STAGES];
-    uint64_t s_full[2], s_empty[2], p_full[2], p_empty[2];
-    uint64_t o_full, o_empty, q_full, q_empty, drain;
+    uint64_t s_full[2], s_empty[2], p_full, p_empty;
+    uint64_t o_full, o_empty, q_full[2], q_empty[2], drain;
     uint32_t tmem;
     int abort_flag;
     int never;
+};
+
+// A CTA's share of one (request, kv head) unit: tiles [t0, t1) of unit u,
+// whose position on the partition axis starts at us.
+struct TcPiece {
+    int u, us, t0, t1, b, g;
 };
 
 // Softmax warps: 4 per column group (one per TMEM lane quarter); each
@@ -135,12 +145,14 @@ struct TcRoles {
 template <int R, int STAGES>
 constexpr size_t tc_smem_fixed() {
     return (size_t)STAGES * 4 * kTcHalf    // K and V stages
-           + 2 * R * 128                   // Q (two 64-d halves)
-           + 2 * 2 * R * 128               // P^T, two buffers of two 64-key halves
+           + 2 * 2 * R * 128               // Q, two buffers of two 64-d halves
+           + 2 * R * 128                   // P^T (two 64-key halves); output staging
            + 4 * R * 4 * 2                 // per-warp row maxima and row sums
            + R * 4                         // per-row causal key limit
            + sizeof(TcShared<STAGES>);
 }
+// plus, per launch: 3 ints per request (kv_len, n_clean, keys) and
+// B * Hkv + 1 ints of unit offsets on the partition axis
 
 // named barrier 1 over the NT softmax threads, OR of a predicate
 template <int NT>
@@ -183,13 +195,16 @@ attention_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_const
         (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     unsigned char* sK = smem;
     unsigned char* sV = sK + STAGES * 2 * kTcHalf;
-    unsigned char* sQ = sV + STAGES * 2 * kTcHalf;
-    unsigned char* sP = sQ + kQBytes;
-    float* red_m = reinterpret_cast<float*>(sP + 2 * kPBytes);  // [4][R]
-    float* red_l = red_m + 4 * R;                                // [4][R]
-    int* lim = reinterpret_cast<int*>(red_l + 4 * R);            // [R]
+    unsigned char* sQ = sV + STAGES * 2 * kTcHalf;  // two buffers
+    unsigned char* sP = sQ + 2 * kQBytes;
+    float* red_m = reinterpret_cast<float*>(sP + kPBytes);   // [4][R]
+    float* red_l = red_m + 4 * R;                             // [4][R]
+    int* lim = reinterpret_cast<int*>(red_l + 4 * R);         // [R]
     TcShared<STAGES>* sh = reinterpret_cast<TcShared<STAGES>*>(lim + R);
-    int* prefix = reinterpret_cast<int*>(sh + 1);                // [B*Hkv + 1]
+    int* kvs = reinterpret_cast<int*>(sh + 1);                // [B] kv_len
+    int* cs = kvs + a.B;                                      // [B] n_clean
+    int* tots = cs + a.B;                                     // [B] keys (0: not served)
+    int* prefix = tots + a.B;                                 // [B*Hkv + 1]
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int n_units = a.B * a.Hkv;
@@ -203,13 +218,13 @@ attention_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_const
         for (int i = 0; i < 2; ++i) {
             mbar_init(&sh->s_full[i], 1);
             mbar_init(&sh->s_empty[i], 4 * CG);
-            mbar_init(&sh->p_full[i], 4 * CG);
-            mbar_init(&sh->p_empty[i], 1);
+            mbar_init(&sh->q_full[i], 1);
+            mbar_init(&sh->q_empty[i], 1);
         }
+        mbar_init(&sh->p_full, 4 * CG);
+        mbar_init(&sh->p_empty, 1);
         mbar_init(&sh->o_full, 1);
         mbar_init(&sh->o_empty, 4 * CG);
-        mbar_init(&sh->q_full, 1);
-        mbar_init(&sh->q_empty, 1);
         mbar_init(&sh->drain, 1);
         sh->abort_flag = 0;
         sh->never = 0;
@@ -223,21 +238,29 @@ attention_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_const
         tmem_relinquish();
     }
     // Q rows past `rows` stay zero (no TMA box covers them)
-    for (int i = threadIdx.x; i < (int)(kQBytes / 16); i += kThreads)
+    for (int i = threadIdx.x; i < (int)(2 * kQBytes / 16); i += kThreads)
         reinterpret_cast<uint4*>(sQ)[i] = make_uint4(0, 0, 0, 0);
+    for (int b = threadIdx.x; b < a.B; b += kThreads) {
+        kvs[b] = a.kv_len[b];
+        cs[b] = a.n_clean[b];
+        tots[b] = tc_total_keys(a, b);
+    }
+    __syncthreads();
     if (warp == 0) {
-        // prefix[u] = tiles of the units before u (unit u = request u / Hkv, kv head u % Hkv)
+        // prefix[u]: start of unit u (request u / Hkv, kv head u % Hkv) on the
+        // partition axis, where a unit of nt > 0 tiles takes nt + kTcUnitCost
         int run = 0;
         for (int u0 = 0; u0 < n_units; u0 += 32) {
             const int u = u0 + lane;
-            const int nt = u < n_units ? (tc_total_keys(a, u / a.Hkv) + kTcKeys - 1) / kTcKeys : 0;
-            int incl = nt;
+            const int nt = u < n_units ? (tots[u / a.Hkv] + kTcKeys - 1) / kTcKeys : 0;
+            const int w = nt > 0 ? nt + kTcUnitCost : 0;
+            int incl = w;
 #pragma unroll
             for (int off = 1; off < 32; off <<= 1) {
                 const int v = __shfl_up_sync(0xffffffffu, incl, off);
                 if (lane >= off) incl += v;
             }
-            if (u < n_units) prefix[u] = run + incl - nt;
+            if (u < n_units) prefix[u] = run + incl - w;
             run += __shfl_sync(0xffffffffu, incl, 31);
         }
         if (lane == 0) prefix[n_units] = run;
@@ -248,20 +271,40 @@ attention_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_const
     tc_fence_after();
     const uint32_t tmem = sh->tmem;
     const int T = prefix[n_units];
-    const int G = (int)gridDim.x < T ? (int)gridDim.x : T;  // every active CTA gets >= 1 tile
+    const int G = (int)gridDim.x < T ? (int)gridDim.x : T;
     const bool active = (int)blockIdx.x < G;
     const int my0 = active ? (int)((long long)T * blockIdx.x / G) : 0;
     const int my1 = active ? (int)((long long)T * (blockIdx.x + 1) / G) : 0;
     volatile int* abort_flag = &sh->abort_flag;
 
-    // unit holding `tile`: the largest u with prefix[u] <= tile
-    auto unit_of = [&](int tile) {
+    // unit holding partition position pos: the largest u with prefix[u] <= pos
+    auto unit_of = [&](int pos) {
         int lo = 0, hi = n_units;
         while (hi - lo > 1) {
             const int mid = (lo + hi) >> 1;
-            if (prefix[mid] <= tile) lo = mid; else hi = mid;
+            if (prefix[mid] <= pos) lo = mid; else hi = mid;
         }
         return lo;
+    };
+    auto unit_tiles = [&](int u) { return (tots[u / a.Hkv] + kTcKeys - 1) / kTcKeys; };
+    // the first piece of this CTA at or after position pos (positions past a
+    // unit's tiles are its epilogue share and hold no tile)
+    auto piece_from = [&](int pos, TcPiece& pc) {
+        while (pos < my1) {
+            const int u = unit_of(pos);
+            const int us = prefix[u], nt = unit_tiles(u);
+            if (pos - us < nt) {
+                pc.u = u;
+                pc.us = us;
+                pc.t0 = pos - us;
+                pc.t1 = min(us + nt, my1) - us;
+                pc.b = u / a.Hkv;
+                pc.g = u - pc.b * a.Hkv;
+                return true;
+            }
+            pos = prefix[u + 1];
+        }
+        return false;
     };
     auto give_up = [&]() {
         *abort_flag = 1;
@@ -273,54 +316,60 @@ attention_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_const
             // ------------------------------------------------ TMA producer
             // The whole warp walks the tiles: page ids come in chunks of 32
             // (lane i holds one), the next chunk's load in flight while the
-            // current one is issued; lane 0 waits and issues the copies.
+            // current one is issued, and the next piece's first chunk in
+            // flight during the current piece; lane 0 waits on the rings, and
+            // the copies of a tile are issued one box per lane (issuing them
+            // from a single thread caps the copy rate with small pages).
             const uint64_t pol_kv = policy_evict_first();  // each K/V byte is read once
             const uint64_t pol_q = policy_evict_last();
             const int np = kTcKeys / a.P;  // pages per tile (<= 16)
-            int st = 0;
-            uint32_t ph = 0, q_use = 0, armed = 0, armed_par = 0;
+            const int tpc = 32 / np;       // tiles per chunk of page ids
+            // page id of page tc0 * np + lane of the piece's request; pages
+            // past the request (or bad ids) read as zeros
+            auto load_ids = [&](const TcPiece& q, int tc0) {
+                const int pidx = tc0 * np + lane;
+                const int need = (tots[q.b] + a.P - 1) / a.P;
+                int id = -1;
+                if (pidx < need) {
+                    id = __ldg(a.page_table + (size_t)q.b * a.max_pages + pidx);
+                    if (id < 0 || id >= a.num_pages) {
+                        raise_flag(a.err_flag, ISD_FLAG_PAGE_OOB);
+                        id = -1;
+                    }
+                }
+                return id;
+            };
+            int st = 0, pi = 0;
+            uint32_t ph = 0, armed = 0, armed_par = 0;
             bool ok = true;
-            for (int tile = my0; ok && tile < my1;) {
-                const int u = unit_of(tile);
-                const int us = prefix[u], ue = prefix[u + 1];
-                const int t0 = tile - us, t1 = min(ue, my1) - us;
-                const int b = u / a.Hkv, g = u % a.Hkv;
-                const int need_pages = (tc_total_keys(a, b) + a.P - 1) / a.P;
+            TcPiece pc;
+            bool has = piece_from(my0, pc);
+            int ids_first = has ? load_ids(pc, pc.t0) : -1;
+            while (ok && has) {
+                TcPiece nx;
+                const bool has_nx = piece_from(pc.us + pc.t1, nx);
+                const int qb = pi & 1;
                 if (lane == 0) {
-                    ok = mbar_wait_bounded(&sh->q_empty, (q_use & 1) ^ 1, abort_flag, kTcWaitNs);
+                    ok = mbar_wait_bounded(&sh->q_empty[qb], ((pi >> 1) & 1) ^ 1, abort_flag, kTcWaitNs);
                     if (!ok) {
                         give_up();
                     } else {
-                        mbar_arrive_expect_tx(&sh->q_full, (uint32_t)a.rows * 256u);
-                        tma_load_4d(sQ, &tm_q, &sh->q_full, 0, g * a.grp, 0, b, pol_q);
-                        tma_load_4d(sQ + R * 128, &tm_q, &sh->q_full, 64, g * a.grp, 0, b, pol_q);
+                        mbar_arrive_expect_tx(&sh->q_full[qb], (uint32_t)a.rows * 256u);
+                        unsigned char* qd = sQ + qb * kQBytes;
+                        tma_load_4d(qd, &tm_q, &sh->q_full[qb], 0, pc.g * a.grp, 0, pc.b, pol_q);
+                        tma_load_4d(qd + R * 128, &tm_q, &sh->q_full[qb], 64, pc.g * a.grp, 0, pc.b, pol_q);
                     }
                 }
                 ok = __shfl_sync(0xffffffffu, ok, 0);
                 if (!ok) break;
-                ++q_use;
-                const int32_t* ptab = a.page_table + (size_t)b * a.max_pages;
-                const int tpc = 32 / np;  // tiles per chunk of page ids
-                // page id of page (first tile of the chunk) * np + lane; pages
-                // past the request (or bad ids) read as zeros
-                auto load_ids = [&](int tc0) {
-                    const int pidx = tc0 * np + lane;
-                    int id = -1;
-                    if (pidx < need_pages) {
-                        id = __ldg(ptab + pidx);
-                        if (id < 0 || id >= a.num_pages) {
-                            raise_flag(a.err_flag, ISD_FLAG_PAGE_OOB);
-                            id = -1;
-                        }
-                    }
-                    return id;
-                };
-                int ids = load_ids(t0), ids_next = load_ids(t0 + tpc);
-                for (int t = t0; t < t1; ++t) {
-                    const int j = (t - t0) % tpc;  // tile within the chunk
-                    if (j == 0 && t > t0) {
+                ++pi;
+                int ids = ids_first, ids_next = load_ids(pc, pc.t0 + tpc);
+                const int ids_nx = has_nx ? load_ids(nx, nx.t0) : -1;
+                for (int t = pc.t0; t < pc.t1; ++t) {
+                    const int j = (t - pc.t0) % tpc;  // tile within the chunk
+                    if (j == 0 && t > pc.t0) {
                         ids = ids_next;
-                        ids_next = load_ids(t + tpc);
+                        ids_next = load_ids(pc, t + tpc);
                     }
                     if (lane == 0) {
                         ok = mbar_wait_bounded(&sh->kv_empty[st], ph ^ 1, abort_flag, kTcWaitNs);
@@ -331,14 +380,16 @@ attention_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_const
                     if (!ok) break;
                     unsigned char* k_dst = sK + st * 2 * kTcHalf;
                     unsigned char* v_dst = sV + st * 2 * kTcHalf;
-                    for (int pg = 0; pg < np; ++pg) {
-                        const int page = __shfl_sync(0xffffffffu, ids, j * np + pg);
-                        if (lane == 0) {
-                            const int off = pg * a.P * 128;
-                            tma_load_4d(k_dst + off, &tm_k, &sh->kv_full[st], 0, g, 0, page, pol_kv);
-                            tma_load_4d(k_dst + kTcHalf + off, &tm_k, &sh->kv_full[st], 64, g, 0, page, pol_kv);
-                            tma_load_4d(v_dst + off, &tm_v, &sh->kv_full[st], 0, g, 0, page, pol_kv);
-                            tma_load_4d(v_dst + kTcHalf + off, &tm_v, &sh->kv_full[st], 64, g, 0, page, pol_kv);
+                    // one box per lane: page lane / 4 of the tile, K or V, 64-d
+                    // half (the expect_tx above precedes them in program order)
+                    for (int box0 = 0; box0 < 4 * np; box0 += 32) {
+                        const int box = box0 + lane;
+                        const int pg = box < 4 * np ? box >> 2 : 0, kind = box & 3;
+                        const int page = __shfl_sync(0xffffffffu, ids, (j * np + pg) & 31);
+                        if (box < 4 * np) {
+                            const int off = pg * a.P * 128 + (kind & 1) * kTcHalf;
+                            tma_load_4d((kind & 2 ? v_dst : k_dst) + off, kind & 2 ? &tm_v : &tm_k,
+                                        &sh->kv_full[st], (kind & 1) * 64, pc.g, 0, page, pol_kv);
                         }
                     }
                     armed |= 1u << st;
@@ -348,14 +399,17 @@ attention_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_const
                         ph ^= 1;
                     }
                 }
-                tile = us + t1;
+                ids_first = ids_nx;
+                pc = nx;
+                has = has_nx;
             }
             // drain: every armed copy has landed before the CTA may exit
             if (lane == 0) {
                 for (int s = 0; s < STAGES; ++s)
                     if (armed >> s & 1)
                         mbar_wait_bounded(&sh->kv_full[s], armed_par >> s & 1, &sh->never, kTcWaitNs);
-                if (q_use) mbar_wait_bounded(&sh->q_full, (q_use - 1) & 1, &sh->never, kTcWaitNs);
+                for (int k = pi - 1; k >= 0 && k >= pi - 2; --k)
+                    mbar_wait_bounded(&sh->q_full[k & 1], (k >> 1) & 1, &sh->never, kTcWaitNs);
             }
         }
     } else if (warp == 1) {
@@ -363,7 +417,7 @@ attention_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_const
             // ------------------------------------------------ MMA issuer
             constexpr uint32_t idesc_s = idesc_bf16_f32(128, R);
             constexpr uint32_t idesc_o = idesc_bf16_f32(128, R) | (1u << 15);  // A = V^T, MN-major
-            const uint64_t dq = smem_desc_sw128(smem_u32(sQ));
+            const uint64_t dq0 = smem_desc_sw128(smem_u32(sQ));
             const uint64_t dk = smem_desc_sw128(smem_u32(sK));
             const uint64_t dp = smem_desc_sw128(smem_u32(sP));
             // V^T as an MN-major operand: the two 64-d blocks are kTcHalf apart
@@ -377,7 +431,9 @@ attention_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_const
             int s_tc = 0, s_st = 0;    // S products issued; stage of the next one
             uint32_t s_ph = 0;
             int pv_tc = 0, pv_st = 0;  // PV products issued; stage of the next one
-            uint32_t q_use = 0, o_use = 0;
+            int pi = 0;                // pieces started
+            uint32_t o_use = 0;
+            uint64_t dq = dq0;
             bool ok = true;
             auto wait = [&](uint64_t* bar, uint32_t par) {
                 if (mbar_try_wait(bar, par) || mbar_wait_bounded(bar, par, abort_flag, kTcWaitNs))
@@ -413,13 +469,14 @@ attention_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_const
                 issue_s();
                 return true;
             };
-            for (int tile = my0; ok && tile < my1;) {
-                const int u = unit_of(tile);
-                const int us = prefix[u], ue = prefix[u + 1];
-                const int t0 = tile - us, t1 = min(ue, my1) - us;
-                const int end_tc = s_tc + (t1 - t0);  // tile numbers of this piece: [s_tc, end_tc)
-                if (!wait(&sh->q_full, q_use & 1)) break;
-                ++q_use;
+            TcPiece pc;
+            bool has = piece_from(my0, pc);
+            while (ok && has) {
+                const int qb = pi & 1;
+                const int end_tc = s_tc + (pc.t1 - pc.t0);  // tile numbers of this piece: [s_tc, end_tc)
+                if (!wait(&sh->q_full[qb], (pi >> 1) & 1)) break;
+                ++pi;
+                dq = dq0 + ((qb * kQBytes) >> 4);
                 if (!issue_s_blocking()) break;
                 bool q_done = false, first_pv = true;
                 while (ok && pv_tc < end_tc) {
@@ -427,7 +484,7 @@ attention_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_const
                     const uint64_t tstart = global_ns();
                     for (uint32_t it = 0;; ++it) {
                         if (s_tc < end_tc && s_inputs_ready()) issue_s();
-                        if (mbar_test(&sh->p_full[pv_tc & 1], (pv_tc >> 1) & 1)) break;
+                        if (mbar_test(&sh->p_full, pv_tc & 1)) break;
                         if ((it & 255) == 255 && (*abort_flag || global_ns() - tstart > kTcWaitNs)) {
                             give_up();
                             ok = false;
@@ -436,21 +493,20 @@ attention_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_const
                     }
                     if (!ok) break;
                     if (s_tc == end_tc && !q_done) {
-                        mma_commit(&sh->q_empty);  // every S product of this unit issued
+                        mma_commit(&sh->q_empty[qb]);  // every S product of this piece issued
                         q_done = true;
                     }
                     if (first_pv && !wait(&sh->o_empty, (o_use & 1) ^ 1)) break;
                     tc_fence_after();
                     const uint32_t v_off = (uint32_t)(pv_st * 2 * kTcHalf);
-                    const uint32_t p_off = (uint32_t)((pv_tc & 1) * kPBytes);
 #pragma unroll
                     for (int kk = 0; kk < kTcKeys / 16; ++kk) {
                         const uint64_t ad = dv + ((v_off + kk * 2048) >> 4);
-                        const uint64_t bd = dp + ((p_off + (kk >> 2) * R * 128 + (kk & 3) * 32) >> 4);
+                        const uint64_t bd = dp + (((kk >> 2) * R * 128 + (kk & 3) * 32) >> 4);
                         mma_f16_ss(tm_o, ad, bd, idesc_o, (first_pv && kk == 0) ? 0u : 1u);
                     }
                     mma_commit(&sh->kv_empty[pv_st]);
-                    mma_commit(&sh->p_empty[pv_tc & 1]);
+                    mma_commit(&sh->p_empty);
                     first_pv = false;
                     if (++pv_st == STAGES) pv_st = 0;
                     ++pv_tc;
@@ -458,10 +514,10 @@ attention_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_const
                     if (pv_tc < end_tc && s_tc == pv_tc && !issue_s_blocking()) break;
                 }
                 if (!ok) break;
-                if (!q_done) mma_commit(&sh->q_empty);
+                if (!q_done) mma_commit(&sh->q_empty[qb]);
                 mma_commit(&sh->o_full);
                 ++o_use;
-                tile = us + t1;
+                has = piece_from(pc.us + pc.t1, pc);
             }
             mma_commit(&sh->drain);
             mbar_wait_bounded(&sh->drain, 0, &sh->never, kTcWaitNs);
@@ -493,13 +549,11 @@ attention_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_const
         int tc = 0, kst = 0;
         uint32_t o_use = 0;
         bool ok = true;
-        for (int tile = my0; ok && tile < my1;) {
-            const int u = unit_of(tile);
-            const int us = prefix[u], ue = prefix[u + 1];
-            const int t0 = tile - us, t1 = min(ue, my1) - us;
-            const int b = u / a.Hkv, g = u % a.Hkv;
-            const int kv = a.kv_len[b], c = a.n_clean[b];
-            const int total = tc_total_keys(a, b);
+        TcPiece pc;
+        bool has = piece_from(my0, pc);
+        while (ok && has) {
+            const int u = pc.u, us = pc.us, t0 = pc.t0, t1 = pc.t1, b = pc.b, g = pc.g;
+            const int kv = kvs[b], c = cs[b], total = tots[b];
             // last visible key of each row (rows are slot-major, then head in
             // the group); read after the next group barrier
             if (et < R) {
@@ -578,8 +632,7 @@ attention_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_const
                     // O^T (thread = d, column = row) is rescaled once the
                     // previous tile's product is complete
                     if (t > t0 && group_or<kSoft>(rescale)) {
-                        const int tp = tc - 1;
-                        if (!group_wait(&sh->p_empty[tp & 1], (tp >> 1) & 1)) {
+                        if (!group_wait(&sh->p_empty, (tc - 1) & 1)) {
                             ok = false;
                             break;
                         }
@@ -599,11 +652,11 @@ attention_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_const
                     }
                 }
                 // P^T[row][key] = 2^(s - m_ref) as bf16, 128-byte-swizzled rows
-                if (tc >= 2 && !group_wait(&sh->p_empty[buf], ((tc - 2) >> 1) & 1)) {
+                if (tc >= 1 && !group_wait(&sh->p_empty, (tc - 1) & 1)) {
                     ok = false;
                     break;
                 }
-                unsigned char* pcol = p_col + buf * kPBytes + r0 * 128;
+                unsigned char* pcol = p_col + r0 * 128;
 #pragma unroll
                 for (int r = 0; r < RC; ++r) {
                     const float m_use = m_ref[r] == -INFINITY ? 0.f : m_ref[r];
@@ -614,7 +667,7 @@ attention_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_const
                 }
                 asm volatile("fence.proxy.async.shared::cta;\n" ::: "memory");
                 __syncwarp();
-                if (lane == 0) mbar_arrive(&sh->p_full[buf]);
+                if (lane == 0) mbar_arrive(&sh->p_full);
                 ++tc;
                 if (++kst == STAGES) kst = 0;
             }
@@ -652,6 +705,7 @@ attention_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_const
             __nv_bfloat16* sO = reinterpret_cast<__nv_bfloat16*>(sP);
             // CTAs whose ranges meet unit u: first .. last (all non-empty)
             const long long TL = T;
+            const int ue = us + unit_tiles(u);  // end of the unit's tiles on the partition axis
             const int first = (int)(((long long)(us + 1) * G + TL - 1) / TL) - 1;
             const int last = (int)(((long long)ue * G + TL - 1) / TL) - 1;
             const int npieces = last - first + 1;
@@ -664,9 +718,14 @@ attention_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_const
                     sO[(r0 + r) * 128 + d] = __float2bfloat16_rn(__uint_as_float(ov[r]) * inv);
                 }
             } else {
-                // partial slot: 0 for the first unit of a CTA's range, 1 for its last
+                // partial slot: 0 when u is the first piece of the CTA's range,
+                // 1 when it is the last one
                 auto slot_of = [&](int cta) {
-                    return (cta > first || (long long)T * cta / G == us) ? 0 : 1;
+                    if (cta > first) return 0;
+                    const int c0 = (int)((long long)T * cta / G);
+                    if (c0 >= us) return 0;
+                    const int v = unit_of(c0);  // a unit before u: does it leave tiles to this CTA?
+                    return (c0 - prefix[v] >= unit_tiles(v) && prefix[v + 1] == us) ? 0 : 1;
                 };
                 auto part_of = [&](int cta) {
                     return a.part + ((size_t)cta * 2 + slot_of(cta)) * a.part_stride;
@@ -745,7 +804,7 @@ attention_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_const
             }
             // lim and the staged rows are rewritten only after the next group barrier
             group_sync<kSoft>();
-            tile = us + t1;
+            has = piece_from(us + t1, pc);
         }
     }
     tc_fence_before();
@@ -806,7 +865,8 @@ cudaError_t launch_attention_tc(const Plan& p, const isd_dims* d, const uint16_t
     int dev = 0, optin = 0;
     cudaGetDevice(&dev);
     cudaDeviceGetAttribute(&optin, cudaDevAttrMaxSharedMemoryPerBlockOptin, dev);
-    const size_t extra = 1024 + (size_t)(d->B * d->Hkv + 1) * 4;  // alignment slack + tile prefix
+    // alignment slack, per-request lengths, unit offsets
+    const size_t extra = 1024 + (size_t)3 * d->B * 4 + (size_t)(d->B * d->Hkv + 1) * 4;
     int stages = 0;
     size_t smem = 0;
     for (int s = 3; s >= 2 && !stages; --s) {
