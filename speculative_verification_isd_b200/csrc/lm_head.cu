@@ -21,6 +21,14 @@
 //  * warps 2-5 drain the accumulator (tcgen05.ld 32 lanes x 32 columns) and
 //    store fp32 logits: lanes are consecutive vocabulary entries, so each
 //    store instruction writes 128 contiguous bytes of one logits row;
+//  * the vocabulary tiles are dealt round-robin in whole waves of gridDim.x;
+//    the L < gridDim.x tiles left over are split along N (the hidden rows)
+//    into chunks of 16-row multiples, one chunk per CTA with the full K
+//    loop, so the last wave is short instead of one tile long; the chunk CTAs
+//    read their shared W tile in the same order with an L2-keep hint, so it
+//    crosses HBM about once.  Each chunk holds complete logits for its rows,
+//    so the fused row statistics need no merge and the result is independent
+//    of timing;
 //  * every mbarrier wait is bounded (about 2 s); on time-out the CTA raises
 //    ISD_FLAG_WAIT_TIMEOUT, every role leaves its loop, outstanding TMA loads
 //    and MMAs are drained with bounded waits, and TMEM is released.
@@ -36,6 +44,9 @@ namespace isd {
 struct LmArgs {
     int V, Mh, H;
     int BN, n_acc, n_tiles;
+    int n_full;                    // tiles dealt in whole waves (a multiple of gridDim.x)
+    int tail_split;                // chunks per left-over tile (1: left-over tiles are whole)
+    int tail_bn;                   // hidden rows per chunk (multiple of 16)
     int w_stages, h_stages;        // depth of the W ring and of the hidden ring (w > h)
     int w_rows, h_rows0, h_rows1;  // TMA box heights (never taller than the tensor)
     uint32_t tmem_cols;
@@ -71,7 +82,8 @@ ISD_DEVINL bool lm_wait(uint64_t* bar, uint32_t parity, volatile int* abort) {
 template <int NB>
 __global__ void __launch_bounds__(kLmThreads, 1)
 lm_head_kernel(const __grid_constant__ CUtensorMap tmap_w, const __grid_constant__ CUtensorMap tmap_h0,
-               const __grid_constant__ CUtensorMap tmap_h1, LmArgs a) {
+               const __grid_constant__ CUtensorMap tmap_h1, const __grid_constant__ CUtensorMap tmap_ht,
+               LmArgs a) {
     using namespace sm100;
     extern __shared__ unsigned char smem_raw[];
     unsigned char* smem = reinterpret_cast<unsigned char*>(
@@ -107,6 +119,7 @@ lm_head_kernel(const __grid_constant__ CUtensorMap tmap_w, const __grid_constant
         prefetch_tmap(&tmap_w);
         prefetch_tmap(&tmap_h0);
         if (NB > 1) prefetch_tmap(&tmap_h1);
+        if (a.tail_split > 1) prefetch_tmap(&tmap_ht);
     }
     if (warp == 1) {
         tmem_alloc(tmem_holder, a.tmem_cols);
@@ -120,9 +133,20 @@ lm_head_kernel(const __grid_constant__ CUtensorMap tmap_w, const __grid_constant
     // Each CTA starts its K loop at a different block so that the 148 CTAs
     // read different hidden slices at any moment.
     const int kb0 = (int)(blockIdx.x % (unsigned)kblocks);
-    int n_my_tiles = 0;
-    for (int t = blockIdx.x; t < a.n_tiles; t += gridDim.x) ++n_my_tiles;
+    // Work items of this CTA: its tiles of the whole waves, then at most one
+    // left-over tile (whole) or one chunk of a left-over tile.
+    const int G = (int)gridDim.x;
+    const int n_wave = a.n_full / G;
+    const int n_left = a.n_tiles - a.n_full;
+    const int S = a.tail_split;
+    const bool has_extra = (int)blockIdx.x < n_left * S;
+    const int n_my_tiles = n_wave + (has_extra ? 1 : 0);
     const int total_kb = n_my_tiles * kblocks;
+    auto item_tile = [&](int i) {
+        return i < n_wave ? (int)blockIdx.x + i * G : a.n_full + (int)blockIdx.x / S;
+    };
+    auto item_is_chunk = [&](int i) { return i >= n_wave && S > 1; };
+    const int chunk_row0 = ((int)blockIdx.x % S) * a.tail_bn;  // first hidden row of this CTA's chunk
 
     auto give_up = [&]() {
         *abort_flag = 1;
@@ -135,9 +159,10 @@ lm_head_kernel(const __grid_constant__ CUtensorMap tmap_w, const __grid_constant
             // the deep ring; warp 6 feeds the L2-resident hidden tiles
             const bool is_w = (warp == 0);
             const uint64_t pol = is_w ? policy_evict_first() : policy_evict_last();
-            const uint32_t tx = is_w ? (uint32_t)a.w_rows * 128u
-                                     : (uint32_t)(a.h_rows0 + a.h_rows1) * 128u;
-            int ws = 0, hs = 0, kb = kb0, tile = blockIdx.x, jt = 0;
+            const uint64_t pol_keep = policy_evict_last();
+            int ws = 0, hs = 0, kb = kb0, item = 0, jt = 0;
+            int tile = item_tile(0);
+            bool chunk = item_is_chunk(0);
             uint32_t wph = 0;
             // hidden producer: the k-block that last used its slot, as a W slot/phase
             int pws = 0;
@@ -156,25 +181,37 @@ lm_head_kernel(const __grid_constant__ CUtensorMap tmap_w, const __grid_constant
                     give_up();
                     break;
                 }
-                mbar_arrive_expect_tx(&full[ws], tx);
+                // a chunk walks K from block 0 like the other chunks of its tile
+                const int kbi = chunk ? jt : kb;
                 if (is_w) {
-                    tma_load_2d(wring + (size_t)ws * kWStageBytes, &tmap_w, &full[ws], kb * 64,
-                                tile * 128, pol);
+                    mbar_arrive_expect_tx(&full[ws], (uint32_t)a.w_rows * 128u);
+                    tma_load_2d(wring + (size_t)ws * kWStageBytes, &tmap_w, &full[ws], kbi * 64,
+                                tile * 128, chunk ? pol_keep : pol);
+                } else if (chunk) {
+                    mbar_arrive_expect_tx(&full[ws], (uint32_t)a.tail_bn * 128u);
+                    tma_load_2d(hring + (size_t)hs * h_bytes, &tmap_ht, &full[ws], kbi * 64, chunk_row0, pol);
                 } else {
+                    mbar_arrive_expect_tx(&full[ws], (uint32_t)(a.h_rows0 + a.h_rows1) * 128u);
                     unsigned char* sb = hring + (size_t)hs * h_bytes;
-                    tma_load_2d(sb, &tmap_h0, &full[ws], kb * 64, 0, pol);
-                    if (NB > 1) tma_load_2d(sb + a.BN * 128, &tmap_h1, &full[ws], kb * 64, a.BN, pol);
+                    tma_load_2d(sb, &tmap_h0, &full[ws], kbi * 64, 0, pol);
+                    if (NB > 1) tma_load_2d(sb + a.BN * 128, &tmap_h1, &full[ws], kbi * 64, a.BN, pol);
                 }
                 if (++ws == a.w_stages) { ws = 0; wph ^= 1; }
                 if (++hs == a.h_stages) hs = 0;
                 if (++kb == kblocks) kb = 0;
-                if (++jt == kblocks) { jt = 0; tile += gridDim.x; }
+                if (++jt == kblocks) {
+                    jt = 0;
+                    ++item;
+                    tile = item_tile(item);
+                    chunk = item_is_chunk(item);
+                }
             }
         }
     } else if (warp == 1) {
         if (lane == 0) {
             // ---------------- MMA issuer
-            const uint32_t idesc = idesc_bf16_f32(128, a.BN);
+            const uint32_t idesc_full = idesc_bf16_f32(128, a.BN);
+            const uint32_t idesc_chunk = idesc_bf16_f32(128, a.tail_bn);
             const uint64_t adesc0 = smem_desc_sw128(smem_u32(wring));
             const uint64_t bdesc0 = smem_desc_sw128(smem_u32(hring));
             const uint64_t astep = kWStageBytes >> 4, bstep = (uint64_t)(h_bytes >> 4);
@@ -190,6 +227,9 @@ lm_head_kernel(const __grid_constant__ CUtensorMap tmap_w, const __grid_constant
                 }
                 tc_fence_after();
                 const uint32_t d0 = tmem_base + (uint32_t)(acc * NB * a.BN);
+                const bool chunk = item_is_chunk(lt);
+                const uint32_t idesc = chunk ? idesc_chunk : idesc_full;
+                const int nbs = chunk ? 1 : NB;
                 for (int j = 0; j < kblocks; ++j) {
                     if (!lm_wait(&full[ws], wph, abort_flag)) {
                         give_up();
@@ -203,8 +243,9 @@ lm_head_kernel(const __grid_constant__ CUtensorMap tmap_w, const __grid_constant
                     for (int k = 0; k < 4; ++k) {
 #pragma unroll
                         for (int nb = 0; nb < NB; ++nb)
-                            mma_f16_ss(d0 + nb * a.BN, ad + 2 * k,
-                                       bd + (uint64_t)(nb * a.BN * 8) + 2 * k, idesc, (j | k) != 0);
+                            if (nb < nbs)
+                                mma_f16_ss(d0 + nb * a.BN, ad + 2 * k,
+                                           bd + (uint64_t)(nb * a.BN * 8) + 2 * k, idesc, (j | k) != 0);
                     }
                     mma_commit(&empty[ws]);
                     if (++ws == a.w_stages) { ws = 0; wph ^= 1; }
@@ -219,8 +260,12 @@ lm_head_kernel(const __grid_constant__ CUtensorMap tmap_w, const __grid_constant
     } else {
         // ---------------- epilogue: warps 2..5 cover TMEM lane quarters 2,3,0,1
         const int quarter = warp & 3;
-        int lt = 0;
-        for (int tile = blockIdx.x; tile < a.n_tiles; tile += gridDim.x, ++lt) {
+        for (int lt = 0; lt < n_my_tiles; ++lt) {
+            const int tile = item_tile(lt);
+            const bool chunk = item_is_chunk(lt);
+            const int bn = chunk ? a.tail_bn : a.BN;    // accumulator columns of this item
+            const int nbs = chunk ? 1 : NB;
+            const int row0 = chunk ? chunk_row0 : 0;    // hidden row of column 0
             const int acc = lt % a.n_acc;
             const uint32_t use = (uint32_t)(lt / a.n_acc);
             int ok = 1;
@@ -241,21 +286,22 @@ lm_head_kernel(const __grid_constant__ CUtensorMap tmap_w, const __grid_constant
             const size_t part_pitch = (size_t)a.n_tiles * 4;
 #pragma unroll
             for (int nb = 0; nb < NB; ++nb) {
-                for (int j0 = 0; j0 < a.BN; j0 += 32) {
+                if (nb >= nbs) break;
+                for (int j0 = 0; j0 < bn; j0 += 32) {
                     uint32_t r[32];
-                    // BN is a multiple of 16: the tail is one 16-column load,
+                    // bn is a multiple of 16: the tail is one 16-column load,
                     // so no load reaches past the allocated columns
-                    if (a.BN - j0 >= 32)
+                    if (bn - j0 >= 32)
                         tmem_ld_32x32b_x32(taddr + nb * a.BN + j0, r);
                     else
                         tmem_ld_32x32b_x16(taddr + nb * a.BN + j0, r);
                     tmem_ld_wait();
-                    const int mbase = nb * a.BN + j0;
+                    const int mbase = row0 + nb * a.BN + j0;
                     if (v_ok) {
 #pragma unroll
                         for (int k = 0; k < 32; ++k) {
                             const int m = mbase + k;
-                            if (j0 + k < a.BN && m < a.Mh)
+                            if (j0 + k < bn && m < a.Mh)
                                 a.logits[(size_t)m * a.V + v] = __uint_as_float(r[k]);
                         }
                     }
@@ -283,7 +329,7 @@ lm_head_kernel(const __grid_constant__ CUtensorMap tmap_w, const __grid_constant
                         for (int i = 0; i < 32; ++i)
                             if (i < nvalid) se += __expf(x[i] - mx);
                         const int m = mbase + lane;
-                        if (j0 + lane < a.BN && m < a.Mh)
+                        if (j0 + lane < bn && m < a.Mh)
                             part[(size_t)m * part_pitch] =
                                 make_float4(mx, se, __int_as_float(tile * 128 + quarter * 32 + arg), 0.f);
                         __syncwarp();
@@ -439,10 +485,34 @@ cudaError_t launch_lm_head(const uint16_t* hidden, const uint16_t* W, int Mh, in
     a.err_flag = err_flag;
     int grid = num_sms_of_current_device();
     if (grid > a.n_tiles) grid = a.n_tiles;
+    // whole waves of tiles, then the left-over tiles split into row chunks
+    a.n_full = (a.n_tiles / grid) * grid;
+    const int left = a.n_tiles - a.n_full;
+    a.tail_split = 1;
+    a.tail_bn = 16;
+    if (left > 0 && Mh >= 32) {
+        int S = grid / left;
+        const int max_chunks = (Mh + 15) / 16;
+        if (S > max_chunks) S = max_chunks;
+        if (S >= 2) {
+            const int bn = ((Mh + S - 1) / S + 15) / 16 * 16;
+            S = (Mh + bn - 1) / bn;
+            if (S >= 2) {
+                a.tail_split = S;
+                a.tail_bn = bn;
+            }
+        }
+    }
+    CUtensorMap tht = th0;
+    if (a.tail_split > 1 &&
+        !encode_bf16_2d(&tht, hidden, (uint64_t)Mh, (uint64_t)H, (uint32_t)a.tail_bn)) {
+        set_error_detail("lm_head: tensor map of hidden (row chunks) rejected");
+        return cudaErrorInvalidValue;
+    }
     if (sh.NB == 1)
-        lm_head_kernel<1><<<grid, kLmThreads, sh.smem, st>>>(tw, th0, th1, a);
+        lm_head_kernel<1><<<grid, kLmThreads, sh.smem, st>>>(tw, th0, th1, tht, a);
     else
-        lm_head_kernel<2><<<grid, kLmThreads, sh.smem, st>>>(tw, th0, th1, a);
+        lm_head_kernel<2><<<grid, kLmThreads, sh.smem, st>>>(tw, th0, th1, tht, a);
     cudaError_t e = cudaGetLastError();
     if (e != cudaSuccess) set_error_detail("lm_head: launch failed");
     return e;

@@ -172,6 +172,36 @@ def test_staged_parity(isd, name, n_clean):
     assert int(sb.err.item()) == 0
 
 
+def test_lm_head_left_over_tiles_by_row_chunks(isd):
+    """V = 151936 on a full GPU leaves a few 128-entry vocabulary tiles after
+    the whole waves; they are computed as 16-row chunks of the hidden rows
+    (M = 56 here, so the last chunk reaches past the matrix).  Every logit of
+    those tiles (and of two tiles of the waves) matches the oracle, every row's
+    statistics match, and a second run is bit-identical."""
+    cfg = I.CONFIGS["qwen3_8b_b8_n4"]
+    inp = I.make_step_inputs(cfg, seed=21)
+    sb = StepBuffers(isd, cfg, inp)
+    sb.attention()
+    sb.lm_head()
+    torch.cuda.synchronize()
+    hid = bf16_host(sb.hidden)
+    z_g = sb.logits.cpu().numpy()
+    n_tiles = (cfg.V + 127) // 128
+    grid = min(torch.cuda.get_device_properties(0).multi_processor_count, n_tiles)
+    first_left = (n_tiles // grid) * grid
+    assert first_left < n_tiles  # the shape does leave tiles over
+    cols = np.r_[0:128, 77 * 128:78 * 128, first_left * 128:cfg.V]
+    z_o = O.lm_head(hid, inp["W"][cols])
+    absdot = np.abs(O.bf16_to_f64(hid)) @ np.abs(O.bf16_to_f64(inp["W"][cols])).T
+    assert np.all(np.abs(z_g[:, cols] - z_o) <= 1e-4 * absdot + 1e-6)
+    check_row_stats(sb, z_g)
+    logits1, stats1 = sb.logits.clone(), sb.row_stats.clone()
+    sb.lm_head()
+    torch.cuda.synchronize()
+    assert torch.equal(sb.logits, logits1) and torch.equal(sb.row_stats, stats1)
+    assert int(sb.err.item()) == 0
+
+
 @pytest.mark.parametrize("name", ["tiny", "ragged_small", "qwen_medium"])
 def test_whole_step_matches_stages(isd, name):
     """isd_step gives bit-identical results to the three stage calls."""
