@@ -383,34 +383,28 @@ def main():
     t_attn, t_lm, t_acc = [float(x) for x in st_ms]
 
     # ---------------- e2e: public API with host buffers, copies inside the timed region
-    host = {}
-    for name in ("q", "k_new", "v_new"):
-        t = getattr(wl, name)
-        host[name] = torch.empty(t.shape, dtype=t.dtype, pin_memory=True).copy_(t)
-    for name in ("kv_len", "n_clean", "clean_tok", "page_table"):
-        t = getattr(wl, name)
-        host[name] = torch.empty(t.shape, dtype=t.dtype, pin_memory=True).copy_(t)
-    host["uniforms"] = torch.empty(wl.uniforms_all.shape, dtype=torch.float32,
-                                   pin_memory=True).copy_(wl.uniforms_all)
-    outs = ("accept_len", "out_tok", "next_n_clean", "next_clean_tok", "next_kv_len")
-    host_out = {n: torch.empty(getattr(wl, n).shape, dtype=torch.int32, pin_memory=True)
-                for n in outs}
-    h2d = sum(host[n].numel() * host[n].element_size() for n in host if n != "uniforms") + \
-        host["uniforms"][0].numel() * 4
-    d2h = sum(v.numel() * 4 for v in host_out.values())
+    # A step's inputs travel in one pinned host buffer (one host-to-device
+    # copy), its integer results come back in one (one device-to-host copy);
+    # the caller waits for each step's result before issuing the next step.
+    in_dev, out_dev, layout = wl.pack_io()
+    host_in = torch.empty(in_dev.numel(), dtype=torch.uint8, pin_memory=True)
+    host_in.copy_(in_dev)
+    u_off, u_nb = next((o, nb) for n, o, nb in layout if n == "uniforms")
+    host_u = host_in[u_off:u_off + u_nb].view(torch.float32)
+    u_steps = wl.uniforms_all.cpu().reshape(wl.uniforms_all.shape[0], -1)
+    host_out = torch.empty(out_dev.numel(), dtype=torch.int32, pin_memory=True)
+    h2d = in_dev.numel()
+    d2h = host_out.numel() * 4
     KE = min(args.e2e_steps, K)
     barrier(world)
     torch.cuda.synchronize()
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     e0.record(stream)
     for k in range(KE):
-        for n in ("q", "k_new", "v_new", "kv_len", "n_clean", "clean_tok", "page_table"):
-            getattr(wl, n).copy_(host[n], non_blocking=True)
-        wl.uniforms = wl.uniforms_all[0]
-        wl.uniforms.copy_(host["uniforms"][k % host["uniforms"].shape[0]], non_blocking=True)
+        host_u.copy_(u_steps[k % u_steps.shape[0]])  # this step's uniforms
+        in_dev.copy_(host_in, non_blocking=True)
         wl.step()
-        for n in outs:
-            host_out[n].copy_(getattr(wl, n), non_blocking=True)
+        host_out.copy_(out_dev, non_blocking=True)
         stream.synchronize()  # the caller needs this step's result before the next one
     e1.record(stream)
     torch.cuda.synchronize()

@@ -74,16 +74,17 @@ row_stats_finalize_kernel(const float4* __restrict__ part, int n_parts,
     const int row = blockIdx.x;
     const float4* pr = part + (size_t)row * n_parts;
     RowStat st = rowstat_empty();
-    // loads issued ahead of the (dependent) merges, in batches of 4
-    for (int k0 = threadIdx.x; k0 < n_parts; k0 += 4 * THREADS) {
-        float4 p[4];
+    // loads issued ahead of the (dependent) merges, in batches of 8 (one
+    // batch covers a 151936-entry vocabulary's 4748 partials)
+    for (int k0 = threadIdx.x; k0 < n_parts; k0 += 8 * THREADS) {
+        float4 p[8];
 #pragma unroll
-        for (int u = 0; u < 4; ++u) {
+        for (int u = 0; u < 8; ++u) {
             const int k = k0 + u * THREADS;
             p[u] = k < n_parts ? __ldcs(pr + k) : make_float4(-INFINITY, 0.f, 0.f, 0.f);
         }
 #pragma unroll
-        for (int u = 0; u < 4; ++u) st = rowstat_merge(st, RowStat{p[u].x, p[u].y, __float_as_int(p[u].z)});
+        for (int u = 0; u < 8; ++u) st = rowstat_merge(st, RowStat{p[u].x, p[u].y, __float_as_int(p[u].z)});
     }
     st = rowstat_block_reduce<THREADS>(st);
     if (threadIdx.x == 0) out[row] = isd_row_stat{st.m, st.s, st.idx, 0};
@@ -428,7 +429,7 @@ cudaError_t launch_row_stats(const Plan& p, const float* logits, int rows, int V
 
 cudaError_t launch_row_stats_finalize(const float4* part, int n_parts, int rows,
                                       isd_row_stat* out, cudaStream_t st) {
-    row_stats_finalize_kernel<kStatsThreads><<<rows, kStatsThreads, 0, st>>>(part, n_parts, out);
+    row_stats_finalize_kernel<kFinalizeThreads><<<rows, kFinalizeThreads, 0, st>>>(part, n_parts, out);
     return cudaGetLastError();
 }
 

@@ -81,36 +81,45 @@ ISD_DEVINL int tc_total_keys(const TcArgs& a, int b) {
     return (int)t;
 }
 
-// a1: the block's K/V rows into their pages (16 bytes per thread and step);
-// a request that cannot be served gets zero attention output here.
+// a1: one CTA per (request, block position): that position's K and V rows
+// for all kv heads go into their page, 16 bytes per thread.  The CTA of block
+// position 0 also clears the request's attention counters (and, if given, one
+// more counter per request for the kernels that follow), and writes zero
+// attention output for a request that cannot be served.
 __global__ void kv_append_kernel(TcArgs a, const __nv_bfloat16* k_new, const __nv_bfloat16* v_new,
-                                 __nv_bfloat16* k_pool, __nv_bfloat16* v_pool) {
-    const int b = blockIdx.x;
+                                 __nv_bfloat16* k_pool, __nv_bfloat16* v_pool, int* clear_extra) {
+    const int b = blockIdx.x, r = blockIdx.y;
     const int kv = a.kv_len[b], c = a.n_clean[b];
     const bool bad_c = (c < 1 || c > a.N);
     const long long want = bad_c ? 0 : (long long)kv + c + a.N - 1;
     const bool over = kv < 0 || (want + a.P - 1) / a.P > a.max_pages;
+    if (r == 0) {
+        for (int i = threadIdx.x; i < a.Hkv; i += blockDim.x) a.ticket[b * a.Hkv + i] = 0;
+        if (clear_extra && threadIdx.x == 0) clear_extra[b] = 0;
+    }
     if (bad_c || over) {
-        if (threadIdx.x == 0) raise_flag(a.err_flag, bad_c ? ISD_FLAG_NCLEAN_RANGE : ISD_FLAG_CAPACITY);
-        uint4* o = reinterpret_cast<uint4*>(a.out + (size_t)b * a.Q * a.Hq * 128);
-        for (int i = threadIdx.x; i < a.Q * a.Hq * 16; i += blockDim.x) o[i] = make_uint4(0, 0, 0, 0);
+        if (r == 0) {
+            if (threadIdx.x == 0) raise_flag(a.err_flag, bad_c ? ISD_FLAG_NCLEAN_RANGE : ISD_FLAG_CAPACITY);
+            uint4* o = reinterpret_cast<uint4*>(a.out + (size_t)b * a.Q * a.Hq * 128);
+            for (int i = threadIdx.x; i < a.Q * a.Hq * 16; i += blockDim.x) o[i] = make_uint4(0, 0, 0, 0);
+        }
         return;
     }
-    const int nblk = c + a.N - 1;
-    const int per_pos = a.Hkv * 16;  // 16-byte chunks of one position, all kv heads
-    for (int i = threadIdx.x; i < nblk * per_pos; i += blockDim.x) {
-        const int r = i / per_pos, rem = i % per_pos;
-        const int t = kv + r;
-        const int slot = r < c ? r : a.N + (r - c);
-        const int page = a.page_table[(size_t)b * a.max_pages + t / a.P];
-        if (page < 0 || page >= a.num_pages) {
-            raise_flag(a.err_flag, ISD_FLAG_PAGE_OOB);
-            continue;
-        }
-        const size_t dst = ((size_t)page * a.P + t % a.P) * a.Hkv * 128 + (size_t)rem * 8;
-        const size_t src = ((size_t)b * a.Q + slot) * a.Hkv * 128 + (size_t)rem * 8;
-        *reinterpret_cast<uint4*>(k_pool + dst) = *reinterpret_cast<const uint4*>(k_new + src);
-        *reinterpret_cast<uint4*>(v_pool + dst) = *reinterpret_cast<const uint4*>(v_new + src);
+    if (r >= c + a.N - 1) return;  // block positions: c clean slots, then N - 1 MASK slots
+    const int t = kv + r;
+    const int slot = r < c ? r : a.N + (r - c);
+    const int page = a.page_table[(size_t)b * a.max_pages + t / a.P];
+    if (page < 0 || page >= a.num_pages) {
+        if (threadIdx.x == 0) raise_flag(a.err_flag, ISD_FLAG_PAGE_OOB);
+        return;
+    }
+    const size_t dst = ((size_t)page * a.P + t % a.P) * a.Hkv * 128;
+    const size_t src = ((size_t)b * a.Q + slot) * a.Hkv * 128;
+    for (int i = threadIdx.x; i < a.Hkv * 16; i += blockDim.x) {
+        *reinterpret_cast<uint4*>(k_pool + dst + (size_t)i * 8) =
+            *reinterpret_cast<const uint4*>(k_new + src + (size_t)i * 8);
+        *reinterpret_cast<uint4*>(v_pool + dst + (size_t)i * 8) =
+            *reinterpret_cast<const uint4*>(v_new + src + (size_t)i * 8);
     }
 }
 
@@ -858,7 +867,7 @@ cudaError_t launch_attention_tc(const Plan& p, const isd_dims* d, const uint16_t
                                 const uint16_t* k_new, const uint16_t* v_new, uint16_t* k_pool,
                                 uint16_t* v_pool, const int32_t* page_table, const int32_t* kv_len,
                                 const int32_t* n_clean, uint16_t* out, void* ws, int32_t* err_flag,
-                                cudaStream_t st, bool* handled) {
+                                cudaStream_t st, int* clear_extra, bool* handled) {
     *handled = false;
     const int R = p.attn_tc_rows;
     if (R == 0) return cudaSuccess;
@@ -917,10 +926,10 @@ cudaError_t launch_attention_tc(const Plan& p, const isd_dims* d, const uint16_t
     a.part_stride = p.attn_tc_part_stride;
     a.ticket = reinterpret_cast<int*>(static_cast<char*>(ws) + p.off_attn_ticket);
     a.err_flag = err_flag;
-    kv_append_kernel<<<d->B, 256, 0, st>>>(a, reinterpret_cast<const __nv_bfloat16*>(k_new),
-                                           reinterpret_cast<const __nv_bfloat16*>(v_new),
-                                           reinterpret_cast<__nv_bfloat16*>(k_pool),
-                                           reinterpret_cast<__nv_bfloat16*>(v_pool));
+    const int append_threads = (Hkv * 16 + 31) / 32 * 32;
+    kv_append_kernel<<<dim3(d->B, 2 * d->N - 1), append_threads > 1024 ? 1024 : append_threads, 0, st>>>(
+        a, reinterpret_cast<const __nv_bfloat16*>(k_new), reinterpret_cast<const __nv_bfloat16*>(v_new),
+        reinterpret_cast<__nv_bfloat16*>(k_pool), reinterpret_cast<__nv_bfloat16*>(v_pool), clear_extra);
     cudaError_t e = cudaGetLastError();
     if (e != cudaSuccess) return e;
     if (R == 16) return stages == 3 ? launch_tc<16, 3>(a, tk, tv, tq, smem, st) : launch_tc<16, 2>(a, tk, tv, tq, smem, st);

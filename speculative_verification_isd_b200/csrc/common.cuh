@@ -114,11 +114,11 @@ ISD_DEVINL RowStat rowstat_block_reduce(RowStat a) {
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
     if (lane == 0) warp_part[warp] = a;
     __syncthreads();
-    if (threadIdx.x == 0) {
-        RowStat r = warp_part[0];
+    if (warp == 0) {
+        // the warp partials, merged by warp 0 in a shuffle tree
+        a = lane < THREADS / 32 ? warp_part[lane] : rowstat_empty();
 #pragma unroll
-        for (int w = 1; w < THREADS / 32; ++w) r = rowstat_merge(r, warp_part[w]);
-        a = r;
+        for (int off = 16; off > 0; off >>= 1) a = rowstat_merge(a, rowstat_shfl_xor(a, off));
     }
     __syncthreads();
     return a;

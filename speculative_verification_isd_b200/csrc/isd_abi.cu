@@ -23,7 +23,7 @@ cudaError_t launch_attention(const Plan& p, const isd_dims* d, const uint16_t* q
                              const uint16_t* k_new, const uint16_t* v_new, uint16_t* k_pool,
                              uint16_t* v_pool, const int32_t* page_table, const int32_t* kv_len,
                              const int32_t* n_clean, uint16_t* out, void* ws, int32_t* err_flag,
-                             cudaStream_t st);
+                             cudaStream_t st, int* clear_extra);
 cudaError_t launch_lm_head(const uint16_t* hidden, const uint16_t* W, int Mh, int H, int V,
                            float* logits, float4* stats_part, int32_t* err_flag, cudaStream_t st);
 cudaError_t launch_row_stats_finalize(const float4* part, int n_parts, int rows,
@@ -118,14 +118,13 @@ isd_status do_attention(const isd_dims* d, const Plan& p, const uint16_t* q,
                         const uint16_t* k_new, const uint16_t* v_new, uint16_t* k_pool,
                         uint16_t* v_pool, const int32_t* page_table, const int32_t* kv_len,
                         const int32_t* n_clean, uint16_t* out, void* ws, int32_t* err_flag,
-                        cudaStream_t st) {
+                        cudaStream_t st, int* clear_extra = nullptr) {
     if (!q || !k_new || !v_new || !k_pool || !v_pool || !page_table || !kv_len || !n_clean || !out)
         return invalid("null attention pointer");
     ISD_TRY(check_attention_shape(d, p));
-    ISD_CUDA(cudaMemsetAsync(static_cast<char*>(ws) + p.off_attn_ticket, 0,
-                             (size_t)d->B * d->Hkv * p.attn_rgb * 4, st));
+    // the launch clears the attention counters (and clear_extra) on the stream
     ISD_CUDA(isd::launch_attention(p, d, q, k_new, v_new, k_pool, v_pool, page_table, kv_len,
-                                   n_clean, out, ws, err_flag, st));
+                                   n_clean, out, ws, err_flag, st, clear_extra));
     return ISD_OK;
 }
 
@@ -209,12 +208,16 @@ isd_status isd_row_stats(const isd_dims* d, const float* logits, int32_t rows,
     return ISD_OK;
 }
 
-isd_status isd_accept(const isd_dims* d, const float* logits, const isd_row_stat* row_stats,
-                      const float* prev_logits, const isd_row_stat* prev_row_stats,
-                      const int32_t* n_clean, const int32_t* clean_tok, const int32_t* kv_len,
-                      const float* uniforms, int32_t* accept_len, int32_t* out_tok,
-                      int32_t* next_n_clean, int32_t* next_clean_tok, int32_t* next_kv_len,
-                      float* ratio, void* ws, size_t ws_bytes, int32_t* err_flag, void* stream) {
+// The accept stage; its counters are cleared first unless the caller has
+// cleared them on the stream already (the whole step clears them in its
+// first kernel).
+static isd_status accept_impl(const isd_dims* d, const float* logits, const isd_row_stat* row_stats,
+                              const float* prev_logits, const isd_row_stat* prev_row_stats,
+                              const int32_t* n_clean, const int32_t* clean_tok, const int32_t* kv_len,
+                              const float* uniforms, int32_t* accept_len, int32_t* out_tok,
+                              int32_t* next_n_clean, int32_t* next_clean_tok, int32_t* next_kv_len,
+                              float* ratio, void* ws, size_t ws_bytes, int32_t* err_flag, void* stream,
+                              bool clear_counters) {
     Plan p;
     ISD_TRY(plan_or_fail(d, &p));
     ISD_TRY(check_ws(p, ws, ws_bytes));
@@ -224,11 +227,23 @@ isd_status isd_accept(const isd_dims* d, const float* logits, const isd_row_stat
         !next_kv_len)
         return invalid("null accept pointer");
     cudaStream_t st = static_cast<cudaStream_t>(stream);
-    ISD_CUDA(cudaMemsetAsync(static_cast<char*>(ws) + p.off_acc_ticket, 0, (size_t)d->B * 4, st));
+    if (clear_counters)
+        ISD_CUDA(cudaMemsetAsync(static_cast<char*>(ws) + p.off_acc_ticket, 0, (size_t)d->B * 4, st));
     ISD_CUDA(isd::launch_accept(p, d, logits, row_stats, prev_logits, prev_row_stats, n_clean,
                                 clean_tok, kv_len, uniforms, accept_len, out_tok, next_n_clean,
                                 next_clean_tok, next_kv_len, ratio, ws, err_flag, st));
     return ISD_OK;
+}
+
+isd_status isd_accept(const isd_dims* d, const float* logits, const isd_row_stat* row_stats,
+                      const float* prev_logits, const isd_row_stat* prev_row_stats,
+                      const int32_t* n_clean, const int32_t* clean_tok, const int32_t* kv_len,
+                      const float* uniforms, int32_t* accept_len, int32_t* out_tok,
+                      int32_t* next_n_clean, int32_t* next_clean_tok, int32_t* next_kv_len,
+                      float* ratio, void* ws, size_t ws_bytes, int32_t* err_flag, void* stream) {
+    return accept_impl(d, logits, row_stats, prev_logits, prev_row_stats, n_clean, clean_tok, kv_len,
+                       uniforms, accept_len, out_tok, next_n_clean, next_clean_tok, next_kv_len,
+                       ratio, ws, ws_bytes, err_flag, stream, true);
 }
 
 isd_status isd_step(const isd_dims* d, const uint16_t* q, const uint16_t* k_new,
@@ -251,12 +266,15 @@ isd_status isd_step(const isd_dims* d, const uint16_t* q, const uint16_t* k_new,
     cudaStream_t st = static_cast<cudaStream_t>(stream);
     uint16_t* h = hidden ? hidden
                          : reinterpret_cast<uint16_t*>(static_cast<char*>(ws) + p.off_hidden);
+    // the attention launch also clears the accept counters, so the step
+    // issues no separate memset
+    int* acc_ticket = reinterpret_cast<int*>(static_cast<char*>(ws) + p.off_acc_ticket);
     ISD_TRY(do_attention(d, p, q, k_new, v_new, k_pool, v_pool, page_table, kv_len, n_clean, h,
-                         ws, err_flag, st));
+                         ws, err_flag, st, acc_ticket));
     ISD_TRY(do_lm_head(d, p, h, W, lora_A, lora_B, logits, row_stats, ws, err_flag, st));
-    return isd_accept(d, logits, row_stats, prev_logits, prev_row_stats, n_clean, clean_tok,
-                      kv_len, uniforms, accept_len, out_tok, next_n_clean, next_clean_tok,
-                      next_kv_len, ratio, ws, ws_bytes, err_flag, stream);
+    return accept_impl(d, logits, row_stats, prev_logits, prev_row_stats, n_clean, clean_tok,
+                       kv_len, uniforms, accept_len, out_tok, next_n_clean, next_clean_tok,
+                       next_kv_len, ratio, ws, ws_bytes, err_flag, stream, false);
 }
 
 }  // extern "C"

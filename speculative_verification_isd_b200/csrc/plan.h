@@ -13,6 +13,7 @@ constexpr int kAttnKeyTile = 64;      // keys per pipeline stage
 constexpr int kAttnRowsPerGroup = 16; // query rows handled by one 4-warp group
 constexpr int kAttnMaxSplit = 2048;   // keys per split at most (bounds the key table)
 constexpr int kStatsThreads = 256;
+constexpr int kFinalizeThreads = 1024;  // one CTA per row merges its statistics partials
 constexpr int kAcceptThreads = 256;
 constexpr int kAcceptChunk = 4096;    // vocabulary entries per accept CTA
 constexpr int kNumSMs = 148;

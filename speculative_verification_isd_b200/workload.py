@@ -126,6 +126,34 @@ class DeviceWorkload:
     def set_uniforms(self, k: int):
         self.uniforms = self.uniforms_all[k % self.uniforms_all.shape[0]]
 
+    IN_NAMES = ("q", "k_new", "v_new", "kv_len", "n_clean", "clean_tok", "page_table", "uniforms")
+    OUT_NAMES = ("accept_len", "out_tok", "next_n_clean", "next_clean_tok", "next_kv_len")
+
+    def pack_io(self):
+        """Rebind a step's inputs to views of one device byte buffer and its
+        integer results to views of one int32 buffer, so that the host traffic
+        of a step is one copy each way.  Returns (in_buf, out_buf, layout) with
+        layout = [(name, byte offset, bytes)]."""
+        layout, off = [], 0
+        for n in self.IN_NAMES:
+            t = getattr(self, n)
+            nb = t.numel() * t.element_size()
+            layout.append((n, off, nb))
+            off = (off + nb + 255) // 256 * 256
+        buf = torch.empty(off, dtype=torch.uint8, device="cuda")
+        for n, o, nb in layout:
+            t = getattr(self, n)
+            v = buf[o:o + nb].view(t.dtype).view(t.shape)
+            v.copy_(t)
+            setattr(self, n, v)
+        sizes = [getattr(self, n).numel() for n in self.OUT_NAMES]
+        obuf = torch.zeros(sum(sizes), dtype=torch.int32, device="cuda")
+        o = 0
+        for n, sz in zip(self.OUT_NAMES, sizes):
+            setattr(self, n, obuf[o:o + sz].view(getattr(self, n).shape))
+            o += sz
+        return buf, obuf, layout
+
     def step(self, stream=None):
         self.isd.step(self.dims, self.q, self.k_new, self.v_new, self.k_pool, self.v_pool,
                       self.page_table, self.kv_len, self.n_clean, self.clean_tok, self.W,
