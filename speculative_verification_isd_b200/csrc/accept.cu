@@ -226,7 +226,7 @@ ISD_DEVINL float chunk_scan(const SweepRow& r, int beg, int end, float target, i
     return total;
 }
 
-__global__ void __launch_bounds__(kAcceptThreads) accept_kernel(AcceptArgs a) {
+__global__ void __launch_bounds__(kAcceptThreads, 8) accept_kernel(AcceptArgs a) {
     const int b = blockIdx.y;
     const int ch = blockIdx.x;
     const int N = a.N, Q = 2 * N - 1, V = a.V;

@@ -25,7 +25,8 @@ cudaError_t launch_attention(const Plan& p, const isd_dims* d, const uint16_t* q
                              const int32_t* n_clean, uint16_t* out, void* ws, int32_t* err_flag,
                              cudaStream_t st, int* clear_extra);
 cudaError_t launch_lm_head(const uint16_t* hidden, const uint16_t* W, int Mh, int H, int V,
-                           float* logits, float4* stats_part, int32_t* err_flag, cudaStream_t st);
+                           float* logits, float4* stats_part, void* tail_ws, int32_t* err_flag,
+                           cudaStream_t st);
 cudaError_t launch_row_stats_finalize(const float4* part, int n_parts, int rows,
                                       isd_row_stat* out, cudaStream_t st);
 cudaError_t launch_lora(const Plan& p, const isd_dims* d, const uint16_t* hidden,
@@ -143,7 +144,8 @@ isd_status do_lm_head(const isd_dims* d, const Plan& p, const uint16_t* hidden, 
     // (no second pass over the logits); a small kernel merges them.
     float4* part = row_stats ? reinterpret_cast<float4*>(static_cast<char*>(ws) + p.off_lm_stats)
                              : nullptr;
-    ISD_CUDA(isd::launch_lm_head(h, W, p.M, p.H, d->V, logits, part, err_flag, st));
+    ISD_CUDA(isd::launch_lm_head(h, W, p.M, p.H, d->V, logits, part,
+                                 static_cast<char*>(ws) + p.off_lm_tail, err_flag, st));
     if (row_stats) ISD_CUDA(isd::launch_row_stats_finalize(part, p.lm_stat_parts, p.M, row_stats, st));
     return ISD_OK;
 }

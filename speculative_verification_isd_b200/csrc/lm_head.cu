@@ -47,16 +47,34 @@ struct LmArgs {
     int n_full;                    // tiles dealt in whole waves (a multiple of gridDim.x)
     int tail_split;                // chunks per left-over tile (1: left-over tiles are whole)
     int tail_bn;                   // hidden rows per chunk (multiple of 16)
+    int tail_ksplit;               // K slices per chunk (1: a chunk runs the whole K loop)
+    float* tail_part;              // [chunk CTA][tail_bn][128] fp32 K-slice partials
+    int* tail_ticket;              // [left-over tiles * tail_split], zero at launch
     int w_stages, h_stages;        // depth of the W ring and of the hidden ring (w > h)
     int w_rows, h_rows0, h_rows1;  // TMA box heights (never taller than the tensor)
     uint32_t tmem_cols;
     float* logits;
-    float4* stats_part;  // [Mh][n_tiles * 4] partial row statistics, or null
+    float4* stats_part;  // [Mh][n_tiles] partial row statistics, or null
     int32_t* err_flag;
 };
 
 constexpr int kEpiPitch = 33;  // floats per row of an epilogue transposition buffer
-constexpr int kEpiSmemBytes = 4 * 32 * kEpiPitch * 4;
+// four transposition buffers, then the four warps' row statistics of one
+// 32-column group (merged into one partial per vocabulary tile)
+constexpr int kEpiSmemBytes = 4 * 32 * kEpiPitch * 4 + 4 * 32 * 16;
+
+// named barrier 1 over the four epilogue warps; OR of a predicate
+ISD_DEVINL bool epi_or(bool v) {
+    uint32_t r;
+    asm volatile(
+        "{\n .reg .pred p, q;\n setp.ne.u32 p, %1, 0;\n bar.red.or.pred q, 1, 128, p;\n"
+        " selp.u32 %0, 1, 0, q;\n}\n"
+        : "=r"(r)
+        : "r"((uint32_t)v)
+        : "memory");
+    return r != 0;
+}
+ISD_DEVINL void epi_sync() { asm volatile("bar.sync 1, 128;\n" ::: "memory"); }
 
 constexpr uint64_t kWaitLimitNs = 2000000000ull;
 constexpr int kLmThreads = 224;  // W producer, MMA, 4 epilogue warps, hidden producer
@@ -138,15 +156,19 @@ lm_head_kernel(const __grid_constant__ CUtensorMap tmap_w, const __grid_constant
     const int G = (int)gridDim.x;
     const int n_wave = a.n_full / G;
     const int n_left = a.n_tiles - a.n_full;
-    const int S = a.tail_split;
-    const bool has_extra = (int)blockIdx.x < n_left * S;
+    const int S = a.tail_split, KS = a.tail_ksplit;
+    const bool has_extra = (int)blockIdx.x < n_left * S * KS;
+    const int grp = (int)blockIdx.x / KS;     // left-over tile * S + row chunk of this CTA
+    const int kslice = (int)blockIdx.x % KS;  // its K slice of that chunk
+    const int kb_lo = kslice * kblocks / KS, kb_hi = (kslice + 1) * kblocks / KS;
     const int n_my_tiles = n_wave + (has_extra ? 1 : 0);
-    const int total_kb = n_my_tiles * kblocks;
     auto item_tile = [&](int i) {
-        return i < n_wave ? (int)blockIdx.x + i * G : a.n_full + (int)blockIdx.x / S;
+        return i < n_wave ? (int)blockIdx.x + i * G : a.n_full + grp / S;
     };
     auto item_is_chunk = [&](int i) { return i >= n_wave && S > 1; };
-    const int chunk_row0 = ((int)blockIdx.x % S) * a.tail_bn;  // first hidden row of this CTA's chunk
+    auto item_len = [&](int i) { return item_is_chunk(i) ? kb_hi - kb_lo : kblocks; };
+    const int total_kb = n_wave * kblocks + (has_extra ? item_len(n_wave) : 0);
+    const int chunk_row0 = (grp % S) * a.tail_bn;  // first hidden row of this CTA's chunk
 
     auto give_up = [&]() {
         *abort_flag = 1;
@@ -181,8 +203,8 @@ lm_head_kernel(const __grid_constant__ CUtensorMap tmap_w, const __grid_constant
                     give_up();
                     break;
                 }
-                // a chunk walks K from block 0 like the other chunks of its tile
-                const int kbi = chunk ? jt : kb;
+                // a chunk walks its K slice in order, like the other chunks of its tile
+                const int kbi = chunk ? kb_lo + jt : kb;
                 if (is_w) {
                     mbar_arrive_expect_tx(&full[ws], (uint32_t)a.w_rows * 128u);
                     tma_load_2d(wring + (size_t)ws * kWStageBytes, &tmap_w, &full[ws], kbi * 64,
@@ -199,7 +221,7 @@ lm_head_kernel(const __grid_constant__ CUtensorMap tmap_w, const __grid_constant
                 if (++ws == a.w_stages) { ws = 0; wph ^= 1; }
                 if (++hs == a.h_stages) hs = 0;
                 if (++kb == kblocks) kb = 0;
-                if (++jt == kblocks) {
+                if (++jt == item_len(item)) {
                     jt = 0;
                     ++item;
                     tile = item_tile(item);
@@ -230,7 +252,8 @@ lm_head_kernel(const __grid_constant__ CUtensorMap tmap_w, const __grid_constant
                 const bool chunk = item_is_chunk(lt);
                 const uint32_t idesc = chunk ? idesc_chunk : idesc_full;
                 const int nbs = chunk ? 1 : NB;
-                for (int j = 0; j < kblocks; ++j) {
+                const int len = item_len(lt);
+                for (int j = 0; j < len; ++j) {
                     if (!lm_wait(&full[ws], wph, abort_flag)) {
                         give_up();
                         ok = false;
@@ -273,8 +296,8 @@ lm_head_kernel(const __grid_constant__ CUtensorMap tmap_w, const __grid_constant
                 ok = lm_wait(&tfull[acc], use & 1, abort_flag);
                 if (!ok) give_up();
             }
-            ok = __shfl_sync(0xffffffffu, ok, 0);
-            if (!ok) break;
+            // the four epilogue warps meet at named barriers: they leave together
+            if (epi_or(!ok)) break;
             tc_fence_after();
             const int v = tile * 128 + quarter * 32 + lane;
             const bool v_ok = v < a.V;
@@ -282,63 +305,118 @@ lm_head_kernel(const __grid_constant__ CUtensorMap tmap_w, const __grid_constant
             const uint32_t taddr =
                 tmem_base + ((uint32_t)(quarter * 32) << 16) + (uint32_t)(acc * NB * a.BN);
             float* tb = epi_buf + quarter * 32 * kEpiPitch;
-            float4* part = a.stats_part ? a.stats_part + (size_t)(tile * 4 + quarter) : nullptr;
-            const size_t part_pitch = (size_t)a.n_tiles * 4;
+            float4* part = a.stats_part;
+            float4* wstat = reinterpret_cast<float4*>(epi_buf + 4 * 32 * kEpiPitch);  // [4][32]
+            // logits and merged row statistics of accumulator columns j0..j0+31
+            // (hidden rows mbase..), one value per column in r[]
+            auto emit = [&](const uint32_t (&r)[32], int j0, int mbase) {
+                if (v_ok) {
 #pragma unroll
-            for (int nb = 0; nb < NB; ++nb) {
-                if (nb >= nbs) break;
-                for (int j0 = 0; j0 < bn; j0 += 32) {
-                    uint32_t r[32];
-                    // bn is a multiple of 16: the tail is one 16-column load,
-                    // so no load reaches past the allocated columns
-                    if (bn - j0 >= 32)
-                        tmem_ld_32x32b_x32(taddr + nb * a.BN + j0, r);
-                    else
-                        tmem_ld_32x32b_x16(taddr + nb * a.BN + j0, r);
-                    tmem_ld_wait();
-                    const int mbase = row0 + nb * a.BN + j0;
-                    if (v_ok) {
-#pragma unroll
-                        for (int k = 0; k < 32; ++k) {
-                            const int m = mbase + k;
-                            if (j0 + k < bn && m < a.Mh)
-                                a.logits[(size_t)m * a.V + v] = __uint_as_float(r[k]);
-                        }
-                    }
-                    if (part) {
-                        // Row statistics of this warp's 32 vocabulary entries:
-                        // transpose through shared memory so that lane k holds
-                        // logits row mbase + k, then max / sum-exp / argmax
-                        // (first index among equal maxima).
-#pragma unroll
-                        for (int k = 0; k < 32; ++k) tb[lane * kEpiPitch + k] = __uint_as_float(r[k]);
-                        __syncwarp();
-                        float x[32];
-                        float mx = -INFINITY;
-                        int arg = 0;
-#pragma unroll
-                        for (int i = 0; i < 32; ++i) {
-                            x[i] = tb[i * kEpiPitch + lane];
-                            if (i < nvalid && x[i] > mx) {
-                                mx = x[i];
-                                arg = i;
-                            }
-                        }
-                        float se = 0.f;
-#pragma unroll
-                        for (int i = 0; i < 32; ++i)
-                            if (i < nvalid) se += __expf(x[i] - mx);
-                        const int m = mbase + lane;
-                        if (j0 + lane < bn && m < a.Mh)
-                            part[(size_t)m * part_pitch] =
-                                make_float4(mx, se, __int_as_float(tile * 128 + quarter * 32 + arg), 0.f);
-                        __syncwarp();
+                    for (int k = 0; k < 32; ++k) {
+                        const int m = mbase + k;
+                        if (j0 + k < bn && m < a.Mh) a.logits[(size_t)m * a.V + v] = __uint_as_float(r[k]);
                     }
                 }
+                if (!part) return;
+                // Row statistics of this warp's 32 vocabulary entries: transpose
+                // through shared memory so that lane k holds logits row mbase + k,
+                // then max / sum-exp / argmax (first index among equal maxima).
+#pragma unroll
+                for (int k = 0; k < 32; ++k) tb[lane * kEpiPitch + k] = __uint_as_float(r[k]);
+                __syncwarp();
+                float x[32];
+                float mx = -INFINITY;
+                int arg = 0;
+#pragma unroll
+                for (int i = 0; i < 32; ++i) {
+                    x[i] = tb[i * kEpiPitch + lane];
+                    if (i < nvalid && x[i] > mx) {
+                        mx = x[i];
+                        arg = i;
+                    }
+                }
+                float se = 0.f;
+#pragma unroll
+                for (int i = 0; i < 32; ++i)
+                    if (i < nvalid) se += __expf(x[i] - mx);
+                // the four warps' statistics of row m merged in vocabulary
+                // order into one partial per tile
+                wstat[quarter * 32 + lane] =
+                    make_float4(mx, se, __int_as_float(tile * 128 + quarter * 32 + arg), 0.f);
+                epi_sync();
+                if (quarter == 0) {
+                    RowStat st = rowstat_empty();
+#pragma unroll
+                    for (int q = 0; q < 4; ++q) {
+                        const float4 e = wstat[q * 32 + lane];
+                        st = rowstat_merge(st, RowStat{e.x, e.y, __float_as_int(e.z)});
+                    }
+                    const int m = mbase + lane;
+                    if (j0 + lane < bn && m < a.Mh)
+                        part[(size_t)m * a.n_tiles + tile] = make_float4(st.m, st.s, __int_as_float(st.idx), 0.f);
+                }
+                epi_sync();
+            };
+            // bn is a multiple of 16: the last column group may be one
+            // 16-column load, so no load reaches past the allocated columns
+            auto load_cols = [&](uint32_t taddr_c, int ncols, uint32_t (&r)[32]) {
+                if (ncols >= 32)
+                    tmem_ld_32x32b_x32(taddr_c, r);
+                else
+                    tmem_ld_32x32b_x16(taddr_c, r);
+                tmem_ld_wait();
+            };
+            if (!(chunk && KS > 1)) {
+#pragma unroll
+                for (int nb = 0; nb < NB; ++nb) {
+                    if (nb >= nbs) break;
+                    for (int j0 = 0; j0 < bn; j0 += 32) {
+                        uint32_t r[32];
+                        load_cols(taddr + nb * a.BN + j0, bn - j0, r);
+                        emit(r, j0, row0 + nb * a.BN + j0);
+                    }
+                }
+                tc_fence_before();
+                __syncwarp();
+                if (lane == 0) mbar_arrive(&tempty[acc]);
+            } else {
+                // One K slice of a row chunk: the fp32 partial goes to this CTA's
+                // slot (column-major, lanes = vocabulary rows); the last slice to
+                // finish sums the slices in K order and emits the chunk.
+                const int vl = quarter * 32 + lane;
+                float* mine = a.tail_part + (size_t)blockIdx.x * bn * 128;
+                for (int j0 = 0; j0 < bn; j0 += 32) {
+                    uint32_t r[32];
+                    load_cols(taddr + j0, bn - j0, r);
+#pragma unroll
+                    for (int k = 0; k < 32; ++k)
+                        if (j0 + k < bn) mine[(size_t)(j0 + k) * 128 + vl] = __uint_as_float(r[k]);
+                }
+                tc_fence_before();
+                __syncwarp();
+                if (lane == 0) mbar_arrive(&tempty[acc]);
+                __threadfence();
+                epi_sync();
+                bool last = false;
+                if (quarter == 0 && lane == 0) last = atomicAdd(&a.tail_ticket[grp], 1) == KS - 1;
+                if (epi_or(last)) {
+                    __threadfence();
+                    const float* slices = a.tail_part + (size_t)grp * KS * bn * 128;
+                    for (int j0 = 0; j0 < bn; j0 += 32) {
+                        uint32_t r[32];
+#pragma unroll
+                        for (int k = 0; k < 32; ++k) {
+                            float acc_v = 0.f;
+                            if (j0 + k < bn)
+                                for (int q = 0; q < KS; ++q)
+                                    acc_v += __ldcg(slices + ((size_t)q * bn + j0 + k) * 128 + vl);
+                            r[k] = __float_as_uint(acc_v);
+                        }
+                        emit(r, j0, row0 + j0);
+                    }
+                    if (quarter == 0 && lane == 0) a.tail_ticket[grp] = 0;
+                }
             }
-            tc_fence_before();
-            __syncwarp();
-            if (lane == 0) mbar_arrive(&tempty[acc]);
         }
     }
     tc_fence_before();
@@ -416,7 +494,8 @@ static int num_sms_of_current_device() {
 void set_error_detail(const char* msg);
 
 cudaError_t launch_lm_head(const uint16_t* hidden, const uint16_t* W, int Mh, int H, int V,
-                           float* logits, float4* stats_part, int32_t* err_flag, cudaStream_t st) {
+                           float* logits, float4* stats_part, void* tail_ws, int32_t* err_flag,
+                           cudaStream_t st) {
     // dynamic shared memory available to this kernel on the current device
     static int smem_limit_dev[64];
     int dev = 0;
@@ -500,6 +579,26 @@ cudaError_t launch_lm_head(const uint16_t* hidden, const uint16_t* W, int Mh, in
             if (S >= 2) {
                 a.tail_split = S;
                 a.tail_bn = bn;
+            }
+        }
+    }
+    // row chunks of at most 64 rows may also be split along K when CTAs are
+    // still idle; the slices' partials and counters live in tail_ws
+    a.tail_ksplit = 1;
+    a.tail_part = nullptr;
+    a.tail_ticket = nullptr;
+    if (a.tail_split > 1 && a.tail_bn <= 64 && grid <= kNumSMs && tail_ws) {
+        int ks = grid / (left * a.tail_split);
+        if (ks > 8) ks = 8;
+        if (ks > H / 64) ks = H / 64;
+        if (ks >= 2) {
+            a.tail_ksplit = ks;
+            a.tail_part = static_cast<float*>(tail_ws);
+            a.tail_ticket = reinterpret_cast<int*>(static_cast<char*>(tail_ws) + kLmTailPartBytes);
+            const cudaError_t me = cudaMemsetAsync(a.tail_ticket, 0, (size_t)left * a.tail_split * 4, st);
+            if (me != cudaSuccess) {
+                set_error_detail("lm_head: clearing the left-over tile counters");
+                return me;
             }
         }
     }

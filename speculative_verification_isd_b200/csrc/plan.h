@@ -13,10 +13,12 @@ constexpr int kAttnKeyTile = 64;      // keys per pipeline stage
 constexpr int kAttnRowsPerGroup = 16; // query rows handled by one 4-warp group
 constexpr int kAttnMaxSplit = 2048;   // keys per split at most (bounds the key table)
 constexpr int kStatsThreads = 256;
-constexpr int kFinalizeThreads = 1024;  // one CTA per row merges its statistics partials
+constexpr int kFinalizeThreads = 256;   // one CTA per row merges its statistics partials
 constexpr int kAcceptThreads = 256;
 constexpr int kAcceptChunk = 4096;    // vocabulary entries per accept CTA
 constexpr int kNumSMs = 148;
+constexpr size_t kLmTailPartBytes = (size_t)kNumSMs * 64 * 128 * 4;
+constexpr size_t kLmTailBytes = kLmTailPartBytes + (size_t)kNumSMs * 4;
 
 struct Plan {
     // derived dims
@@ -36,12 +38,12 @@ struct Plan {
     int acc_chunks;
     // R-ISD LoRA
     int lora_rows, lora_ksplit;
-    // LM-head row-statistics partials: one per (128-entry vocabulary tile, warp)
+    // LM-head row-statistics partials: one per 128-entry vocabulary tile
     int lm_stat_parts;
     // workspace offsets (bytes)
     size_t off_attn_part, off_attn_ticket, off_hidden, off_hidden_lora, off_lora_t,
         off_stats_part, off_stats_ticket, off_acc_part, off_acc_ticket, off_lora_part,
-        off_lm_stats, total;
+        off_lm_stats, off_lm_tail, total;
 };
 
 inline size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
@@ -120,8 +122,11 @@ inline bool make_plan(const isd_dims* d, Plan* p) {
     p->off_acc_part = take((size_t)d->B * (d->N + 1) * p->acc_chunks * 4);
     p->off_acc_ticket = take((size_t)d->B * 4);
     p->off_lora_part = take(d->lora_rank ? (size_t)p->lora_ksplit * p->lora_rows * d->lora_rank * 4 : 0);
-    p->lm_stat_parts = ((d->V + 127) / 128) * 4;
+    p->lm_stat_parts = (d->V + 127) / 128;
     p->off_lm_stats = take((size_t)p->M * p->lm_stat_parts * 16);
+    // LM head, left-over vocabulary tiles: K-slice partials (at most one per
+    // CTA, up to 64 hidden rows x 128 entries) and their counters
+    p->off_lm_tail = take(kLmTailBytes);
     p->total = off;
     return true;
 }
