@@ -382,6 +382,23 @@ def main():
     st_ms = stage.mean(axis=0)
     t_attn, t_lm, t_acc = [float(x) for x in st_ms]
 
+    # ---------------- R-ISD gated LoRA: cost of the adapter (same steps with it off)
+    lora_alpha = None
+    if cfg.lora_rank:
+        KL = min(K, 300)
+        for k in range(W):
+            wl.set_uniforms(k)
+            wl.step(without_lora=True)
+        f0, f1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        f0.record(stream)
+        for k in range(KL):
+            wl.set_uniforms(k)
+            wl.step(without_lora=True)
+        f1.record(stream)
+        torch.cuda.synchronize()
+        t_plain = allreduce_max(f0.elapsed_time(f1), world) / KL
+        lora_alpha = (t_ms / K) / t_plain
+
     # ---------------- e2e: public API with host buffers, copies inside the timed region
     # A step's inputs travel in one pinned host buffer (one host-to-device
     # copy), its integer results come back in one (one device-to-host copy);
@@ -446,10 +463,13 @@ def main():
                                        "accept": t_acc}},
         "e2e": {"value": e2e_value, "unit": "ISD steps/s", "h2d_bytes_per_step": int(h2d),
                 "d2h_bytes_per_step": int(d2h), "steps": KE},
-        # attention, LM head, row-stats merge, accept (+ 3 LoRA kernels)
-        "gpu_launches": K * (4 + (3 if cfg.lora_rank else 0)),
+        # KV append, attention, LM head, row-stats merge, accept (+ 3 LoRA kernels)
+        "gpu_launches": K * (5 + (3 if cfg.lora_rank else 0)),
         "clocks": clk, "err_flags": flags,
     }
+    if lora_alpha is not None:
+        # step time with the adapter / without it (the pages report about 1.12)
+        line["lora_alpha"] = lora_alpha
     if world == 1 and rank == 0 and not args.no_cpu_baseline:
         line["cpu_baseline"] = cpu_baseline(wl, cfg, args.cpu_budget_s)
     if rank == 0:

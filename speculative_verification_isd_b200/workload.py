@@ -154,13 +154,20 @@ class DeviceWorkload:
             o += sz
         return buf, obuf, layout
 
-    def step(self, stream=None):
-        self.isd.step(self.dims, self.q, self.k_new, self.v_new, self.k_pool, self.v_pool,
+    def step(self, stream=None, without_lora=False):
+        """One isd_step; without_lora runs the same step with the adapter off
+        (dims with lora_rank 0), for measuring the adapter's cost."""
+        dims, la, lb = self.dims, self.lora_A, self.lora_B
+        if without_lora:
+            dims = type(self.dims).from_buffer_copy(self.dims)
+            dims.lora_rank = 0
+            la = lb = None
+        self.isd.step(dims, self.q, self.k_new, self.v_new, self.k_pool, self.v_pool,
                       self.page_table, self.kv_len, self.n_clean, self.clean_tok, self.W,
                       self.prev_logits, self.prev_row_stats, self.uniforms, self.logits,
                       self.row_stats, self.accept_len, self.out_tok, self.next_n_clean,
                       self.next_clean_tok, self.next_kv_len, self.ws, hidden=self.hidden,
-                      ratio=self.ratio, lora_A=self.lora_A, lora_B=self.lora_B,
+                      ratio=self.ratio, lora_A=la, lora_B=lb,
                       err_flag=self.err, stream=stream)
 
     def outputs(self) -> Dict[str, np.ndarray]:
