@@ -175,6 +175,8 @@ isd_status isd_accept(const isd_dims* d, const float* logits, const isd_row_stat
  * `hidden` [B*Q, H] bf16 receives the attention output if non-NULL (else it
  * stays in ws).  `logits` and `row_stats` are outputs of this step and become
  * the caller's prev_logits / prev_row_stats for the next one.
+ * The step issues no memset and no host synchronisation: its first kernel
+ * also clears the counters the later kernels use.
  */
 isd_status isd_step(const isd_dims* d, const uint16_t* q, const uint16_t* k_new,
                     const uint16_t* v_new, uint16_t* k_pool, uint16_t* v_pool,

@@ -16,6 +16,7 @@
 // last-block-done ticket: every CTA publishes its partial, fences, and the
 // CTA that draws the last ticket combines; nothing spins.
 #include "common.cuh"
+#include "launch.h"
 #include "plan.h"
 
 namespace isd {
@@ -71,6 +72,8 @@ template <int THREADS>
 __global__ void __launch_bounds__(THREADS)
 row_stats_finalize_kernel(const float4* __restrict__ part, int n_parts,
                           isd_row_stat* __restrict__ out) {
+    pdl_trigger();
+    pdl_wait();
     const int row = blockIdx.x;
     const float4* pr = part + (size_t)row * n_parts;
     RowStat st = rowstat_empty();
@@ -227,6 +230,8 @@ ISD_DEVINL float chunk_scan(const SweepRow& r, int beg, int end, float target, i
 }
 
 __global__ void __launch_bounds__(kAcceptThreads, 8) accept_kernel(AcceptArgs a) {
+    pdl_trigger();
+    pdl_wait();
     const int b = blockIdx.y;
     const int ch = blockIdx.x;
     const int N = a.N, Q = 2 * N - 1, V = a.V;
@@ -428,9 +433,9 @@ cudaError_t launch_row_stats(const Plan& p, const float* logits, int rows, int V
 }
 
 cudaError_t launch_row_stats_finalize(const float4* part, int n_parts, int rows,
-                                      isd_row_stat* out, cudaStream_t st) {
-    row_stats_finalize_kernel<kFinalizeThreads><<<rows, kFinalizeThreads, 0, st>>>(part, n_parts, out);
-    return cudaGetLastError();
+                                      isd_row_stat* out, cudaStream_t st, bool pdl) {
+    return launch_kernel(pdl, row_stats_finalize_kernel<kFinalizeThreads>, dim3(rows),
+                         dim3(kFinalizeThreads), 0, st, part, n_parts, out);
 }
 
 cudaError_t launch_accept(const Plan& p, const isd_dims* d, const float* logits,
@@ -439,7 +444,7 @@ cudaError_t launch_accept(const Plan& p, const isd_dims* d, const float* logits,
                           const int32_t* clean_tok, const int32_t* kv_len, const float* uniforms,
                           int32_t* accept_len, int32_t* out_tok, int32_t* next_n_clean,
                           int32_t* next_clean_tok, int32_t* next_kv_len, float* ratio, void* ws,
-                          int32_t* err_flag, cudaStream_t st) {
+                          int32_t* err_flag, cudaStream_t st, bool pdl) {
     char* w = static_cast<char*>(ws);
     AcceptArgs a;
     a.B = d->B;
@@ -465,8 +470,7 @@ cudaError_t launch_accept(const Plan& p, const isd_dims* d, const float* logits,
     a.n_chunks = p.acc_chunks;
     a.err_flag = err_flag;
     dim3 grid(p.acc_chunks, d->B);
-    accept_kernel<<<grid, kAcceptThreads, 0, st>>>(a);
-    return cudaGetLastError();
+    return launch_kernel(pdl, accept_kernel, grid, dim3(kAcceptThreads), 0, st, a);
 }
 
 }  // namespace isd

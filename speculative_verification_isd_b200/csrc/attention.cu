@@ -504,25 +504,30 @@ cudaError_t launch_attention_tc(const Plan& p, const isd_dims* d, const uint16_t
                                 const uint16_t* k_new, const uint16_t* v_new, uint16_t* k_pool,
                                 uint16_t* v_pool, const int32_t* page_table, const int32_t* kv_len,
                                 const int32_t* n_clean, uint16_t* out, void* ws, int32_t* err_flag,
-                                cudaStream_t st, int* clear_extra, bool* handled);
+                                cudaStream_t st, int* clear_extra, int* clear_range, int clear_count,
+                                bool pdl, bool* handled);
 
 // The tensor-core kernel (attention_tc.cu) where the shape fits it, else the
 // general mma.sync kernel above.  Either way the attention counters in the
 // workspace are cleared on the stream first, and so are the B counters at
-// clear_extra when it is not null.
+// clear_extra and the clear_count counters at clear_range when not null.
+// pdl: launched as part of the whole step (programmatic dependent launch).
 cudaError_t launch_attention(const Plan& p, const isd_dims* d, const uint16_t* q,
                              const uint16_t* k_new, const uint16_t* v_new, uint16_t* k_pool,
                              uint16_t* v_pool, const int32_t* page_table, const int32_t* kv_len,
                              const int32_t* n_clean, uint16_t* out, void* ws, int32_t* err_flag,
-                             cudaStream_t st, int* clear_extra) {
+                             cudaStream_t st, int* clear_extra, int* clear_range, int clear_count,
+                             bool pdl) {
     bool handled = false;
     const cudaError_t te = launch_attention_tc(p, d, q, k_new, v_new, k_pool, v_pool, page_table,
                                                kv_len, n_clean, out, ws, err_flag, st, clear_extra,
-                                               &handled);
+                                               clear_range, clear_count, pdl, &handled);
     if (handled || te != cudaSuccess) return te;
     cudaError_t me = cudaMemsetAsync(static_cast<char*>(ws) + p.off_attn_ticket, 0,
                                      (size_t)d->B * d->Hkv * p.attn_rgb * 4, st);
     if (me == cudaSuccess && clear_extra) me = cudaMemsetAsync(clear_extra, 0, (size_t)d->B * 4, st);
+    if (me == cudaSuccess && clear_range && clear_count > 0)
+        me = cudaMemsetAsync(clear_range, 0, (size_t)clear_count * 4, st);
     if (me != cudaSuccess) return me;
     char* w = static_cast<char*>(ws);
     AttnArgs a;

@@ -36,6 +36,7 @@
 #include "common.cuh"
 #include "plan.h"
 #include "sm100.cuh"
+#include "launch.h"
 #include "tmap.h"
 
 namespace isd {
@@ -85,10 +86,16 @@ ISD_DEVINL int tc_total_keys(const TcArgs& a, int b) {
 // for all kv heads go into their page, 16 bytes per thread.  The CTA of block
 // position 0 also clears the request's attention counters (and, if given, one
 // more counter per request for the kernels that follow), and writes zero
-// attention output for a request that cannot be served.
+// attention output for a request that cannot be served; CTA (0, 0) clears
+// clear_count more counters at clear_range (for later kernels of the step).
 __global__ void kv_append_kernel(TcArgs a, const __nv_bfloat16* k_new, const __nv_bfloat16* v_new,
-                                 __nv_bfloat16* k_pool, __nv_bfloat16* v_pool, int* clear_extra) {
+                                 __nv_bfloat16* k_pool, __nv_bfloat16* v_pool, int* clear_extra,
+                                 int* clear_range, int clear_count) {
+    pdl_trigger();
+    pdl_wait();
     const int b = blockIdx.x, r = blockIdx.y;
+    if (clear_range && b == 0 && r == 0)
+        for (int i = threadIdx.x; i < clear_count; i += blockDim.x) clear_range[i] = 0;
     const int kv = a.kv_len[b], c = a.n_clean[b];
     const bool bad_c = (c < 1 || c > a.N);
     const long long want = bad_c ? 0 : (long long)kv + c + a.N - 1;
@@ -217,6 +224,7 @@ attention_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_const
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int n_units = a.B * a.Hkv;
+    pdl_trigger();
 
     // ---- set-up
     if (threadIdx.x == 0) {
@@ -249,6 +257,8 @@ attention_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_const
     // Q rows past `rows` stay zero (no TMA box covers them)
     for (int i = threadIdx.x; i < (int)(2 * kQBytes / 16); i += kThreads)
         reinterpret_cast<uint4*>(sQ)[i] = make_uint4(0, 0, 0, 0);
+    // everything below reads what the KV append (the preceding kernel) wrote
+    pdl_wait();
     for (int b = threadIdx.x; b < a.B; b += kThreads) {
         kvs[b] = a.kv_len[b];
         cs[b] = a.n_clean[b];
@@ -840,7 +850,7 @@ bool encode_bf16_4d(CUtensorMap* m, const void* ptr, const uint64_t dims[4],
 
 template <int R, int STAGES>
 cudaError_t launch_tc(const TcArgs& a, const CUtensorMap& tk, const CUtensorMap& tv,
-                      const CUtensorMap& tq, size_t smem, cudaStream_t st) {
+                      const CUtensorMap& tq, size_t smem, cudaStream_t st, bool pdl) {
     static unsigned long long configured = 0;  // bit per device
     int dev = 0;
     cudaGetDevice(&dev);
@@ -853,8 +863,8 @@ cudaError_t launch_tc(const TcArgs& a, const CUtensorMap& tk, const CUtensorMap&
         if (e != cudaSuccess) return e;
         configured |= 1ull << dev;
     }
-    attention_tc_kernel<R, STAGES><<<kNumSMs, TcRoles<R>::kThreads, smem, st>>>(tk, tv, tq, a);
-    return cudaGetLastError();
+    return launch_kernel(pdl, attention_tc_kernel<R, STAGES>, dim3(kNumSMs), dim3(TcRoles<R>::kThreads),
+                         smem, st, tk, tv, tq, a);
 }
 
 }  // namespace
@@ -867,7 +877,8 @@ cudaError_t launch_attention_tc(const Plan& p, const isd_dims* d, const uint16_t
                                 const uint16_t* k_new, const uint16_t* v_new, uint16_t* k_pool,
                                 uint16_t* v_pool, const int32_t* page_table, const int32_t* kv_len,
                                 const int32_t* n_clean, uint16_t* out, void* ws, int32_t* err_flag,
-                                cudaStream_t st, int* clear_extra, bool* handled) {
+                                cudaStream_t st, int* clear_extra, int* clear_range, int clear_count,
+                                bool pdl, bool* handled) {
     *handled = false;
     const int R = p.attn_tc_rows;
     if (R == 0) return cudaSuccess;
@@ -927,14 +938,17 @@ cudaError_t launch_attention_tc(const Plan& p, const isd_dims* d, const uint16_t
     a.ticket = reinterpret_cast<int*>(static_cast<char*>(ws) + p.off_attn_ticket);
     a.err_flag = err_flag;
     const int append_threads = (Hkv * 16 + 31) / 32 * 32;
-    kv_append_kernel<<<dim3(d->B, 2 * d->N - 1), append_threads > 1024 ? 1024 : append_threads, 0, st>>>(
-        a, reinterpret_cast<const __nv_bfloat16*>(k_new), reinterpret_cast<const __nv_bfloat16*>(v_new),
-        reinterpret_cast<__nv_bfloat16*>(k_pool), reinterpret_cast<__nv_bfloat16*>(v_pool), clear_extra);
-    cudaError_t e = cudaGetLastError();
+    cudaError_t e = launch_kernel(pdl, kv_append_kernel, dim3(d->B, 2 * d->N - 1),
+                                  dim3(append_threads > 1024 ? 1024 : append_threads), 0, st, a,
+                                  reinterpret_cast<const __nv_bfloat16*>(k_new),
+                                  reinterpret_cast<const __nv_bfloat16*>(v_new),
+                                  reinterpret_cast<__nv_bfloat16*>(k_pool),
+                                  reinterpret_cast<__nv_bfloat16*>(v_pool), clear_extra, clear_range,
+                                  clear_count);
     if (e != cudaSuccess) return e;
-    if (R == 16) return stages == 3 ? launch_tc<16, 3>(a, tk, tv, tq, smem, st) : launch_tc<16, 2>(a, tk, tv, tq, smem, st);
-    if (R == 32) return stages == 3 ? launch_tc<32, 3>(a, tk, tv, tq, smem, st) : launch_tc<32, 2>(a, tk, tv, tq, smem, st);
-    return stages == 3 ? launch_tc<64, 3>(a, tk, tv, tq, smem, st) : launch_tc<64, 2>(a, tk, tv, tq, smem, st);
+    if (R == 16) return stages == 3 ? launch_tc<16, 3>(a, tk, tv, tq, smem, st, pdl) : launch_tc<16, 2>(a, tk, tv, tq, smem, st, pdl);
+    if (R == 32) return stages == 3 ? launch_tc<32, 3>(a, tk, tv, tq, smem, st, pdl) : launch_tc<32, 2>(a, tk, tv, tq, smem, st, pdl);
+    return stages == 3 ? launch_tc<64, 3>(a, tk, tv, tq, smem, st, pdl) : launch_tc<64, 2>(a, tk, tv, tq, smem, st, pdl);
 }
 
 }  // namespace isd

@@ -11,6 +11,13 @@
 
 namespace isd {
 
+// Programmatic dependent launch: wait until the preceding kernel of the
+// stream has completed and its memory is visible (a no-op for a kernel
+// launched without the attribute); allow the next kernel to be scheduled.
+ISD_DEVINL void pdl_wait() { asm volatile("griddepcontrol.wait;\n" ::: "memory"); }
+ISD_DEVINL void pdl_trigger() { asm volatile("griddepcontrol.launch_dependents;\n" ::: "memory"); }
+
+
 ISD_DEVINL void raise_flag(int32_t* err_flag, int32_t bit) {
     if (err_flag) atomicOr(err_flag, bit);
 }

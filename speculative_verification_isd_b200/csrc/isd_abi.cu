@@ -23,12 +23,13 @@ cudaError_t launch_attention(const Plan& p, const isd_dims* d, const uint16_t* q
                              const uint16_t* k_new, const uint16_t* v_new, uint16_t* k_pool,
                              uint16_t* v_pool, const int32_t* page_table, const int32_t* kv_len,
                              const int32_t* n_clean, uint16_t* out, void* ws, int32_t* err_flag,
-                             cudaStream_t st, int* clear_extra);
+                             cudaStream_t st, int* clear_extra, int* clear_range, int clear_count,
+                             bool pdl);
 cudaError_t launch_lm_head(const uint16_t* hidden, const uint16_t* W, int Mh, int H, int V,
                            float* logits, float4* stats_part, void* tail_ws, int32_t* err_flag,
-                           cudaStream_t st);
+                           cudaStream_t st, bool pdl, bool counters_cleared);
 cudaError_t launch_row_stats_finalize(const float4* part, int n_parts, int rows,
-                                      isd_row_stat* out, cudaStream_t st);
+                                      isd_row_stat* out, cudaStream_t st, bool pdl);
 cudaError_t launch_lora(const Plan& p, const isd_dims* d, const uint16_t* hidden,
                         const uint16_t* lora_A, const uint16_t* lora_B, uint16_t* hidden_out,
                         void* ws, cudaStream_t st);
@@ -40,7 +41,7 @@ cudaError_t launch_accept(const Plan& p, const isd_dims* d, const float* logits,
                           const int32_t* clean_tok, const int32_t* kv_len, const float* uniforms,
                           int32_t* accept_len, int32_t* out_tok, int32_t* next_n_clean,
                           int32_t* next_clean_tok, int32_t* next_kv_len, float* ratio, void* ws,
-                          int32_t* err_flag, cudaStream_t st);
+                          int32_t* err_flag, cudaStream_t st, bool pdl);
 }  // namespace isd
 
 using isd::Plan;
@@ -115,23 +116,39 @@ isd_status check_accept_shape(const isd_dims* d) {
         if (e_ != cudaSuccess) return cuda_fail(e_); \
     } while (0)
 
+// The step's kernels can be launched with programmatic dependent launch
+// (launch.h).  On B200 at B=32, N=4 that measured slower than plain stream
+// order (0.516 vs 0.500 ms per step, alternating runs in one process: the LM
+// head's early W stream competes with the attention's last CTAs for HBM), so
+// it is off.
+constexpr bool kStepPdl = false;
+
 isd_status do_attention(const isd_dims* d, const Plan& p, const uint16_t* q,
                         const uint16_t* k_new, const uint16_t* v_new, uint16_t* k_pool,
                         uint16_t* v_pool, const int32_t* page_table, const int32_t* kv_len,
                         const int32_t* n_clean, uint16_t* out, void* ws, int32_t* err_flag,
-                        cudaStream_t st, int* clear_extra = nullptr) {
+                        cudaStream_t st, bool in_step = false) {
     if (!q || !k_new || !v_new || !k_pool || !v_pool || !page_table || !kv_len || !n_clean || !out)
         return invalid("null attention pointer");
     ISD_TRY(check_attention_shape(d, p));
-    // the launch clears the attention counters (and clear_extra) on the stream
+    // The launch clears the attention counters on the stream; inside the whole
+    // step it also clears the step's accept and LM-head counters.
+    int* acc_ticket = nullptr;
+    int* lm_ticket = nullptr;
+    if (in_step) {
+        acc_ticket = reinterpret_cast<int*>(static_cast<char*>(ws) + p.off_acc_ticket);
+        lm_ticket = reinterpret_cast<int*>(static_cast<char*>(ws) + p.off_lm_tail + isd::kLmTailPartBytes);
+    }
     ISD_CUDA(isd::launch_attention(p, d, q, k_new, v_new, k_pool, v_pool, page_table, kv_len,
-                                   n_clean, out, ws, err_flag, st, clear_extra));
+                                   n_clean, out, ws, err_flag, st, acc_ticket, lm_ticket,
+                                   in_step ? isd::kNumSMs : 0, kStepPdl));
     return ISD_OK;
 }
 
 isd_status do_lm_head(const isd_dims* d, const Plan& p, const uint16_t* hidden, const uint16_t* W,
                       const uint16_t* lora_A, const uint16_t* lora_B, float* logits,
-                      isd_row_stat* row_stats, void* ws, int32_t* err_flag, cudaStream_t st) {
+                      isd_row_stat* row_stats, void* ws, int32_t* err_flag, cudaStream_t st,
+                      bool in_step = false) {
     if (!hidden || !W || !logits) return invalid("null lm-head pointer");
     ISD_TRY(check_lm_shape(d, p, lora_A, lora_B));
     const uint16_t* h = hidden;
@@ -145,8 +162,11 @@ isd_status do_lm_head(const isd_dims* d, const Plan& p, const uint16_t* hidden, 
     float4* part = row_stats ? reinterpret_cast<float4*>(static_cast<char*>(ws) + p.off_lm_stats)
                              : nullptr;
     ISD_CUDA(isd::launch_lm_head(h, W, p.M, p.H, d->V, logits, part,
-                                 static_cast<char*>(ws) + p.off_lm_tail, err_flag, st));
-    if (row_stats) ISD_CUDA(isd::launch_row_stats_finalize(part, p.lm_stat_parts, p.M, row_stats, st));
+                                 static_cast<char*>(ws) + p.off_lm_tail, err_flag, st,
+                                 in_step && kStepPdl, in_step));
+    if (row_stats)
+        ISD_CUDA(isd::launch_row_stats_finalize(part, p.lm_stat_parts, p.M, row_stats, st,
+                                                in_step && kStepPdl));
     return ISD_OK;
 }
 
@@ -233,7 +253,8 @@ static isd_status accept_impl(const isd_dims* d, const float* logits, const isd_
         ISD_CUDA(cudaMemsetAsync(static_cast<char*>(ws) + p.off_acc_ticket, 0, (size_t)d->B * 4, st));
     ISD_CUDA(isd::launch_accept(p, d, logits, row_stats, prev_logits, prev_row_stats, n_clean,
                                 clean_tok, kv_len, uniforms, accept_len, out_tok, next_n_clean,
-                                next_clean_tok, next_kv_len, ratio, ws, err_flag, st));
+                                next_clean_tok, next_kv_len, ratio, ws, err_flag, st,
+                                !clear_counters && kStepPdl));
     return ISD_OK;
 }
 
@@ -268,12 +289,11 @@ isd_status isd_step(const isd_dims* d, const uint16_t* q, const uint16_t* k_new,
     cudaStream_t st = static_cast<cudaStream_t>(stream);
     uint16_t* h = hidden ? hidden
                          : reinterpret_cast<uint16_t*>(static_cast<char*>(ws) + p.off_hidden);
-    // the attention launch also clears the accept counters, so the step
-    // issues no separate memset
-    int* acc_ticket = reinterpret_cast<int*>(static_cast<char*>(ws) + p.off_acc_ticket);
+    // The attention launch also clears the accept and LM-head counters, so the
+    // step issues no separate memset.
     ISD_TRY(do_attention(d, p, q, k_new, v_new, k_pool, v_pool, page_table, kv_len, n_clean, h,
-                         ws, err_flag, st, acc_ticket));
-    ISD_TRY(do_lm_head(d, p, h, W, lora_A, lora_B, logits, row_stats, ws, err_flag, st));
+                         ws, err_flag, st, true));
+    ISD_TRY(do_lm_head(d, p, h, W, lora_A, lora_B, logits, row_stats, ws, err_flag, st, true));
     return accept_impl(d, logits, row_stats, prev_logits, prev_row_stats, n_clean, clean_tok,
                        kv_len, uniforms, accept_len, out_tok, next_n_clean, next_clean_tok,
                        next_kv_len, ratio, ws, ws_bytes, err_flag, stream, false);

@@ -37,6 +37,7 @@
 #include "common.cuh"
 #include "plan.h"
 #include "sm100.cuh"
+#include "launch.h"
 #include "tmap.h"
 
 namespace isd {
@@ -121,6 +122,7 @@ lm_head_kernel(const __grid_constant__ CUtensorMap tmap_w, const __grid_constant
     __shared__ int never;  // a flag nothing sets: used by the final drains
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    pdl_trigger();
     if (threadIdx.x == 0) {
         for (int s = 0; s < a.w_stages; ++s) {
             mbar_init(&full[s], 2);
@@ -180,6 +182,10 @@ lm_head_kernel(const __grid_constant__ CUtensorMap tmap_w, const __grid_constant
             // ---------------- TMA producers: warp 0 streams W from HBM through
             // the deep ring; warp 6 feeds the L2-resident hidden tiles
             const bool is_w = (warp == 0);
+            // under programmatic dependent launch W (which no earlier kernel
+            // of the step writes) streams at once; the hidden rows come from
+            // the preceding kernel and wait for it
+            if (!is_w) pdl_wait();
             const uint64_t pol = is_w ? policy_evict_first() : policy_evict_last();
             const uint64_t pol_keep = policy_evict_last();
             int ws = 0, hs = 0, kb = kb0, item = 0, jt = 0;
@@ -283,6 +289,7 @@ lm_head_kernel(const __grid_constant__ CUtensorMap tmap_w, const __grid_constant
     } else {
         // ---------------- epilogue: warps 2..5 cover TMEM lane quarters 2,3,0,1
         const int quarter = warp & 3;
+        pdl_wait();  // logits, statistics and counters are shared with earlier kernels
         for (int lt = 0; lt < n_my_tiles; ++lt) {
             const int tile = item_tile(lt);
             const bool chunk = item_is_chunk(lt);
@@ -493,9 +500,12 @@ static int num_sms_of_current_device() {
 
 void set_error_detail(const char* msg);
 
+// pdl: launched as part of the whole step (programmatic dependent launch);
+// counters_cleared: an earlier kernel of the step already cleared the
+// left-over-tile counters in tail_ws.
 cudaError_t launch_lm_head(const uint16_t* hidden, const uint16_t* W, int Mh, int H, int V,
                            float* logits, float4* stats_part, void* tail_ws, int32_t* err_flag,
-                           cudaStream_t st) {
+                           cudaStream_t st, bool pdl, bool counters_cleared) {
     // dynamic shared memory available to this kernel on the current device
     static int smem_limit_dev[64];
     int dev = 0;
@@ -595,7 +605,9 @@ cudaError_t launch_lm_head(const uint16_t* hidden, const uint16_t* W, int Mh, in
             a.tail_ksplit = ks;
             a.tail_part = static_cast<float*>(tail_ws);
             a.tail_ticket = reinterpret_cast<int*>(static_cast<char*>(tail_ws) + kLmTailPartBytes);
-            const cudaError_t me = cudaMemsetAsync(a.tail_ticket, 0, (size_t)left * a.tail_split * 4, st);
+            const cudaError_t me =
+                counters_cleared ? cudaSuccess
+                                 : cudaMemsetAsync(a.tail_ticket, 0, (size_t)left * a.tail_split * 4, st);
             if (me != cudaSuccess) {
                 set_error_detail("lm_head: clearing the left-over tile counters");
                 return me;
@@ -608,11 +620,9 @@ cudaError_t launch_lm_head(const uint16_t* hidden, const uint16_t* W, int Mh, in
         set_error_detail("lm_head: tensor map of hidden (row chunks) rejected");
         return cudaErrorInvalidValue;
     }
-    if (sh.NB == 1)
-        lm_head_kernel<1><<<grid, kLmThreads, sh.smem, st>>>(tw, th0, th1, tht, a);
-    else
-        lm_head_kernel<2><<<grid, kLmThreads, sh.smem, st>>>(tw, th0, th1, tht, a);
-    cudaError_t e = cudaGetLastError();
+    cudaError_t e = sh.NB == 1
+        ? launch_kernel(pdl, lm_head_kernel<1>, dim3(grid), dim3(kLmThreads), sh.smem, st, tw, th0, th1, tht, a)
+        : launch_kernel(pdl, lm_head_kernel<2>, dim3(grid), dim3(kLmThreads), sh.smem, st, tw, th0, th1, tht, a);
     if (e != cudaSuccess) set_error_detail("lm_head: launch failed");
     return e;
 }
