@@ -117,10 +117,9 @@ isd_status check_accept_shape(const isd_dims* d) {
     } while (0)
 
 // The step's kernels can be launched with programmatic dependent launch
-// (launch.h).  On B200 at B=32, N=4 that measured slower than plain stream
-// order (0.516 vs 0.500 ms per step, alternating runs in one process: the LM
-// head's early W stream competes with the attention's last CTAs for HBM), so
-// it is off.
+// (launch.h).  On B200 at B=32, N=4 that measured about 3% slower than plain
+// stream order (alternating runs in one process, with or without the LM head
+// streaming W early), so it is off.
 constexpr bool kStepPdl = false;
 
 isd_status do_attention(const isd_dims* d, const Plan& p, const uint16_t* q,

@@ -344,6 +344,25 @@ def test_bad_page_and_bad_nclean_raise_flags(isd):
     assert np.all(np.isfinite(sb.logits.cpu().numpy()))
 
 
+def test_attention_long_request_split_across_many_ctas(isd):
+    """A 30000-token request next to a short one (Qwen3-8B heads): each of the
+    long request's (request, kv head) units spans a dozen or more persistent
+    CTAs, whose partial results the last of them merges (four at a time, in
+    CTA order).  Matches the oracle, and a second run is bit-identical."""
+    cfg = I.IsdConfig("long_request", B=2, N=4, Hq=32, Hkv=8, D=128, V=1000, page_size=16,
+                      prefix_lo=0, prefix_hi=30000, fixed_prefix=(30000, 700), w_std=0.05,
+                      qkv_std=0.3, kv_std=1.0)
+    inp = I.make_step_inputs(cfg, seed=31, n_clean="mixed")
+    sb = StepBuffers(isd, cfg, inp)
+    sb.attention()
+    check_attention(sb, inp, cfg)
+    first = sb.hidden.clone()
+    sb.attention()  # the block rows are appended again at the same positions
+    torch.cuda.synchronize()
+    assert torch.equal(sb.hidden, first)
+    assert int(sb.err.item()) == 0
+
+
 def test_poisoned_unused_pages_do_not_leak(isd):
     """NaN in every pool row that no request may read leaves outputs finite."""
     cfg = I.CONFIGS["ragged_small"]
