@@ -110,7 +110,10 @@ const char* isd_last_error(void);
  *   out    [B*Q, Hq*D] bf16: for each active slot s and head h, the softmax
  *          (sm_scale q.k) weighted sum of v over keys at positions <= pos_s,
  *          query head h reading KV head h / (Hq/Hkv); inactive slots -> 0.
- * Supported: D in {64, 128}; (Hq/Hkv)*Q <= 128.
+ * Supported: D in {64, 128}; (Hq/Hkv)*Q <= 128.  D = 128 with (Hq/Hkv)*Q
+ * <= 64 and page sizes 8, 16, 32, 64 or 128 run on the tensor cores
+ * (tcgen05); other supported shapes on a general (mma.sync) kernel.  Both
+ * give results that do not depend on timing (fixed-order merges).
  */
 isd_status isd_attention(const isd_dims* d, const uint16_t* q, const uint16_t* k_new,
                          const uint16_t* v_new, uint16_t* k_pool, uint16_t* v_pool,
@@ -197,7 +200,7 @@ isd_status isd_step(const isd_dims* d, const uint16_t* q, const uint16_t* k_new,
  * gave all free device memory to its KV-cache pool at start-up, or code that
  * must not call the CUDA allocator (cudaMalloc/cudaFree can synchronise the
  * device).  This call takes the same inputs and outputs as isd_attention, but
- * its scratch (the split-KV partial results and counters) lives in a fixed
+ * its scratch (the attention's partial results and counters) lives in a fixed
  * array inside the library of ISD_NOALLOC_SCRATCH_BYTES bytes, which every
  * GPU that loads the library keeps until the process exits.  It allocates
  * nothing and calls no allocating routine.

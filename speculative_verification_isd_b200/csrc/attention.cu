@@ -1,4 +1,8 @@
-// KV append (a1) and strict-causal GQA attention over the paged cache (a2).
+// KV append (a1) and strict-causal GQA attention over the paged cache (a2):
+// the general kernel, for the shapes the tensor-core kernel in
+// attention_tc.cu does not take (D = 64, more than 64 query rows per kv head,
+// pages that are not 8..128 tokens dividing 128).  launch_attention at the
+// end of this file picks the kernel.
 //
 // Strict causal attention over clean and MASK slots alike is the first of the
 // training changes on "I-DLM：扩散模型如何用“自省一致性”追上自回归模型质量"
