@@ -200,48 +200,6 @@ def cpu_baseline(wl, cfg, budget_s):
 
 
 # ---------------------------------------------------------------------------
-def setup_dist(args):
-    import torch
-    world = int(os.environ.get("WORLD_SIZE", "1"))
-    rank = int(os.environ.get("RANK", "0"))
-    local = int(os.environ.get("LOCAL_RANK", "0"))
-    if world > 1:
-        import datetime
-        import torch.distributed as dist
-        torch.cuda.set_device(local)
-        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
-                                device_id=torch.device("cuda", local))
-    else:
-        torch.cuda.set_device(0)
-    return world, rank, local
-
-
-def allreduce_max(x: float, world: int) -> float:
-    if world == 1:
-        return x
-    import torch
-    import torch.distributed as dist
-    t = torch.tensor([x], dtype=torch.float64, device="cuda")
-    dist.all_reduce(t, op=dist.ReduceOp.MAX)
-    return float(t.item())
-
-
-def allreduce_sum(x: float, world: int) -> float:
-    if world == 1:
-        return x
-    import torch
-    import torch.distributed as dist
-    t = torch.tensor([x], dtype=torch.float64, device="cuda")
-    dist.all_reduce(t, op=dist.ReduceOp.SUM)
-    return float(t.item())
-
-
-def barrier(world):
-    if world > 1:
-        import torch.distributed as dist
-        dist.barrier()
-
-
 def run_reference(args):
     """--impl reference: the CPU oracle, timed on host cores (rank 0 only)."""
     import torch
@@ -302,11 +260,13 @@ def main():
         return run_reference(args)
     import numpy as np
     import torch
-    world, rank, local = setup_dist(args)
+    from speculative_verification_isd_b200 import ranks as RK
+    R = RK.setup(use_cuda=True)
+    world, rank = R.world, R.rank
     from speculative_verification_isd_b200 import build as B
     if rank == 0:
         B.build()
-    barrier(world)
+    R.barrier()
     from speculative_verification_isd_b200 import inputs as I
     from speculative_verification_isd_b200 import isd
     from speculative_verification_isd_b200.workload import DeviceWorkload
@@ -314,7 +274,7 @@ def main():
     hbm, tf_burst, tf_sus, peak_src = measured_peaks()
     # weak scaling: every rank runs its own batch of B requests (requests are
     # independent), so there is no collective on the data path
-    wl = DeviceWorkload(isd, cfg, seed=rank, n_uniform_steps=max(64, args.warmup + 1))
+    wl = DeviceWorkload(isd, cfg, seed=RK.rank_seed(0, rank), n_uniform_steps=max(64, args.warmup + 1))
     d = wl.dims
     K, W = args.steps, args.warmup
     stream = torch.cuda.current_stream()
@@ -339,7 +299,7 @@ def main():
     clocks.start()
     time.sleep(0.3)
     # ---------------- timed region: K steps through isd_step
-    barrier(world)
+    R.barrier()
     torch.cuda.synchronize()
     ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     ev0.record(stream)
@@ -347,13 +307,13 @@ def main():
         run_step(k, acc_hist[k])
     ev1.record(stream)
     torch.cuda.synchronize()
-    barrier(world)
+    R.barrier()
     clk = clocks.stop()
-    t_ms = allreduce_max(ev0.elapsed_time(ev1), world)
+    t_ms = R.max(ev0.elapsed_time(ev1))
     wl.accept_len = torch.empty(cfg.B, dtype=torch.int32, device="cuda")
-    accepted = allreduce_sum(float(acc_hist.sum().item()), world)
+    accepted = R.sum(float(acc_hist.sum().item()))
     steps_total = K * world
-    value = steps_total / (t_ms / 1e3)
+    value = RK.job_throughput(K, R, t_ms)  # all ranks' steps over the slowest rank's time
     tok_s = accepted / (t_ms / 1e3)
     mean_acc = accepted / (steps_total * cfg.B)
     flags = int(wl.err.item())
@@ -396,7 +356,7 @@ def main():
             wl.step(without_lora=True)
         f1.record(stream)
         torch.cuda.synchronize()
-        t_plain = allreduce_max(f0.elapsed_time(f1), world) / KL
+        t_plain = R.max(f0.elapsed_time(f1)) / KL
         lora_alpha = (t_ms / K) / t_plain
 
     # ---------------- e2e: public API with host buffers, copies inside the timed region
@@ -413,7 +373,7 @@ def main():
     h2d = in_dev.numel()
     d2h = host_out.numel() * 4
     KE = min(args.e2e_steps, K)
-    barrier(world)
+    R.barrier()
     torch.cuda.synchronize()
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     e0.record(stream)
@@ -425,8 +385,8 @@ def main():
         stream.synchronize()  # the caller needs this step's result before the next one
     e1.record(stream)
     torch.cuda.synchronize()
-    barrier(world)
-    e2e_ms = allreduce_max(e0.elapsed_time(e1), world)
+    R.barrier()
+    e2e_ms = R.max(e0.elapsed_time(e1))
     e2e_value = KE * world / (e2e_ms / 1e3)
 
     # ---------------- roofline of the dominant kernel (LM head)
@@ -474,9 +434,7 @@ def main():
         line["cpu_baseline"] = cpu_baseline(wl, cfg, args.cpu_budget_s)
     if rank == 0:
         print(json.dumps(line), flush=True)
-    if world > 1:
-        import torch.distributed as dist
-        dist.destroy_process_group()
+    R.close()
     return 0
 
 
