@@ -186,7 +186,7 @@ def cpu_baseline(wl, cfg, budget_s):
     sampler = OracleSampler(wl, cfg)
     vs = 8192
     ests, spent, k = [], 0.0, 0
-    while spent < budget_s and k < 50:
+    while spent < budget_s and k < 400:
         est, used = sampler.estimate_step_seconds(k, vs)
         ests.append(est)
         spent += used
