@@ -152,6 +152,9 @@ CONFIGS: Dict[str, IsdConfig] = {
     "ragged_lora": IsdConfig("ragged_lora", B=5, N=3, Hq=8, Hkv=2, D=128, V=2053, page_size=16,
                              prefix_lo=0, prefix_hi=700, lora_rank=128, w_std=0.2, qkv_std=0.5,
                              kv_std=1.0, lora_std=0.05),
+    # Stride 8 (60 query rows per kv head) in 64-token pages, ragged prefixes.
+    "ragged_n8": IsdConfig("ragged_n8", B=3, N=8, Hq=8, Hkv=2, D=128, V=1000, page_size=64,
+                           prefix_lo=1, prefix_hi=400, w_std=0.5, qkv_std=0.5, kv_std=1.0),
     "qwen_medium": IsdConfig("qwen_medium", B=4, N=4, page_size=16, prefix_lo=100, prefix_hi=2500,
                              w_std=0.05, qkv_std=0.3, kv_std=1.0, **QWEN3_8B),
 }

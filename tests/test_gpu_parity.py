@@ -146,7 +146,7 @@ def check_row_stats(sb, z_g):
     assert np.all(np.abs(s_g - s_o) <= NEAR * s_o)
 
 
-PARITY_CONFIGS = ["tiny", "ragged_small", "ragged_lora", "qwen_medium"]
+PARITY_CONFIGS = ["tiny", "ragged_small", "ragged_lora", "ragged_n8", "qwen_medium"]
 
 
 @pytest.mark.parametrize("name", PARITY_CONFIGS)
