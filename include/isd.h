@@ -164,6 +164,7 @@ isd_status isd_row_stats(const isd_dims* d, const float* logits, int32_t rows,
  *   (-1 padded); next_kv_len [B] = kv_len + A
  *   ratio [B, max(N-1,1)] fp32 or NULL: p/q of each tested proposal, -1 if
  *   not tested.
+ * Supported: N <= 16, V <= 524288 (else ISD_ERR_UNSUPPORTED_SHAPE).
  */
 isd_status isd_accept(const isd_dims* d, const float* logits, const isd_row_stat* row_stats,
                       const float* prev_logits, const isd_row_stat* prev_row_stats,

@@ -100,8 +100,9 @@ isd_status check_lm_shape(const isd_dims* d, const Plan& p, const void* A, const
 
 isd_status check_accept_shape(const isd_dims* d) {
     if (d->N > 16) return unsupported("stride N must be <= 16");
+    static_assert(isd::kAcceptThreads * isd::kAcceptChunk == 524288, "update the message below");
     if ((long long)d->V > (long long)isd::kAcceptThreads * isd::kAcceptChunk)
-        return unsupported("vocabulary must be <= 1048576 entries");
+        return unsupported("vocabulary must be <= 524288 entries");
     return ISD_OK;
 }
 
