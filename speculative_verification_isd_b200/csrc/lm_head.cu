@@ -23,12 +23,13 @@
 //    store instruction writes 128 contiguous bytes of one logits row;
 //  * the vocabulary tiles are dealt round-robin in whole waves of gridDim.x;
 //    the L < gridDim.x tiles left over are split along N (the hidden rows)
-//    into chunks of 16-row multiples, one chunk per CTA with the full K
-//    loop, so the last wave is short instead of one tile long; the chunk CTAs
-//    read their shared W tile in the same order with an L2-keep hint, so it
-//    crosses HBM about once.  Each chunk holds complete logits for its rows,
-//    so the fused row statistics need no merge and the result is independent
-//    of timing;
+//    into chunks of 16-row multiples, so the last wave is short instead of
+//    one tile long; the chunk CTAs read their shared W tile in the same order
+//    with an L2-keep hint, so it crosses HBM about once.  When CTAs are still
+//    idle, each chunk is also split into K slices: every slice writes an fp32
+//    partial, and the last slice to finish sums them in K order before the
+//    usual epilogue (logits and fused row statistics), so the result does not
+//    depend on timing;
 //  * every mbarrier wait is bounded (about 2 s); on time-out the CTA raises
 //    ISD_FLAG_WAIT_TIMEOUT, every role leaves its loop, outstanding TMA loads
 //    and MMAs are drained with bounded waits, and TMEM is released.
