@@ -101,15 +101,20 @@ def test_mean_accept_length_matches_table(golden, N):
 def test_closed_loop_tpf_matches_table(golden, N):
     """Run the oracle's state machine in closed loop; tokens per forward must
     equal the table's TPF column (and the TPF^2/Q identity must hold on the
-    counters, as derived on the project page, step 6)."""
+    counters, as derived on the project page, step 6).
+
+    The tolerance is 4 standard errors of the mean TPF, estimated from the
+    per-request TPFs (requests are independent; consecutive forwards of one
+    request are not, so a per-forward standard error would be too small),
+    plus the table's rounding to two decimals."""
     table = {n: t for n, _, t in load_table(golden)}
     rng = np.random.default_rng(77 + N)
-    B, steps, V, a = 40, 350, 64, 0.9
+    B, steps, V, a = 160, 350, 64, 0.9
     Q = 2 * N - 1
     nc = np.ones(B, dtype=np.int32)
     tok = rng.integers(0, V, size=(B, N)).astype(np.int32)
     kv = np.zeros(B, dtype=np.int32)
-    total_tokens = 0
+    per_request = np.zeros(B)
     for _ in range(steps):
         logits = (rng.standard_normal((B, Q, V)) * 0.5).astype(np.float32)
         prev = (rng.standard_normal((B, Q, V)) * 0.5).astype(np.float32)
@@ -120,14 +125,17 @@ def test_closed_loop_tpf_matches_table(golden, N):
                 prev[b, N + j - 2] = zq
         u = rng.random((B, 2 * N)).astype(np.float32)
         res = O.accept(logits, prev, nc, tok, kv, u, N)
-        total_tokens += int(res["accept_len"].sum())
+        per_request += res["accept_len"]
         assert np.array_equal(res["next_kv_len"], kv + res["accept_len"])
         nc, tok, kv = res["next_n_clean"], res["next_clean_tok"], res["next_kv_len"]
         assert set(np.unique(nc)) <= {1, N}
+    total_tokens = int(per_request.sum())
     forwards = B * steps
     tpf = total_tokens / forwards
-    assert abs(tpf - table[N]) < 0.06, (tpf, table[N])
-    assert abs(tpf - tpf_restart_model(a, N)) < 0.06
+    se = (per_request / steps).std(ddof=1) / math.sqrt(B)
+    assert se < 0.02  # the run is long enough for the bound to mean something
+    assert abs(tpf - tpf_restart_model(a, N)) < 4 * se, (tpf, se)
+    assert abs(tpf - table[N]) < 4 * se + 0.005, (tpf, table[N], se)
     oh = forwards * Q / total_tokens
     assert tpf / oh == pytest.approx(tpf * tpf / Q, rel=1e-12)
     # kv_len counts exactly the emitted tokens
@@ -305,3 +313,41 @@ def test_argmax_ties_go_to_lowest_index():
     assert (m, a) == (3.0, 1)
     assert s == pytest.approx(3.0 + math.exp(-1.0) + math.exp(-2.0), rel=1e-15)
     assert O.row_stats(np.zeros(10))[1] == 10.0
+
+
+def test_zero_residual_mass_falls_back_to_argmax_p():
+    """A proposal with zero probability under both rows: p(x)/q(x) is 0/0
+    (NaN), so u < p(x)/q(x) is false for every u and the proposal is rejected;
+    p and q are otherwise equal, so max(0, p - q) has no mass and the
+    replacement is the argmax of p (the reading taken for the empty residual),
+    here worked out by hand: entry 1 holds the largest logit."""
+    N, V = 2, 5
+    Q = 2 * N - 1
+    zp = np.array([0.1, 2.0, -np.inf, 0.5, -1.0], np.float32)
+    logits = np.zeros((1, Q, V), np.float32)
+    prev = np.zeros((1, Q, V), np.float32)
+    logits[0, 0] = zp          # p for t_2
+    prev[0, N] = zp            # q for t_2: the same distribution
+    tok = np.array([[3, 2]], np.int32)   # t_2 = 2 has p = q = 0
+    u = np.array([[0.0, 0.7, 0.2, 0.3]], np.float32)
+    with np.errstate(invalid="ignore"):
+        res = O.accept(logits, prev, np.array([2], np.int32), tok, np.array([5], np.int32), u, N)
+        w = O.residual_distribution(zp, zp)
+    assert w.sum() == 0.0
+    assert np.isnan(res["ratio"][0, 0])
+    assert res["rejected_at"][0] == 2
+    assert res["accept_len"][0] == 1
+    assert list(res["out_tok"][0]) == [1, -1]
+    assert res["next_n_clean"][0] == 1 and list(res["next_clean_tok"][0]) == [1, -1]
+    assert res["next_kv_len"][0] == 6
+
+
+def test_inverse_cdf_falls_back_to_last_positive_weight():
+    """When no prefix sum exceeds u * total (u = 1 makes the target equal to
+    the total), the draw is the last entry with positive weight -- never a
+    trailing zero-weight entry."""
+    w = np.array([0.0, 0.25, 0.0, 0.5, 0.25, 0.0, 0.0])
+    assert O.inverse_cdf(w, 1.0) == 4
+    assert O.inverse_cdf(np.array([0.0, 3.0, 0.0]), 1.0) == 1
+    # the main branch just below: the largest uniform in [0, 1) of float32
+    assert O.inverse_cdf(w, float(np.nextafter(np.float32(1), np.float32(0)))) == 4
