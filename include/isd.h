@@ -210,8 +210,9 @@ isd_status isd_step(const isd_dims* d, const uint16_t* q, const uint16_t* k_new,
  *    grows with B * Hkv * (longest context); B=32, 8 KV heads and 8 K
  *    contexts fit.
  *  - The first call on each device (made with that device current) looks up
- *    the array's device address; make that first call before any stream
- *    capture.
+ *    the array's device address, and so does the first call after the
+ *    device's context was destroyed and recreated (cudaDeviceReset); make
+ *    those calls before any stream capture.
  *  - All calls on a device share the array: calls that overlap on the GPU
  *    (e.g. on two unordered streams) race on it.  Each call clears the
  *    counters it needs on its own stream.

@@ -17,11 +17,17 @@
 //
 // Host code cannot use the array's name as a device address, so the first
 // call on each device (with that device current) looks the address up with
-// cudaGetSymbolAddress and keeps it; make that first call before any stream
+// cudaGetSymbolAddress and keeps it, together with the unique id of the
+// context it was looked up in; a later call in another context on the same
+// device (after cudaDeviceReset, for instance) looks it up again.  Make the
+// first call on a device, and the first one after a reset, before any stream
 // capture.
+#include <cuda.h>
 #include <cuda_runtime.h>
 #include <stdint.h>
 #include <stdio.h>
+
+#include <mutex>
 
 #include "common.cuh"
 #include "plan.h"
@@ -34,7 +40,41 @@ constexpr size_t kNoAllocScratchBytes = (size_t)ISD_NOALLOC_SCRATCH_BYTES;
 
 static __device__ __align__(256) unsigned char g_attn_scratch[kNoAllocScratchBytes];
 
-void* g_scratch_ptr[ISD_NOALLOC_MAX_DEVICES];  // per device, filled on first use
+struct ScratchSlot {
+    void* ptr;             // device address of g_attn_scratch in that context
+    unsigned long long ctx_id;  // unique id of the context of the lookup
+};
+ScratchSlot g_scratch[ISD_NOALLOC_MAX_DEVICES];  // per device, filled on first use
+std::mutex g_scratch_mu;
+
+typedef CUresult (*CtxGetCurrentFn)(CUcontext*);
+typedef CUresult (*CtxGetIdFn)(CUcontext, unsigned long long*);
+
+// Unique id of the calling thread's current context (0 if there is none yet
+// or the driver cannot say).
+unsigned long long current_ctx_id() {
+    static CtxGetCurrentFn get_cur = nullptr;
+    static CtxGetIdFn get_id = nullptr;
+    static bool looked = false;
+    if (!looked) {
+        void* p = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuCtxGetCurrent", &p, cudaEnableDefault, &q) == cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            get_cur = reinterpret_cast<CtxGetCurrentFn>(p);
+        p = nullptr;
+        if (cudaGetDriverEntryPoint("cuCtxGetId", &p, cudaEnableDefault, &q) == cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            get_id = reinterpret_cast<CtxGetIdFn>(p);
+        looked = true;
+    }
+    CUcontext ctx = nullptr;
+    unsigned long long id = 0;
+    if (get_cur && get_id && get_cur(&ctx) == CUDA_SUCCESS && ctx &&
+        get_id(ctx, &id) == CUDA_SUCCESS)
+        return id;
+    return 0;
+}
 
 }  // namespace
 
@@ -84,16 +124,25 @@ extern "C" isd_status isd_attention_noalloc(const isd_dims* d, const uint16_t* q
         isd::set_last_error("isd_attention_noalloc: no usable current device");
         return ISD_ERR_CUDA;
     }
-    if (!g_scratch_ptr[dev]) {
-        void* ptr = nullptr;
-        const cudaError_t e = cudaGetSymbolAddress(&ptr, g_attn_scratch);
-        if (e != cudaSuccess || !ptr) {
-            isd::set_last_error("isd_attention_noalloc: device address of the scratch array");
-            return ISD_ERR_CUDA;
+    void* scratch = nullptr;
+    {
+        std::lock_guard<std::mutex> lock(g_scratch_mu);
+        ScratchSlot& slot = g_scratch[dev];
+        const unsigned long long id = current_ctx_id();
+        if (!slot.ptr || id == 0 || id != slot.ctx_id) {
+            void* ptr = nullptr;
+            const cudaError_t e = cudaGetSymbolAddress(&ptr, g_attn_scratch);
+            if (e != cudaSuccess || !ptr) {
+                isd::set_last_error("isd_attention_noalloc: device address of the scratch array");
+                return ISD_ERR_CUDA;
+            }
+            slot.ptr = ptr;
+            // the lookup has made the context current if it was not yet
+            slot.ctx_id = current_ctx_id();
         }
-        g_scratch_ptr[dev] = ptr;
+        scratch = slot.ptr;
     }
-    char* ws = static_cast<char*>(g_scratch_ptr[dev]);
+    char* ws = static_cast<char*>(scratch);
     cudaStream_t st = static_cast<cudaStream_t>(stream);
     // launch_attention clears the counters on the stream before the attention
     if (isd::launch_attention(p, d, q, k_new, v_new, k_pool, v_pool, page_table, kv_len, n_clean,

@@ -865,7 +865,7 @@ cudaError_t launch_tc(const TcArgs& a, const CUtensorMap& tk, const CUtensorMap&
         if (e != cudaSuccess) return e;
         configured |= 1ull << dev;
     }
-    return launch_kernel(pdl, attention_tc_kernel<R, STAGES>, dim3(kNumSMs), dim3(TcRoles<R>::kThreads),
+    return launch_kernel(pdl, attention_tc_kernel<R, STAGES>, dim3(persistent_grid()), dim3(TcRoles<R>::kThreads),
                          smem, st, tk, tv, tq, a);
 }
 

@@ -19,6 +19,18 @@ namespace isd {
 void set_error_detail(const char* msg) { snprintf(g_detail, sizeof(g_detail), "%s", msg); }
 // The message isd_last_error() returns (this thread).
 void set_last_error(const char* msg) { snprintf(g_last_error, sizeof(g_last_error), "%s", msg); }
+
+int persistent_grid() {
+    static int sms[64];
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return kPlanSMs;
+    if (!sms[dev]) {
+        int n = 0;
+        cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev);
+        sms[dev] = n < 1 ? kPlanSMs : (n > kMaxSMs ? kMaxSMs : n);
+    }
+    return sms[dev];
+}
 cudaError_t launch_attention(const Plan& p, const isd_dims* d, const uint16_t* q,
                              const uint16_t* k_new, const uint16_t* v_new, uint16_t* k_pool,
                              uint16_t* v_pool, const int32_t* page_table, const int32_t* kv_len,
@@ -141,7 +153,7 @@ isd_status do_attention(const isd_dims* d, const Plan& p, const uint16_t* q,
     }
     ISD_CUDA(isd::launch_attention(p, d, q, k_new, v_new, k_pool, v_pool, page_table, kv_len,
                                    n_clean, out, ws, err_flag, st, acc_ticket, lm_ticket,
-                                   in_step ? isd::kNumSMs : 0, kStepPdl));
+                                   in_step ? isd::kMaxSMs : 0, kStepPdl));
     return ISD_OK;
 }
 

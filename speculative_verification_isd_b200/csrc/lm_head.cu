@@ -492,13 +492,6 @@ bool lm_head_shape(int Mh, int smem_limit, LmShape* s) {
     return true;
 }
 
-static int num_sms_of_current_device() {
-    int dev = 0, n = 0;
-    cudaGetDevice(&dev);
-    cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev);
-    return n > 0 ? n : 148;
-}
-
 void set_error_detail(const char* msg);
 
 // pdl: launched as part of the whole step (programmatic dependent launch);
@@ -573,7 +566,7 @@ cudaError_t launch_lm_head(const uint16_t* hidden, const uint16_t* W, int Mh, in
     a.logits = logits;
     a.stats_part = stats_part;
     a.err_flag = err_flag;
-    int grid = num_sms_of_current_device();
+    int grid = persistent_grid();
     if (grid > a.n_tiles) grid = a.n_tiles;
     // whole waves of tiles, then the left-over tiles split into row chunks
     a.n_full = (a.n_tiles / grid) * grid;
@@ -598,7 +591,7 @@ cudaError_t launch_lm_head(const uint16_t* hidden, const uint16_t* W, int Mh, in
     a.tail_ksplit = 1;
     a.tail_part = nullptr;
     a.tail_ticket = nullptr;
-    if (a.tail_split > 1 && a.tail_bn <= 64 && grid <= kNumSMs && tail_ws) {
+    if (a.tail_split > 1 && a.tail_bn <= 64 && grid <= kMaxSMs && tail_ws) {
         int ks = grid / (left * a.tail_split);
         if (ks > 8) ks = 8;
         if (ks > H / 64) ks = H / 64;

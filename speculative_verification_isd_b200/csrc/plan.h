@@ -19,9 +19,13 @@ constexpr int kAcceptThreads = 256;
 // kernel than 4096 at B=32, N=4, V=151936; the chunk totals of a request are
 // scanned by one CTA, so V <= kAcceptThreads * kAcceptChunk).
 constexpr int kAcceptChunk = 2048;
-constexpr int kNumSMs = 148;
-constexpr size_t kLmTailPartBytes = (size_t)kNumSMs * 64 * 128 * 4;
-constexpr size_t kLmTailBytes = kLmTailPartBytes + (size_t)kNumSMs * 4;
+// Persistent kernels (attention, LM head) run one CTA per SM of the current
+// device, at most kMaxSMs (a B200 has 148); the workspace is sized for
+// kMaxSMs, and the split heuristics below aim at a B200-sized grid.
+constexpr int kMaxSMs = 192;
+constexpr int kPlanSMs = 148;
+constexpr size_t kLmTailPartBytes = (size_t)kMaxSMs * 64 * 128 * 4;
+constexpr size_t kLmTailBytes = kLmTailPartBytes + (size_t)kMaxSMs * 4;
 
 struct Plan {
     // derived dims
@@ -51,6 +55,10 @@ struct Plan {
 
 inline size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
 
+// SMs of the current device, capped at kMaxSMs (cached per device).  The one
+// place the persistent kernels take their grid size from.
+int persistent_grid();
+
 // Returns false if the dims are invalid.
 inline bool make_plan(const isd_dims* d, Plan* p) {
     if (!d || d->B < 1 || d->N < 1 || d->Hq < 1 || d->Hkv < 1 || d->D < 1 || d->V < 1 ||
@@ -70,7 +78,7 @@ inline bool make_plan(const isd_dims* d, Plan* p) {
     // Aim for about 3 waves of 2 CTAs per SM over the expected keys (half
     // the longest context per request on average).
     long long est = (long long)d->B * d->Hkv * p->attn_rgb * (max_ctx / 2 + 1);
-    long long split = est / (kNumSMs * 2 * 3);
+    long long split = est / (kPlanSMs * 2 * 3);
     if (split < 256) split = 256;
     if (split > kAttnMaxSplit) split = kAttnMaxSplit;
     split = (split + kAttnKeyTile - 1) / kAttnKeyTile * kAttnKeyTile;
@@ -85,7 +93,7 @@ inline bool make_plan(const isd_dims* d, Plan* p) {
         p->attn_tc_rows = p->rows <= 16 ? 16 : (p->rows <= 32 ? 32 : 64);
     p->attn_tc_part_stride = 2 * p->attn_tc_rows + 128 * p->attn_tc_rows;
     // row statistics: enough CTAs to fill the GPU, chunks of >= 2048 entries
-    int target = (kNumSMs * 8 + p->M - 1) / p->M;
+    int target = (kPlanSMs * 8 + p->M - 1) / p->M;
     int max_chunks = (d->V + 2047) / 2048;
     p->stats_chunks = target < 1 ? 1 : (target > max_chunks ? max_chunks : target);
     if (p->stats_chunks < 1) p->stats_chunks = 1;
@@ -113,7 +121,7 @@ inline bool make_plan(const isd_dims* d, Plan* p) {
     // split partials of the general kernel, or two partials per persistent
     // CTA of the tensor-core kernel: whichever is larger
     size_t part_bytes = n_units * p->attn_max_splits * p->attn_part_stride;
-    const size_t tc_bytes = (size_t)kNumSMs * 2 * p->attn_tc_part_stride * 4;
+    const size_t tc_bytes = (size_t)kMaxSMs * 2 * p->attn_tc_part_stride * 4;
     if (tc_bytes > part_bytes) part_bytes = tc_bytes;
     p->off_attn_part = take(part_bytes);
     p->off_attn_ticket = take(n_units * 4);

@@ -218,13 +218,13 @@ def accept(d: Dims, logits, row_stats, prev_logits, prev_row_stats, n_clean, cle
         _ptr(err_flag, torch.int32, 1, "err_flag"), _stream(stream)))
 
 
-def step(d: Dims, q, k_new, v_new, k_pool, v_pool, page_table, kv_len, n_clean, clean_tok, W,
-         prev_logits, prev_row_stats, uniforms, logits, row_stats, accept_len, out_tok,
-         next_n_clean, next_clean_tok, next_kv_len, ws, hidden=None, ratio=None, lora_A=None,
-         lora_B=None, err_flag=None, stream=None):
+def _step_args(d: Dims, q, k_new, v_new, k_pool, v_pool, page_table, kv_len, n_clean, clean_tok,
+               W, prev_logits, prev_row_stats, uniforms, logits, row_stats, accept_len, out_tok,
+               next_n_clean, next_clean_tok, next_kv_len, ws, hidden=None, ratio=None,
+               lora_A=None, lora_B=None, err_flag=None, stream=None):
     B, N = d.B, d.N
     kvrow = d.page_size * d.Hkv * d.D
-    _check(_lib.isd_step(
+    return [
         ctypes.byref(d), _ptr(q, _BF16, d.M * d.Hq * d.D, "q"),
         _ptr(k_new, _BF16, d.M * d.Hkv * d.D, "k_new"),
         _ptr(v_new, _BF16, d.M * d.Hkv * d.D, "v_new"),
@@ -247,7 +247,39 @@ def step(d: Dims, q, k_new, v_new, k_pool, v_pool, page_table, kv_len, n_clean, 
         _ptr(next_kv_len, torch.int32, B, "next_kv_len"),
         _ptr(ratio, torch.float32, B * max(N - 1, 1), "ratio"),
         _ptr(ws, torch.uint8, None, "ws"), ws.numel(),
-        _ptr(err_flag, torch.int32, 1, "err_flag"), _stream(stream)))
+        _ptr(err_flag, torch.int32, 1, "err_flag"), _stream(stream)]
+
+
+def step(d: Dims, q, k_new, v_new, k_pool, v_pool, page_table, kv_len, n_clean, clean_tok, W,
+         prev_logits, prev_row_stats, uniforms, logits, row_stats, accept_len, out_tok,
+         next_n_clean, next_clean_tok, next_kv_len, ws, hidden=None, ratio=None, lora_A=None,
+         lora_B=None, err_flag=None, stream=None):
+    _check(_lib.isd_step(*_step_args(
+        d, q, k_new, v_new, k_pool, v_pool, page_table, kv_len, n_clean, clean_tok, W,
+        prev_logits, prev_row_stats, uniforms, logits, row_stats, accept_len, out_tok,
+        next_n_clean, next_clean_tok, next_kv_len, ws, hidden, ratio, lora_A, lora_B, err_flag,
+        stream)))
+
+
+class StepCall:
+    """isd_step with its arguments checked and marshalled once.
+
+    For a loop that issues the same step on the same buffers many times (a
+    serving loop whose tensors stay in place): the constructor takes the
+    arguments of ``step`` (stream included) and validates them; calling the
+    object only passes the cached pointers to the library.  The tensors must
+    stay alive and in place while the object is used."""
+
+    def __init__(self, d: Dims, *args, **kwargs):
+        self._dims = d  # keeps the struct alive: the cached arguments point at it
+        self._keep = (args, kwargs)
+        self._args = tuple(_step_args(d, *args, **kwargs))
+        self._fn = _lib.isd_step
+
+    def __call__(self):
+        st = self._fn(*self._args)
+        if st != ISD_OK:
+            raise IsdError(st)
 
 
 def row_stats_view(rs: torch.Tensor):

@@ -10,6 +10,15 @@ import torch
 
 from speculative_verification_isd_b200 import inputs as I
 
+# (label, counts) of every accept comparison in this session; printed by the
+# terminal-summary hook in conftest.py so that near-threshold decisions and
+# rounding-excused draws are reported, not only counted
+PARITY_REPORT = []
+
+
+def record_parity(label: str, rep: dict):
+    PARITY_REPORT.append((label, dict(rep)))
+
 
 def bf16_dev(a: np.ndarray) -> torch.Tensor:
     return torch.from_numpy(np.ascontiguousarray(a).view(np.int16)).view(torch.bfloat16).cuda()

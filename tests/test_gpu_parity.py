@@ -17,9 +17,10 @@ import pytest
 import torch
 
 from oracle import isd_oracle as O
+from oracle import parity as P
 from speculative_verification_isd_b200 import inputs as I
 
-from gpu_util import StepBuffers, bf16_host, f32_dev, i32_dev, row_stats_host
+from gpu_util import StepBuffers, bf16_host, f32_dev, i32_dev, record_parity, row_stats_host
 
 pytestmark = pytest.mark.gpu
 
@@ -30,75 +31,16 @@ def isd():
     return lib
 
 
-NEAR = 1e-5
+NEAR = P.NEAR
 
 
-def ratio_near(b, c, u, ores):
-    """Is an accept decision of request b within NEAR of its uniform?"""
-    for j in range(2, c + 1):
-        r = ores["ratio"][b, j - 2]
-        if abs(float(u[b, j - 2]) - r) < NEAR:
-            return True
-        if not (float(u[b, j - 2]) < r):
-            break
-    return False
-
-
-def draw_explained(w, u, y):
-    """Is bucket y within NEAR * sum(w) of the oracle's inverse-CDF target?"""
-    cum = np.cumsum(np.asarray(w, dtype=np.float64))
-    tot = cum[-1]
-    if not (0 <= y < len(w)) or w[y] <= 0 or tot <= 0:
-        return False
-    t = float(u) * tot
-    lo = cum[y - 1] if y > 0 else 0.0
-    dist = max(0.0, lo - t, t - cum[y])
-    return dist <= NEAR * tot
-
-
-def compare_accept(gpu, ores, logits, prev, inp, N, mode):
-    """Decisions, lengths and states bit-exact; every differing token must be an
-    inverse-CDF draw whose GPU pick lies within NEAR * sum(w) of the oracle's
-    target.  Returns the number of requests excused (near-threshold ratio or
-    a rounding-explained draw)."""
-    B = logits.shape[0]
-    u = inp["uniforms"]
-    near = 0
-    for b in range(B):
-        c = int(inp["n_clean"][b])
-        if ratio_near(b, c, u, ores):
-            near += 1
-            continue
-        for key in ("accept_len", "next_n_clean", "next_kv_len"):
-            assert gpu[key][b] == ores[key][b], (key, b, gpu[key][b], ores[key][b])
-        A = int(ores["accept_len"][b])
-        # draws of this request: (position in out_tok / next_clean_tok, weights, uniform)
-        draws = {}
-        rej = int(ores["rejected_at"][b])
-        if rej > 0:
-            draws[("out", A - 1)] = (O.residual_distribution(logits[b, rej - 2], prev[b, N + rej - 2]),
-                                     u[b, N - 1])
-            draws[("next", 0)] = draws[("out", A - 1)]
-        elif mode == O.PROPOSE_SAMPLE:
-            rows = [c - 1] + [N + m for m in range(N - 1)]
-            for k, r in enumerate(rows):
-                draws[("next", k)] = (O.softmax(logits[b, r]), u[b, N + k])
-            draws[("out", A - 1)] = draws[("next", 0)]
-        excused = False
-        for kind, key in (("out", "out_tok"), ("next", "next_clean_tok")):
-            g, o = gpu[key][b], ores[key][b]
-            for i in np.nonzero(g != o)[0]:
-                assert (kind, int(i)) in draws, (key, b, i, g, o)
-                w, uu = draws[(kind, int(i))]
-                assert draw_explained(w, uu, int(g[i])), (key, b, i, g[i], o[i])
-                excused = True
-        near += excused
-        # ratios of the tested proposals
-        for j in range(2, A + 2):
-            if j - 2 >= ores["ratio"].shape[1] or ores["ratio"][b, j - 2] < 0:
-                break
-            assert gpu["ratio"][b, j - 2] == pytest.approx(ores["ratio"][b, j - 2], rel=NEAR)
-    return near
+def accept_parity(gpu, ores, logits, prev, inp, N, mode, label):
+    """oracle.parity.compare_accept, recorded for the session's parity report
+    (printed at the end of the run), with no unexplained difference allowed."""
+    rep = P.compare_accept(gpu, ores, logits, prev, inp, N, mode)
+    record_parity(label, rep)
+    assert rep["mismatches"] == 0, rep["first_mismatch"]
+    return rep
 
 
 def check_attention(sb, inp, cfg):
@@ -167,8 +109,9 @@ def test_staged_parity(isd, name, n_clean):
     logits = z_g.reshape(cfg.B, cfg.Q, cfg.V)
     ores = O.accept(logits, prev, inp["n_clean"], inp["clean_tok"], inp["kv_len"],
                     inp["uniforms"], cfg.N)
-    near = compare_accept(gpu, ores, logits, prev, inp, cfg.N, O.PROPOSE_ARGMAX)
-    assert near <= max(1, cfg.B // 10)
+    rep = accept_parity(gpu, ores, logits, prev, inp, cfg.N, O.PROPOSE_ARGMAX,
+                        f"staged {name} n_clean={n_clean}")
+    assert rep["near_threshold"] + rep["excused_draws"] <= max(1, cfg.B // 10)
     assert int(sb.err.item()) == 0
 
 
@@ -270,15 +213,76 @@ def test_accept_on_random_logits(isd, mode, V, N, B):
     gpu = {k: v.cpu().numpy() for k, v in outs.items()}
     ores = O.accept(logits, prev, nc, tok, kv, u, N, mode)
     inp = dict(n_clean=nc, clean_tok=tok, uniforms=u)
-    near = compare_accept(gpu, ores, logits, prev, inp, N, mode)
-    print(f"requests excused by rounding near a threshold: {near} of {B}")
-    assert near <= max(2, B // 20)
+    rep = accept_parity(gpu, ores, logits, prev, inp, N, mode,
+                        f"random logits V={V} N={N} B={B} mode={mode}")
+    # a decision within 1e-5 of its uniform has probability ~2e-5 per test
+    assert rep["near_threshold"] <= max(1, B // 50)
+    # fp32 prefix sums over V entries move a draw by about V * 2^-24 of its
+    # mass; over a large vocabulary that lands in a neighbouring bucket for a
+    # measurable fraction of the draws (counted and reported, each checked by
+    # draw_explained); a small vocabulary should almost never need it
+    assert rep["excused_draws"] <= max(1, rep["draws"] // 50 if V < 100000 else rep["draws"] // 4)
     assert (ores["rejected_at"] > 0).sum() > 0 or N == 1
     assert int(err.item()) == 0
     # row stats of both inputs
     m_g, s_g, a_g = row_stats_host(rs)
     m_o, s_o, a_o = O.row_stats_all(logits)
     assert np.array_equal(a_g, a_o) and np.all(np.abs(s_g - s_o) <= NEAR * s_o)
+
+
+def _accept_only(isd, logits, prev, nc, tok, kv, u, N, mode=0):
+    """Row statistics of both logits arrays and the accept kernel, through the
+    C ABI, on host-given logits.  Returns the host copies of the outputs."""
+    B, Q, V = logits.shape
+    d = isd.make_dims(B, N, 1, 1, 64, V, 16, 1, 1, 0, mode)
+    ws = isd.alloc_workspace(d)
+    zl, zp = f32_dev(logits.reshape(B * Q, V)), f32_dev(prev.reshape(B * Q, V))
+    rs = torch.empty(B * Q, 4, dtype=torch.int32, device="cuda")
+    prs = torch.empty_like(rs)
+    isd.row_stats(d, zl, B * Q, rs, ws)
+    isd.row_stats(d, zp, B * Q, prs, ws)
+    outs = dict(accept_len=torch.empty(B, dtype=torch.int32, device="cuda"),
+                out_tok=torch.empty(B, N, dtype=torch.int32, device="cuda"),
+                next_n_clean=torch.empty(B, dtype=torch.int32, device="cuda"),
+                next_clean_tok=torch.empty(B, N, dtype=torch.int32, device="cuda"),
+                next_kv_len=torch.empty(B, dtype=torch.int32, device="cuda"),
+                ratio=torch.empty(B, max(N - 1, 1), dtype=torch.float32, device="cuda"))
+    err = torch.zeros(1, dtype=torch.int32, device="cuda")
+    isd.accept(d, zl, rs, zp, prs, i32_dev(nc), i32_dev(tok), i32_dev(kv), f32_dev(u),
+               outs["accept_len"], outs["out_tok"], outs["next_n_clean"], outs["next_clean_tok"],
+               outs["next_kv_len"], ws, ratio=outs["ratio"], err_flag=err)
+    torch.cuda.synchronize()
+    assert int(err.item()) == 0
+    return {k: v.cpu().numpy() for k, v in outs.items()}
+
+
+def test_zero_residual_mass_falls_back_to_argmax_gpu(isd):
+    """Proposals with zero probability under both rows (logit -inf in p and
+    q, the rows otherwise equal): the ratio is 0/0, the proposal is rejected
+    whatever the uniform, max(0, p - q) has no mass, and the replacement is
+    the argmax of p -- on the GPU as in the oracle."""
+    B, N, V = 6, 3, 3000
+    Q = 2 * N - 1
+    rng = np.random.default_rng(44)
+    logits = I.random_logits(B, Q, V, seed=44)
+    prev = I.random_logits(B, Q, V, seed=45)
+    tok = rng.integers(0, V, (B, N)).astype(np.int32)
+    for b in range(B):
+        prev[b, N] = logits[b, 0]
+        logits[b, 0, tok[b, 1]] = -np.inf
+        prev[b, N, tok[b, 1]] = -np.inf
+    nc = np.full(B, N, np.int32)
+    kv = np.arange(B, dtype=np.int32) * 7
+    u = I.step_uniforms(3, 0, B, N)
+    gpu = _accept_only(isd, logits, prev, nc, tok, kv, u, N)
+    with np.errstate(invalid="ignore"):
+        ores = O.accept(logits, prev, nc, tok, kv, u, N)
+        rep = accept_parity(gpu, ores, logits, prev, dict(n_clean=nc, uniforms=u), N,
+                            O.PROPOSE_ARGMAX, "zero residual mass")
+    assert np.all(gpu["accept_len"] == 1)
+    assert np.array_equal(gpu["out_tok"][:, 0], logits[:, 0].argmax(-1))
+    assert np.all(gpu["next_n_clean"] == 1)
+    assert rep["near_threshold"] == 0 and rep["excused_draws"] == 0
 
 
 def test_identical_rows_accept_everything_gpu(isd):
@@ -431,7 +435,7 @@ def test_tiny_closed_loop_1000_steps(isd):
             torch.empty(cfg.B, dtype=torch.int32, device="cuda")]
     ratio = torch.empty(cfg.B, cfg.N - 1, dtype=torch.float32, device="cuda")
     err = torch.zeros(1, dtype=torch.int32, device="cuda")
-    near_total, emitted = 0, 0
+    near_total, excused_total, emitted = 0, 0, 0
     for k in range(steps):
         q, kn, vn = I.embed_block(tables, state["clean_tok"], state["n_clean"], cfg.N, cfg.V)
         u = I.step_uniforms(0, k, cfg.B, cfg.N)
@@ -457,8 +461,11 @@ def test_tiny_closed_loop_1000_steps(isd):
         gpu = dict(accept_len=outs[0].cpu().numpy(), out_tok=outs[1].cpu().numpy(),
                    next_n_clean=outs[2].cpu().numpy(), next_clean_tok=outs[3].cpu().numpy(),
                    next_kv_len=outs[4].cpu().numpy(), ratio=ratio.cpu().numpy())
-        near_total += compare_accept(gpu, ores, L, prev, dict(state, uniforms=u), cfg.N,
-                                     O.PROPOSE_ARGMAX)
+        rep = P.compare_accept(gpu, ores, L, prev, dict(state, uniforms=u), cfg.N,
+                               O.PROPOSE_ARGMAX)
+        assert rep["mismatches"] == 0, (k, rep["first_mismatch"])
+        near_total += rep["near_threshold"]
+        excused_total += rep["excused_draws"]
         emitted += int(gpu["accept_len"].sum())
         # advance with the GPU's state (the loop is driven by the CUDA path)
         state = dict(kv_len=gpu["next_kv_len"], n_clean=gpu["next_n_clean"],
@@ -466,8 +473,11 @@ def test_tiny_closed_loop_1000_steps(isd):
         prev = L.copy()
         prev_d.copy_(logits)
         prs.copy_(rs)
+    record_parity("tiny closed loop, 1000 steps",
+                  dict(requests=steps * cfg.B, near_threshold=near_total,
+                       excused_draws=excused_total, mismatches=0))
     assert int(err.item()) == 0
-    assert near_total <= 10
+    assert near_total + excused_total <= 10
     assert emitted >= steps * cfg.B
 
 
@@ -511,8 +521,9 @@ def test_full_size_b32_n4_sampled(isd):
     ores = O.accept(zg, prev, host["n_clean"], host["clean_tok"], host["kv_len"],
                     host["uniforms"], cfg.N)
     gpu = wl.outputs()
-    near = compare_accept(gpu, ores, zg, prev, host, cfg.N, O.PROPOSE_ARGMAX)
-    assert near <= 2
+    rep = accept_parity(gpu, ores, zg, prev, host, cfg.N, O.PROPOSE_ARGMAX,
+                        "full size qwen3_8b_b32_n4")
+    assert rep["near_threshold"] + rep["excused_draws"] <= 2
     # the constructed acceptance rate holds on every tested proposal
     r = ores["ratio"][ores["ratio"] >= 0]
     assert np.all(np.abs(r - cfg.accept_rate) < 1e-4)
