@@ -17,7 +17,7 @@ import pytest
 import torch
 
 from oracle import isd_oracle as O
-from oracle import parity as P
+from oracle import parity as OP
 from speculative_verification_isd_b200 import inputs as I
 
 from gpu_util import StepBuffers, bf16_host, f32_dev, i32_dev, record_parity, row_stats_host
@@ -31,13 +31,13 @@ def isd():
     return lib
 
 
-NEAR = P.NEAR
+NEAR = OP.NEAR
 
 
 def accept_parity(gpu, ores, logits, prev, inp, N, mode, label):
     """oracle.parity.compare_accept, recorded for the session's parity report
     (printed at the end of the run), with no unexplained difference allowed."""
-    rep = P.compare_accept(gpu, ores, logits, prev, inp, N, mode)
+    rep = OP.compare_accept(gpu, ores, logits, prev, inp, N, mode)
     record_parity(label, rep)
     assert rep["mismatches"] == 0, rep["first_mismatch"]
     return rep
@@ -215,13 +215,12 @@ def test_accept_on_random_logits(isd, mode, V, N, B):
     inp = dict(n_clean=nc, clean_tok=tok, uniforms=u)
     rep = accept_parity(gpu, ores, logits, prev, inp, N, mode,
                         f"random logits V={V} N={N} B={B} mode={mode}")
-    # a decision within 1e-5 of its uniform has probability ~2e-5 per test
+    # a decision within 1e-5 of its uniform has probability about 2e-5 per
+    # tested proposal; a GPU draw lands in a neighbouring bucket only when the
+    # target is within the fp32 prefix sums' rounding of a bucket edge.  Both
+    # were 0 in every case on B200 (1098 draws); the caps leave room for a rare one.
     assert rep["near_threshold"] <= max(1, B // 50)
-    # fp32 prefix sums over V entries move a draw by about V * 2^-24 of its
-    # mass; over a large vocabulary that lands in a neighbouring bucket for a
-    # measurable fraction of the draws (counted and reported, each checked by
-    # draw_explained); a small vocabulary should almost never need it
-    assert rep["excused_draws"] <= max(1, rep["draws"] // 50 if V < 100000 else rep["draws"] // 4)
+    assert rep["excused_draws"] <= max(1, rep["draws"] // 50)
     assert (ores["rejected_at"] > 0).sum() > 0 or N == 1
     assert int(err.item()) == 0
     # row stats of both inputs
@@ -461,8 +460,8 @@ def test_tiny_closed_loop_1000_steps(isd):
         gpu = dict(accept_len=outs[0].cpu().numpy(), out_tok=outs[1].cpu().numpy(),
                    next_n_clean=outs[2].cpu().numpy(), next_clean_tok=outs[3].cpu().numpy(),
                    next_kv_len=outs[4].cpu().numpy(), ratio=ratio.cpu().numpy())
-        rep = P.compare_accept(gpu, ores, L, prev, dict(state, uniforms=u), cfg.N,
-                               O.PROPOSE_ARGMAX)
+        rep = OP.compare_accept(gpu, ores, L, prev, dict(state, uniforms=u), cfg.N,
+                                O.PROPOSE_ARGMAX)
         assert rep["mismatches"] == 0, (k, rep["first_mismatch"])
         near_total += rep["near_threshold"]
         excused_total += rep["excused_draws"]
