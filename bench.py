@@ -546,8 +546,8 @@ def main():
         "e2e": {"value": e2e_value, "unit": "ISD steps/s", "h2d_bytes_per_step": int(h2d),
                 "d2h_bytes_per_step": int(d2h), "steps": KE, "warmup": max(3, W)},
         "sustained": sustained,
-        # KV append, attention, LM head, row-stats merge, accept (+ 3 LoRA kernels)
-        "gpu_launches": K * (5 + (3 if cfg.lora_rank else 0)),
+        # KV append, attention, LM head, accept (+ 3 LoRA kernels)
+        "gpu_launches": K * (4 + (3 if cfg.lora_rank else 0)),
         "clocks": clk, "err_flags": flags,
     }
     if lora_alpha is not None:

@@ -66,33 +66,6 @@ row_stats_kernel(const float* __restrict__ logits, int V, int n_chunks, int chun
     ticket[row] = 0;
 }
 
-// Row statistics from the LM head's per-(vocabulary tile, warp) partials:
-// part[row][k], k = 0..n_parts-1, merged in a fixed order.
-template <int THREADS>
-__global__ void __launch_bounds__(THREADS)
-row_stats_finalize_kernel(const float4* __restrict__ part, int n_parts,
-                          isd_row_stat* __restrict__ out) {
-    pdl_trigger();
-    pdl_wait();
-    const int row = blockIdx.x;
-    const float4* pr = part + (size_t)row * n_parts;
-    RowStat st = rowstat_empty();
-    // loads issued ahead of the (dependent) merges, in batches of 8 (one
-    // batch covers a 151936-entry vocabulary's 4748 partials)
-    for (int k0 = threadIdx.x; k0 < n_parts; k0 += 8 * THREADS) {
-        float4 p[8];
-#pragma unroll
-        for (int u = 0; u < 8; ++u) {
-            const int k = k0 + u * THREADS;
-            p[u] = k < n_parts ? __ldcs(pr + k) : make_float4(-INFINITY, 0.f, 0.f, 0.f);
-        }
-#pragma unroll
-        for (int u = 0; u < 8; ++u) st = rowstat_merge(st, RowStat{p[u].x, p[u].y, __float_as_int(p[u].z)});
-    }
-    st = rowstat_block_reduce<THREADS>(st);
-    if (threadIdx.x == 0) out[row] = isd_row_stat{st.m, st.s, st.idx, 0};
-}
-
 // ---------------------------------------------------------------------------
 // a6-a9
 // ---------------------------------------------------------------------------
@@ -116,6 +89,12 @@ struct AcceptArgs {
     int* ticket;     // [B]
     int n_chunks;
     int32_t* err_flag;
+    // inside a whole step: this step's row statistics come as the LM head's
+    // partials ([B*Q][n_parts]); the kernel merges the rows it needs and the
+    // CTA of chunk 0 writes each request's merged rows to stats_out
+    const float4* stats_part;
+    int n_parts;
+    isd_row_stat* stats_out;
 };
 
 // Weight of vocabulary entry i for "row" r of a sweep.
@@ -239,28 +218,57 @@ __global__ void __launch_bounds__(kAcceptThreads, 8) accept_kernel(AcceptArgs a)
     __shared__ int s_state;  // -1 invalid request, 0 no rejection, j = rejected proposal index
     __shared__ int s_last, s_bad;
     __shared__ float s_ratio[16];
+    __shared__ isd_row_stat s_stats[32];  // this request's merged rows (Q <= 31)
     const float* ub = a.uniforms + (size_t)b * 2 * N;
     const int c_in = __ldg(&a.n_clean[b]);
     const bool bad_c = (c_in < 1 || c_in > N);
+    const bool fused = a.stats_part != nullptr;
     if (threadIdx.x == 0) s_bad = 0;
     __syncthreads();
-    // all p/q ratios of this request at once (one gather round, not a chain)
-    {
-        const int j = (int)threadIdx.x + 2;
-        if (!bad_c && j <= c_in) {
-            const int x = __ldg(&a.clean_tok[(size_t)b * N + j - 1]);
-            if (x < 0 || x >= V) {
-                s_bad = 1;
-            } else {
-                const size_t rp = (size_t)b * Q + (j - 2);
-                const size_t rq = (size_t)b * Q + (N + j - 2);
-                const isd_row_stat sp = a.stats[rp], sq = a.prev_stats[rq];
-                const float zp = a.logits[rp * V + x];
-                const float zq = a.prev_logits[rq * V + x];
-                // p(x)/q(x) = exp((zp - mp) - (zq - mq)) * Sq / Sp
-                s_ratio[j - 2] = expf((zp - sp.max) - (zq - sq.max)) * (sq.sumexp / sp.sumexp);
+    // the gathered p/q operands of every tested proposal (one round of loads,
+    // in flight while the row statistics are merged)
+    const int jt = (int)threadIdx.x + 2;
+    float zp = 0.f, zq = 0.f;
+    isd_row_stat sq = isd_row_stat{0.f, 1.f, 0, 0};
+    bool have = false;
+    if (!bad_c && jt <= c_in) {
+        const int x = __ldg(&a.clean_tok[(size_t)b * N + jt - 1]);
+        if (x < 0 || x >= V) {
+            s_bad = 1;
+        } else {
+            const size_t rp = (size_t)b * Q + (jt - 2);
+            const size_t rq = (size_t)b * Q + (N + jt - 2);
+            zp = a.logits[rp * V + x];
+            zq = a.prev_logits[rq * V + x];
+            sq = a.prev_stats[rq];
+            have = true;
+        }
+    }
+    if (fused) {
+        // one warp per row: chunk 0 merges every row of the request (it writes
+        // them out); the other chunks the rows they read (tested proposals,
+        // and in sample mode the proposal rows they sweep)
+        const int wid = (int)threadIdx.x >> 5;
+        for (int k = wid; k < Q; k += kAcceptThreads / 32) {
+            const bool need = ch == 0 || k < c_in - 1 ||
+                              (a.mode == ISD_PROPOSE_SAMPLE && (k == c_in - 1 || k >= N));
+            if (!need) continue;
+            const RowStat st = warp_merge_partials(a.stats_part + ((size_t)b * Q + k) * a.n_parts, a.n_parts);
+            if ((threadIdx.x & 31) == 0) {
+                s_stats[k] = isd_row_stat{st.m, st.s, st.idx, 0};
+                if (ch == 0) a.stats_out[(size_t)b * Q + k] = s_stats[k];
             }
         }
+    }
+    __syncthreads();
+    // row statistics of row k of this request (this step's logits)
+    auto stat_of = [&](int k) -> isd_row_stat {
+        return fused ? s_stats[k] : a.stats[(size_t)b * Q + k];
+    };
+    // p(x)/q(x) = exp((zp - mp) - (zq - mq)) * Sq / Sp
+    if (have) {
+        const isd_row_stat sp = stat_of(jt - 2);
+        s_ratio[jt - 2] = expf((zp - sp.max) - (zq - sq.max)) * (sq.sumexp / sp.sumexp);
     }
     __syncthreads();
     if (threadIdx.x == 0) {
@@ -310,12 +318,12 @@ __global__ void __launch_bounds__(kAcceptThreads, 8) accept_kernel(AcceptArgs a)
         if (state > 0) {
             const size_t rp = (size_t)b * Q + (state - 2);
             const size_t rq = (size_t)b * Q + (N + state - 2);
-            const isd_row_stat sp = a.stats[rp], sq = a.prev_stats[rq];
+            const isd_row_stat sp = stat_of(state - 2), sq = a.prev_stats[rq];
             *r = SweepRow{a.logits + rp * V, a.prev_logits + rq * V, sp.max, sq.max,
                           1.f / sq.sumexp, (sq.max - sp.max) + logf(sq.sumexp / sp.sumexp)};
         } else {
             const size_t rr = (size_t)b * Q + (k == 0 ? c - 1 : N + k - 1);
-            const isd_row_stat s = a.stats[rr];
+            const isd_row_stat s = stat_of(k == 0 ? c - 1 : N + k - 1);
             *r = SweepRow{a.logits + rr * V, nullptr, s.max, 0.f, 0.f, 0.f};
         }
     };
@@ -376,9 +384,7 @@ __global__ void __launch_bounds__(kAcceptThreads, 8) accept_kernel(AcceptArgs a)
             __syncthreads();
             int y;
             if (q == -2) {  // argmax of the anchor (or proposal) row
-                const size_t fr = state > 0 ? (size_t)b * Q + (state - 2)
-                                            : (size_t)b * Q + (k == 0 ? c - 1 : N + k - 1);
-                y = a.stats[fr].argmax;
+                y = stat_of(state > 0 ? state - 2 : (k == 0 ? c - 1 : N + k - 1)).argmax;
             } else {
                 const int beg2 = q * kAcceptChunk, end2 = min(V, beg2 + kAcceptChunk);
                 chunk_scan(r, beg2, end2, tgt, &y);
@@ -389,8 +395,8 @@ __global__ void __launch_bounds__(kAcceptThreads, 8) accept_kernel(AcceptArgs a)
     } else {
         if (ch != 0) return;
         if (threadIdx.x == 0) {
-            picked[0] = a.stats[(size_t)b * Q + c - 1].argmax;
-            for (int m = 0; m + 1 < N; ++m) picked[m + 1] = a.stats[(size_t)b * Q + N + m].argmax;
+            picked[0] = stat_of(c - 1).argmax;
+            for (int m = 0; m + 1 < N; ++m) picked[m + 1] = stat_of(N + m).argmax;
         }
     }
     if (threadIdx.x != 0) return;
@@ -432,21 +438,19 @@ cudaError_t launch_row_stats(const Plan& p, const float* logits, int rows, int V
     return cudaGetLastError();
 }
 
-cudaError_t launch_row_stats_finalize(const float4* part, int n_parts, int rows,
-                                      isd_row_stat* out, cudaStream_t st, bool pdl) {
-    return launch_kernel(pdl, row_stats_finalize_kernel<kFinalizeThreads>, dim3(rows),
-                         dim3(kFinalizeThreads), 0, st, part, n_parts, out);
-}
-
 cudaError_t launch_accept(const Plan& p, const isd_dims* d, const float* logits,
                           const isd_row_stat* stats, const float* prev_logits,
                           const isd_row_stat* prev_stats, const int32_t* n_clean,
                           const int32_t* clean_tok, const int32_t* kv_len, const float* uniforms,
                           int32_t* accept_len, int32_t* out_tok, int32_t* next_n_clean,
                           int32_t* next_clean_tok, int32_t* next_kv_len, float* ratio, void* ws,
-                          int32_t* err_flag, cudaStream_t st, bool pdl) {
+                          int32_t* err_flag, cudaStream_t st, bool pdl, const float4* stats_part,
+                          int n_parts, isd_row_stat* stats_out) {
     char* w = static_cast<char*>(ws);
     AcceptArgs a;
+    a.stats_part = stats_part;
+    a.n_parts = n_parts;
+    a.stats_out = stats_out;
     a.B = d->B;
     a.N = d->N;
     a.V = d->V;

@@ -6,6 +6,7 @@
 #include <stdint.h>
 
 #include "../../include/isd.h"
+#include "plan.h"
 
 #define ISD_DEVINL __device__ __forceinline__
 
@@ -129,6 +130,35 @@ ISD_DEVINL RowStat rowstat_block_reduce(RowStat a) {
     }
     __syncthreads();
     return a;
+}
+
+
+// Row statistics from n <= kMaxStatParts partials p[0..n), merged by
+// one warp in a fixed order: lane l folds p[l], p[l + 32], ... in index order,
+// then the lanes meet in a fixed shuffle tree and lane 0's result is
+// broadcast.  Every caller (the LM head's merge kernel, the accept kernel)
+// uses this one routine, so the merged statistics are bit-identical.
+constexpr int kMaxPartsPerLane = kMaxStatParts / 32;
+ISD_DEVINL RowStat warp_merge_partials(const float4* p, int n) {
+    const int lane = threadIdx.x & 31;
+    RowStat st = rowstat_empty();
+    // batches of 4 loads per lane keep the register need small
+    for (int u0 = 0; u0 < kMaxPartsPerLane && 32 * u0 < n; u0 += 4) {
+        float4 v[4];
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
+            const int k = lane + 32 * (u0 + u);
+            v[u] = k < n ? __ldcg(p + k) : make_float4(-INFINITY, 0.f, 0.f, 0.f);
+        }
+#pragma unroll
+        for (int u = 0; u < 4; ++u) st = rowstat_merge(st, RowStat{v[u].x, v[u].y, __float_as_int(v[u].z)});
+    }
+#pragma unroll
+    for (int off = 16; off > 0; off >>= 1) st = rowstat_merge(st, rowstat_shfl_xor(st, off));
+    st.m = __shfl_sync(0xffffffffu, st.m, 0);
+    st.s = __shfl_sync(0xffffffffu, st.s, 0);
+    st.idx = __shfl_sync(0xffffffffu, st.idx, 0);
+    return st;
 }
 
 }  // namespace isd

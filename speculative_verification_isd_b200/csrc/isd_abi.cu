@@ -40,8 +40,9 @@ cudaError_t launch_attention(const Plan& p, const isd_dims* d, const uint16_t* q
 cudaError_t launch_lm_head(const uint16_t* hidden, const uint16_t* W, int Mh, int H, int V,
                            float* logits, float4* stats_part, void* tail_ws, int32_t* err_flag,
                            cudaStream_t st, bool pdl, bool counters_cleared);
-cudaError_t launch_row_stats_finalize(const float4* part, int n_parts, int rows,
-                                      isd_row_stat* out, cudaStream_t st, bool pdl);
+cudaError_t launch_lm_stats_merge(const float4* part, int n_parts, int rows, isd_row_stat* out,
+                                  cudaStream_t st, bool pdl);
+int lm_head_stat_parts(int Mh, int H, int V);
 cudaError_t launch_lora(const Plan& p, const isd_dims* d, const uint16_t* hidden,
                         const uint16_t* lora_A, const uint16_t* lora_B, uint16_t* hidden_out,
                         void* ws, cudaStream_t st);
@@ -53,7 +54,8 @@ cudaError_t launch_accept(const Plan& p, const isd_dims* d, const float* logits,
                           const int32_t* clean_tok, const int32_t* kv_len, const float* uniforms,
                           int32_t* accept_len, int32_t* out_tok, int32_t* next_n_clean,
                           int32_t* next_clean_tok, int32_t* next_kv_len, float* ratio, void* ws,
-                          int32_t* err_flag, cudaStream_t st, bool pdl);
+                          int32_t* err_flag, cudaStream_t st, bool pdl, const float4* stats_part,
+                          int n_parts, isd_row_stat* stats_out);
 }  // namespace isd
 
 using isd::Plan;
@@ -149,7 +151,8 @@ isd_status do_attention(const isd_dims* d, const Plan& p, const uint16_t* q,
     int* lm_ticket = nullptr;
     if (in_step) {
         acc_ticket = reinterpret_cast<int*>(static_cast<char*>(ws) + p.off_acc_ticket);
-        lm_ticket = reinterpret_cast<int*>(static_cast<char*>(ws) + p.off_lm_tail + isd::kLmTailPartBytes);
+        lm_ticket = reinterpret_cast<int*>(static_cast<char*>(ws) + p.off_lm_tail +
+                                           (size_t)isd::kMaxSMs * isd::lm_part_floats(p.M) * 4);
     }
     ISD_CUDA(isd::launch_attention(p, d, q, k_new, v_new, k_pool, v_pool, page_table, kv_len,
                                    n_clean, out, ws, err_flag, st, acc_ticket, lm_ticket,
@@ -169,16 +172,18 @@ isd_status do_lm_head(const isd_dims* d, const Plan& p, const uint16_t* hidden, 
         ISD_CUDA(isd::launch_lora(p, d, hidden, lora_A, lora_B, hl, ws, st));
         h = hl;
     }
-    // Row statistics come out of the LM head's epilogue as per-tile partials
-    // (no second pass over the logits); a small kernel merges them.
+    // Row statistics come out of the LM head's epilogue as partials (one per
+    // row and CTA; no second pass over the logits).  On its own the LM head
+    // merges them with a small kernel; inside the whole step the accept
+    // kernel merges them as it reads them.
     float4* part = row_stats ? reinterpret_cast<float4*>(static_cast<char*>(ws) + p.off_lm_stats)
                              : nullptr;
     ISD_CUDA(isd::launch_lm_head(h, W, p.M, p.H, d->V, logits, part,
                                  static_cast<char*>(ws) + p.off_lm_tail, err_flag, st,
                                  in_step && kStepPdl, in_step));
-    if (row_stats)
-        ISD_CUDA(isd::launch_row_stats_finalize(part, p.lm_stat_parts, p.M, row_stats, st,
-                                                in_step && kStepPdl));
+    if (row_stats && !in_step)
+        ISD_CUDA(isd::launch_lm_stats_merge(part, isd::lm_head_stat_parts(p.M, p.H, d->V), p.M,
+                                            row_stats, st, false));
     return ISD_OK;
 }
 
@@ -251,7 +256,8 @@ static isd_status accept_impl(const isd_dims* d, const float* logits, const isd_
                               const float* uniforms, int32_t* accept_len, int32_t* out_tok,
                               int32_t* next_n_clean, int32_t* next_clean_tok, int32_t* next_kv_len,
                               float* ratio, void* ws, size_t ws_bytes, int32_t* err_flag, void* stream,
-                              bool clear_counters) {
+                              bool clear_counters, const float4* stats_part = nullptr,
+                              int n_parts = 0, isd_row_stat* stats_out = nullptr) {
     Plan p;
     ISD_TRY(plan_or_fail(d, &p));
     ISD_TRY(check_ws(p, ws, ws_bytes));
@@ -266,7 +272,7 @@ static isd_status accept_impl(const isd_dims* d, const float* logits, const isd_
     ISD_CUDA(isd::launch_accept(p, d, logits, row_stats, prev_logits, prev_row_stats, n_clean,
                                 clean_tok, kv_len, uniforms, accept_len, out_tok, next_n_clean,
                                 next_clean_tok, next_kv_len, ratio, ws, err_flag, st,
-                                !clear_counters && kStepPdl));
+                                !clear_counters && kStepPdl, stats_part, n_parts, stats_out));
     return ISD_OK;
 }
 
@@ -306,9 +312,13 @@ isd_status isd_step(const isd_dims* d, const uint16_t* q, const uint16_t* k_new,
     ISD_TRY(do_attention(d, p, q, k_new, v_new, k_pool, v_pool, page_table, kv_len, n_clean, h,
                          ws, err_flag, st, true));
     ISD_TRY(do_lm_head(d, p, h, W, lora_A, lora_B, logits, row_stats, ws, err_flag, st, true));
+    // the accept kernel merges this step's row statistics from the LM head's
+    // partials and writes them to row_stats
+    const float4* part = reinterpret_cast<const float4*>(static_cast<char*>(ws) + p.off_lm_stats);
     return accept_impl(d, logits, row_stats, prev_logits, prev_row_stats, n_clean, clean_tok,
                        kv_len, uniforms, accept_len, out_tok, next_n_clean, next_clean_tok,
-                       next_kv_len, ratio, ws, ws_bytes, err_flag, stream, false);
+                       next_kv_len, ratio, ws, ws_bytes, err_flag, stream, false, part,
+                       isd::lm_head_stat_parts(p.M, p.H, d->V), row_stats);
 }
 
 }  // extern "C"

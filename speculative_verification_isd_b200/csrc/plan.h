@@ -24,8 +24,17 @@ constexpr int kAcceptChunk = 2048;
 // kMaxSMs, and the split heuristics below aim at a B200-sized grid.
 constexpr int kMaxSMs = 192;
 constexpr int kPlanSMs = 148;
-constexpr size_t kLmTailPartBytes = (size_t)kMaxSMs * 64 * 128 * 4;
-constexpr size_t kLmTailBytes = kLmTailPartBytes + (size_t)kMaxSMs * 4;
+// row-statistics partials per logits row at most (the LM head's epilogue
+// writes one per CTA plus two per left-over pair tile; merged by one warp)
+constexpr int kMaxStatParts = 384;
+// LM head: accumulator columns for Mh hidden rows (one block of <= 256
+// columns, or two equal blocks), each a multiple of 16
+inline int lm_cols(int Mh) {
+    if (Mh <= 256) return (Mh + 15) / 16 * 16;
+    return 2 * (((Mh + 1) / 2 + 15) / 16 * 16);
+}
+// floats of one CTA's tile-tail buffer: its 128 vocabulary rows x lm_cols
+inline size_t lm_part_floats(int Mh) { return (size_t)128 * lm_cols(Mh); }
 
 struct Plan {
     // derived dims
@@ -45,7 +54,8 @@ struct Plan {
     int acc_chunks;
     // R-ISD LoRA
     int lora_rows, lora_ksplit;
-    // LM-head row-statistics partials: one per 128-entry vocabulary tile
+    // LM-head row-statistics partials per row: room for one per CTA and two
+    // per left-over pair tile (the launch decides how many are used)
     int lm_stat_parts;
     // workspace offsets (bytes)
     size_t off_attn_part, off_attn_ticket, off_hidden, off_hidden_lora, off_lora_t,
@@ -133,11 +143,10 @@ inline bool make_plan(const isd_dims* d, Plan* p) {
     p->off_acc_part = take((size_t)d->B * (d->N + 1) * p->acc_chunks * 4);
     p->off_acc_ticket = take((size_t)d->B * 4);
     p->off_lora_part = take(d->lora_rank ? (size_t)p->lora_ksplit * p->lora_rows * d->lora_rank * 4 : 0);
-    p->lm_stat_parts = (d->V + 127) / 128;
+    p->lm_stat_parts = kMaxStatParts;
     p->off_lm_stats = take((size_t)p->M * p->lm_stat_parts * 16);
-    // LM head, left-over vocabulary tiles: K-slice partials (at most one per
-    // CTA, up to 64 hidden rows x 128 entries) and their counters
-    p->off_lm_tail = take(kLmTailBytes);
+    // LM head: one tile-tail accumulator buffer and one flag per CTA
+    p->off_lm_tail = take((size_t)kMaxSMs * lm_part_floats(p->M) * 4 + (size_t)kMaxSMs * 4);
     p->total = off;
     return true;
 }

@@ -115,12 +115,13 @@ def test_staged_parity(isd, name, n_clean):
     assert int(sb.err.item()) == 0
 
 
-def test_lm_head_left_over_tiles_by_row_chunks(isd):
-    """V = 151936 on a full GPU leaves a few 128-entry vocabulary tiles after
-    the whole waves; they are computed as 16-row chunks of the hidden rows
-    (M = 56 here, so the last chunk reaches past the matrix).  Every logit of
-    those tiles (and of two tiles of the waves) matches the oracle, every row's
-    statistics match, and a second run is bit-identical."""
+def test_lm_head_tiles_split_between_clusters(isd):
+    """The LM head splits the pair tiles' k-blocks evenly over clusters of two
+    CTAs ("stream-K"): a tile cut by a range boundary is summed from two
+    clusters' accumulators.  At V = 151936, M = 56 (full vocabulary, 8 heads'
+    worth of rows) every logit of the first split tiles, of the last (ragged)
+    tile and of one unsplit tile matches the oracle, every row's statistics
+    match, and a second run is bit-identical."""
     cfg = I.CONFIGS["qwen3_8b_b8_n4"]
     inp = I.make_step_inputs(cfg, seed=21)
     sb = StepBuffers(isd, cfg, inp)
@@ -129,11 +130,16 @@ def test_lm_head_left_over_tiles_by_row_chunks(isd):
     torch.cuda.synchronize()
     hid = bf16_host(sb.hidden)
     z_g = sb.logits.cpu().numpy()
-    n_tiles = (cfg.V + 127) // 128
-    grid = min(torch.cuda.get_device_properties(0).multi_processor_count, n_tiles)
-    first_left = (n_tiles // grid) * grid
-    assert first_left < n_tiles  # the shape does leave tiles over
-    cols = np.r_[0:128, 77 * 128:78 * 128, first_left * 128:cfg.V]
+    n_pairs = ((cfg.V + 127) // 128 + 1) // 2
+    grid = min(torch.cuda.get_device_properties(0).multi_processor_count & ~1, 192, 2 * n_pairs)
+    G2, kb = grid // 2, cfg.H // 64
+    U = n_pairs * kb
+    split = sorted({(U * c // G2) // kb for c in range(1, G2) if (U * c // G2) % kb})
+    assert len(split) > 8  # the shape does cut tiles
+    tiles = split[:6] + [n_pairs - 1]
+    unsplit = next(t for t in range(n_pairs) if t not in split)
+    tiles.append(unsplit)
+    cols = np.concatenate([np.arange(256 * t, min(256 * t + 256, cfg.V)) for t in tiles])
     z_o = O.lm_head(hid, inp["W"][cols])
     absdot = np.abs(O.bf16_to_f64(hid)) @ np.abs(O.bf16_to_f64(inp["W"][cols])).T
     assert np.all(np.abs(z_g[:, cols] - z_o) <= 1e-4 * absdot + 1e-6)
