@@ -194,6 +194,79 @@ isd_status isd_step(const isd_dims* d, const uint16_t* q, const uint16_t* k_new,
                     size_t ws_bytes, int32_t* err_flag, void* stream);
 
 /*
+ * isd_prepare_block -- the block activations of one step from each request's
+ * state, and on-device page bookkeeping.  The pages give no layer internals,
+ * so the per-layer forward that turns the block's tokens into q, k and v is
+ * stood in for by a table lookup:
+ *   Eq [V+1, Hq, D], Ek, Ev [V+1, Hkv, D] bf16: row t is token t, row V the
+ *   MASK token; slot s < n_clean[b] of request b reads row clean_tok[b][s],
+ *   every other slot (inactive clean slots, MASK slots) row V.
+ *   q [B, Q, Hq, D], k_new, v_new [B, Q, Hkv, D] bf16 (outputs)
+ * Page bookkeeping: request b's pages page_table[b][0 .. pages_used[b]) are
+ * extended to ceil((kv_len[b] + Q) / P) pages (at most max_pages_per_req)
+ * with pages taken in request order from *next_free_page (a bump allocator
+ * over [*next_free_page, num_pages), updated).  Running out of pages or
+ * columns raises ISD_FLAG_CAPACITY; an out-of-range token ISD_FLAG_TOKEN_OOB
+ * (the slot reads the MASK row).
+ */
+isd_status isd_prepare_block(const isd_dims* d, const uint16_t* Eq, const uint16_t* Ek,
+                             const uint16_t* Ev, const int32_t* n_clean, const int32_t* clean_tok,
+                             const int32_t* kv_len, int32_t* page_table, int32_t* pages_used,
+                             int32_t* next_free_page, uint16_t* q, uint16_t* k_new,
+                             uint16_t* v_new, int32_t* err_flag, void* stream);
+
+/*
+ * isd_loop -- n_steps ISD steps of a stationary batch, enqueued back to back
+ * with no host read between them: each step is isd_prepare_block followed by
+ * isd_step on the state of that step, so every request advances on its own
+ * ([PRJ], the paragraph on requests advancing independently; [ENG
+ * §服务部署与 SGLang 集成]: stationary batch, CUDA-graph capture).  The call is
+ * capturable into a CUDA graph.
+ * State and outputs are double buffers; step s reads buffer s & 1 and writes
+ * buffer (s + 1) & 1 (so the final state is in buffer n_steps & 1):
+ *   kv_len [2][B], n_clean [2][B], clean_tok [2][B][N] int32
+ *   logits [2][B*Q][V] fp32, row_stats [2][B*Q]: step s writes buffer s & 1
+ *          and reads buffer (s + 1) & 1 as the previous step's (step 0 reads
+ *          buffer 1, needed only for requests with n_clean > 1)
+ *   uniforms [n_steps][B][2N] fp32 (as isd_accept's, per step)
+ *   accept_len_hist [n_steps][B], out_tok_hist [n_steps][B][N] int32: the
+ *          accept lengths and emitted tokens of every step
+ *   q, k_new, v_new, hidden: one block's activations (caller-owned scratch,
+ *          the sizes of isd_step's arguments); page_table, pages_used,
+ *          next_free_page, k_pool, v_pool, W, lora_A, lora_B, Eq, Ek, Ev as
+ *          in isd_prepare_block and isd_step.
+ * ws: isd_workspace_bytes(d) bytes, as for isd_step.
+ */
+typedef struct {
+    const uint16_t* Eq;
+    const uint16_t* Ek;
+    const uint16_t* Ev;
+    const uint16_t* W;
+    const uint16_t* lora_A;
+    const uint16_t* lora_B;
+    uint16_t* k_pool;
+    uint16_t* v_pool;
+    int32_t* page_table;
+    int32_t* pages_used;
+    int32_t* next_free_page;
+    int32_t* kv_len;
+    int32_t* n_clean;
+    int32_t* clean_tok;
+    float* logits;
+    isd_row_stat* row_stats;
+    const float* uniforms;
+    uint16_t* q;
+    uint16_t* k_new;
+    uint16_t* v_new;
+    uint16_t* hidden;
+    int32_t* accept_len_hist;
+    int32_t* out_tok_hist;
+} isd_loop_args;
+
+isd_status isd_loop(const isd_dims* d, int32_t n_steps, const isd_loop_args* a, void* ws,
+                    size_t ws_bytes, int32_t* err_flag, void* stream);
+
+/*
  * isd_attention_noalloc -- isd_attention for callers that cannot provide a
  * workspace.  The paper has no counterpart: this is a deployment convenience.
  *

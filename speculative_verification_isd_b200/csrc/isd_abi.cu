@@ -48,6 +48,11 @@ cudaError_t launch_lora(const Plan& p, const isd_dims* d, const uint16_t* hidden
                         void* ws, cudaStream_t st);
 cudaError_t launch_row_stats(const Plan& p, const float* logits, int rows, int V,
                              isd_row_stat* out, void* ws, cudaStream_t st);
+cudaError_t launch_prepare_block(const isd_dims* d, const uint16_t* Eq, const uint16_t* Ek,
+                                 const uint16_t* Ev, const int32_t* n_clean, const int32_t* clean_tok,
+                                 const int32_t* kv_len, int32_t* page_table, int32_t* pages_used,
+                                 int32_t* next_free, uint16_t* q, uint16_t* k_new, uint16_t* v_new,
+                                 int32_t* err_flag, cudaStream_t st, bool pdl);
 cudaError_t launch_accept(const Plan& p, const isd_dims* d, const float* logits,
                           const isd_row_stat* stats, const float* prev_logits,
                           const isd_row_stat* prev_stats, const int32_t* n_clean,
@@ -131,11 +136,13 @@ isd_status check_accept_shape(const isd_dims* d) {
         if (e_ != cudaSuccess) return cuda_fail(e_); \
     } while (0)
 
-// The step's kernels can be launched with programmatic dependent launch
-// (launch.h).  On B200 at B=32, N=4 that measured about 3% slower than plain
-// stream order (alternating runs in one process, with or without the LM head
-// streaming W early), so it is off.
-constexpr bool kStepPdl = false;
+// The step's kernels are launched with programmatic dependent launch
+// (launch.h): each kernel may start its set-up (barriers, TMEM, tensor-map
+// prefetch; the LM head also streams W, which no kernel writes) while its
+// predecessor finishes, and waits for it before touching anything an earlier
+// kernel produces.  At B=32, N=4 on B200 this measured 3 us per step faster
+// than plain stream order (paired runs in one process).
+constexpr bool kStepPdl = true;
 
 isd_status do_attention(const isd_dims* d, const Plan& p, const uint16_t* q,
                         const uint16_t* k_new, const uint16_t* v_new, uint16_t* k_pool,
@@ -156,7 +163,7 @@ isd_status do_attention(const isd_dims* d, const Plan& p, const uint16_t* q,
     }
     ISD_CUDA(isd::launch_attention(p, d, q, k_new, v_new, k_pool, v_pool, page_table, kv_len,
                                    n_clean, out, ws, err_flag, st, acc_ticket, lm_ticket,
-                                   in_step ? isd::kMaxSMs : 0, kStepPdl));
+                                   in_step ? isd::kMaxSMs : 0, in_step && kStepPdl));
     return ISD_OK;
 }
 
@@ -287,6 +294,47 @@ isd_status isd_accept(const isd_dims* d, const float* logits, const isd_row_stat
                        ratio, ws, ws_bytes, err_flag, stream, true);
 }
 
+}  // extern "C"
+
+// The whole step on validated dims: attention (its first kernel also clears
+// the counters of the later ones, so the step issues no memset), LM head,
+// accept (which merges this step's row statistics from the LM head's
+// partials and writes them to row_stats).
+static isd_status step_impl(const isd_dims* d, const Plan& p, const uint16_t* q,
+                            const uint16_t* k_new, const uint16_t* v_new, uint16_t* k_pool,
+                            uint16_t* v_pool, const int32_t* page_table, const int32_t* kv_len,
+                            const int32_t* n_clean, const int32_t* clean_tok, const uint16_t* W,
+                            const uint16_t* lora_A, const uint16_t* lora_B, const float* prev_logits,
+                            const isd_row_stat* prev_row_stats, const float* uniforms,
+                            uint16_t* hidden, float* logits, isd_row_stat* row_stats,
+                            int32_t* accept_len, int32_t* out_tok, int32_t* next_n_clean,
+                            int32_t* next_clean_tok, int32_t* next_kv_len, float* ratio, void* ws,
+                            size_t ws_bytes, int32_t* err_flag, void* stream) {
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    uint16_t* h = hidden ? hidden
+                         : reinterpret_cast<uint16_t*>(static_cast<char*>(ws) + p.off_hidden);
+    ISD_TRY(do_attention(d, p, q, k_new, v_new, k_pool, v_pool, page_table, kv_len, n_clean, h,
+                         ws, err_flag, st, true));
+    ISD_TRY(do_lm_head(d, p, h, W, lora_A, lora_B, logits, row_stats, ws, err_flag, st, true));
+    const float4* part = reinterpret_cast<const float4*>(static_cast<char*>(ws) + p.off_lm_stats);
+    return accept_impl(d, logits, row_stats, prev_logits, prev_row_stats, n_clean, clean_tok,
+                       kv_len, uniforms, accept_len, out_tok, next_n_clean, next_clean_tok,
+                       next_kv_len, ratio, ws, ws_bytes, err_flag, stream, false, part,
+                       isd::lm_head_stat_parts(p.M, p.H, d->V), row_stats);
+}
+
+static isd_status check_step(const isd_dims* d, Plan* p, void* ws, size_t ws_bytes,
+                             const uint16_t* lora_A, const uint16_t* lora_B) {
+    ISD_TRY(plan_or_fail(d, p));
+    ISD_TRY(check_ws(*p, ws, ws_bytes));
+    ISD_TRY(check_attention_shape(d, *p));
+    ISD_TRY(check_lm_shape(d, *p, lora_A, lora_B));
+    ISD_TRY(check_accept_shape(d));
+    return ISD_OK;
+}
+
+extern "C" {
+
 isd_status isd_step(const isd_dims* d, const uint16_t* q, const uint16_t* k_new,
                     const uint16_t* v_new, uint16_t* k_pool, uint16_t* v_pool,
                     const int32_t* page_table, const int32_t* kv_len, const int32_t* n_clean,
@@ -298,27 +346,73 @@ isd_status isd_step(const isd_dims* d, const uint16_t* q, const uint16_t* k_new,
                     int32_t* next_kv_len, float* ratio, void* ws, size_t ws_bytes,
                     int32_t* err_flag, void* stream) {
     Plan p;
-    ISD_TRY(plan_or_fail(d, &p));
-    ISD_TRY(check_ws(p, ws, ws_bytes));
-    ISD_TRY(check_attention_shape(d, p));
-    ISD_TRY(check_lm_shape(d, p, lora_A, lora_B));
-    ISD_TRY(check_accept_shape(d));
+    ISD_TRY(check_step(d, &p, ws, ws_bytes, lora_A, lora_B));
     if (!row_stats || !logits) return invalid("null logits/row_stats");
+    return step_impl(d, p, q, k_new, v_new, k_pool, v_pool, page_table, kv_len, n_clean,
+                     clean_tok, W, lora_A, lora_B, prev_logits, prev_row_stats, uniforms, hidden,
+                     logits, row_stats, accept_len, out_tok, next_n_clean, next_clean_tok,
+                     next_kv_len, ratio, ws, ws_bytes, err_flag, stream);
+}
+
+static isd_status check_prepare(const isd_dims* d, const uint16_t* Eq, const uint16_t* Ek,
+                                const uint16_t* Ev, const void* n_clean, const void* clean_tok,
+                                const void* kv_len, const void* page_table, const void* pages_used,
+                                const void* next_free, const void* q, const void* k_new,
+                                const void* v_new) {
+    if (!Eq || !Ek || !Ev || !n_clean || !clean_tok || !kv_len || !page_table || !pages_used ||
+        !next_free || !q || !k_new || !v_new)
+        return invalid("null prepare-block pointer");
+    if ((d->Hkv * d->D) % 8) return unsupported("Hkv * D must be a multiple of 8");
+    return ISD_OK;
+}
+
+isd_status isd_prepare_block(const isd_dims* d, const uint16_t* Eq, const uint16_t* Ek,
+                             const uint16_t* Ev, const int32_t* n_clean, const int32_t* clean_tok,
+                             const int32_t* kv_len, int32_t* page_table, int32_t* pages_used,
+                             int32_t* next_free_page, uint16_t* q, uint16_t* k_new,
+                             uint16_t* v_new, int32_t* err_flag, void* stream) {
+    Plan p;
+    ISD_TRY(plan_or_fail(d, &p));
+    ISD_TRY(check_prepare(d, Eq, Ek, Ev, n_clean, clean_tok, kv_len, page_table, pages_used,
+                          next_free_page, q, k_new, v_new));
+    ISD_CUDA(isd::launch_prepare_block(d, Eq, Ek, Ev, n_clean, clean_tok, kv_len, page_table,
+                                       pages_used, next_free_page, q, k_new, v_new, err_flag,
+                                       static_cast<cudaStream_t>(stream), false));
+    return ISD_OK;
+}
+
+isd_status isd_loop(const isd_dims* d, int32_t n_steps, const isd_loop_args* a, void* ws,
+                    size_t ws_bytes, int32_t* err_flag, void* stream) {
+    Plan p;
+    if (!a) return invalid("null loop arguments");
+    ISD_TRY(check_step(d, &p, ws, ws_bytes, a->lora_A, a->lora_B));
+    if (n_steps < 0) return invalid("n_steps must be >= 0");
+    ISD_TRY(check_prepare(d, a->Eq, a->Ek, a->Ev, a->n_clean, a->clean_tok, a->kv_len,
+                          a->page_table, a->pages_used, a->next_free_page, a->q, a->k_new,
+                          a->v_new));
+    if (!a->W || !a->k_pool || !a->v_pool || !a->logits || !a->row_stats || !a->uniforms ||
+        !a->accept_len_hist || !a->out_tok_hist)
+        return invalid("null loop pointer");
+    const int B = d->B, N = d->N;
     cudaStream_t st = static_cast<cudaStream_t>(stream);
-    uint16_t* h = hidden ? hidden
-                         : reinterpret_cast<uint16_t*>(static_cast<char*>(ws) + p.off_hidden);
-    // The attention launch also clears the accept and LM-head counters, so the
-    // step issues no separate memset.
-    ISD_TRY(do_attention(d, p, q, k_new, v_new, k_pool, v_pool, page_table, kv_len, n_clean, h,
-                         ws, err_flag, st, true));
-    ISD_TRY(do_lm_head(d, p, h, W, lora_A, lora_B, logits, row_stats, ws, err_flag, st, true));
-    // the accept kernel merges this step's row statistics from the LM head's
-    // partials and writes them to row_stats
-    const float4* part = reinterpret_cast<const float4*>(static_cast<char*>(ws) + p.off_lm_stats);
-    return accept_impl(d, logits, row_stats, prev_logits, prev_row_stats, n_clean, clean_tok,
-                       kv_len, uniforms, accept_len, out_tok, next_n_clean, next_clean_tok,
-                       next_kv_len, ratio, ws, ws_bytes, err_flag, stream, false, part,
-                       isd::lm_head_stat_parts(p.M, p.H, d->V), row_stats);
+    for (int s = 0; s < n_steps; ++s) {
+        const int cur = s & 1, nxt = cur ^ 1;
+        ISD_CUDA(isd::launch_prepare_block(
+            d, a->Eq, a->Ek, a->Ev, a->n_clean + (size_t)cur * B, a->clean_tok + (size_t)cur * B * N,
+            a->kv_len + (size_t)cur * B, a->page_table, a->pages_used, a->next_free_page, a->q,
+            a->k_new, a->v_new, err_flag, st, kStepPdl));
+        ISD_TRY(step_impl(
+            d, p, a->q, a->k_new, a->v_new, a->k_pool, a->v_pool, a->page_table,
+            a->kv_len + (size_t)cur * B, a->n_clean + (size_t)cur * B,
+            a->clean_tok + (size_t)cur * B * N, a->W, a->lora_A, a->lora_B,
+            a->logits + (size_t)nxt * p.M * d->V, a->row_stats + (size_t)nxt * p.M,
+            a->uniforms + (size_t)s * B * 2 * N, a->hidden, a->logits + (size_t)cur * p.M * d->V,
+            a->row_stats + (size_t)cur * p.M, a->accept_len_hist + (size_t)s * B,
+            a->out_tok_hist + (size_t)s * B * N, a->n_clean + (size_t)nxt * B,
+            a->clean_tok + (size_t)nxt * B * N, a->kv_len + (size_t)nxt * B, nullptr, ws, ws_bytes,
+            err_flag, stream));
+    }
+    return ISD_OK;
 }
 
 }  // extern "C"

@@ -36,7 +36,8 @@ PROPOSE_ARGMAX = 0
 PROPOSE_SAMPLE = 1
 
 EXPORTED = ("isd_workspace_bytes", "isd_status_string", "isd_last_error", "isd_attention",
-            "isd_lm_head", "isd_row_stats", "isd_accept", "isd_step", "isd_attention_noalloc")
+            "isd_lm_head", "isd_row_stats", "isd_accept", "isd_step", "isd_prepare_block",
+            "isd_loop", "isd_attention_noalloc")
 NOALLOC_SCRATCH_BYTES = 32 * 1024 * 1024  # ISD_NOALLOC_SCRATCH_BYTES in include/isd.h
 
 
@@ -62,6 +63,16 @@ class Dims(ctypes.Structure):
 
 ROW_STAT_FIELDS = 4  # isd_row_stat = {float max, float sumexp, int32 argmax, int32 reserved}
 
+LOOP_FIELDS = ("Eq", "Ek", "Ev", "W", "lora_A", "lora_B", "k_pool", "v_pool", "page_table",
+               "pages_used", "next_free_page", "kv_len", "n_clean", "clean_tok", "logits",
+               "row_stats", "uniforms", "q", "k_new", "v_new", "hidden", "accept_len_hist",
+               "out_tok_hist")
+
+
+class LoopArgs(ctypes.Structure):
+    """isd_loop_args (include/isd.h): device pointers, in declaration order."""
+    _fields_ = [(n, ctypes.c_void_p) for n in LOOP_FIELDS]
+
 _vp = ctypes.c_void_p
 _sz = ctypes.c_size_t
 _i32 = ctypes.c_int32
@@ -83,6 +94,10 @@ _lib.isd_accept.argtypes = [_dims_p] + [_vp] * 15 + [_sz, _vp, _vp]
 _lib.isd_accept.restype = _i32
 _lib.isd_step.argtypes = [_dims_p] + [_vp] * 25 + [_sz, _vp, _vp]
 _lib.isd_step.restype = _i32
+_lib.isd_prepare_block.argtypes = [_dims_p] + [_vp] * 14
+_lib.isd_prepare_block.restype = _i32
+_lib.isd_loop.argtypes = [_dims_p, _i32, ctypes.POINTER(LoopArgs), _vp, _sz, _vp, _vp]
+_lib.isd_loop.restype = _i32
 _lib.isd_attention_noalloc.argtypes = [_dims_p] + [_vp] * 9 + [_vp, _vp]
 _lib.isd_attention_noalloc.restype = _i32
 
@@ -280,6 +295,56 @@ class StepCall:
         st = self._fn(*self._args)
         if st != ISD_OK:
             raise IsdError(st)
+
+
+def prepare_block(d: Dims, Eq, Ek, Ev, n_clean, clean_tok, kv_len, page_table, pages_used,
+                  next_free_page, q, k_new, v_new, err_flag=None, stream=None):
+    """isd_prepare_block: block activations by table lookup + page bookkeeping."""
+    B, N = d.B, d.N
+    _check(_lib.isd_prepare_block(
+        ctypes.byref(d), _ptr(Eq, _BF16, (d.V + 1) * d.Hq * d.D, "Eq"),
+        _ptr(Ek, _BF16, (d.V + 1) * d.Hkv * d.D, "Ek"), _ptr(Ev, _BF16, (d.V + 1) * d.Hkv * d.D, "Ev"),
+        _ptr(n_clean, torch.int32, B, "n_clean"), _ptr(clean_tok, torch.int32, B * N, "clean_tok"),
+        _ptr(kv_len, torch.int32, B, "kv_len"),
+        _ptr(page_table, torch.int32, B * d.max_pages_per_req, "page_table"),
+        _ptr(pages_used, torch.int32, B, "pages_used"),
+        _ptr(next_free_page, torch.int32, 1, "next_free_page"),
+        _ptr(q, _BF16, d.M * d.Hq * d.D, "q"), _ptr(k_new, _BF16, d.M * d.Hkv * d.D, "k_new"),
+        _ptr(v_new, _BF16, d.M * d.Hkv * d.D, "v_new"), _ptr(err_flag, torch.int32, 1, "err_flag"),
+        _stream(stream)))
+
+
+def loop_args(d: Dims, n_steps: int, **t) -> LoopArgs:
+    """Checked isd_loop_args from tensors named as its fields (lora_A / lora_B
+    may be omitted when lora_rank is 0)."""
+    B, N, M = d.B, d.N, d.M
+    kvrow = d.page_size * d.Hkv * d.D
+    want = dict(
+        Eq=(_BF16, (d.V + 1) * d.Hq * d.D), Ek=(_BF16, (d.V + 1) * d.Hkv * d.D),
+        Ev=(_BF16, (d.V + 1) * d.Hkv * d.D), W=(_BF16, d.V * d.H),
+        lora_A=(_BF16, d.H * d.lora_rank), lora_B=(_BF16, d.lora_rank * d.H),
+        k_pool=(_BF16, d.num_pages * kvrow), v_pool=(_BF16, d.num_pages * kvrow),
+        page_table=(torch.int32, B * d.max_pages_per_req), pages_used=(torch.int32, B),
+        next_free_page=(torch.int32, 1), kv_len=(torch.int32, 2 * B), n_clean=(torch.int32, 2 * B),
+        clean_tok=(torch.int32, 2 * B * N), logits=(torch.float32, 2 * M * d.V),
+        row_stats=((torch.int32, torch.float32), 2 * M * ROW_STAT_FIELDS),
+        uniforms=(torch.float32, n_steps * B * 2 * N), q=(_BF16, M * d.Hq * d.D),
+        k_new=(_BF16, M * d.Hkv * d.D), v_new=(_BF16, M * d.Hkv * d.D), hidden=(_BF16, M * d.H),
+        accept_len_hist=(torch.int32, n_steps * B), out_tok_hist=(torch.int32, n_steps * B * N))
+    vals = {}
+    for n in LOOP_FIELDS:
+        dt, numel = want[n]
+        vals[n] = _ptr(t.get(n), dt, numel, n)
+    return LoopArgs(**vals)
+
+
+def loop(d: Dims, n_steps: int, ws, err_flag=None, stream=None, args: Optional[LoopArgs] = None,
+         **tensors):
+    """isd_loop: n_steps ISD steps of a stationary batch on the device."""
+    a = args if args is not None else loop_args(d, n_steps, **tensors)
+    _check(_lib.isd_loop(ctypes.byref(d), int(n_steps), ctypes.byref(a),
+                         _ptr(ws, torch.uint8, None, "ws"), ws.numel(),
+                         _ptr(err_flag, torch.int32, 1, "err_flag"), _stream(stream)))
 
 
 def row_stats_view(rs: torch.Tensor):
