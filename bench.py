@@ -40,6 +40,10 @@ def parse_args():
     ap.add_argument("--e2e-steps", type=int, default=200)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-budget-s", type=float, default=20.0)
+    ap.add_argument("--sustained-s", type=float, default=2.5,
+                    help="seconds of the sustained leg; 0 skips it")
+    ap.add_argument("--loop-steps", type=int, default=400,
+                    help="timed steps of the closed-loop leg (isd_loop); 0 skips it")
     return ap.parse_args()
 
 
@@ -287,6 +291,70 @@ def accept_parity(wl, cfg, k):
 
 
 # ---------------------------------------------------------------------------
+# LM head scale of the closed-loop model.  The proposal acceptance of the loop
+# is a property of its synthetic model (see LoopWorkload); at this scale the
+# measured rate at B=32, N=4 is about 0.9, the rate of the tokens-per-forward
+# table on the engineering page (section on the core parameters of token
+# generation).  Attention inputs N(0, 0.5), cache N(0, 1.0).
+LOOP_W_STD, LOOP_QKV_STD, LOOP_KV_STD = 0.1, 0.5, 1.0
+
+
+def restart_model_tpf(a, N):
+    """Tokens per forward of the restart state machine when every proposal is
+    kept with probability a: a cycle that keeps all N-1 proposals (probability
+    a^(N-1)) is one forward; any other adds a restart forward (one clean
+    token) and emits one replacement token."""
+    f = a ** (N - 1)
+    eacc = (1.0 - a ** N) / (1.0 - a) if a < 1.0 else float(N)
+    return (eacc + 1.0 - f) / (2.0 - f)
+
+
+def closed_loop(isd, cfg, R, K, bus, seed):
+    """Closed-loop leg: isd_loop runs K steps of a stationary batch on the
+    device (block activations by table lookup, pages from the on-device
+    allocator, accept state and logits in double buffers; five kernels per
+    step), after 16 untimed steps.  Tokens/s counts every token the requests
+    emitted in the timed steps, over the slowest rank's time."""
+    import torch
+    from speculative_verification_isd_b200.workload import LoopWorkload
+    W = 16
+    K += K % 2
+    lw = LoopWorkload(isd, cfg, capacity_steps=W + K, seed=seed, w_std=LOOP_W_STD,
+                      qkv_std=LOOP_QKV_STD, kv_std=LOOP_KV_STD)
+    stream = torch.cuda.current_stream()
+    lw.run(W)
+    torch.cuda.synchronize()
+    args = lw.args(W, K)
+    clocks = ClockSampler(bus)
+    clocks.start()
+    time.sleep(0.2)
+    R.barrier()
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    lw.run(K, args=args)
+    e1.record(stream)
+    torch.cuda.synchronize()
+    R.barrier()
+    clk = clocks.stop()
+    ms = R.max(e0.elapsed_time(e1))
+    st = lw.stats(W, W + K)
+    tokens = R.sum(st["tokens"])
+    kv_end = lw.kv_len[0].float().mean().item()
+    out = {"workload": cfg.name + " closed loop", "steps": K, "warmup": W,
+           "ms_per_step": ms / K, "steps_per_s": K * R.world / (ms / 1e3),
+           "tokens_per_s": tokens / (ms / 1e3), "tpf": st["tpf"], "tpf_se": st["tpf_se"],
+           "accept_rate": st["accept_rate"],
+           "accept_rate_by_position": st["accept_rate_by_position"],
+           "tpf_restart_model_at_measured_rate": restart_model_tpf(st["accept_rate"], cfg.N),
+           "model": {"w_std": LOOP_W_STD, "qkv_std": LOOP_QKV_STD, "kv_std": LOOP_KV_STD},
+           "mean_kv_len": {"start": float(lw.kv0.mean()), "end": kv_end},
+           "gpu_launches": 5 * K, "err_flags": int(lw.err.item()), "clocks": clk}
+    del lw
+    torch.cuda.empty_cache()
+    return out
+
+
 def config_dict(cfg, world):
     return {"workload": cfg.name, "B": cfg.B, "N": cfg.N, "Q": cfg.Q, "V": cfg.V,
             "hidden": cfg.H, "heads": f"{cfg.Hq}q/{cfg.Hkv}kv x {cfg.D}",
@@ -414,24 +482,26 @@ def main():
     flags = int(wl.err.item())
 
     # ---------------- sustained: the same step back to back for >= 2.5 s, own clock record
-    n_sus = max(K, int(2.5e3 / max(1e-3, t_ms / K)))
-    clocks2 = ClockSampler(bus)
-    clocks2.start()
-    time.sleep(0.2)
-    R.barrier()
-    torch.cuda.synchronize()
-    s0, s1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    s0.record(stream)
-    for k in range(n_sus):
-        run_step(k)
-    s1.record(stream)
-    torch.cuda.synchronize()
-    R.barrier()
-    clk_sus = clocks2.stop()
-    sus_ms = R.max(s0.elapsed_time(s1))
-    sustained = {"value": RK.job_throughput(n_sus, R, sus_ms), "unit": "ISD steps/s",
-                 "steps": n_sus, "seconds": sus_ms / 1e3, "ms_per_step": sus_ms / n_sus,
-                 "clocks": clk_sus}
+    sustained = None
+    if args.sustained_s > 0:
+        n_sus = max(K, int(args.sustained_s * 1e3 / max(1e-3, t_ms / K)))
+        clocks2 = ClockSampler(bus)
+        clocks2.start()
+        time.sleep(0.2)
+        R.barrier()
+        torch.cuda.synchronize()
+        s0, s1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        s0.record(stream)
+        for k in range(n_sus):
+            run_step(k)
+        s1.record(stream)
+        torch.cuda.synchronize()
+        R.barrier()
+        clk_sus = clocks2.stop()
+        sus_ms = R.max(s0.elapsed_time(s1))
+        sustained = {"value": RK.job_throughput(n_sus, R, sus_ms), "unit": "ISD steps/s",
+                     "steps": n_sus, "seconds": sus_ms / 1e3, "ms_per_step": sus_ms / n_sus,
+                     "clocks": clk_sus}
 
     # ---------------- stage breakdown (same work, stage by stage, events between)
     KS = min(K, 300)
@@ -516,6 +586,10 @@ def main():
     e2e_ms = R.max(e0.elapsed_time(e1))
     e2e_value = KE * world / (e2e_ms / 1e3)
 
+    loop_line = None
+    if args.loop_steps > 0:
+        loop_line = closed_loop(isd, cfg, R, args.loop_steps, bus, RK.rank_seed(0, rank))
+
     # ---------------- roofline of the dominant kernel (LM head)
     lm_bytes = float(cfg.V) * cfg.H * 2 + float(cfg.M) * cfg.H * 2 + float(cfg.M) * cfg.V * 4
     lm_flops = 2.0 * cfg.M * cfg.H * cfg.V
@@ -550,6 +624,8 @@ def main():
         "gpu_launches": K * (4 + (3 if cfg.lora_rank else 0)),
         "clocks": clk, "err_flags": flags,
     }
+    if loop_line is not None:
+        line["closed_loop"] = loop_line
     if lora_alpha is not None:
         # step time with the adapter / without it (the pages report about 1.12)
         line["lora_alpha"] = lora_alpha

@@ -203,4 +203,138 @@ def request_slice(host: Dict, cfg: I.IsdConfig, b: int) -> Dict[str, np.ndarray]
         kv_len=host["kv_len"][b:b + 1], n_clean=host["n_clean"][b:b + 1])
 
 
-__all__ = ["DeviceWorkload", "request_slice"]
+class LoopWorkload:
+    """Device buffers of the stationary-batch loop (isd_loop) at a config.
+
+    The block's activations come from token -> (q, k, v) tables of V + 1 rows
+    (row V is the MASK token) drawn N(0, qkv_std); the prefix pages hold
+    N(0, kv_std) keys and values; the LM head is N(0, w_std).  The pool has
+    room for every request's prefix plus ``capacity_steps`` steps of growth,
+    handed out on the device.  Every request starts with one clean token.  With
+    a LoRA rank in the config, the gated adapter (N(0, lora_std)) is applied
+    to the MASK rows as in the single step.
+
+    The acceptance rate of the loop is a property of this synthetic model: a
+    proposal x (argmax of the previous step's MASK row q) is kept with
+    probability min(1, p(x)/q(x)), and p and q are the LM head applied to two
+    attention outputs over almost the same context; w_std scales the logit
+    gap between them, so it sets the rate.
+    """
+
+    FIELDS = ("Eq", "Ek", "Ev", "W", "k_pool", "v_pool", "page_table", "pages_used",
+              "next_free_page", "kv_len", "n_clean", "clean_tok", "logits", "row_stats", "q",
+              "k_new", "v_new", "hidden")
+
+    def __init__(self, isd, cfg: I.IsdConfig, capacity_steps: int, seed: int = 0,
+                 w_std: Optional[float] = None, qkv_std: Optional[float] = None,
+                 kv_std: Optional[float] = None):
+        self.isd, self.cfg, self.seed = isd, cfg, seed
+        B, N, Q, V, P = cfg.B, cfg.N, cfg.Q, cfg.V, cfg.page_size
+        w_std = cfg.w_std if w_std is None else w_std
+        qkv_std = cfg.qkv_std if qkv_std is None else qkv_std
+        kv_std = cfg.kv_std if kv_std is None else kv_std
+        self.w_std, self.qkv_std, self.kv_std = w_std, qkv_std, kv_std
+        kv0 = I.prefix_lengths(cfg, seed)
+        pre = (kv0.astype(np.int64) + P - 1) // P
+        max_pages = int((kv0.max() + capacity_steps * N + Q + P - 1) // P + 1)
+        num_pages = int(pre.sum()) + B * max_pages
+        table = np.full((B, max_pages), -1, np.int32)
+        nxt = 0
+        for b in range(B):
+            table[b, : pre[b]] = np.arange(nxt, nxt + pre[b], dtype=np.int32)
+            nxt += int(pre[b])
+        rng = np.random.default_rng([seed, 37])
+        tok0 = np.full((B, N), -1, np.int32)
+        tok0[:, 0] = rng.integers(0, V, B)
+        self.kv0 = kv0
+        self.capacity_steps = capacity_steps
+        self.dims = isd.make_dims(B, N, cfg.Hq, cfg.Hkv, cfg.D, V, P, num_pages, max_pages,
+                                  cfg.lora_rank)
+        d = self.dims
+        gen = torch.Generator(device="cuda")
+        gen.manual_seed(seed)
+        self.Eq = _randn_bf16((V + 1, cfg.Hq, cfg.D), qkv_std, gen)
+        self.Ek = _randn_bf16((V + 1, cfg.Hkv, cfg.D), qkv_std, gen)
+        self.Ev = _randn_bf16((V + 1, cfg.Hkv, cfg.D), qkv_std, gen)
+        self.W = _randn_bf16((V, cfg.H), w_std, gen)
+        self.k_pool = _randn_bf16((num_pages, P, cfg.Hkv, cfg.D), kv_std, gen)
+        self.v_pool = _randn_bf16((num_pages, P, cfg.Hkv, cfg.D), kv_std, gen)
+        r = cfg.lora_rank
+        self.lora_A = _randn_bf16((cfg.H, r), cfg.lora_std, gen) if r else None
+        self.lora_B = _randn_bf16((r, cfg.H), cfg.lora_std, gen) if r else None
+        dev = lambda x: torch.from_numpy(np.ascontiguousarray(x)).cuda()
+        self.page_table = dev(table)
+        self.pages_used = dev(pre.astype(np.int32))
+        self.next_free_page = dev(np.array([nxt], np.int32))
+        self.kv_len = dev(np.stack([kv0.astype(np.int32), np.zeros(B, np.int32)]))
+        self.n_clean = dev(np.stack([np.ones(B, np.int32), np.zeros(B, np.int32)]))
+        self.clean_tok = dev(np.stack([tok0, np.full((B, N), -1, np.int32)]))
+        M = d.M
+        self.logits = torch.zeros(2 * M * V, dtype=torch.float32, device="cuda")
+        self.row_stats = torch.zeros(2 * M * 4, dtype=torch.int32, device="cuda")
+        self.q = torch.empty(M * cfg.Hq * cfg.D, dtype=torch.bfloat16, device="cuda")
+        self.k_new = torch.empty(M * cfg.Hkv * cfg.D, dtype=torch.bfloat16, device="cuda")
+        self.v_new = torch.empty(M * cfg.Hkv * cfg.D, dtype=torch.bfloat16, device="cuda")
+        self.hidden = torch.empty(M * d.H, dtype=torch.bfloat16, device="cuda")
+        self.uniforms = dev(np.stack([I.step_uniforms(seed, k, B, N)
+                                      for k in range(capacity_steps)]))
+        self.accept_len_hist = torch.zeros(capacity_steps, B, dtype=torch.int32, device="cuda")
+        self.out_tok_hist = torch.zeros(capacity_steps, B, N, dtype=torch.int32, device="cuda")
+        self.ws = isd.alloc_workspace(d)
+        self.err = torch.zeros(1, dtype=torch.int32, device="cuda")
+        self.done = 0
+
+    def args(self, start: int, n: int):
+        """Checked isd_loop arguments for steps start .. start+n-1 (start even,
+        so that the state and logits of step ``start`` are in buffer 0)."""
+        if start % 2 or start + n > self.capacity_steps:
+            raise ValueError("loop steps must start even and stay within capacity")
+        t = {f: getattr(self, f) for f in self.FIELDS}
+        if self.cfg.lora_rank:
+            t["lora_A"], t["lora_B"] = self.lora_A, self.lora_B
+        t["uniforms"] = self.uniforms[start:start + n]
+        t["accept_len_hist"] = self.accept_len_hist[start:start + n]
+        t["out_tok_hist"] = self.out_tok_hist[start:start + n]
+        return self.isd.loop_args(self.dims, n, **t)
+
+    def run(self, n: int, stream=None, args=None):
+        """Enqueue the next n steps (n even keeps the next call's start even)."""
+        a = args if args is not None else self.args(self.done, n)
+        self.isd.loop(self.dims, n, self.ws, err_flag=self.err, stream=stream, args=a)
+        self.done += n
+
+    def stats(self, start: int, stop: int) -> Dict[str, float]:
+        """Tokens per forward and the proposal acceptance rate of steps
+        start .. stop-1, from the accept-length history.
+
+        The clean count c of each step follows from the history: every request
+        starts at c = 1; a step that keeps all of its c tokens continues with
+        c = N, any other with c = 1 (the restart).  A step with c clean tokens
+        tests proposals 2..c in order and stops at the first rejection, so it
+        accepted A - 1 of them and made one more (rejected) test if A < c."""
+        N = self.cfg.N
+        al = self.accept_len_hist[:stop].cpu().numpy().astype(np.int64)
+        c = np.ones(al.shape[1], np.int64)
+        acc = tests = 0
+        acc_pos = np.zeros(max(N - 1, 1))
+        tests_pos = np.zeros(max(N - 1, 1))
+        for s in range(stop):
+            A = al[s]
+            if s >= start:
+                full = A == c
+                tested = np.where(full, c - 1, A)
+                acc += int((A - 1).sum())
+                tests += int(tested.sum())
+                for j in range(N - 1):
+                    tests_pos[j] += int((tested > j).sum())
+                    acc_pos[j] += int((A - 1 > j).sum())
+            c = np.where(A == c, N, 1)
+        window = al[start:stop]
+        tpf = float(window.mean())
+        se = float(window.mean(axis=0).std(ddof=1) / math.sqrt(window.shape[1]))
+        return dict(tokens=int(window.sum()), tpf=tpf, tpf_se=se,
+                    accept_rate=acc / max(tests, 1), tests=tests,
+                    accept_rate_by_position=[float(a / max(t, 1)) for a, t in zip(acc_pos, tests_pos)])
+
+
+__all__ = ["DeviceWorkload", "LoopWorkload", "request_slice"]

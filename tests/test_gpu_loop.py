@@ -208,3 +208,136 @@ def test_loop_with_rejections(isd):
     later = al[1:]
     assert (later == 1).any() and (later == cfg.N).any() and ((later > 1) & (later < cfg.N)).any()
     assert rejections >= 20 and draws >= 20
+
+
+def _ids(tok, nc, N, V):
+    Q = 2 * N - 1
+    ids = np.full((tok.shape[0], Q), V, np.int64)
+    for b in range(tok.shape[0]):
+        ids[b, : int(nc[b])] = tok[b, : int(nc[b])]
+    return ids
+
+
+def test_loop_full_shape_b32_n4(isd):
+    """Headline shape (B=32, N=4, Qwen3-8B sizes, prefixes U[512, 8192], the
+    benchmark's closed-loop model).  Ten steps one per call: every block row
+    equals its table row, the page table follows the allocator's rule, the KV
+    append put each block slot's key/value at its position, the row statistics
+    match the GPU's logits, sampled logits match the oracle's dot products,
+    and the accept decisions, tokens and next states match the oracle's on the
+    GPU's logits.  Then the same ten steps in one call are bit-identical."""
+    from speculative_verification_isd_b200.workload import LoopWorkload
+    cfg = I.CONFIGS["qwen3_8b_b32_n4"]
+    B, N, Q, V, P = cfg.B, cfg.N, cfg.Q, cfg.V, cfg.page_size
+    steps = 10
+    mk = lambda: LoopWorkload(isd, cfg, capacity_steps=steps, seed=2, w_std=0.1, qkv_std=0.5,
+                              kv_std=1.0)
+    lw = mk()
+    d, M = lw.dims, lw.dims.M
+    maxp = d.max_pages_per_req
+    t = {f: getattr(lw, f) for f in lw.FIELDS}
+    hist_al = torch.zeros(1, B, dtype=torch.int32, device="cuda")
+    hist_ot = torch.zeros(1, B, N, dtype=torch.int32, device="cuda")
+    o_table = lw.page_table.cpu().numpy().reshape(B, maxp).copy()
+    o_used = (lw.kv0.astype(np.int64) + P - 1) // P
+    o_next = int(lw.next_free_page.item())
+    W_h = bf16_host(lw.W).reshape(V, d.H)
+    rng = np.random.default_rng(4)
+    prev = np.zeros((B, Q, V), np.float32)
+    al_step, ot_step = [], []
+    near = excused = draws = 0
+    for s in range(steps):
+        kv = lw.kv_len[0].cpu().numpy()
+        nc = lw.n_clean[0].cpu().numpy()
+        tok = lw.clean_tok[0].cpu().numpy()
+        u = lw.uniforms[s].cpu().numpy()
+        isd.loop(d, 1, lw.ws, err_flag=lw.err, uniforms=lw.uniforms[s:s + 1],
+                 accept_len_hist=hist_al, out_tok_hist=hist_ot, **t)
+        torch.cuda.synchronize()
+        # block rows are table rows
+        ids = torch.from_numpy(_ids(tok, nc, N, V).reshape(-1)).cuda()
+        assert torch.equal(lw.q.view(M, -1), lw.Eq.view(V + 1, -1)[ids])
+        assert torch.equal(lw.k_new.view(M, -1), lw.Ek.view(V + 1, -1)[ids])
+        assert torch.equal(lw.v_new.view(M, -1), lw.Ev.view(V + 1, -1)[ids])
+        # pages: ceil((kv_len + Q) / P) per request, new ones in request order
+        for b in range(B):
+            need = min((int(kv[b]) + Q + P - 1) // P, maxp)
+            while o_used[b] < need:
+                o_table[b, o_used[b]] = o_next
+                o_used[b] += 1
+                o_next += 1
+        table = lw.page_table.cpu().numpy().reshape(B, maxp)
+        assert np.array_equal(table, o_table)
+        # the KV append: every active block slot's key/value at its position
+        rows, pos = [], []
+        for b in range(B):
+            p_b = O.slot_positions(int(kv[b]), int(nc[b]), N)
+            for i in range(Q):
+                if p_b[i] >= 0:
+                    rows.append(b * Q + i)
+                    pos.append(int(p_b[i]))
+        rows_t = torch.tensor(rows, dtype=torch.long, device="cuda")
+        pos = np.array(pos)
+        bidx = np.array(rows) // Q
+        pages = torch.from_numpy(table[bidx, pos // P].astype(np.int64)).cuda()
+        offs = torch.from_numpy(pos % P).long().cuda()
+        assert torch.equal(lw.k_pool[pages, offs].view(len(rows), -1), lw.k_new.view(M, -1)[rows_t])
+        assert torch.equal(lw.v_pool[pages, offs].view(len(rows), -1), lw.v_new.view(M, -1)[rows_t])
+        # logits: sampled entries against the oracle's dot products on the
+        # GPU's hidden, row statistics of every row against the GPU's logits
+        z_g = lw.logits[: M * V].view(M, V).cpu().numpy()
+        hid = bf16_host(lw.hidden).reshape(M, d.H)
+        for m, v in zip(rng.integers(0, M, 48), rng.integers(0, V, 48)):
+            ref = O.lm_head_entry(hid[m], W_h[v])
+            bound = 1e-4 * float(np.abs(O.bf16_to_f64(hid[m])) @ np.abs(O.bf16_to_f64(W_h[v]))) + 1e-6
+            assert abs(float(z_g[m, v]) - ref) <= bound, (s, m, v)
+        m_g, s_g, a_g = row_stats_host(lw.row_stats[: M * 4])
+        m_o, s_o, a_o = O.row_stats_all(z_g)
+        assert np.array_equal(m_g, m_o.astype(np.float32).astype(np.float64))
+        assert np.array_equal(a_g, a_o)
+        assert np.all(np.abs(s_g - s_o) <= OP.NEAR * s_o)
+        # acceptance on the GPU's logits
+        L = z_g.reshape(B, Q, V)
+        ores = O.accept(L, prev, nc, tok, kv, u, N)
+        al = hist_al[0].cpu().numpy()
+        ot = hist_ot[0].cpu().numpy()
+        gpu = dict(accept_len=al, out_tok=ot, next_n_clean=lw.n_clean[1].cpu().numpy(),
+                   next_clean_tok=lw.clean_tok[1].cpu().numpy(),
+                   next_kv_len=lw.kv_len[1].cpu().numpy(), ratio=ores["ratio"])
+        rep = OP.compare_accept(gpu, ores, L, prev, dict(n_clean=nc, uniforms=u), N,
+                                O.PROPOSE_ARGMAX)
+        assert rep["mismatches"] == 0, (s, rep["first_mismatch"])
+        near += rep["near_threshold"]
+        excused += rep["excused_draws"]
+        draws += rep["draws"]
+        al_step.append(al.copy())
+        ot_step.append(ot.copy())
+        for k in ("kv_len", "n_clean", "clean_tok"):
+            getattr(lw, k)[0].copy_(getattr(lw, k)[1])
+        lw.logits[M * V:].copy_(lw.logits[: M * V])
+        lw.row_stats[M * 4:].copy_(lw.row_stats[: M * 4])
+        prev = L.copy()
+    assert int(lw.err.item()) == 0
+    record_parity("device loop, B=32 N=4 full shape, one step per call",
+                  dict(requests=steps * B, near_threshold=near, draws=draws,
+                       excused_draws=excused, mismatches=0))
+    assert near <= max(1, steps * B // 50) and excused <= max(1, draws // 50)
+    # restarts and full accepts both occur
+    al_all = np.stack(al_step)
+    assert (al_all[1:] == N).any() and (al_all[2:] < N).any()
+
+    # the same steps in one call
+    lw2 = mk()
+    lw2.run(steps)
+    torch.cuda.synchronize()
+    assert int(lw2.err.item()) == 0
+    assert np.array_equal(lw2.accept_len_hist.cpu().numpy(), al_all)
+    assert np.array_equal(lw2.out_tok_hist.cpu().numpy(), np.stack(ot_step))
+    fin = steps & 1
+    for k in ("kv_len", "n_clean", "clean_tok"):
+        assert torch.equal(getattr(lw2, k)[fin], getattr(lw, k)[0]), k
+    assert torch.equal(lw2.page_table, lw.page_table)
+    assert torch.equal(lw2.next_free_page, lw.next_free_page)
+    assert torch.equal(lw2.k_pool, lw.k_pool) and torch.equal(lw2.v_pool, lw.v_pool)
+    last = (steps - 1) & 1
+    assert torch.equal(lw2.logits[last * M * V:(last + 1) * M * V], lw.logits[: M * V])
