@@ -18,6 +18,12 @@
 //    (request, kv head) cut by a range boundary leaves a partial result per
 //    CTA; the CTA that draws the last ticket merges them in CTA order, so the
 //    result does not depend on timing;
+//  * K and V halves of a stage have their own ring barriers and their own
+//    TMA producer warp: the K half is refilled as soon as S = K.Q^T has
+//    read it, the V half after P.V, so a stage's bytes wait in shared memory
+//    only about one product's latency (with a 3-stage ring of 128 keys,
+//    holding a stage for the whole S -> softmax -> P.V chain measured about
+//    3% slower for the whole step at B=32, N=4);
 //  * per 128-key tile two tensor-core products, issued by one thread:
 //      S^T[128 keys, R rows] = K . Q^T         (M=128, N=R, K=128 d)
 //      O^T[128 d,   R rows] += V^T . P^T       (M=128, N=R, K=128 keys)
@@ -132,7 +138,7 @@ __global__ void kv_append_kernel(TcArgs a, const __nv_bfloat16* k_new, const __n
 
 template <int STAGES>
 struct TcShared {
-    uint64_t kv_full[STAGES], kv_empty[STAGES];
+    uint64_t k_full[STAGES], k_empty[STAGES], v_full[STAGES], v_empty[STAGES];
     uint64_t s_full[2], s_empty[2], p_full, p_empty;
     uint64_t o_full, o_empty, q_full[2], q_empty[2], drain;
     uint32_t tmem;
@@ -157,7 +163,8 @@ struct TcRoles {
     static constexpr int RC = R == 64 ? 32 : 16;  // rows per softmax thread
     static constexpr int CG = R / RC;           // column groups
     static constexpr int kSoft = 128 * CG;      // softmax threads
-    static constexpr int kThreads = 64 + kSoft; // + TMA warp + MMA warp
+    static constexpr int kVWarp = 2 + 4 * CG;   // the V producer follows the softmax warps
+    static constexpr int kThreads = 96 + kSoft; // + K/Q TMA warp + MMA warp + V TMA warp
 };
 
 template <int R, int STAGES>
@@ -231,8 +238,10 @@ attention_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_const
     // ---- set-up
     if (threadIdx.x == 0) {
         for (int s = 0; s < STAGES; ++s) {
-            mbar_init(&sh->kv_full[s], 1);
-            mbar_init(&sh->kv_empty[s], 1);
+            mbar_init(&sh->k_full[s], 1);
+            mbar_init(&sh->k_empty[s], 1);
+            mbar_init(&sh->v_full[s], 1);
+            mbar_init(&sh->v_empty[s], 1);
         }
         for (int i = 0; i < 2; ++i) {
             mbar_init(&sh->s_full[i], 1);
@@ -332,15 +341,24 @@ attention_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_const
         raise_flag(a.err_flag, ISD_FLAG_WAIT_TIMEOUT);
     };
 
-    if (warp == 0) {
+    if (warp == 0 || warp == TcRoles<R>::kVWarp) {
         if (active) {
-            // ------------------------------------------------ TMA producer
-            // The whole warp walks the tiles: page ids come in chunks of 32
-            // (lane i holds one), the next chunk's load in flight while the
-            // current one is issued, and the next piece's first chunk in
-            // flight during the current piece; lane 0 waits on the rings, and
-            // the copies of a tile are issued one box per lane (issuing them
-            // from a single thread caps the copy rate with small pages).
+            // ------------------------------------------------ TMA producers
+            // Warp 0 loads Q and the K halves of the stages, the last warp the
+            // V halves: each half has its own ring barriers, so a K half is
+            // refilled as soon as S = K.Q^T has read it and K runs ahead of V
+            // (the V half is held until P.V).  Each producer walks the tiles
+            // with the whole warp: page ids come in chunks of 32 (lane i holds
+            // one), the next chunk's load in flight while the current one is
+            // issued, and the next piece's first chunk in flight during the
+            // current piece; lane 0 waits on the ring, and the copies of a
+            // half are issued one box per lane (issuing them from a single
+            // thread caps the copy rate with small pages).
+            const bool is_v = warp != 0;
+            uint64_t* full = is_v ? sh->v_full : sh->k_full;
+            uint64_t* empty = is_v ? sh->v_empty : sh->k_empty;
+            unsigned char* ring = is_v ? sV : sK;
+            const CUtensorMap* map = is_v ? &tm_v : &tm_k;
             const uint64_t pol_kv = policy_evict_first();  // each K/V byte is read once
             const uint64_t pol_q = policy_evict_last();
             const int np = kTcKeys / a.P;  // pages per tile (<= 16)
@@ -369,20 +387,22 @@ attention_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_const
             while (ok && has) {
                 TcPiece nx;
                 const bool has_nx = piece_from(pc.us + pc.t1, nx);
-                const int qb = pi & 1;
-                if (lane == 0) {
-                    ok = mbar_wait_bounded(&sh->q_empty[qb], ((pi >> 1) & 1) ^ 1, abort_flag, kTcWaitNs);
-                    if (!ok) {
-                        give_up();
-                    } else {
-                        mbar_arrive_expect_tx(&sh->q_full[qb], (uint32_t)a.rows * 256u);
-                        unsigned char* qd = sQ + qb * kQBytes;
-                        tma_load_4d(qd, &tm_q, &sh->q_full[qb], 0, pc.g * a.grp, 0, pc.b, pol_q);
-                        tma_load_4d(qd + R * 128, &tm_q, &sh->q_full[qb], 64, pc.g * a.grp, 0, pc.b, pol_q);
+                if (!is_v) {
+                    const int qb = pi & 1;
+                    if (lane == 0) {
+                        ok = mbar_wait_bounded(&sh->q_empty[qb], ((pi >> 1) & 1) ^ 1, abort_flag, kTcWaitNs);
+                        if (!ok) {
+                            give_up();
+                        } else {
+                            mbar_arrive_expect_tx(&sh->q_full[qb], (uint32_t)a.rows * 256u);
+                            unsigned char* qd = sQ + qb * kQBytes;
+                            tma_load_4d(qd, &tm_q, &sh->q_full[qb], 0, pc.g * a.grp, 0, pc.b, pol_q);
+                            tma_load_4d(qd + R * 128, &tm_q, &sh->q_full[qb], 64, pc.g * a.grp, 0, pc.b, pol_q);
+                        }
                     }
+                    ok = __shfl_sync(0xffffffffu, ok, 0);
+                    if (!ok) break;
                 }
-                ok = __shfl_sync(0xffffffffu, ok, 0);
-                if (!ok) break;
                 ++pi;
                 int ids = ids_first, ids_next = load_ids(pc, pc.t0 + tpc);
                 const int ids_nx = has_nx ? load_ids(nx, nx.t0) : -1;
@@ -393,25 +413,22 @@ attention_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_const
                         ids_next = load_ids(pc, t + tpc);
                     }
                     if (lane == 0) {
-                        ok = mbar_wait_bounded(&sh->kv_empty[st], ph ^ 1, abort_flag, kTcWaitNs);
+                        ok = mbar_wait_bounded(&empty[st], ph ^ 1, abort_flag, kTcWaitNs);
                         if (!ok) give_up();
-                        else mbar_arrive_expect_tx(&sh->kv_full[st], 4u * kTcHalf);
+                        else mbar_arrive_expect_tx(&full[st], 2u * kTcHalf);
                     }
                     ok = __shfl_sync(0xffffffffu, ok, 0);
                     if (!ok) break;
-                    unsigned char* k_dst = sK + st * 2 * kTcHalf;
-                    unsigned char* v_dst = sV + st * 2 * kTcHalf;
-                    // one box per lane: page lane / 4 of the tile, K or V, 64-d
-                    // half (the expect_tx above precedes them in program order)
-                    for (int box0 = 0; box0 < 4 * np; box0 += 32) {
+                    unsigned char* dst = ring + st * 2 * kTcHalf;
+                    // one box per lane: page lane / 2 of the tile, 64-d half lane % 2
+                    // (the expect_tx above precedes them in program order)
+                    for (int box0 = 0; box0 < 2 * np; box0 += 32) {
                         const int box = box0 + lane;
-                        const int pg = box < 4 * np ? box >> 2 : 0, kind = box & 3;
+                        const int pg = box < 2 * np ? box >> 1 : 0, hf = box & 1;
                         const int page = __shfl_sync(0xffffffffu, ids, (j * np + pg) & 31);
-                        if (box < 4 * np) {
-                            const int off = pg * a.P * 128 + (kind & 1) * kTcHalf;
-                            tma_load_4d((kind & 2 ? v_dst : k_dst) + off, kind & 2 ? &tm_v : &tm_k,
-                                        &sh->kv_full[st], (kind & 1) * 64, pc.g, 0, page, pol_kv);
-                        }
+                        if (box < 2 * np)
+                            tma_load_4d(dst + pg * a.P * 128 + hf * kTcHalf, map, &full[st], hf * 64,
+                                        pc.g, 0, page, pol_kv);
                     }
                     armed |= 1u << st;
                     armed_par = (armed_par & ~(1u << st)) | (ph << st);
@@ -428,9 +445,10 @@ attention_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_const
             if (lane == 0) {
                 for (int s = 0; s < STAGES; ++s)
                     if (armed >> s & 1)
-                        mbar_wait_bounded(&sh->kv_full[s], armed_par >> s & 1, &sh->never, kTcWaitNs);
-                for (int k = pi - 1; k >= 0 && k >= pi - 2; --k)
-                    mbar_wait_bounded(&sh->q_full[k & 1], (k >> 1) & 1, &sh->never, kTcWaitNs);
+                        mbar_wait_bounded(&full[s], armed_par >> s & 1, &sh->never, kTcWaitNs);
+                if (!is_v)
+                    for (int k = pi - 1; k >= 0 && k >= pi - 2; --k)
+                        mbar_wait_bounded(&sh->q_full[k & 1], (k >> 1) & 1, &sh->never, kTcWaitNs);
             }
         }
     } else if (warp == 1) {
@@ -447,11 +465,13 @@ attention_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_const
                                 ((uint64_t)(kTcHalf >> 4) << 16);
             const uint32_t tm_o = tmem + 2 * R;
             // S products run ahead of the P.V products: S(t+1) is issued as
-            // soon as its K tile and S buffer are ready, PV(t) as soon as P(t)
-            // is, so a stage is released right after its PV completes
+            // soon as its K half and S buffer are ready, PV(t) as soon as P(t)
+            // and its V half are; the K half of a stage is released when its
+            // S product completes, the V half when its P.V product does
             int s_tc = 0, s_st = 0;    // S products issued; stage of the next one
             uint32_t s_ph = 0;
             int pv_tc = 0, pv_st = 0;  // PV products issued; stage of the next one
+            uint32_t pv_ph = 0;
             int pi = 0;                // pieces started
             uint32_t o_use = 0;
             uint64_t dq = dq0;
@@ -474,6 +494,7 @@ attention_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_const
                     mma_f16_ss(tmem + buf * R, ad, bd, idesc_s, kk != 0);
                 }
                 mma_commit(&sh->s_full[buf]);
+                mma_commit(&sh->k_empty[s_st]);  // the K half may be refilled once S is done
                 if (++s_st == STAGES) {
                     s_st = 0;
                     s_ph ^= 1;
@@ -481,11 +502,11 @@ attention_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_const
                 ++s_tc;
             };
             auto s_inputs_ready = [&]() {
-                return mbar_test(&sh->kv_full[s_st], s_ph) &&
+                return mbar_test(&sh->k_full[s_st], s_ph) &&
                        mbar_test(&sh->s_empty[s_tc & 1], ((s_tc >> 1) & 1) ^ 1);
             };
             auto issue_s_blocking = [&]() {
-                if (!wait(&sh->kv_full[s_st], s_ph)) return false;
+                if (!wait(&sh->k_full[s_st], s_ph)) return false;
                 if (!wait(&sh->s_empty[s_tc & 1], ((s_tc >> 1) & 1) ^ 1)) return false;
                 issue_s();
                 return true;
@@ -518,6 +539,7 @@ attention_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_const
                         q_done = true;
                     }
                     if (first_pv && !wait(&sh->o_empty, (o_use & 1) ^ 1)) break;
+                    if (!wait(&sh->v_full[pv_st], pv_ph)) break;
                     tc_fence_after();
                     const uint32_t v_off = (uint32_t)(pv_st * 2 * kTcHalf);
 #pragma unroll
@@ -526,10 +548,13 @@ attention_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_const
                         const uint64_t bd = dp + (((kk >> 2) * R * 128 + (kk & 3) * 32) >> 4);
                         mma_f16_ss(tm_o, ad, bd, idesc_o, (first_pv && kk == 0) ? 0u : 1u);
                     }
-                    mma_commit(&sh->kv_empty[pv_st]);
+                    mma_commit(&sh->v_empty[pv_st]);
                     mma_commit(&sh->p_empty);
                     first_pv = false;
-                    if (++pv_st == STAGES) pv_st = 0;
+                    if (++pv_st == STAGES) {
+                        pv_st = 0;
+                        pv_ph ^= 1;
+                    }
                     ++pv_tc;
                     // the softmax continues with S(pv_tc): issue it now if it is still missing
                     if (pv_tc < end_tc && s_tc == pv_tc && !issue_s_blocking()) break;
@@ -545,6 +570,7 @@ attention_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_const
         }
     } else if (active) {
         // ------------------------------------------------ softmax + epilogue
+        // (warps 2 .. kVWarp - 1)
         // thread = key kl of the tile (S^T lane) and rows r0 .. r0+RC-1;
         // in the epilogue thread = output dimension d = kl of O^T
         const int q4 = warp & 3;             // TMEM lane quarter of this warp
@@ -568,7 +594,7 @@ attention_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_const
         };
         float m_ref[RC], l_part[RC];
         int tc = 0, kst = 0;
-        uint32_t o_use = 0;
+        uint32_t kph = 0, o_use = 0;
         bool ok = true;
         TcPiece pc;
         bool has = piece_from(my0, pc);
@@ -609,9 +635,16 @@ attention_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_const
 #pragma unroll
                     for (int r = 0; r < RC; ++r)
                         if (key > lim[r0 + r]) s[r] = -INFINITY;
+                }
+                if (t * kTcKeys + kTcKeys > total) {
+                    // a V row past the request's keys may hold anything: zero it,
+                    // once the V half has landed, so that 0 * V stays 0 in the
+                    // second product (the fence before p_full orders it)
+                    if (!group_wait(&sh->v_full[kst], kph)) {
+                        ok = false;
+                        break;
+                    }
                     if (key >= total && cg == 0) {
-                        // a V row past the request's keys may hold anything:
-                        // zero it so that 0 * V stays 0 in the second product
                         uint4* vr = reinterpret_cast<uint4*>(sV + kst * 2 * kTcHalf + kl * 128);
 #pragma unroll
                         for (int j = 0; j < 8; ++j) {
@@ -690,7 +723,10 @@ attention_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_const
                 __syncwarp();
                 if (lane == 0) mbar_arrive(&sh->p_full);
                 ++tc;
-                if (++kst == STAGES) kst = 0;
+                if (++kst == STAGES) {
+                    kst = 0;
+                    kph ^= 1;
+                }
             }
             if (!ok) break;
 
