@@ -18,6 +18,7 @@
 #include "common.cuh"
 #include "launch.h"
 #include "plan.h"
+#include "sm100.cuh"
 
 namespace isd {
 
@@ -86,8 +87,9 @@ struct AcceptArgs {
     int32_t* next_kv_len;
     float* ratio;
     float* part;     // [B][N+1][n_chunks] chunk totals
-    int* ticket;     // [B]
+    int* ticket;     // [B] tickets, then [B] decision flags, then [B] decided states
     int n_chunks;
+    bool vec;        // logits rows 16-byte aligned (V % 4 == 0, aligned bases)
     int32_t* err_flag;
     // inside a whole step: this step's row statistics come as the LM head's
     // partials ([B*Q][n_parts]); the kernel merges the rows it needs and the
@@ -121,16 +123,53 @@ ISD_DEVINL float expm1_pos(float d) {
     return __expf(d) - 1.f;
 }
 
-ISD_DEVINL float sweep_weight(const SweepRow& r, int i) {
-    const float zp = __ldg(r.zp + i);
+ISD_DEVINL float weight_of(const SweepRow& r, float zp, float zq) {
     if (!r.zq) return __expf(zp - r.mp);
-    const float zq = __ldg(r.zq + i);
     const float d = (zp - zq) + r.k;
     if (!(d > 0.f)) return 0.f;
     return __expf(zq - r.mq) * r.inv_sq * expm1_pos(d);
 }
 
 constexpr int kSeg = kAcceptChunk / kAcceptThreads;  // contiguous entries per thread
+static_assert(kSeg % 4 == 0, "a thread's segment is whole float4s");
+
+// Weights of entries s0 .. s0+kSeg-1 (zero at and past end).  With vec (rows
+// 16-byte aligned) a full segment is read as float4s, every load of the
+// segment issued before the first is used.
+ISD_DEVINL void seg_weights(const SweepRow& r, int s0, int end, bool vec, float (&w)[kSeg]) {
+    float zp[kSeg], zq[kSeg];
+    if (vec && s0 + kSeg <= end) {
+#pragma unroll
+        for (int v = 0; v < kSeg / 4; ++v) {
+            const float4 t = __ldg(reinterpret_cast<const float4*>(r.zp + s0) + v);
+            zp[4 * v] = t.x;
+            zp[4 * v + 1] = t.y;
+            zp[4 * v + 2] = t.z;
+            zp[4 * v + 3] = t.w;
+        }
+        if (r.zq) {
+#pragma unroll
+            for (int v = 0; v < kSeg / 4; ++v) {
+                const float4 t = __ldg(reinterpret_cast<const float4*>(r.zq + s0) + v);
+                zq[4 * v] = t.x;
+                zq[4 * v + 1] = t.y;
+                zq[4 * v + 2] = t.z;
+                zq[4 * v + 3] = t.w;
+            }
+        }
+#pragma unroll
+        for (int k = 0; k < kSeg; ++k) w[k] = weight_of(r, zp[k], r.zq ? zq[k] : 0.f);
+        return;
+    }
+#pragma unroll
+    for (int k = 0; k < kSeg; ++k) {
+        const int i = s0 + k;
+        zp[k] = i < end ? __ldg(r.zp + i) : 0.f;
+        zq[k] = (i < end && r.zq) ? __ldg(r.zq + i) : 0.f;
+    }
+#pragma unroll
+    for (int k = 0; k < kSeg; ++k) w[k] = s0 + k < end ? weight_of(r, zp[k], zq[k]) : 0.f;
+}
 
 // Exclusive block scan of one float per thread (fixed order); returns the
 // exclusive prefix and writes the block total to *total.
@@ -159,16 +198,14 @@ ISD_DEVINL float block_exclusive_scan(float v, float* total) {
 // Chunk [beg, end): per-thread contiguous segments; returns the chunk total
 // (identical bits every time it is recomputed) and, if target >= 0, the first
 // index whose prefix exceeds target (or -1).
-ISD_DEVINL float chunk_scan(const SweepRow& r, int beg, int end, float target, int* found) {
+ISD_DEVINL float chunk_scan(const SweepRow& r, int beg, int end, bool vec, float target,
+                            int* found) {
     float w[kSeg];
-    float local = 0.f;
     const int s0 = beg + threadIdx.x * kSeg;
+    seg_weights(r, s0, end, vec, w);
+    float local = 0.f;
 #pragma unroll
-    for (int k = 0; k < kSeg; ++k) {
-        const int i = s0 + k;
-        w[k] = (i < end) ? sweep_weight(r, i) : 0.f;
-        local += w[k];
-    }
+    for (int k = 0; k < kSeg; ++k) local += w[k];
     float total;
     const float excl = block_exclusive_scan(local, &total);
     if (target >= 0.f) {
@@ -208,11 +245,19 @@ ISD_DEVINL float chunk_scan(const SweepRow& r, int beg, int end, float target, i
     return total;
 }
 
-__global__ void __launch_bounds__(kAcceptThreads, 8) accept_kernel(AcceptArgs a) {
+// Grid (request, chunk), requests fastest, so the chunk-0 CTAs of all requests
+// are dispatched first.  The chunk-0 CTA of request b decides it (merging
+// all of its rows, written to stats_out in fused mode) and publishes the
+// decision with a release flag; the other CTAs of b take it from there
+// rather than repeating the merges, and leave at once when b draws nothing.
+// A CTA that does not see the flag within kAcceptFlagWaitNs decides b itself
+// (the same arithmetic, so the same decision).
+__global__ void __launch_bounds__(kAcceptThreads, kAcceptMinBlocks)
+accept_kernel(const __grid_constant__ AcceptArgs a) {
     pdl_trigger();
     pdl_wait();
-    const int b = blockIdx.y;
-    const int ch = blockIdx.x;
+    const int b = blockIdx.x;
+    const int ch = blockIdx.y;
     const int N = a.N, Q = 2 * N - 1, V = a.V;
     const int rcols = N > 1 ? N - 1 : 1;
     __shared__ int s_state;  // -1 invalid request, 0 no rejection, j = rejected proposal index
@@ -223,15 +268,36 @@ __global__ void __launch_bounds__(kAcceptThreads, 8) accept_kernel(AcceptArgs a)
     const int c_in = __ldg(&a.n_clean[b]);
     const bool bad_c = (c_in < 1 || c_in > N);
     const bool fused = a.stats_part != nullptr;
-    if (threadIdx.x == 0) s_bad = 0;
+    int* flag = a.ticket + a.B;
+    int* req_state = a.ticket + 2 * a.B;
+    constexpr int kNone = -0x7fffffff;
+    __shared__ int s_pub;  // the decider's published state, or kNone
+    if (threadIdx.x == 0) {
+        s_bad = 0;
+        int st = kNone;
+        if (ch != 0) {
+            const uint64_t t0 = sm100::global_ns();
+            for (uint32_t it = 0;; ++it) {
+                int v;
+                asm volatile("ld.acquire.gpu.global.b32 %0, [%1];\n" : "=r"(v) : "l"(flag + b) : "memory");
+                if (v) {
+                    st = __ldcg(req_state + b);
+                    break;
+                }
+                if ((it & 15) == 15 && sm100::global_ns() - t0 > kAcceptFlagWaitNs) break;
+            }
+        }
+        s_pub = st;
+    }
     __syncthreads();
+    const bool published = s_pub != kNone;
     // the gathered p/q operands of every tested proposal (one round of loads,
     // in flight while the row statistics are merged)
     const int jt = (int)threadIdx.x + 2;
     float zp = 0.f, zq = 0.f;
     isd_row_stat sq = isd_row_stat{0.f, 1.f, 0, 0};
     bool have = false;
-    if (!bad_c && jt <= c_in) {
+    if (!published && !bad_c && jt <= c_in) {
         const int x = __ldg(&a.clean_tok[(size_t)b * N + jt - 1]);
         if (x < 0 || x >= V) {
             s_bad = 1;
@@ -244,10 +310,10 @@ __global__ void __launch_bounds__(kAcceptThreads, 8) accept_kernel(AcceptArgs a)
             have = true;
         }
     }
-    if (fused) {
+    if (fused && !published) {
         // one warp per row: chunk 0 merges every row of the request (it writes
-        // them out); the other chunks the rows they read (tested proposals,
-        // and in sample mode the proposal rows they sweep)
+        // them out); a CTA deciding for itself the rows it reads (tested
+        // proposals, and in sample mode the proposal rows it sweeps)
         const int wid = (int)threadIdx.x >> 5;
         for (int k = wid; k < Q; k += kAcceptThreads / 32) {
             const bool need = ch == 0 || k < c_in - 1 ||
@@ -256,14 +322,23 @@ __global__ void __launch_bounds__(kAcceptThreads, 8) accept_kernel(AcceptArgs a)
             const RowStat st = warp_merge_partials(a.stats_part + ((size_t)b * Q + k) * a.n_parts, a.n_parts);
             if ((threadIdx.x & 31) == 0) {
                 s_stats[k] = isd_row_stat{st.m, st.s, st.idx, 0};
-                if (ch == 0) a.stats_out[(size_t)b * Q + k] = s_stats[k];
+                if (ch == 0) {
+                    a.stats_out[(size_t)b * Q + k] = s_stats[k];
+                    __threadfence();  // before the decision is published
+                }
             }
         }
     }
     __syncthreads();
-    // row statistics of row k of this request (this step's logits)
+    // row statistics of row k of this request (this step's logits): merged
+    // here, merged by the decider (stats_out, read from L2), or given
     auto stat_of = [&](int k) -> isd_row_stat {
-        return fused ? s_stats[k] : a.stats[(size_t)b * Q + k];
+        if (!fused) return a.stats[(size_t)b * Q + k];
+        if (published) {
+            const float4 v = __ldcg(reinterpret_cast<const float4*>(a.stats_out + (size_t)b * Q + k));
+            return isd_row_stat{v.x, v.y, __float_as_int(v.z), __float_as_int(v.w)};
+        }
+        return s_stats[k];
     };
     // p(x)/q(x) = exp((zp - mp) - (zq - mq)) * Sq / Sp
     if (have) {
@@ -271,7 +346,7 @@ __global__ void __launch_bounds__(kAcceptThreads, 8) accept_kernel(AcceptArgs a)
         s_ratio[jt - 2] = expf((zp - sp.max) - (zq - sq.max)) * (sq.sumexp / sp.sumexp);
     }
     __syncthreads();
-    if (threadIdx.x == 0) {
+    if (threadIdx.x == 0 && !published) {
         int state = 0;
         if (bad_c) {
             raise_flag(a.err_flag, ISD_FLAG_NCLEAN_RANGE);
@@ -292,8 +367,14 @@ __global__ void __launch_bounds__(kAcceptThreads, 8) accept_kernel(AcceptArgs a)
             for (int k = 0; k < rcols; ++k)
                 a.ratio[(size_t)b * rcols + k] = k < tested ? s_ratio[k] : -1.f;
         }
+        if (ch == 0) {  // publish the decision
+            req_state[b] = state;
+            __threadfence();
+            asm volatile("st.release.gpu.global.b32 [%0], %1;\n" ::"l"(flag + b), "r"(1) : "memory");
+        }
         s_state = state;
     }
+    if (threadIdx.x == 0 && published) s_state = s_pub;
     __syncthreads();
     const int state = s_state, c = c_in;
     const int* tok = a.clean_tok + (size_t)b * N;
@@ -327,7 +408,7 @@ __global__ void __launch_bounds__(kAcceptThreads, 8) accept_kernel(AcceptArgs a)
             *r = SweepRow{a.logits + rr * V, nullptr, s.max, 0.f, 0.f, 0.f};
         }
     };
-    int picked[16];  // N <= 16 (checked on the host)
+    __shared__ int picked[16];  // N <= 16 (checked on the host); written by thread 0
     if (sweep) {
         const int beg = ch * kAcceptChunk, end = min(V, beg + kAcceptChunk);
         float* part = a.part + (size_t)b * (N + 1) * a.n_chunks;
@@ -335,7 +416,7 @@ __global__ void __launch_bounds__(kAcceptThreads, 8) accept_kernel(AcceptArgs a)
             SweepRow r;
             row_of(k, &r);
             int dummy;
-            const float tot = chunk_scan(r, beg, end, -1.f, &dummy);
+            const float tot = chunk_scan(r, beg, end, a.vec, -1.f, &dummy);
             if (threadIdx.x == 0) part[(size_t)k * a.n_chunks + ch] = tot;
         }
         __threadfence();
@@ -387,7 +468,7 @@ __global__ void __launch_bounds__(kAcceptThreads, 8) accept_kernel(AcceptArgs a)
                 y = stat_of(state > 0 ? state - 2 : (k == 0 ? c - 1 : N + k - 1)).argmax;
             } else {
                 const int beg2 = q * kAcceptChunk, end2 = min(V, beg2 + kAcceptChunk);
-                chunk_scan(r, beg2, end2, tgt, &y);
+                chunk_scan(r, beg2, end2, a.vec, tgt, &y);
             }
             if (threadIdx.x == 0) picked[k] = y;
         }
@@ -472,8 +553,10 @@ cudaError_t launch_accept(const Plan& p, const isd_dims* d, const float* logits,
     a.part = reinterpret_cast<float*>(w + p.off_acc_part);
     a.ticket = reinterpret_cast<int*>(w + p.off_acc_ticket);
     a.n_chunks = p.acc_chunks;
+    a.vec = d->V % 4 == 0 && reinterpret_cast<uintptr_t>(logits) % 16 == 0 &&
+            reinterpret_cast<uintptr_t>(prev_logits) % 16 == 0;
     a.err_flag = err_flag;
-    dim3 grid(p.acc_chunks, d->B);
+    dim3 grid(d->B, p.acc_chunks);
     return launch_kernel(pdl, accept_kernel, grid, dim3(kAcceptThreads), 0, st, a);
 }
 

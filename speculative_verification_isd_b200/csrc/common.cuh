@@ -139,19 +139,21 @@ ISD_DEVINL RowStat rowstat_block_reduce(RowStat a) {
 // broadcast.  Every caller (the LM head's merge kernel, the accept kernel)
 // uses this one routine, so the merged statistics are bit-identical.
 constexpr int kMaxPartsPerLane = kMaxStatParts / 32;
+template <int BATCH = 4>
 ISD_DEVINL RowStat warp_merge_partials(const float4* p, int n) {
     const int lane = threadIdx.x & 31;
     RowStat st = rowstat_empty();
-    // batches of 4 loads per lane keep the register need small
-    for (int u0 = 0; u0 < kMaxPartsPerLane && 32 * u0 < n; u0 += 4) {
-        float4 v[4];
+    // loads in batches of BATCH per lane (more in flight, more registers);
+    // the order of the merge does not depend on BATCH
+    for (int u0 = 0; u0 < kMaxPartsPerLane && 32 * u0 < n; u0 += BATCH) {
+        float4 v[BATCH];
 #pragma unroll
-        for (int u = 0; u < 4; ++u) {
+        for (int u = 0; u < BATCH; ++u) {
             const int k = lane + 32 * (u0 + u);
             v[u] = k < n ? __ldcg(p + k) : make_float4(-INFINITY, 0.f, 0.f, 0.f);
         }
 #pragma unroll
-        for (int u = 0; u < 4; ++u) st = rowstat_merge(st, RowStat{v[u].x, v[u].y, __float_as_int(v[u].z)});
+        for (int u = 0; u < BATCH; ++u) st = rowstat_merge(st, RowStat{v[u].x, v[u].y, __float_as_int(v[u].z)});
     }
 #pragma unroll
     for (int off = 16; off > 0; off >>= 1) st = rowstat_merge(st, rowstat_shfl_xor(st, off));

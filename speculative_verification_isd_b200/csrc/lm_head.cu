@@ -206,7 +206,7 @@ ISD_DEVINL RowStat column_stats(const uint32_t (&x)[32], int v, bool ok) {
 template <int NB>
 __global__ void __launch_bounds__(kLmThreads, 1)
 lm_head_kernel(const __grid_constant__ CUtensorMap tmap_w, const __grid_constant__ CUtensorMap tmap_h,
-               LmArgs a) {
+               const __grid_constant__ LmArgs a) {
     using namespace sm100;
     extern __shared__ unsigned char smem_raw[];
     unsigned char* smem = reinterpret_cast<unsigned char*>(

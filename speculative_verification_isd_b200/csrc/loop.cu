@@ -50,7 +50,7 @@ constexpr int kPrepThreads = 256;
 // grid (Q, B): block slot s of request b copies its table rows (16 bytes per
 // thread); CTA (0, 0) also extends every request's page list, in request
 // order, from the bump allocator.
-__global__ void __launch_bounds__(kPrepThreads) prepare_block_kernel(PrepArgs a) {
+__global__ void __launch_bounds__(kPrepThreads) prepare_block_kernel(const __grid_constant__ PrepArgs a) {
     pdl_trigger();
     pdl_wait();  // the state was written by the previous step's accept
     const int s = blockIdx.x, b = blockIdx.y;

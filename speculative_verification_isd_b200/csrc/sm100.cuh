@@ -97,6 +97,18 @@ ISD_DEVINL void tmem_alloc(uint32_t* holder_smem, uint32_t ncols) {
                  "r"(ncols)
                  : "memory");
 }
+// Register reallocation between warpgroups: every thread of a warpgroup
+// executes the same one.  The increases must fit in what the decreases free
+// from the block's launch allocation (threads x registers per thread).
+template <uint32_t N>
+ISD_DEVINL void setmaxnreg_inc() {
+    asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;\n" ::"n"(N));
+}
+template <uint32_t N>
+ISD_DEVINL void setmaxnreg_dec() {
+    asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;\n" ::"n"(N));
+}
+
 ISD_DEVINL void tmem_relinquish() {
     asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;\n" ::: "memory");
 }
