@@ -87,7 +87,7 @@ struct AcceptArgs {
     int32_t* next_kv_len;
     float* ratio;
     float* part;     // [B][N+1][n_chunks] chunk totals
-    int* ticket;     // [B] tickets, then [B] decision flags, then [B] decided states
+    int* ticket;     // [B] tickets, then [B] decided states, then the decided count
     int n_chunks;
     bool vec;        // logits rows 16-byte aligned (V % 4 == 0, aligned bases)
     int32_t* err_flag;
@@ -245,243 +245,12 @@ ISD_DEVINL float chunk_scan(const SweepRow& r, int beg, int end, bool vec, float
     return total;
 }
 
-// Grid (request, chunk), requests fastest, so the chunk-0 CTAs of all requests
-// are dispatched first.  The chunk-0 CTA of request b decides it (merging
-// all of its rows, written to stats_out in fused mode) and publishes the
-// decision with a release flag; the other CTAs of b take it from there
-// rather than repeating the merges, and leave at once when b draws nothing.
-// A CTA that does not see the flag within kAcceptFlagWaitNs decides b itself
-// (the same arithmetic, so the same decision).
-__global__ void __launch_bounds__(kAcceptThreads, kAcceptMinBlocks)
-accept_kernel(const __grid_constant__ AcceptArgs a) {
-    pdl_trigger();
-    pdl_wait();
-    const int b = blockIdx.x;
-    const int ch = blockIdx.y;
-    const int N = a.N, Q = 2 * N - 1, V = a.V;
-    const int rcols = N > 1 ? N - 1 : 1;
-    __shared__ int s_state;  // -1 invalid request, 0 no rejection, j = rejected proposal index
-    __shared__ int s_last, s_bad;
-    __shared__ float s_ratio[16];
-    __shared__ isd_row_stat s_stats[32];  // this request's merged rows (Q <= 31)
-    const float* ub = a.uniforms + (size_t)b * 2 * N;
-    const int c_in = __ldg(&a.n_clean[b]);
-    const bool bad_c = (c_in < 1 || c_in > N);
-    const bool fused = a.stats_part != nullptr;
-    int* flag = a.ticket + a.B;
-    int* req_state = a.ticket + 2 * a.B;
-    constexpr int kNone = -0x7fffffff;
-    __shared__ int s_pub;  // the decider's published state, or kNone
-    if (threadIdx.x == 0) {
-        s_bad = 0;
-        int st = kNone;
-        if (ch != 0) {
-            const uint64_t t0 = sm100::global_ns();
-            for (uint32_t it = 0;; ++it) {
-                int v;
-                asm volatile("ld.acquire.gpu.global.b32 %0, [%1];\n" : "=r"(v) : "l"(flag + b) : "memory");
-                if (v) {
-                    st = __ldcg(req_state + b);
-                    break;
-                }
-                if ((it & 15) == 15 && sm100::global_ns() - t0 > kAcceptFlagWaitNs) break;
-            }
-        }
-        s_pub = st;
-    }
-    __syncthreads();
-    const bool published = s_pub != kNone;
-    // the gathered p/q operands of every tested proposal (one round of loads,
-    // in flight while the row statistics are merged)
-    const int jt = (int)threadIdx.x + 2;
-    float zp = 0.f, zq = 0.f;
-    isd_row_stat sq = isd_row_stat{0.f, 1.f, 0, 0};
-    bool have = false;
-    if (!published && !bad_c && jt <= c_in) {
-        const int x = __ldg(&a.clean_tok[(size_t)b * N + jt - 1]);
-        if (x < 0 || x >= V) {
-            s_bad = 1;
-        } else {
-            const size_t rp = (size_t)b * Q + (jt - 2);
-            const size_t rq = (size_t)b * Q + (N + jt - 2);
-            zp = a.logits[rp * V + x];
-            zq = a.prev_logits[rq * V + x];
-            sq = a.prev_stats[rq];
-            have = true;
-        }
-    }
-    if (fused && !published) {
-        // one warp per row: chunk 0 merges every row of the request (it writes
-        // them out); a CTA deciding for itself the rows it reads (tested
-        // proposals, and in sample mode the proposal rows it sweeps)
-        const int wid = (int)threadIdx.x >> 5;
-        for (int k = wid; k < Q; k += kAcceptThreads / 32) {
-            const bool need = ch == 0 || k < c_in - 1 ||
-                              (a.mode == ISD_PROPOSE_SAMPLE && (k == c_in - 1 || k >= N));
-            if (!need) continue;
-            const RowStat st = warp_merge_partials(a.stats_part + ((size_t)b * Q + k) * a.n_parts, a.n_parts);
-            if ((threadIdx.x & 31) == 0) {
-                s_stats[k] = isd_row_stat{st.m, st.s, st.idx, 0};
-                if (ch == 0) {
-                    a.stats_out[(size_t)b * Q + k] = s_stats[k];
-                    __threadfence();  // before the decision is published
-                }
-            }
-        }
-    }
-    __syncthreads();
-    // row statistics of row k of this request (this step's logits): merged
-    // here, merged by the decider (stats_out, read from L2), or given
-    auto stat_of = [&](int k) -> isd_row_stat {
-        if (!fused) return a.stats[(size_t)b * Q + k];
-        if (published) {
-            const float4 v = __ldcg(reinterpret_cast<const float4*>(a.stats_out + (size_t)b * Q + k));
-            return isd_row_stat{v.x, v.y, __float_as_int(v.z), __float_as_int(v.w)};
-        }
-        return s_stats[k];
-    };
-    // p(x)/q(x) = exp((zp - mp) - (zq - mq)) * Sq / Sp
-    if (have) {
-        const isd_row_stat sp = stat_of(jt - 2);
-        s_ratio[jt - 2] = expf((zp - sp.max) - (zq - sq.max)) * (sq.sumexp / sp.sumexp);
-    }
-    __syncthreads();
-    if (threadIdx.x == 0 && !published) {
-        int state = 0;
-        if (bad_c) {
-            raise_flag(a.err_flag, ISD_FLAG_NCLEAN_RANGE);
-            state = -1;
-        } else if (s_bad) {
-            raise_flag(a.err_flag, ISD_FLAG_TOKEN_OOB);
-            state = -1;
-        } else {
-            // the first rejection stops the pass
-            for (int j = 2; j <= c_in; ++j)
-                if (!(ub[j - 2] < s_ratio[j - 2])) {
-                    state = j;
-                    break;
-                }
-        }
-        if (ch == 0 && a.ratio && state >= 0) {
-            const int tested = state > 0 ? state - 1 : c_in - 1;
-            for (int k = 0; k < rcols; ++k)
-                a.ratio[(size_t)b * rcols + k] = k < tested ? s_ratio[k] : -1.f;
-        }
-        if (ch == 0) {  // publish the decision
-            req_state[b] = state;
-            __threadfence();
-            asm volatile("st.release.gpu.global.b32 [%0], %1;\n" ::"l"(flag + b), "r"(1) : "memory");
-        }
-        s_state = state;
-    }
-    if (threadIdx.x == 0 && published) s_state = s_pub;
-    __syncthreads();
-    const int state = s_state, c = c_in;
+// Emitted tokens and next state of request b (thread 0): state > 0 is the
+// rejected proposal index j (the first j - 2 proposals kept, then the draw
+// picked[0]); state 0 keeps all c clean tokens and proposes picked[0..N-1].
+ISD_DEVINL void emit_request(const AcceptArgs& a, int b, int state, int c, const int* picked) {
+    const int N = a.N;
     const int* tok = a.clean_tok + (size_t)b * N;
-    if (state < 0) {  // invalid request: emit nothing, carry the state over
-        if (ch == 0 && threadIdx.x == 0) {
-            a.accept_len[b] = 0;
-            a.next_n_clean[b] = c;
-            a.next_kv_len[b] = a.kv_len[b];
-            for (int k = 0; k < N; ++k) {
-                a.out_tok[(size_t)b * N + k] = -1;
-                a.next_clean_tok[(size_t)b * N + k] = tok[k];
-            }
-            if (a.ratio)
-                for (int k = 0; k < rcols; ++k) a.ratio[(size_t)b * rcols + k] = -1.f;
-        }
-        return;
-    }
-    const bool sweep = state > 0 || a.mode == ISD_PROPOSE_SAMPLE;
-    const int nrows = state > 0 ? 1 : N;
-    // Describe the rows to sweep (or the argmax rows).
-    auto row_of = [&](int k, SweepRow* r) {
-        if (state > 0) {
-            const size_t rp = (size_t)b * Q + (state - 2);
-            const size_t rq = (size_t)b * Q + (N + state - 2);
-            const isd_row_stat sp = stat_of(state - 2), sq = a.prev_stats[rq];
-            *r = SweepRow{a.logits + rp * V, a.prev_logits + rq * V, sp.max, sq.max,
-                          1.f / sq.sumexp, (sq.max - sp.max) + logf(sq.sumexp / sp.sumexp)};
-        } else {
-            const size_t rr = (size_t)b * Q + (k == 0 ? c - 1 : N + k - 1);
-            const isd_row_stat s = stat_of(k == 0 ? c - 1 : N + k - 1);
-            *r = SweepRow{a.logits + rr * V, nullptr, s.max, 0.f, 0.f, 0.f};
-        }
-    };
-    __shared__ int picked[16];  // N <= 16 (checked on the host); written by thread 0
-    if (sweep) {
-        const int beg = ch * kAcceptChunk, end = min(V, beg + kAcceptChunk);
-        float* part = a.part + (size_t)b * (N + 1) * a.n_chunks;
-        for (int k = 0; k < nrows; ++k) {
-            SweepRow r;
-            row_of(k, &r);
-            int dummy;
-            const float tot = chunk_scan(r, beg, end, a.vec, -1.f, &dummy);
-            if (threadIdx.x == 0) part[(size_t)k * a.n_chunks + ch] = tot;
-        }
-        __threadfence();
-        __syncthreads();
-        if (threadIdx.x == 0) s_last = (atomicAdd(&a.ticket[b], 1) == a.n_chunks - 1);
-        __syncthreads();
-        if (!s_last) return;
-        __threadfence();
-        for (int k = 0; k < nrows; ++k) {
-            SweepRow r;
-            row_of(k, &r);
-            const float u = state > 0 ? ub[N - 1] : ub[N + k];
-            // chunk totals in chunk order, scanned by the whole block
-            __shared__ float s_target;
-            __shared__ int s_chunk, s_hit, s_lastpos;
-            const float tv = (int)threadIdx.x < a.n_chunks
-                                 ? __ldcg(&part[(size_t)k * a.n_chunks + threadIdx.x]) : 0.f;
-            float total;
-            const float excl = block_exclusive_scan(tv, &total);
-            const float target = u * total;
-            if (threadIdx.x == 0) {
-                s_hit = 0x7fffffff;
-                s_lastpos = -1;
-            }
-            __syncthreads();
-            if (tv > 0.f) atomicMax(&s_lastpos, (int)threadIdx.x);
-            if ((int)threadIdx.x < a.n_chunks && excl + tv > target) atomicMin(&s_hit, (int)threadIdx.x);
-            __syncthreads();
-            if (threadIdx.x == 0) {
-                if (!(total > 0.f)) {
-                    s_chunk = -2;  // no mass: residual falls back to argmax p
-                    s_target = 0.f;
-                } else if (s_hit == 0x7fffffff) {
-                    s_chunk = s_lastpos;
-                    s_target = 3.0e38f;  // take the last positive entry of that chunk
-                } else {
-                    s_chunk = s_hit;
-                }
-            }
-            __syncthreads();
-            if (s_chunk >= 0 && s_chunk == s_hit && (int)threadIdx.x == s_hit)
-                s_target = fmaxf(target - excl, 0.f);
-            __syncthreads();
-            const int q = s_chunk;
-            const float tgt = s_target;
-            __syncthreads();
-            int y;
-            if (q == -2) {  // argmax of the anchor (or proposal) row
-                y = stat_of(state > 0 ? state - 2 : (k == 0 ? c - 1 : N + k - 1)).argmax;
-            } else {
-                const int beg2 = q * kAcceptChunk, end2 = min(V, beg2 + kAcceptChunk);
-                chunk_scan(r, beg2, end2, a.vec, tgt, &y);
-            }
-            if (threadIdx.x == 0) picked[k] = y;
-        }
-        if (threadIdx.x == 0) a.ticket[b] = 0;
-    } else {
-        if (ch != 0) return;
-        if (threadIdx.x == 0) {
-            picked[0] = stat_of(c - 1).argmax;
-            for (int m = 0; m + 1 < N; ++m) picked[m + 1] = stat_of(N + m).argmax;
-        }
-    }
-    if (threadIdx.x != 0) return;
-    // a9: emitted tokens and next state
     int32_t* ot = a.out_tok + (size_t)b * N;
     int32_t* nt = a.next_clean_tok + (size_t)b * N;
     int A;
@@ -503,6 +272,264 @@ accept_kernel(const __grid_constant__ AcceptArgs a) {
     }
     a.accept_len[b] = A;
     a.next_kv_len[b] = a.kv_len[b] + A;
+}
+
+// One CTA per (sweep item) slot, B x n_chunks in all.  CTAs 0 .. B-1 decide
+// the requests (merging every row of theirs, written to stats_out in fused
+// mode), write the ratios and, when a request draws nothing, its outputs;
+// then each counts itself in `decided`.  Every CTA waits (bounded) until all
+// B are decided and takes the item of its index among the chunks of the
+// requests that draw (a rejection's residual, or sample-mode proposals), in
+// request order; the CTAs past them leave at once.  The CTA holding a
+// request's last ticket scans its chunk totals in chunk order and draws.
+// Decisions and draws do not depend on which CTA computes them, so a
+// repeated call is bit-identical.
+__global__ void __launch_bounds__(kAcceptThreads, kAcceptMinBlocks)
+accept_kernel(const __grid_constant__ AcceptArgs a) {
+    pdl_trigger();
+    pdl_wait();
+    const int cta = blockIdx.x;
+    const int N = a.N, Q = 2 * N - 1, V = a.V;
+    const int rcols = N > 1 ? N - 1 : 1;
+    const bool fused = a.stats_part != nullptr;
+    int* req_state = a.ticket + a.B;
+    int* decided = a.ticket + 2 * a.B;
+    __shared__ int s_state, s_last, s_bad, s_b, s_ok;
+    __shared__ float s_ratio[16];
+    __shared__ isd_row_stat s_stats[32];  // the decided request's merged rows (Q <= 31)
+    __shared__ int picked[16];            // N <= 16 (checked on the host); written by thread 0
+    // this step's statistics of row k of request b outside the decision:
+    // merged by the decider (stats_out, read from L2), or given
+    auto stat_of = [&](int b, int k) -> isd_row_stat {
+        if (!fused) return a.stats[(size_t)b * Q + k];
+        const float4 v = __ldcg(reinterpret_cast<const float4*>(a.stats_out + (size_t)b * Q + k));
+        return isd_row_stat{v.x, v.y, __float_as_int(v.z), __float_as_int(v.w)};
+    };
+
+    // ------------------------------------------------------------ decisions
+    if (cta < a.B) {
+        const int b = cta;
+        const float* ub = a.uniforms + (size_t)b * 2 * N;
+        const int c_in = __ldg(&a.n_clean[b]);
+        const bool bad_c = (c_in < 1 || c_in > N);
+        if (threadIdx.x == 0) s_bad = 0;
+        __syncthreads();
+        // the gathered p/q operands of every tested proposal (one round of
+        // loads, in flight while the row statistics are merged)
+        const int jt = (int)threadIdx.x + 2;
+        float zp = 0.f, zq = 0.f;
+        isd_row_stat sq = isd_row_stat{0.f, 1.f, 0, 0};
+        bool have = false;
+        if (!bad_c && jt <= c_in) {
+            const int x = __ldg(&a.clean_tok[(size_t)b * N + jt - 1]);
+            if (x < 0 || x >= V) {
+                s_bad = 1;
+            } else {
+                const size_t rp = (size_t)b * Q + (jt - 2);
+                const size_t rq = (size_t)b * Q + (N + jt - 2);
+                zp = a.logits[rp * V + x];
+                zq = a.prev_logits[rq * V + x];
+                sq = a.prev_stats[rq];
+                have = true;
+            }
+        }
+        // every row of the request: merged here (one warp per row) and
+        // written out, or given
+        const int wid = (int)threadIdx.x >> 5;
+        for (int k = wid; k < Q; k += kAcceptThreads / 32) {
+            isd_row_stat v;
+            if (fused) {
+                const RowStat st = warp_merge_partials<8>(a.stats_part + ((size_t)b * Q + k) * a.n_parts, a.n_parts);
+                v = isd_row_stat{st.m, st.s, st.idx, 0};
+                if ((threadIdx.x & 31) == 0) {
+                    a.stats_out[(size_t)b * Q + k] = v;
+                    __threadfence();  // before the decision is counted
+                }
+            } else {
+                v = a.stats[(size_t)b * Q + k];
+            }
+            if ((threadIdx.x & 31) == 0) s_stats[k] = v;
+        }
+        __syncthreads();
+        // p(x)/q(x) = exp((zp - mp) - (zq - mq)) * Sq / Sp
+        if (have) {
+            const isd_row_stat sp = s_stats[jt - 2];
+            s_ratio[jt - 2] = expf((zp - sp.max) - (zq - sq.max)) * (sq.sumexp / sp.sumexp);
+        }
+        __syncthreads();
+        if (threadIdx.x == 0) {
+            int state = 0;
+            if (bad_c) {
+                raise_flag(a.err_flag, ISD_FLAG_NCLEAN_RANGE);
+                state = -1;
+            } else if (s_bad) {
+                raise_flag(a.err_flag, ISD_FLAG_TOKEN_OOB);
+                state = -1;
+            } else {
+                // the first rejection stops the pass
+                for (int j = 2; j <= c_in; ++j)
+                    if (!(ub[j - 2] < s_ratio[j - 2])) {
+                        state = j;
+                        break;
+                    }
+            }
+            if (a.ratio) {
+                const int tested = state > 0 ? state - 1 : (state == 0 ? c_in - 1 : 0);
+                for (int k = 0; k < rcols; ++k)
+                    a.ratio[(size_t)b * rcols + k] = k < tested ? s_ratio[k] : -1.f;
+            }
+            if (state < 0) {  // invalid request: emit nothing, carry the state over
+                const int* tok = a.clean_tok + (size_t)b * N;
+                a.accept_len[b] = 0;
+                a.next_n_clean[b] = c_in;
+                a.next_kv_len[b] = a.kv_len[b];
+                for (int k = 0; k < N; ++k) {
+                    a.out_tok[(size_t)b * N + k] = -1;
+                    a.next_clean_tok[(size_t)b * N + k] = tok[k];
+                }
+            } else if (state == 0 && a.mode != ISD_PROPOSE_SAMPLE) {
+                // every proposal kept, argmax proposals: nothing to draw
+                picked[0] = s_stats[c_in - 1].argmax;
+                for (int m = 0; m + 1 < N; ++m) picked[m + 1] = s_stats[N + m].argmax;
+                emit_request(a, b, 0, c_in, picked);
+            }
+            req_state[b] = state;
+            __threadfence();
+            asm volatile("red.release.gpu.global.add.s32 [%0], 1;\n" ::"l"(decided) : "memory");
+        }
+    }
+
+    // ------------------------------------------------------------ draws
+    if (threadIdx.x == 0) {
+        // bounded wait until every request is decided (the deciders are the
+        // first B CTAs of the grid; they wait for nothing)
+        int ok = 0;
+        const uint64_t t0 = sm100::global_ns();
+        for (uint32_t it = 0;; ++it) {
+            int v;
+            asm volatile("ld.acquire.gpu.global.b32 %0, [%1];\n" : "=r"(v) : "l"(decided) : "memory");
+            if (v >= a.B) {
+                ok = 1;
+                break;
+            }
+            if ((it & 63) == 63 && sm100::global_ns() - t0 > 2000000000ull) {
+                raise_flag(a.err_flag, ISD_FLAG_WAIT_TIMEOUT);
+                break;
+            }
+        }
+        s_ok = ok;
+        s_b = -1;
+    }
+    __syncthreads();
+    if (!s_ok) return;
+    // this CTA's item: request number cta / n_chunks among those that draw
+    const int r_idx = cta / a.n_chunks, ch = cta - r_idx * a.n_chunks;
+    {
+        int base = 0;
+        for (int t0 = 0; t0 < a.B && base <= r_idx; t0 += kAcceptThreads) {
+            const int t = t0 + (int)threadIdx.x;
+            int f = 0;
+            if (t < a.B) {
+                const int st = __ldcg(req_state + t);
+                f = st > 0 || (st == 0 && a.mode == ISD_PROPOSE_SAMPLE);
+            }
+            float tot;
+            const int excl = base + (int)block_exclusive_scan((float)f, &tot);
+            if (f && excl == r_idx) s_b = t;
+            base += (int)tot;
+            __syncthreads();
+        }
+    }
+    __syncthreads();
+    const int b = s_b;
+    if (b < 0) return;  // past the drawing requests' chunks
+    const int state = __ldcg(req_state + b);
+    const int c = __ldg(&a.n_clean[b]);
+    const int nrows = state > 0 ? 1 : N;
+    const float* ub = a.uniforms + (size_t)b * 2 * N;
+    // the inverse-CDF rows of request b: the residual max(0, p - q) of the
+    // rejected proposal, or (sample mode) the N proposal rows
+    auto row_of = [&](int k, SweepRow* r) {
+        if (state > 0) {
+            const size_t rp = (size_t)b * Q + (state - 2);
+            const size_t rq = (size_t)b * Q + (N + state - 2);
+            const isd_row_stat sp = stat_of(b, state - 2), sq = a.prev_stats[rq];
+            *r = SweepRow{a.logits + rp * V, a.prev_logits + rq * V, sp.max, sq.max,
+                          1.f / sq.sumexp, (sq.max - sp.max) + logf(sq.sumexp / sp.sumexp)};
+        } else {
+            const size_t rr = (size_t)b * Q + (k == 0 ? c - 1 : N + k - 1);
+            const isd_row_stat st = stat_of(b, k == 0 ? c - 1 : N + k - 1);
+            *r = SweepRow{a.logits + rr * V, nullptr, st.max, 0.f, 0.f, 0.f};
+        }
+    };
+    float* part = a.part + (size_t)b * (N + 1) * a.n_chunks;
+    {
+        const int beg = ch * kAcceptChunk, end = min(V, beg + kAcceptChunk);
+        for (int k = 0; k < nrows; ++k) {
+            SweepRow r;
+            row_of(k, &r);
+            int dummy;
+            const float tot = chunk_scan(r, beg, end, a.vec, -1.f, &dummy);
+            if (threadIdx.x == 0) part[(size_t)k * a.n_chunks + ch] = tot;
+        }
+    }
+    __threadfence();
+    __syncthreads();
+    if (threadIdx.x == 0) s_last = (atomicAdd(&a.ticket[b], 1) == a.n_chunks - 1);
+    __syncthreads();
+    if (!s_last) return;
+    __threadfence();
+    for (int k = 0; k < nrows; ++k) {
+        SweepRow r;
+        row_of(k, &r);
+        const float u = state > 0 ? ub[N - 1] : ub[N + k];
+        // chunk totals in chunk order, scanned by the whole block
+        __shared__ float s_target;
+        __shared__ int s_chunk, s_hit, s_lastpos;
+        const float tv = (int)threadIdx.x < a.n_chunks
+                             ? __ldcg(&part[(size_t)k * a.n_chunks + threadIdx.x]) : 0.f;
+        float total;
+        const float excl = block_exclusive_scan(tv, &total);
+        const float target = u * total;
+        if (threadIdx.x == 0) {
+            s_hit = 0x7fffffff;
+            s_lastpos = -1;
+        }
+        __syncthreads();
+        if (tv > 0.f) atomicMax(&s_lastpos, (int)threadIdx.x);
+        if ((int)threadIdx.x < a.n_chunks && excl + tv > target) atomicMin(&s_hit, (int)threadIdx.x);
+        __syncthreads();
+        if (threadIdx.x == 0) {
+            if (!(total > 0.f)) {
+                s_chunk = -2;  // no mass: residual falls back to argmax p
+                s_target = 0.f;
+            } else if (s_hit == 0x7fffffff) {
+                s_chunk = s_lastpos;
+                s_target = 3.0e38f;  // take the last positive entry of that chunk
+            } else {
+                s_chunk = s_hit;
+            }
+        }
+        __syncthreads();
+        if (s_chunk >= 0 && s_chunk == s_hit && (int)threadIdx.x == s_hit)
+            s_target = fmaxf(target - excl, 0.f);
+        __syncthreads();
+        const int q = s_chunk;
+        const float tgt = s_target;
+        __syncthreads();
+        int y;
+        if (q == -2) {  // argmax of the anchor (or proposal) row
+            y = stat_of(b, state > 0 ? state - 2 : (k == 0 ? c - 1 : N + k - 1)).argmax;
+        } else {
+            const int beg2 = q * kAcceptChunk, end2 = min(V, beg2 + kAcceptChunk);
+            chunk_scan(r, beg2, end2, a.vec, tgt, &y);
+        }
+        if (threadIdx.x == 0) picked[k] = y;
+    }
+    if (threadIdx.x == 0) {
+        emit_request(a, b, state, c, picked);
+        a.ticket[b] = 0;
+    }
 }
 
 // ---------------------------------------------------------------------------
@@ -556,7 +583,7 @@ cudaError_t launch_accept(const Plan& p, const isd_dims* d, const float* logits,
     a.vec = d->V % 4 == 0 && reinterpret_cast<uintptr_t>(logits) % 16 == 0 &&
             reinterpret_cast<uintptr_t>(prev_logits) % 16 == 0;
     a.err_flag = err_flag;
-    dim3 grid(d->B, p.acc_chunks);
+    dim3 grid(d->B * p.acc_chunks);
     return launch_kernel(pdl, accept_kernel, grid, dim3(kAcceptThreads), 0, st, a);
 }
 

@@ -514,7 +514,7 @@ cudaError_t launch_attention_tc(const Plan& p, const isd_dims* d, const uint16_t
 // The tensor-core kernel (attention_tc.cu) where the shape fits it, else the
 // general mma.sync kernel above.  Either way the attention counters in the
 // workspace are cleared on the stream first, and so are the B counters at
-// clear_extra (2 B: the accept kernel's tickets and decision flags) and the
+// clear_extra (2 B + 1: the accept kernel's tickets, states and decided count) and the
 // clear_count counters at clear_range when not null.
 // pdl: launched as part of the whole step (programmatic dependent launch).
 cudaError_t launch_attention(const Plan& p, const isd_dims* d, const uint16_t* q,
@@ -530,7 +530,7 @@ cudaError_t launch_attention(const Plan& p, const isd_dims* d, const uint16_t* q
     if (handled || te != cudaSuccess) return te;
     cudaError_t me = cudaMemsetAsync(static_cast<char*>(ws) + p.off_attn_ticket, 0,
                                      (size_t)d->B * d->Hkv * p.attn_rgb * 4, st);
-    if (me == cudaSuccess && clear_extra) me = cudaMemsetAsync(clear_extra, 0, (size_t)d->B * 2 * 4, st);
+    if (me == cudaSuccess && clear_extra) me = cudaMemsetAsync(clear_extra, 0, (size_t)d->B * 2 * 4 + 4, st);
     if (me == cudaSuccess && clear_range && clear_count > 0)
         me = cudaMemsetAsync(clear_range, 0, (size_t)clear_count * 4, st);
     if (me != cudaSuccess) return me;

@@ -113,8 +113,8 @@ __global__ void kv_append_kernel(TcArgs a, const __nv_bfloat16* k_new, const __n
     if (r == 0) {
         for (int i = threadIdx.x; i < a.Hkv; i += blockDim.x) a.ticket[b * a.Hkv + i] = 0;
         if (clear_extra && threadIdx.x == 0) {
-            clear_extra[b] = 0;        // accept ticket
-            clear_extra[a.B + b] = 0;  // accept decision flag
+            clear_extra[b] = 0;  // accept ticket
+            if (b == 0) clear_extra[2 * a.B] = 0;  // accept decided count
         }
     }
     if (bad_c || over) {

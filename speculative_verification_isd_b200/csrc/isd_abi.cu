@@ -275,7 +275,7 @@ static isd_status accept_impl(const isd_dims* d, const float* logits, const isd_
         return invalid("null accept pointer");
     cudaStream_t st = static_cast<cudaStream_t>(stream);
     if (clear_counters)
-        ISD_CUDA(cudaMemsetAsync(static_cast<char*>(ws) + p.off_acc_ticket, 0, (size_t)d->B * 2 * 4, st));  // tickets, flags
+        ISD_CUDA(cudaMemsetAsync(static_cast<char*>(ws) + p.off_acc_ticket, 0, (size_t)d->B * 2 * 4 + 4, st));  // tickets, states, count
     ISD_CUDA(isd::launch_accept(p, d, logits, row_stats, prev_logits, prev_row_stats, n_clean,
                                 clean_tok, kv_len, uniforms, accept_len, out_tok, next_n_clean,
                                 next_clean_tok, next_kv_len, ratio, ws, err_flag, st,

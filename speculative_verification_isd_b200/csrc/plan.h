@@ -19,10 +19,8 @@ constexpr int kAcceptThreads = 256;
 // kernel than 4096 at B=32, N=4, V=151936; the chunk totals of a request are
 // scanned by one CTA, so V <= kAcceptThreads * kAcceptChunk).
 constexpr int kAcceptChunk = 2048;
-// accept CTAs resident per SM (launch bounds), and how long a CTA waits for
-// its request's published decision before deciding itself
+// accept CTAs resident per SM (launch bounds: 64 registers a thread)
 constexpr int kAcceptMinBlocks = 4;
-constexpr unsigned long long kAcceptFlagWaitNs = 30000;
 // Persistent kernels (attention, LM head) run one CTA per SM of the current
 // device, at most kMaxSMs (a B200 has 148); the workspace is sized for
 // kMaxSMs, and the split heuristics below aim at a B200-sized grid.
@@ -145,7 +143,7 @@ inline bool make_plan(const isd_dims* d, Plan* p) {
     p->off_stats_part = take((size_t)p->M * p->stats_chunks * 16);
     p->off_stats_ticket = take((size_t)p->M * 4);
     p->off_acc_part = take((size_t)d->B * (d->N + 1) * p->acc_chunks * 4);
-    p->off_acc_ticket = take((size_t)d->B * 3 * 4);  // tickets, decision flags, decided states
+    p->off_acc_ticket = take((size_t)d->B * 2 * 4 + 4);  // tickets, decided states, decided count
     p->off_lora_part = take(d->lora_rank ? (size_t)p->lora_ksplit * p->lora_rows * d->lora_rank * 4 : 0);
     p->lm_stat_parts = kMaxStatParts;
     p->off_lm_stats = take((size_t)p->M * p->lm_stat_parts * 16);
