@@ -13,6 +13,7 @@ instead (host cores, bounded samples of the same workload).
 from __future__ import annotations
 
 import argparse
+import dataclasses
 import hashlib
 import json
 import os
@@ -37,6 +38,8 @@ def parse_args():
     ap.add_argument("--warmup", type=int, default=20)
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--config", default="qwen3_8b_b32_n4")
+    ap.add_argument("--accept-rate", type=float, default=None,
+                    help="constructed per-proposal acceptance (default: the config's)")
     ap.add_argument("--e2e-steps", type=int, default=200)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-budget-s", type=float, default=20.0)
@@ -437,6 +440,8 @@ def main():
     hbm, tf_burst, tf_sus, peak_src = measured_peaks()
     # weak scaling: every rank runs its own batch of B requests (requests are
     # independent), so there is no collective on the data path
+    if args.accept_rate is not None:
+        cfg = dataclasses.replace(cfg, accept_rate=args.accept_rate)
     wl = DeviceWorkload(isd, cfg, seed=RK.rank_seed(0, rank), n_uniform_steps=max(64, args.warmup + 1))
     d = wl.dims
     K, W = args.steps, args.warmup
