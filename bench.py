@@ -344,6 +344,34 @@ def closed_loop(isd, cfg, R, K, bus, seed):
     st = lw.stats(W, W + K)
     tokens = R.sum(st["tokens"])
     kv_end = lw.kv_len[0].float().mean().item()
+    # the same steps again, the timed K captured once in a CUDA graph: back to
+    # the initial state, W steps eagerly, capture, one timed replay (the same
+    # work as the eager timed run, and the same results)
+    graph = None
+    al_eager = lw.accept_len_hist[W:W + K].clone()
+    try:
+        lw.reset()
+        lw.run(W)
+        torch.cuda.synchronize()
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g):
+            lw.isd.loop(lw.dims, K, lw.ws, err_flag=lw.err, stream=torch.cuda.current_stream(), args=args)
+        R.barrier()
+        torch.cuda.synchronize()
+        g0, g1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        g0.record(stream)
+        g.replay()
+        g1.record(stream)
+        torch.cuda.synchronize()
+        R.barrier()
+        gms = R.max(g0.elapsed_time(g1))
+        graph = {"steps": K, "ms_per_step": gms / K, "steps_per_s": K * R.world / (gms / 1e3),
+                 "tokens_per_s": tokens / (gms / 1e3),
+                 "same_accept_lengths_as_eager": bool(torch.equal(al_eager, lw.accept_len_hist[W:W + K])),
+                 "err_flags": int(lw.err.item())}
+        del g
+    except RuntimeError as e:  # capture unsupported in this process: report why
+        graph = {"unavailable": str(e).splitlines()[0][:200]}
     out = {"workload": cfg.name + " closed loop", "steps": K, "warmup": W,
            "ms_per_step": ms / K, "steps_per_s": K * R.world / (ms / 1e3),
            "tokens_per_s": tokens / (ms / 1e3), "tpf": st["tpf"], "tpf_se": st["tpf_se"],
@@ -352,7 +380,8 @@ def closed_loop(isd, cfg, R, K, bus, seed):
            "tpf_restart_model_at_measured_rate": restart_model_tpf(st["accept_rate"], cfg.N),
            "model": {"w_std": LOOP_W_STD, "qkv_std": LOOP_QKV_STD, "kv_std": LOOP_KV_STD},
            "mean_kv_len": {"start": float(lw.kv0.mean()), "end": kv_end},
-           "gpu_launches": 5 * K, "err_flags": int(lw.err.item()), "clocks": clk}
+           "gpu_launches": 5 * K, "err_flags": int(lw.err.item()), "clocks": clk,
+           "cuda_graph": graph}
     del lw
     torch.cuda.empty_cache()
     return out

@@ -283,6 +283,17 @@ class LoopWorkload:
         self.ws = isd.alloc_workspace(d)
         self.err = torch.zeros(1, dtype=torch.int32, device="cuda")
         self.done = 0
+        self._initial = {f: getattr(self, f).clone() for f in self.STATE}
+
+    # the requests' state and the page bookkeeping; the KV pool needs no reset
+    # (a position past a request's prefix is appended before it is read)
+    STATE = ("page_table", "pages_used", "next_free_page", "kv_len", "n_clean", "clean_tok")
+
+    def reset(self):
+        """Back to the state before the first step (stream-ordered copies)."""
+        for f in self.STATE:
+            getattr(self, f).copy_(self._initial[f])
+        self.done = 0
 
     def args(self, start: int, n: int):
         """Checked isd_loop arguments for steps start .. start+n-1 (start even,
@@ -303,9 +314,14 @@ class LoopWorkload:
         self.isd.loop(self.dims, n, self.ws, err_flag=self.err, stream=stream, args=a)
         self.done += n
 
-    def stats(self, start: int, stop: int) -> Dict[str, float]:
+    def state_host(self):
+        """n_clean of the current state (buffer 0 after an even number of steps)."""
+        return self.n_clean[self.done & 1].cpu().numpy()
+
+    def stats(self, start: int, stop: int, c_start=None) -> Dict[str, float]:
         """Tokens per forward and the proposal acceptance rate of steps
-        start .. stop-1, from the accept-length history.
+        start .. stop-1, from the accept-length history (c_start: the clean
+        counts at step `start`, when the history before it is not the same run).
 
         The clean count c of each step follows from the history: every request
         starts at c = 1; a step that keeps all of its c tokens continues with
@@ -315,10 +331,14 @@ class LoopWorkload:
         N = self.cfg.N
         al = self.accept_len_hist[:stop].cpu().numpy().astype(np.int64)
         c = np.ones(al.shape[1], np.int64)
+        first = 0
+        if c_start is not None:  # the clean counts at step `start` are known
+            c = np.asarray(c_start, np.int64).copy()
+            first = start
         acc = tests = 0
         acc_pos = np.zeros(max(N - 1, 1))
         tests_pos = np.zeros(max(N - 1, 1))
-        for s in range(stop):
+        for s in range(first, stop):
             A = al[s]
             if s >= start:
                 full = A == c

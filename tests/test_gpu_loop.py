@@ -341,3 +341,28 @@ def test_loop_full_shape_b32_n4(isd):
     assert torch.equal(lw2.k_pool, lw.k_pool) and torch.equal(lw2.v_pool, lw.v_pool)
     last = (steps - 1) & 1
     assert torch.equal(lw2.logits[last * M * V:(last + 1) * M * V], lw.logits[: M * V])
+
+
+def test_loop_captured_in_cuda_graph(isd):
+    """isd_loop captured once in a CUDA graph (the launches are capturable: no
+    host reads, allocations or memsets) replays bit-identically to the same
+    steps run eagerly from the same state."""
+    cfg = I.CONFIGS["tiny"]
+    steps = 64
+    d, host = setup(isd, cfg, steps, 3)
+    ws = isd.alloc_workspace(d)
+    err = torch.zeros(1, dtype=torch.int32, device="cuda")
+    eager = device_buffers(d, cfg, host, steps)
+    isd.loop(d, steps, ws, err_flag=err, **eager)
+    torch.cuda.synchronize()
+    cap = device_buffers(d, cfg, host, steps)
+    args = isd.loop_args(d, steps, **cap)
+    graph = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(graph):
+        isd.loop(d, steps, ws, err_flag=err, stream=torch.cuda.current_stream(), args=args)
+    graph.replay()
+    torch.cuda.synchronize()
+    assert int(err.item()) == 0
+    for k in eager:
+        assert torch.equal(eager[k], cap[k]), k
+    assert int(cap["accept_len_hist"].sum().item()) >= steps * cfg.B
