@@ -486,50 +486,72 @@ def test_tiny_closed_loop_1000_steps(isd):
     assert emitted >= steps * cfg.B
 
 
+FULL_SIZE = ["qwen3_8b_b32_n4", "qwen3_8b_b32_n8", "qwen3_8b_b64_n4_lora"]
+
+
 @pytest.mark.slow
-def test_full_size_b32_n4_sampled(isd):
-    """Qwen3-8B shapes, B=32, N=4 (the benchmark workload and launch
-    configuration): sampled attention rows, sampled logits, row statistics of
-    sampled rows, and the full accept decision checked against the oracle."""
+@pytest.mark.parametrize("name", FULL_SIZE)
+def test_full_size_sampled(isd, name):
+    """Full-size workloads in the benchmark's launch configuration (Qwen3-8B
+    shapes): B=32 N=4 (the headline), B=32 N=8 (64-token pages, 16-32 K
+    prefixes), B=64 N=4 with the rank-128 gated LoRA.  Checked against the
+    oracle: attention of whole requests; every logit of whole 256-row
+    vocabulary tiles (the first, tiles across the LM head's partition and the
+    half-full last one) for all rows; the statistics of every row; the full
+    accept decision."""
     from speculative_verification_isd_b200 import workload as Wk
-    cfg = I.CONFIGS["qwen3_8b_b32_n4"]
+    cfg = I.CONFIGS[name]
     wl = Wk.DeviceWorkload(isd, cfg, seed=0)
+    wl.set_uniforms(1)
     wl.step()
     torch.cuda.synchronize()
+    assert int(wl.err.item()) == 0
     rng = np.random.default_rng(0)
-    # attention: a few (request, slot, head) rows
     host = wl.host_view()
-    for b in rng.choice(cfg.B, 3, replace=False):
+    # attention: whole requests (all slots and heads)
+    for b in rng.choice(cfg.B, 2, replace=False):
         sub = Wk.request_slice(host, cfg, int(b))
         out_o, _, _ = O.attention(sub["q"], sub["k_new"], sub["v_new"], sub["k_pool"],
                                   sub["v_pool"], sub["page_table"], sub["kv_len"],
                                   sub["n_clean"], cfg.N, cfg.page_size, cfg.D ** -0.5)
         got = O.bf16_to_f64(bf16_host(wl.hidden[b * cfg.Q:(b + 1) * cfg.Q]))
-        assert np.abs(got - O.bf16_to_f64(out_o)).max() <= 2e-2
-    # logits: sampled entries, one float64 dot product each
+        err = np.abs(got - O.bf16_to_f64(out_o))
+        assert err.max() <= 2e-2 and err.mean() <= 3e-3, (b, err.max(), err.mean())
+    # logits: whole vocabulary tiles, every row
     hid = bf16_host(wl.hidden)
-    z = wl.logits
-    for _ in range(64):
-        m = int(rng.integers(0, cfg.M))
-        v = int(rng.integers(0, cfg.V))
-        w_row = bf16_host(wl.W[v:v + 1])[0]
-        ref = O.lm_head_entry(hid[m], w_row)
-        absdot = float(np.abs(O.bf16_to_f64(hid[m])) @ np.abs(O.bf16_to_f64(w_row)))
-        assert abs(float(z[m, v].item()) - ref) <= 1e-4 * absdot + 1e-6
-    # row statistics of a few rows and the complete accept step on GPU logits
-    zg = z.cpu().numpy().reshape(cfg.B, cfg.Q, cfg.V)
+    h_in = hid
+    if cfg.lora_rank:
+        h_in = O.gated_lora(hid, bf16_host(wl.lora_A), bf16_host(wl.lora_B), cfg.B, cfg.N)
+    h64 = O.bf16_to_f64(h_in)
+    n_tiles = (cfg.V + 255) // 256
+    tiles = sorted({0, 1, n_tiles // 4, n_tiles // 2, (3 * n_tiles) // 4, n_tiles - 2, n_tiles - 1,
+                    int(rng.integers(2, n_tiles - 2))})
+    for t in tiles:
+        v0, v1 = t * 256, min(cfg.V, t * 256 + 256)
+        w = O.bf16_to_f64(bf16_host(wl.W[v0:v1]))
+        ref = h64 @ w.T
+        bound = 1e-4 * (np.abs(h64) @ np.abs(w).T) + 1e-6
+        if cfg.lora_rank:  # one bf16 ulp of h' per product (intermediate roundings)
+            bound = bound + (np.abs(h64) @ np.abs(w).T) * 2.0 ** -8
+        got = wl.logits[:, v0:v1].cpu().numpy().astype(np.float64)
+        assert np.all(np.abs(got - ref) <= bound), (t, float(np.max(np.abs(got - ref) - bound)))
+    # statistics of every row, on the GPU's logits
+    zg = wl.logits.cpu().numpy()
     m_g, s_g, a_g = row_stats_host(wl.row_stats)
-    for r in rng.choice(cfg.M, 8, replace=False):
-        m_o, s_o, a_o = O.row_stats(zg.reshape(cfg.M, -1)[r])
-        assert m_g[r] == m_o and a_g[r] == a_o and abs(s_g[r] - s_o) <= NEAR * s_o
+    m_o, s_o, a_o = O.row_stats_all(zg)
+    assert np.array_equal(m_g, m_o.astype(np.float32).astype(np.float64))
+    assert np.array_equal(a_g, a_o)
+    assert np.all(np.abs(s_g - s_o) <= NEAR * s_o)
+    # the complete accept step on the GPU's logits
+    zg = zg.reshape(cfg.B, cfg.Q, cfg.V)
     prev = wl.prev_logits.cpu().numpy().reshape(cfg.B, cfg.Q, cfg.V)
     ores = O.accept(zg, prev, host["n_clean"], host["clean_tok"], host["kv_len"],
                     host["uniforms"], cfg.N)
-    gpu = wl.outputs()
-    rep = accept_parity(gpu, ores, zg, prev, host, cfg.N, O.PROPOSE_ARGMAX,
-                        "full size qwen3_8b_b32_n4")
-    assert rep["near_threshold"] + rep["excused_draws"] <= 2
-    # the constructed acceptance rate holds on every tested proposal
-    r = ores["ratio"][ores["ratio"] >= 0]
-    assert np.all(np.abs(r - cfg.accept_rate) < 1e-4)
-    assert int(wl.err.item()) == 0
+    rep = accept_parity(wl.outputs(), ores, zg, prev, host, cfg.N, O.PROPOSE_ARGMAX,
+                        f"full size {name}")
+    assert rep["near_threshold"] <= max(1, cfg.B // 50)
+    assert rep["excused_draws"] <= max(1, rep["draws"] // 50)
+    if cfg.accept_rate is not None:
+        # the constructed acceptance rate holds on every tested proposal
+        r = ores["ratio"][ores["ratio"] >= 0]
+        assert np.all(np.abs(r - cfg.accept_rate) < 1e-4)
