@@ -58,6 +58,10 @@ constexpr int kTcKeys = 128;            // keys per tile (M of S^T)
 constexpr int kTcUnitCost = 4;
 constexpr int kTcHalf = kTcKeys * 128;  // bytes of one 64-d half of a K or V tile
 constexpr uint64_t kTcWaitNs = 2000000000ull;
+// K and V ring depths (stages of 128 keys) when shared memory allows: a K
+// half is held only until its S product completes, a V half until its P.V
+// product, after the softmax of the tile
+constexpr int kTcDeepK = 3, kTcDeepV = 3;
 
 struct TcArgs {
     int B, N, Q, Hq, Hkv, grp, rows, P, num_pages, max_pages;
@@ -143,9 +147,9 @@ __global__ void kv_append_kernel(TcArgs a, const __nv_bfloat16* k_new, const __n
     }
 }
 
-template <int STAGES>
+template <int KS, int VS>
 struct TcShared {
-    uint64_t k_full[STAGES], k_empty[STAGES], v_full[STAGES], v_empty[STAGES];
+    uint64_t k_full[KS], k_empty[KS], v_full[VS], v_empty[VS];
     uint64_t s_full[2], s_empty[2], p_full, p_empty;
     uint64_t o_full, o_empty, q_full[2], q_empty[2], drain;
     uint32_t tmem;
@@ -186,14 +190,14 @@ struct TcRoles {
                   "register split exceeds the launch allocation");
 };
 
-template <int R, int STAGES>
+template <int R, int KS, int VS>
 constexpr size_t tc_smem_fixed() {
-    return (size_t)STAGES * 4 * kTcHalf    // K and V stages
+    return (size_t)(KS + VS) * 2 * kTcHalf  // K and V stages
            + 2 * 2 * R * 128               // Q, two buffers of two 64-d halves
            + 2 * R * 128                   // P^T (two 64-key halves); output staging
            + 4 * R * 4 * 2                 // per-warp row maxima and row sums
            + R * 4                         // per-row causal key limit
-           + sizeof(TcShared<STAGES>);
+           + sizeof(TcShared<KS, VS>);
 }
 // plus, per launch: 3 ints per request (kv_len, n_clean, keys) and
 // B * Hkv + 1 ints of unit offsets on the partition axis
@@ -224,7 +228,7 @@ ISD_DEVINL void tmem_store_cols(uint32_t taddr, const uint32_t (&v)[C]) {
     for (int j = 0; j < C / 16; ++j) sm100::tmem_st16(taddr + j * 16, v + j * 16);
 }
 
-template <int R, int STAGES>
+template <int R, int KS, int VS>
 __global__ void __launch_bounds__(TcRoles<R>::kThreads, 1)
 attention_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_v,
                     const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ TcArgs a) {
@@ -238,13 +242,13 @@ attention_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_const
     unsigned char* smem = reinterpret_cast<unsigned char*>(
         (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     unsigned char* sK = smem;
-    unsigned char* sV = sK + STAGES * 2 * kTcHalf;
-    unsigned char* sQ = sV + STAGES * 2 * kTcHalf;  // two buffers
+    unsigned char* sV = sK + KS * 2 * kTcHalf;
+    unsigned char* sQ = sV + VS * 2 * kTcHalf;  // two buffers
     unsigned char* sP = sQ + 2 * kQBytes;
     float* red_m = reinterpret_cast<float*>(sP + kPBytes);   // [4][R]
     float* red_l = red_m + 4 * R;                             // [4][R]
     int* lim = reinterpret_cast<int*>(red_l + 4 * R);         // [R]
-    TcShared<STAGES>* sh = reinterpret_cast<TcShared<STAGES>*>(lim + R);
+    TcShared<KS, VS>* sh = reinterpret_cast<TcShared<KS, VS>*>(lim + R);
     int* kvs = reinterpret_cast<int*>(sh + 1);                // [B] kv_len
     int* cs = kvs + a.B;                                      // [B] n_clean
     int* tots = cs + a.B;                                     // [B] keys (0: not served)
@@ -256,9 +260,11 @@ attention_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_const
 
     // ---- set-up
     if (threadIdx.x == 0) {
-        for (int s = 0; s < STAGES; ++s) {
+        for (int s = 0; s < KS; ++s) {
             mbar_init(&sh->k_full[s], 1);
             mbar_init(&sh->k_empty[s], 1);
+        }
+        for (int s = 0; s < VS; ++s) {
             mbar_init(&sh->v_full[s], 1);
             mbar_init(&sh->v_empty[s], 1);
         }
@@ -396,6 +402,7 @@ attention_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_const
                 // half are issued one box per lane (issuing them from a single
                 // thread caps the copy rate with small pages).
                 const bool is_v = warp != 0;
+            const int nst = is_v ? VS : KS;  // this producer's ring
                 uint64_t* full = is_v ? sh->v_full : sh->k_full;
                 uint64_t* empty = is_v ? sh->v_empty : sh->k_empty;
                 unsigned char* ring = is_v ? sV : sK;
@@ -473,7 +480,7 @@ attention_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_const
                         }
                         armed |= 1u << st;
                         armed_par = (armed_par & ~(1u << st)) | (ph << st);
-                        if (++st == STAGES) {
+                        if (++st == nst) {
                             st = 0;
                             ph ^= 1;
                         }
@@ -484,7 +491,7 @@ attention_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_const
                 }
                 // drain: every armed copy has landed before the CTA may exit
                 if (lane == 0) {
-                    for (int s = 0; s < STAGES; ++s)
+                    for (int s = 0; s < nst; ++s)
                         if (armed >> s & 1)
                             mbar_wait_bounded(&full[s], armed_par >> s & 1, &sh->never, kTcWaitNs);
                     if (!is_v)
@@ -536,7 +543,7 @@ attention_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_const
                     }
                     mma_commit(&sh->s_full[buf]);
                     mma_commit(&sh->k_empty[s_st]);  // the K half may be refilled once S is done
-                    if (++s_st == STAGES) {
+                    if (++s_st == KS) {
                         s_st = 0;
                         s_ph ^= 1;
                     }
@@ -592,7 +599,7 @@ attention_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_const
                         mma_commit(&sh->v_empty[pv_st]);
                         mma_commit(&sh->p_empty);
                         first_pv = false;
-                        if (++pv_st == STAGES) {
+                        if (++pv_st == VS) {
                             pv_st = 0;
                             pv_ph ^= 1;
                         }
@@ -766,7 +773,7 @@ attention_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_const
                     __syncwarp();
                     if (lane == 0) mbar_arrive(&sh->p_full);
                     ++tc;
-                    if (++kst == STAGES) {
+                    if (++kst == VS) {
                         kst = 0;
                         kph ^= 1;
                     }
@@ -955,7 +962,7 @@ bool encode_bf16_4d(CUtensorMap* m, const void* ptr, const uint64_t dims[4],
               CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
-template <int R, int STAGES>
+template <int R, int KS, int VS>
 cudaError_t launch_tc(const TcArgs& a, const CUtensorMap& tk, const CUtensorMap& tv,
                       const CUtensorMap& tq, size_t smem, cudaStream_t st, bool pdl) {
     static unsigned long long configured = 0;  // bit per device
@@ -967,7 +974,7 @@ cudaError_t launch_tc(const TcArgs& a, const CUtensorMap& tk, const CUtensorMap&
             // the register split assumes the launch allocation; a build that
             // allots fewer registers would leave the increase waiting forever
             cudaFuncAttributes fa;
-            const cudaError_t ae = cudaFuncGetAttributes(&fa, attention_tc_kernel<R, STAGES>);
+            const cudaError_t ae = cudaFuncGetAttributes(&fa, attention_tc_kernel<R, KS, VS>);
             if (ae != cudaSuccess) return ae;
             if (fa.numRegs < TcRoles<R>::kLaunchRegs) {
                 set_error_detail("attention: registers at launch below the warpgroup split");
@@ -976,12 +983,12 @@ cudaError_t launch_tc(const TcArgs& a, const CUtensorMap& tk, const CUtensorMap&
         }
         int optin = 0;
         cudaDeviceGetAttribute(&optin, cudaDevAttrMaxSharedMemoryPerBlockOptin, dev);
-        const cudaError_t e = cudaFuncSetAttribute(attention_tc_kernel<R, STAGES>,
+        const cudaError_t e = cudaFuncSetAttribute(attention_tc_kernel<R, KS, VS>,
                                                    cudaFuncAttributeMaxDynamicSharedMemorySize, optin);
         if (e != cudaSuccess) return e;
         configured |= 1ull << dev;
     }
-    return launch_kernel(pdl, attention_tc_kernel<R, STAGES>, dim3(persistent_grid()), dim3(TcRoles<R>::kThreads),
+    return launch_kernel(pdl, attention_tc_kernel<R, KS, VS>, dim3(persistent_grid()), dim3(TcRoles<R>::kThreads),
                          smem, st, tk, tv, tq, a);
 }
 
@@ -1005,13 +1012,14 @@ cudaError_t launch_attention_tc(const Plan& p, const isd_dims* d, const uint16_t
     cudaDeviceGetAttribute(&optin, cudaDevAttrMaxSharedMemoryPerBlockOptin, dev);
     // alignment slack, per-request lengths, unit offsets
     const size_t extra = 1024 + (size_t)3 * d->B * 4 + (size_t)(d->B * d->Hkv + 1) * 4;
+    // the deep rings when they fit, else two stages each
     int stages = 0;
     size_t smem = 0;
     for (int s = 3; s >= 2 && !stages; --s) {
         size_t f = 0;
-        if (R == 16) f = s == 3 ? tc_smem_fixed<16, 3>() : tc_smem_fixed<16, 2>();
-        if (R == 32) f = s == 3 ? tc_smem_fixed<32, 3>() : tc_smem_fixed<32, 2>();
-        if (R == 64) f = s == 3 ? tc_smem_fixed<64, 3>() : tc_smem_fixed<64, 2>();
+        if (R == 16) f = s == 3 ? tc_smem_fixed<16, kTcDeepK, kTcDeepV>() : tc_smem_fixed<16, 2, 2>();
+        if (R == 32) f = s == 3 ? tc_smem_fixed<32, kTcDeepK, kTcDeepV>() : tc_smem_fixed<32, 2, 2>();
+        if (R == 64) f = s == 3 ? tc_smem_fixed<64, kTcDeepK, kTcDeepV>() : tc_smem_fixed<64, 2, 2>();
         if (f + extra <= (size_t)optin) {
             stages = s;
             smem = f + extra;
@@ -1066,9 +1074,14 @@ cudaError_t launch_attention_tc(const Plan& p, const isd_dims* d, const uint16_t
                                   reinterpret_cast<__nv_bfloat16*>(v_pool), clear_extra, clear_range,
                                   clear_count);
     if (e != cudaSuccess) return e;
-    if (R == 16) return stages == 3 ? launch_tc<16, 3>(a, tk, tv, tq, smem, st, pdl) : launch_tc<16, 2>(a, tk, tv, tq, smem, st, pdl);
-    if (R == 32) return stages == 3 ? launch_tc<32, 3>(a, tk, tv, tq, smem, st, pdl) : launch_tc<32, 2>(a, tk, tv, tq, smem, st, pdl);
-    return stages == 3 ? launch_tc<64, 3>(a, tk, tv, tq, smem, st, pdl) : launch_tc<64, 2>(a, tk, tv, tq, smem, st, pdl);
+    if (R == 16)
+        return stages == 3 ? launch_tc<16, kTcDeepK, kTcDeepV>(a, tk, tv, tq, smem, st, pdl)
+                           : launch_tc<16, 2, 2>(a, tk, tv, tq, smem, st, pdl);
+    if (R == 32)
+        return stages == 3 ? launch_tc<32, kTcDeepK, kTcDeepV>(a, tk, tv, tq, smem, st, pdl)
+                           : launch_tc<32, 2, 2>(a, tk, tv, tq, smem, st, pdl);
+    return stages == 3 ? launch_tc<64, kTcDeepK, kTcDeepV>(a, tk, tv, tq, smem, st, pdl)
+                       : launch_tc<64, 2, 2>(a, tk, tv, tq, smem, st, pdl);
 }
 
 }  // namespace isd
