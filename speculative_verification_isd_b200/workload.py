@@ -320,41 +320,48 @@ class LoopWorkload:
 
     def stats(self, start: int, stop: int, c_start=None) -> Dict[str, float]:
         """Tokens per forward and the proposal acceptance rate of steps
-        start .. stop-1, from the accept-length history (c_start: the clean
-        counts at step `start`, when the history before it is not the same run).
-
-        The clean count c of each step follows from the history: every request
-        starts at c = 1; a step that keeps all of its c tokens continues with
-        c = N, any other with c = 1 (the restart).  A step with c clean tokens
-        tests proposals 2..c in order and stops at the first rejection, so it
-        accepted A - 1 of them and made one more (rejected) test if A < c."""
-        N = self.cfg.N
-        al = self.accept_len_hist[:stop].cpu().numpy().astype(np.int64)
-        c = np.ones(al.shape[1], np.int64)
-        first = 0
-        if c_start is not None:  # the clean counts at step `start` are known
-            c = np.asarray(c_start, np.int64).copy()
-            first = start
-        acc = tests = 0
-        acc_pos = np.zeros(max(N - 1, 1))
-        tests_pos = np.zeros(max(N - 1, 1))
-        for s in range(first, stop):
-            A = al[s]
-            if s >= start:
-                full = A == c
-                tested = np.where(full, c - 1, A)
-                acc += int((A - 1).sum())
-                tests += int(tested.sum())
-                for j in range(N - 1):
-                    tests_pos[j] += int((tested > j).sum())
-                    acc_pos[j] += int((A - 1 > j).sum())
-            c = np.where(A == c, N, 1)
-        window = al[start:stop]
-        tpf = float(window.mean())
-        se = float(window.mean(axis=0).std(ddof=1) / math.sqrt(window.shape[1]))
-        return dict(tokens=int(window.sum()), tpf=tpf, tpf_se=se,
-                    accept_rate=acc / max(tests, 1), tests=tests,
-                    accept_rate_by_position=[float(a / max(t, 1)) for a, t in zip(acc_pos, tests_pos)])
+        start .. stop-1 of this loop (see ``loop_stats``)."""
+        al = self.accept_len_hist[:stop].cpu().numpy()
+        return loop_stats(al, self.cfg.N, start, stop, c_start)
 
 
-__all__ = ["DeviceWorkload", "LoopWorkload", "request_slice"]
+def loop_stats(al: np.ndarray, N: int, start: int, stop: int, c_start=None) -> Dict[str, float]:
+    """Tokens per forward and the proposal acceptance rate of steps
+    start .. stop-1 from an accept-length history al [steps, B].
+
+    The clean count c of each step follows from the history: every request
+    starts at c = 1; a step that keeps all of its c tokens continues with
+    c = N, any other with c = 1 (the restart).  A step with c clean tokens
+    tests proposals 2..c in order and stops at the first rejection, so it
+    accepted A - 1 of them and made one more (rejected) test if A < c.
+    c_start: the clean counts at step `start`, when the history before it is
+    not the same run."""
+    al = np.asarray(al, np.int64)
+    c = np.ones(al.shape[1], np.int64)
+    first = 0
+    if c_start is not None:
+        c = np.asarray(c_start, np.int64).copy()
+        first = start
+    acc = tests = 0
+    acc_pos = np.zeros(max(N - 1, 1))
+    tests_pos = np.zeros(max(N - 1, 1))
+    for s in range(first, stop):
+        A = al[s]
+        if s >= start:
+            full = A == c
+            tested = np.where(full, c - 1, A)
+            acc += int((A - 1).sum())
+            tests += int(tested.sum())
+            for j in range(N - 1):
+                tests_pos[j] += int((tested > j).sum())
+                acc_pos[j] += int((A - 1 > j).sum())
+        c = np.where(A == c, N, 1)
+    window = al[start:stop]
+    tpf = float(window.mean())
+    se = float(window.mean(axis=0).std(ddof=1) / math.sqrt(window.shape[1]))
+    return dict(tokens=int(window.sum()), tpf=tpf, tpf_se=se,
+                accept_rate=acc / max(tests, 1), tests=tests,
+                accept_rate_by_position=[float(a / max(t, 1)) for a, t in zip(acc_pos, tests_pos)])
+
+
+__all__ = ["DeviceWorkload", "LoopWorkload", "loop_stats", "request_slice"]

@@ -351,3 +351,59 @@ def test_inverse_cdf_falls_back_to_last_positive_weight():
     assert O.inverse_cdf(np.array([0.0, 3.0, 0.0]), 1.0) == 1
     # the main branch just below: the largest uniform in [0, 1) of float32
     assert O.inverse_cdf(w, float(np.nextafter(np.float32(1), np.float32(0)))) == 4
+
+
+def test_loop_stats_counts_match_the_oracle_loop():
+    """The device loop's statistics (speculative_verification_isd_b200.workload.
+    loop_stats) rebuild each step's clean count from the accept lengths alone;
+    on the oracle's own closed loop their test and acceptance counts equal the
+    oracle's (tested = proposals with a ratio, accepted = u < ratio), and
+    tokens per forward is the mean accept length."""
+    from speculative_verification_isd_b200.workload import loop_stats
+    rng = np.random.default_rng(11)
+    B, steps, V, N, a = 40, 120, 64, 4, 0.85
+    Q = 2 * N - 1
+    nc = np.ones(B, dtype=np.int32)
+    tok = rng.integers(0, V, size=(B, N)).astype(np.int32)
+    kv = np.zeros(B, dtype=np.int32)
+    hist = np.zeros((steps, B), np.int64)
+    tests = acc = 0
+    for s in range(steps):
+        logits = (rng.standard_normal((B, Q, V)) * 0.5).astype(np.float32)
+        prev = (rng.standard_normal((B, Q, V)) * 0.5).astype(np.float32)
+        for b in range(B):
+            for j in range(2, int(nc[b]) + 1):
+                z, zq = constructed_pair(rng, V, int(tok[b, j - 1]), a)
+                logits[b, j - 2] = z
+                prev[b, N + j - 2] = zq
+        u = rng.random((B, 2 * N)).astype(np.float32)
+        res = O.accept(logits, prev, nc, tok, kv, u, N)
+        hist[s] = res["accept_len"]
+        if s >= 10:
+            r = res["ratio"]
+            tested = r >= 0
+            tests += int(tested.sum())
+            acc += int((tested & (u[:, : N - 1] < r)).sum())
+        nc, tok, kv = res["next_n_clean"], res["next_clean_tok"], res["next_kv_len"]
+    st = loop_stats(hist, N, 10, steps)
+    assert st["tests"] == tests
+    assert st["accept_rate"] == pytest.approx(acc / tests, abs=1e-12)
+    assert st["tpf"] == pytest.approx(hist[10:].mean(), abs=1e-12)
+    assert abs(st["accept_rate"] - a) < 0.03
+    # starting the count mid-run from the known clean counts gives the same
+    c10 = np.ones(B, np.int64)
+    for s in range(10):
+        c10 = np.where(hist[s] == c10, N, 1)
+    assert loop_stats(hist, N, 10, steps, c_start=c10) == st
+
+
+def test_bench_restart_model_matches_the_closed_form():
+    """bench.py's restart-model TPF (reported beside the closed-loop figure)
+    is the same function of (a, N) as this file's, and gives the table's
+    2.92 at a = 0.9, N = 4; a = 1 keeps every proposal (TPF = N)."""
+    import bench
+    for N in (2, 3, 4, 8):
+        for a in (0.5, 0.8, 0.9, 0.95):
+            assert bench.restart_model_tpf(a, N) == pytest.approx(tpf_restart_model(a, N), rel=1e-12)
+        assert bench.restart_model_tpf(1.0, N) == pytest.approx(float(N))
+    assert round(bench.restart_model_tpf(0.9, 4), 2) == 2.92
