@@ -561,22 +561,34 @@ def main():
     st_ms = stage.mean(axis=0)
     t_attn, t_lm, t_acc = [float(x) for x in st_ms]
 
-    # ---------------- R-ISD gated LoRA: cost of the adapter (same steps with it off)
+    # ---------------- R-ISD gated LoRA: cost of the adapter.  The same steps with
+    # the adapter on and off, in alternating rounds (so that clock changes hit
+    # both alike); alpha = median of the rounds' time ratios
     lora_alpha = None
     if cfg.lora_rank:
-        KL = min(K, 300)
-        for k in range(W):
-            wl.set_uniforms(k)
-            wl.step(without_lora=True)
-        f0, f1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-        f0.record(stream)
-        for k in range(KL):
-            wl.set_uniforms(k)
-            wl.step(without_lora=True)
-        f1.record(stream)
-        torch.cuda.synchronize()
-        t_plain = R.max(f0.elapsed_time(f1)) / KL
-        lora_alpha = (t_ms / K) / t_plain
+        rounds, per = 10, max(10, min(K, 300) // 10)
+
+        def timed(off):
+            for k in range(3):
+                wl.set_uniforms(k)
+                wl.step(without_lora=off)
+            f0, f1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            f0.record(stream)
+            for k in range(per):
+                wl.set_uniforms(k)
+                wl.step(without_lora=off)
+            f1.record(stream)
+            torch.cuda.synchronize()
+            return R.max(f0.elapsed_time(f1)) / per
+
+        ratios = []
+        for rnd in range(rounds):
+            if rnd % 2 == 0:
+                t_on, t_off = timed(False), timed(True)
+            else:
+                t_off, t_on = timed(True), timed(False)
+            ratios.append(t_on / t_off)
+        lora_alpha = statistics.median(ratios)
 
     # ---------------- e2e: public API with host buffers, copies inside the timed region
     # A step's inputs travel in one pinned host buffer (one host-to-device

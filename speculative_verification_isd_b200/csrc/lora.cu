@@ -7,10 +7,13 @@
 // the LM head.  The work is two thin GEMMs (at B=64, N=4: 192 rows x 4096 x
 // 128 and back), about 0.4 GFLOP, done on mma.sync tiles:
 //   1. T_part[z] = H_mask . A over K-slice z (fp32, split-K for parallelism)
-//   2. T = bf16(sum_z T_part[z]) in a fixed order
-//   3. h' = bf16(h + T . B) written over the MASK rows of a copy of hidden.
+//   2. T = bf16(sum_z T_part[z]) in slice order
+//   3. h' = bf16(h + T . B) on the MASK rows, h' = h copied on the clean rows
+//      (a second plane of the grid, so no separate copy of hidden).
+// The kernels wait for their predecessor when launched as dependents (pdl).
 #include "common.cuh"
 #include "plan.h"
+#include "launch.h"
 
 namespace isd {
 
@@ -28,6 +31,7 @@ struct LoraGemmArgs {
     float* part;                 // mode 0 output [ksplit][rows][r]
     const __nv_bfloat16* hidden; // mode 1 addend
     __nv_bfloat16* out;          // mode 1 output (hidden' [M,H])
+    int clean_rows;              // mode 1: B * N rows copied by the grid's second plane
 };
 
 // Row of the A operand for logical row m.
@@ -41,10 +45,24 @@ ISD_DEVINL const __nv_bfloat16* lora_a_row(const LoraGemmArgs& g, int m) {
 }
 
 template <int MODE>
-__global__ void __launch_bounds__(128) lora_gemm_kernel(LoraGemmArgs g) {
+__global__ void __launch_bounds__(128) lora_gemm_kernel(const __grid_constant__ LoraGemmArgs g) {
     __shared__ __align__(16) __nv_bfloat16 As[2][kLBM * kAStride];
     __shared__ __align__(16) __nv_bfloat16 Bs[2][kLBK * kBStride];
+    pdl_trigger();
+    pdl_wait();  // hidden (attention) or T (the first kernel) comes from the preceding kernel
     const int m0 = blockIdx.x * kLBM, n0 = blockIdx.y * kLBN, z = blockIdx.z;
+    if (MODE == 1 && z == 1) {
+        // clean rows: h' = h, 64 columns of 64 rows, 16 bytes per thread and step
+        for (int i = threadIdx.x; i < kLBM * (kLBN / 8); i += 128) {
+            const int cr = m0 + i / (kLBN / 8), c8 = (i % (kLBN / 8)) * 8;
+            if (cr >= g.clean_rows || n0 + c8 >= g.H) continue;
+            const int b = cr / g.N, s = cr % g.N;
+            const size_t off = ((size_t)b * g.Q + s) * g.H + n0 + c8;
+            *reinterpret_cast<uint4*>(g.out + off) = *reinterpret_cast<const uint4*>(g.hidden + off);
+        }
+        return;
+    }
+    if (m0 >= g.rows) return;
     const int kbeg = z * g.k_per_split;
     const int kend = min(g.K, kbeg + g.k_per_split);
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
@@ -148,6 +166,8 @@ __global__ void __launch_bounds__(128) lora_gemm_kernel(LoraGemmArgs g) {
 // T[m][n] = bf16(sum_z part[z][m][n]) in z order.
 __global__ void lora_reduce_kernel(const float* __restrict__ part, int ksplit, int count,
                                    __nv_bfloat16* __restrict__ t) {
+    pdl_trigger();
+    pdl_wait();  // the partials come from the preceding kernel
     const int i = blockIdx.x * blockDim.x + threadIdx.x;
     if (i >= count) return;
     float s = 0.f;
@@ -155,43 +175,44 @@ __global__ void lora_reduce_kernel(const float* __restrict__ part, int ksplit, i
     t[i] = __float2bfloat16_rn(s);
 }
 
-// hidden' = hidden with the adapter applied to the MASK rows.
+// hidden' = hidden with the adapter applied to the MASK rows (pdl: launch the
+// kernels as programmatic dependents of the preceding ones).
 cudaError_t launch_lora(const Plan& p, const isd_dims* d, const uint16_t* hidden,
                         const uint16_t* lora_A, const uint16_t* lora_B, uint16_t* hidden_out,
-                        void* ws, cudaStream_t st) {
+                        void* ws, cudaStream_t st, bool pdl) {
     char* w = static_cast<char*>(ws);
-    cudaError_t e = cudaMemcpyAsync(hidden_out, hidden, (size_t)p.M * p.H * 2,
-                                    cudaMemcpyDeviceToDevice, st);
-    if (e != cudaSuccess || p.lora_rows == 0) return e;
+    cudaError_t e = cudaSuccess;
     const int r = d->lora_rank;
-    LoraGemmArgs g;
+    LoraGemmArgs g = {};
     g.rows = p.lora_rows;
     g.N = d->N;
     g.Q = p.Q;
     g.H = p.H;
     g.r = r;
+    g.clean_rows = d->B * d->N;
     float* part = reinterpret_cast<float*>(w + p.off_lora_part);
     __nv_bfloat16* t = reinterpret_cast<__nv_bfloat16*>(w + p.off_lora_t);
-    // 1. partial h.A
-    const int kiters = p.H / kLBK;
-    const int per = (kiters + p.lora_ksplit - 1) / p.lora_ksplit;
-    g.K = p.H;
-    g.ncols = r;
-    g.k_per_split = per * kLBK;
-    g.a_src = reinterpret_cast<const __nv_bfloat16*>(hidden);
-    g.bmat = reinterpret_cast<const __nv_bfloat16*>(lora_A);
-    g.part = part;
-    g.hidden = nullptr;
-    g.out = nullptr;
-    const int ks = (kiters + per - 1) / per;
-    dim3 g1((g.rows + kLBM - 1) / kLBM, (r + kLBN - 1) / kLBN, ks);
-    lora_gemm_kernel<0><<<g1, 128, 0, st>>>(g);
-    if ((e = cudaGetLastError()) != cudaSuccess) return e;
-    // 2. fixed-order reduction, rounded to bf16
-    const int count = g.rows * r;
-    lora_reduce_kernel<<<(count + 255) / 256, 256, 0, st>>>(part, ks, count, t);
-    if ((e = cudaGetLastError()) != cudaSuccess) return e;
-    // 3. h' = bf16(h + T.B) on the MASK rows
+    if (p.lora_rows > 0) {
+        // 1. partial h.A
+        const int kiters = p.H / kLBK;
+        const int per = (kiters + p.lora_ksplit - 1) / p.lora_ksplit;
+        g.K = p.H;
+        g.ncols = r;
+        g.k_per_split = per * kLBK;
+        g.a_src = reinterpret_cast<const __nv_bfloat16*>(hidden);
+        g.bmat = reinterpret_cast<const __nv_bfloat16*>(lora_A);
+        g.part = part;
+        const int ks = (kiters + per - 1) / per;
+        dim3 g1((g.rows + kLBM - 1) / kLBM, (r + kLBN - 1) / kLBN, ks);
+        if ((e = launch_kernel(pdl, lora_gemm_kernel<0>, g1, dim3(128), 0, st, g)) != cudaSuccess)
+            return e;
+        // 2. fixed-order reduction, rounded to bf16
+        const int count = g.rows * r;
+        if ((e = launch_kernel(pdl, lora_reduce_kernel, dim3((count + 255) / 256), dim3(256), 0, st,
+                               (const float*)part, ks, count, t)) != cudaSuccess)
+            return e;
+    }
+    // 3. h' = bf16(h + T.B) on the MASK rows (plane 0), h' = h on the clean rows (plane 1)
     g.K = r;
     g.ncols = p.H;
     g.k_per_split = r;
@@ -200,9 +221,9 @@ cudaError_t launch_lora(const Plan& p, const isd_dims* d, const uint16_t* hidden
     g.part = nullptr;
     g.hidden = reinterpret_cast<const __nv_bfloat16*>(hidden);
     g.out = reinterpret_cast<__nv_bfloat16*>(hidden_out);
-    dim3 g2((g.rows + kLBM - 1) / kLBM, (p.H + kLBN - 1) / kLBN, 1);
-    lora_gemm_kernel<1><<<g2, 128, 0, st>>>(g);
-    return cudaGetLastError();
+    const int mtiles = (max(g.rows, g.clean_rows) + kLBM - 1) / kLBM;
+    dim3 g2(mtiles, (p.H + kLBN - 1) / kLBN, 2);
+    return launch_kernel(pdl, lora_gemm_kernel<1>, g2, dim3(128), 0, st, g);
 }
 
 }  // namespace isd
