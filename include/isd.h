@@ -236,6 +236,14 @@ isd_status isd_prepare_block(const isd_dims* d, const uint16_t* Eq, const uint16
  *          next_free_page, k_pool, v_pool, W, lora_A, lora_B, Eq, Ek, Ev as
  *          in isd_prepare_block and isd_step.
  * ws: isd_workspace_bytes(d) bytes, as for isd_step.
+ * Ownership: every buffer is the caller's device memory; the call allocates
+ * nothing and reads nothing back to the host.
+ * Errors: invalid dims, a null pointer among the required ones (lora_A and
+ * lora_B may be null when lora_rank is 0), n_steps < 0 or a short workspace
+ * return ISD_ERR_* before anything is enqueued; a launch failure part-way
+ * returns ISD_ERR_CUDA with the earlier steps enqueued.  Device-side faults
+ * (a page or token out of range, a request out of pages) set err_flag bits
+ * and never trap; the affected requests carry their state over.
  */
 typedef struct {
     const uint16_t* Eq;
@@ -268,7 +276,7 @@ isd_status isd_loop(const isd_dims* d, int32_t n_steps, const isd_loop_args* a, 
 
 /*
  * isd_attention_noalloc -- isd_attention for callers that cannot provide a
- * workspace.  The paper has no counterpart: this is a deployment convenience.
+ * workspace.  The pages have no counterpart: this is a deployment convenience.
  *
  * Some callers cannot allocate device memory for us: a serving engine that
  * gave all free device memory to its KV-cache pool at start-up, or code that
