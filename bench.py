@@ -47,6 +47,9 @@ def parse_args():
                     help="seconds of the sustained leg; 0 skips it")
     ap.add_argument("--loop-steps", type=int, default=400,
                     help="timed steps of the closed-loop leg (isd_loop); 0 skips it")
+    ap.add_argument("--sdar-steps", type=int, default=400,
+                    help="timed forwards of the SDAR-style comparison leg (isd_sdar_loop), "
+                         "per scheduling mode; 0 skips it")
     return ap.parse_args()
 
 
@@ -387,6 +390,72 @@ def closed_loop(isd, cfg, R, K, bus, seed):
     return out
 
 
+# SDAR-style comparison leg: confidence threshold of the unmask rule on the
+# same table model (q and k rotated by position).  Confidences of this model
+# at V = 151936 are small (flat synthetic logits); tau sits near the median
+# confidence of fresh-block rows, so blocks need 1..N forwards.
+SDAR_TAU = 1.1e-5
+
+
+def sdar_leg(isd, cfg, R, K, bus, seed):
+    """SDAR-style block decoding on the same batch shape, in both scheduling
+    modes: batch-synchronous (a round ends when every request's block is
+    complete and stored, so it costs max_b S_b + 1 forwards) and free-running
+    (each request moves on by itself after S_b + 1, as ISD requests do).  Each mode: 16 untimed forwards,
+    then K timed ones of isd_sdar_loop (five kernels per forward).  Tokens
+    count the blocks that left the batch in the timed window."""
+    import torch
+    from speculative_verification_isd_b200.workload import (SdarLoopWorkload, expected_max_of,
+                                                            sdar_round_stats)
+    W = 16
+    stream = torch.cuda.current_stream()
+    out = {"workload": cfg.name + " SDAR-style blocks", "block": cfg.N, "queries_per_forward": cfg.N,
+           "tau": SDAR_TAU,
+           "model": {"w_std": LOOP_W_STD, "qkv_std": LOOP_QKV_STD, "kv_std": LOOP_KV_STD,
+                     "rope_base": 1.0e6}}
+    for sync in (True, False):
+        sw = SdarLoopWorkload(isd, cfg, capacity_steps=W + K, seed=seed, w_std=LOOP_W_STD,
+                              qkv_std=LOOP_QKV_STD, kv_std=LOOP_KV_STD)
+        sw.run(W, SDAR_TAU, sync)
+        torch.cuda.synchronize()
+        args = sw.args(W, K)
+        clocks = ClockSampler(bus)
+        clocks.start()
+        time.sleep(0.2)
+        R.barrier()
+        torch.cuda.synchronize()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        sw.run(K, SDAR_TAU, sync, args=args)
+        e1.record(stream)
+        torch.cuda.synchronize()
+        R.barrier()
+        clk = clocks.stop()
+        ms = R.max(e0.elapsed_time(e1))
+        st = sdar_round_stats(sw.block_steps_hist[W:W + K].cpu().numpy(), cfg.N)
+        tokens = R.sum(st["blocks"] * cfg.N)
+        mode = {"forwards": K, "ms_per_forward": ms / K, "forwards_per_s": K * R.world / (ms / 1e3),
+                "tokens_per_s": tokens / (ms / 1e3), "blocks": st["blocks"],
+                "mean_S": st["mean_S"], "S_pmf": st["pmf"],
+                "tokens_per_forward_per_request": st["blocks"] * cfg.N / (K * cfg.B),
+                "err_flags": int(sw.err.item()), "gpu_launches": 5 * K, "clocks": clk}
+        if sync:
+            # forwards per block with the sync over those without it
+            mode.update(rounds=st["rounds"], mean_max_S=st["mean_max_S"],
+                        sync_penalty=(st["mean_max_S"] + 1.0) / (st["mean_S"] + 1.0))
+        out["sync" if sync else "free"] = mode
+        del sw
+        torch.cuda.empty_cache()
+    # E[max S_b] over a batch of B requests, from the free-running S pmf (the
+    # distribution of one request's block on its own), and the tokens per
+    # forward of a request that a synchronised batch of B would leave
+    pmf = out["free"]["S_pmf"]
+    emax = {b: expected_max_of(pmf, b) for b in (1, 2, 4, 8, 16, 32, 64)}
+    out["expected_max_S_by_batch"] = {str(b): v for b, v in emax.items()}
+    out["sync_tokens_per_forward_by_batch"] = {str(b): cfg.N / (v + 1.0) for b, v in emax.items()}
+    return out
+
+
 def config_dict(cfg, world):
     return {"workload": cfg.name, "B": cfg.B, "N": cfg.N, "Q": cfg.Q, "V": cfg.V,
             "hidden": cfg.H, "heads": f"{cfg.Hq}q/{cfg.Hkv}kv x {cfg.D}",
@@ -635,6 +704,9 @@ def main():
     loop_line = None
     if args.loop_steps > 0:
         loop_line = closed_loop(isd, cfg, R, args.loop_steps, bus, RK.rank_seed(0, rank))
+    sdar_line = None
+    if args.sdar_steps > 0:
+        sdar_line = sdar_leg(isd, cfg, R, args.sdar_steps, bus, RK.rank_seed(0, rank))
 
     # ---------------- roofline of the dominant kernel (LM head)
     lm_bytes = float(cfg.V) * cfg.H * 2 + float(cfg.M) * cfg.H * 2 + float(cfg.M) * cfg.V * 4
@@ -672,6 +744,8 @@ def main():
     }
     if loop_line is not None:
         line["closed_loop"] = loop_line
+    if sdar_line is not None:
+        line["sdar_comparison"] = sdar_line
     if lora_alpha is not None:
         # step time with the adapter / without it (the pages report about 1.12)
         line["lora_alpha"] = lora_alpha

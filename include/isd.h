@@ -305,6 +305,117 @@ isd_status isd_attention_noalloc(const isd_dims* d, const uint16_t* q, const uin
                                  const int32_t* n_clean, uint16_t* out, int32_t* err_flag,
                                  void* stream);
 
+/*
+ * ---------------------------------------------------------------------------
+ * SDAR-style confidence-threshold block decoding: the batch-synchronous
+ * comparison workload.  The I-DLM project page (paragraphs comparing ISD with
+ * SDAR) says SDAR denoises a block of N positions by confidence with N queries
+ * per forward, and that a batch waits for its slowest block, so a round costs
+ * max(S_1..S_B) forwards, a cost ISD does not pay.  The rule is not spelled
+ * out; these calls take the plain reading:
+ *  - block: positions kv_len .. kv_len+N-1, all N rows computed every forward;
+ *    a committed position carries its token, an uncommitted one MASK;
+ *  - attention is block-causal: every block row sees the prefix and all N
+ *    rows of its block; each forward writes the N rows' K/V at their
+ *    positions, and they stay in the cache when the block is committed;
+ *  - row s predicts position s; confidence = the row's largest softmax
+ *    probability, fl32(1) / fl32(sum_i exp(z_i - max)); candidate = argmax;
+ *  - unmask: every uncommitted position with confidence >= tau commits its
+ *    candidate; if none does, the most confident uncommitted one does (ties:
+ *    lowest position); a block takes S_b in [1, N] such forwards;
+ *  - a complete block gets one more forward over its final tokens (its
+ *    store pass: the K/V that forward appends stay in the cache), after
+ *    which it may leave: kv_len += N, a fresh block of MASK;
+ *  - sync != 0: the batch moves on only when every request's block is
+ *    complete and stored (a round costs max_b S_b + 1 forwards); requests
+ *    that finished early idle.  sync == 0: each stored block moves on by
+ *    itself (S_b + 1 forwards).
+ * Dims: isd_dims with N = the block size (<= 16) and lora_rank 0; the block
+ * has Q = N rows (not 2N-1).  isd_workspace_bytes(d) covers these calls.
+ * State (device, int32, updated in place): block_tok [B, N] (-1 = MASK),
+ * steps [B] (forwards spent on the current block), kv_len [B].
+ * Per call outputs: unmasked [B] (positions committed by this forward),
+ * out_tok [B, N] (a block's tokens when it leaves the batch in this call,
+ * else -1), block_steps [B] (its S_b, denoising forwards without the store
+ * pass, then; else 0).
+ * Errors: invalid pointers or dims -> ISD_ERR_INVALID_ARG; N > 16, lora_rank
+ * != 0 or shapes the attention / LM head do not support ->
+ * ISD_ERR_UNSUPPORTED_SHAPE.  On the device, a page id outside the pool
+ * raises ISD_FLAG_PAGE_OOB, a block that does not fit the request's pages
+ * ISD_FLAG_CAPACITY, a committed token outside [0, V) ISD_FLAG_TOKEN_OOB.
+ * ---------------------------------------------------------------------------
+ */
+
+/*
+ * isd_sdar_step -- one forward and decision of the batch: KV append +
+ * block-causal attention, LM head (logits [B*N, V] fp32), row statistics
+ * (row_stats [B*N], optional), unmask.  q [B, N, Hq, D], k_new / v_new
+ * [B, N, Hkv, D] bf16; pools, page_table as for isd_attention; hidden
+ * [B*N, H] bf16 or NULL (workspace).  No host synchronisation; capturable.
+ */
+isd_status isd_sdar_step(const isd_dims* d, float tau, int32_t sync, const uint16_t* q,
+                         const uint16_t* k_new, const uint16_t* v_new, uint16_t* k_pool,
+                         uint16_t* v_pool, const int32_t* page_table, int32_t* kv_len,
+                         const uint16_t* W, uint16_t* hidden, float* logits,
+                         isd_row_stat* row_stats, int32_t* block_tok, int32_t* steps,
+                         int32_t* unmasked, int32_t* out_tok, int32_t* block_steps, void* ws,
+                         size_t ws_bytes, int32_t* err_flag, void* stream);
+
+/*
+ * isd_sdar_unmask -- the decision alone, on given row statistics
+ * (row_stats [B*N]); same state and outputs as isd_sdar_step.
+ */
+isd_status isd_sdar_unmask(const isd_dims* d, float tau, int32_t sync,
+                           const isd_row_stat* row_stats, int32_t* block_tok, int32_t* steps,
+                           int32_t* kv_len, int32_t* unmasked, int32_t* out_tok,
+                           int32_t* block_steps, void* ws, size_t ws_bytes, int32_t* err_flag,
+                           void* stream);
+
+/*
+ * isd_sdar_loop -- n_steps forwards of a stationary batch on the device, each
+ * one: block activations by table lookup (Eq/Ek/Ev [V+1, heads, D], row V =
+ * MASK, as isd_prepare_block does for an ISD block) with the page list grown
+ * to cover kv_len + N, then isd_sdar_step on the state in place.  Step s
+ * writes unmasked_hist[s] [B], out_tok_hist[s] [B, N], block_steps_hist[s]
+ * [B]; logits, row_stats, q, k_new, v_new and hidden hold the last step's.
+ * rope (optional): [rope_positions, D/2, 2] fp32 (cos, sin) per position and
+ * pair; when given, the q and k rows of block position s are rotated by
+ * position kv_len + s (pairs (i, i + D/2), each product and sum rounded in
+ * fp32, then to bf16), as a rotary-embedded model's are; a position past the
+ * table raises ISD_FLAG_CAPACITY and is left unrotated.  NULL: no rotation.
+ * Ownership: every pointer is the caller's device memory, which must stay
+ * valid until the enqueued work completes; nothing is allocated.
+ */
+typedef struct {
+    const uint16_t* Eq;
+    const uint16_t* Ek;
+    const uint16_t* Ev;
+    const uint16_t* W;
+    uint16_t* k_pool;
+    uint16_t* v_pool;
+    int32_t* page_table;
+    int32_t* pages_used;
+    int32_t* next_free_page;
+    int32_t* kv_len;
+    int32_t* block_tok;
+    int32_t* steps;
+    float* logits;
+    isd_row_stat* row_stats;
+    uint16_t* q;
+    uint16_t* k_new;
+    uint16_t* v_new;
+    uint16_t* hidden;
+    int32_t* unmasked_hist;
+    int32_t* out_tok_hist;
+    int32_t* block_steps_hist;
+    const float* rope;
+    int32_t rope_positions;
+} isd_sdar_loop_args;
+
+isd_status isd_sdar_loop(const isd_dims* d, float tau, int32_t sync, int32_t n_steps,
+                         const isd_sdar_loop_args* a, void* ws, size_t ws_bytes,
+                         int32_t* err_flag, void* stream);
+
 #ifdef __cplusplus
 }
 #endif

@@ -20,8 +20,11 @@ it out.  The readings taken here (plainest ones the text supports):
       all N rows of its own block (bidirectional inside the block, causal
       across blocks), the usual mask of block-diffusion models.
   R3  Each forward writes the block's K/V rows (from that forward's inputs)
-      at their positions.  When the batch commits the block, kv_len advances
-      by N and those rows stay in the cache; there is no separate store pass.
+      at their positions.  A block leaves (kv_len += N, a fresh block of
+      MASK) only after a forward whose inputs were its final tokens, so the
+      cache keeps K/V computed from them: once its last position is committed,
+      the request's next forward is the block's store pass, as block-diffusion
+      decoders run one forward over a finished block to extend the cache.
   R4  Row s predicts block position s (no logit shift).
   R5  Confidence of position s = its largest softmax probability,
       1 / sum_i exp(z_i - max z); its candidate token is the argmax (ties to
@@ -29,12 +32,13 @@ it out.  The readings taken here (plainest ones the text supports):
   R6  Unmask rule: every uncommitted position whose confidence is >= tau is
       committed with its candidate; if none is, the one uncommitted position
       of highest confidence is (ties to the lowest position).  A block
-      therefore takes S_b in [1, N] forwards.  Committed tokens never change.
+      therefore takes S_b in [1, N] denoising forwards, then its store pass.
+      Committed tokens never change.
   R7  Batch sync: the batch moves to the next block only once every
-      request's block is committed.  A request that finished early idles
-      (its rows are still computed, its block is unchanged) until then.  A
-      round of the batch costs max_b S_b forwards.  Without sync (the ISD way)
-      a request moves on as soon as its own block is committed.
+      request's block is complete and stored.  A request that finished early
+      idles (its rows, final tokens, are still computed) until then.  A round
+      of the batch costs max_b S_b + 1 forwards.  Without sync (the ISD way)
+      a request moves on after its own block's store pass: S_b + 1 forwards.
   R8  Decisions (>= tau, the highest confidence) are taken on float32
       confidences conf = fl32(1) / fl32(S), the precision the kernel decides
       in; the oracle rounds its float64 sum to float32 first.
@@ -129,14 +133,15 @@ def unmask(block_tok: np.ndarray, conf: np.ndarray, cand: np.ndarray, tau: float
 
 
 def unmask_batch(block_tok, steps, kv_len, conf, cand, tau: float, sync: bool):
-    """One decision step of the whole batch (R6, R7).
+    """One decision step of the whole batch (R3, R6, R7).
 
-    block_tok [B, N], steps [B] (forwards spent on the current block before
-    this one), kv_len [B]; conf, cand [B, N] of this forward.
-    Returns a dict with the next block_tok / steps / kv_len and, per request,
-    unmasked (positions committed now), out_tok [N] (the block's tokens when
-    it leaves the batch in this step, else -1) and block_steps (its S_b then,
-    else 0)."""
+    block_tok [B, N], steps [B] (denoising forwards spent on the current
+    block before this one), kv_len [B]; conf, cand [B, N] of this forward.
+    A block that was complete when this forward began had its store pass in
+    this forward and may leave.  Returns a dict with the next block_tok /
+    steps / kv_len and, per request, unmasked (positions committed now),
+    out_tok [N] (the block's tokens when it leaves the batch in this step,
+    else -1) and block_steps (its S_b then, else 0)."""
     B, N = block_tok.shape
     tok = np.array(block_tok, dtype=np.int64, copy=True)
     st = np.array(steps, dtype=np.int64, copy=True)
@@ -144,13 +149,13 @@ def unmask_batch(block_tok, steps, kv_len, conf, cand, tau: float, sync: bool):
     unmasked = np.zeros(B, np.int64)
     out_tok = np.full((B, N), -1, np.int64)
     block_steps = np.zeros(B, np.int64)
+    stored = ~(tok == MASK).any(axis=1)   # complete at entry: this forward stored it
     for b in range(B):
-        if (tok[b] == MASK).any():
+        if not stored[b]:
             tok[b], ch = unmask(tok[b], conf[b], cand[b], tau)
             unmasked[b] = len(ch)
             st[b] += 1
-    done = ~(tok == MASK).any(axis=1)
-    leave = np.ones(B, bool) * bool(done.all()) if sync else done
+    leave = np.ones(B, bool) * bool(stored.all()) if sync else stored
     for b in range(B):
         if leave[b]:
             out_tok[b] = tok[b]
@@ -165,11 +170,38 @@ def unmask_batch(block_tok, steps, kv_len, conf, cand, tau: float, sync: bool):
 # ---------------------------------------------------------------------------
 # Whole step and closed loop on the synthetic table model
 # ---------------------------------------------------------------------------
-def embed_block(tables: Dict[str, np.ndarray], block_tok: np.ndarray, V: int):
+def rope_rotate(x_bits: np.ndarray, cs: np.ndarray) -> np.ndarray:
+    """Rotary embedding of bf16 head vectors x [..., D] with the (cos, sin)
+    table row cs [D/2, 2] of their position: element i pairs with i + D/2
+    (the rotate-half layout of Qwen3), x_i' = x_i cos - x_{i+D/2} sin and
+    x_{i+D/2}' = x_{i+D/2} cos + x_i sin.  The stand-in model fixes the
+    arithmetic: float32, each product and sum rounded, then one bf16 rounding."""
+    x = O.bf16_to_f64(x_bits).astype(np.float32)
+    h = x.shape[-1] // 2
+    c = cs[:, 0].astype(np.float32)
+    s = cs[:, 1].astype(np.float32)
+    lo, hi = x[..., :h], x[..., h:]
+    out = np.concatenate([lo * c - hi * s, hi * c + lo * s], axis=-1).astype(np.float32)
+    return O.f64_to_bf16(out.astype(np.float64))
+
+
+def embed_block(tables: Dict[str, np.ndarray], block_tok: np.ndarray, V: int,
+                kv_len: np.ndarray = None, rope: np.ndarray = None):
     """q, k_new, v_new of the N block rows: a committed position looks up its
-    token's row, an uncommitted one the MASK row V (R1)."""
+    token's row, an uncommitted one the MASK row V (R1).  With a rotary table
+    rope [positions, D/2, 2], the q and k rows of block position s are rotated
+    by position kv_len + s (v is not)."""
     ids = np.where(block_tok >= 0, block_tok, V).astype(np.int64)
-    return tables["Eq"][ids], tables["Ek"][ids], tables["Ev"][ids]
+    q, k, v = tables["Eq"][ids], tables["Ek"][ids], tables["Ev"][ids]
+    if rope is not None:
+        q, k = q.copy(), k.copy()
+        B, N = block_tok.shape
+        for b in range(B):
+            for s in range(N):
+                cs = rope[int(kv_len[b]) + s]
+                q[b, s] = rope_rotate(q[b, s], cs)
+                k[b, s] = rope_rotate(k[b, s], cs)
+    return q, k, v
 
 
 def sdar_step(q, k_new, v_new, k_pool, v_pool, page_table, kv_len, W, block_tok, steps,
@@ -188,14 +220,15 @@ def sdar_step(q, k_new, v_new, k_pool, v_pool, page_table, kv_len, W, block_tok,
 
 
 def round_stats(block_steps_hist: np.ndarray, N: int) -> Dict[str, float]:
-    """Forwards per block of a batch-synchronous decision history (R7).
+    """Forwards per block of a decision history (R3, R7).
 
     block_steps_hist [steps, B]: S_b of a block that left the batch at that
-    step, else 0.  Under sync every request's block leaves at the same step,
-    so each step with leavers closes one round, which cost max_b S_b
-    forwards.  Returns the number of blocks and rounds, the mean S_b (the
-    forwards a block needed on its own), the mean round length (max_b S_b)
-    and the tokens per forward of a request with and without the sync."""
+    step, else 0.  A block costs S_b denoising forwards plus its store pass.
+    Under sync every request's block leaves at the same step, so each step
+    with leavers closes one round, which cost max_b S_b + 1 forwards.
+    Returns the number of blocks and rounds, the mean S_b, the mean of
+    max_b S_b over rounds, and the tokens per forward of a request without
+    the sync, N / (E[S_b] + 1), and with it, N / (E[max_b S_b] + 1)."""
     h = np.asarray(block_steps_hist)
     rounds = [r[r > 0] for r in h if (r > 0).any()]
     if not rounds:
@@ -204,8 +237,8 @@ def round_stats(block_steps_hist: np.ndarray, N: int) -> Dict[str, float]:
     s_all = np.concatenate(rounds).astype(np.float64)
     maxes = np.array([r.max() for r in rounds], dtype=np.float64)
     return dict(blocks=int(s_all.size), rounds=len(rounds), mean_S=float(s_all.mean()),
-                mean_max_S=float(maxes.mean()), tpf_free=N / float(s_all.mean()),
-                tpf_sync=N / float(maxes.mean()))
+                mean_max_S=float(maxes.mean()), tpf_free=N / (float(s_all.mean()) + 1.0),
+                tpf_sync=N / (float(maxes.mean()) + 1.0))
 
 
 def expected_max(pmf: np.ndarray, B: int) -> float:
@@ -219,4 +252,4 @@ def expected_max(pmf: np.ndarray, B: int) -> float:
 
 
 __all__ = ["MASK", "kv_append", "block_attention", "confidence", "unmask", "unmask_batch",
-           "embed_block", "sdar_step", "round_stats", "expected_max"]
+           "rope_rotate", "embed_block", "sdar_step", "round_stats", "expected_max"]

@@ -44,7 +44,8 @@ struct AttnArgs {
     __nv_bfloat16* v_pool;
     const int32_t* page_table;
     const int32_t* kv_len;
-    const int32_t* n_clean;
+    const int32_t* n_clean;  // null: every one of the N first slots is active (c = N)
+    int bidir;               // 1: every row sees the whole block (block-causal mask)
     __nv_bfloat16* out;
     char* part;
     size_t part_stride;
@@ -86,9 +87,10 @@ __global__ void __launch_bounds__(128 * RG, (RG <= 2 ? 2 : 1)) attention_kernel(
     const int kw = (warp & 3) * 16;    // this warp's keys within a tile
 
     const int kv = a.kv_len[b];
-    const int c = a.n_clean[b];
+    const int c = a.n_clean ? a.n_clean[b] : a.N;
     const bool bad_c = (c < 1 || c > a.N);
-    const long long want = bad_c ? 0 : (long long)kv + c + a.N - 1;  // keys incl. the block
+    // keys incl. the block: c clean slots, then the Q - N slots after them
+    const long long want = bad_c ? 0 : (long long)kv + c + a.Q - a.N;
     const bool over = kv < 0 || (want + a.P - 1) / a.P > a.max_pages;
     // a request that cannot be served (bad n_clean, negative or over-capacity
     // length) is one empty split: its rows are written as zeros
@@ -106,7 +108,7 @@ __global__ void __launch_bounds__(128 * RG, (RG <= 2 ? 2 : 1)) attention_kernel(
 
     // ---- a1: the last split's CTA appends the block's K/V rows to the pages
     if (sp == ns - 1 && rgb == 0 && total > 0) {
-        const int nblk = c + a.N - 1;
+        const int nblk = c + a.Q - a.N;
         for (int i = tid; i < nblk * CH; i += THREADS) {
             const int r = i / CH, cc = i % CH;
             const int t = kv + r;
@@ -143,6 +145,7 @@ __global__ void __launch_bounds__(128 * RG, (RG <= 2 ? 2 : 1)) attention_kernel(
     for (int i = 0; i < 2; ++i) {
         const int rr = row0 + rg * 16 + i * 8 + (lane >> 2);
         rpos[i] = (rr < a.rows && total > 0) ? slot_pos(rr % a.Q, kv, c, a.N) : -1;
+        if (a.bidir && rpos[i] >= 0) rpos[i] = total - 1;
     }
 
     // ---- key -> cache-row table of this split (one page lookup per key):
@@ -509,7 +512,7 @@ cudaError_t launch_attention_tc(const Plan& p, const isd_dims* d, const uint16_t
                                 uint16_t* v_pool, const int32_t* page_table, const int32_t* kv_len,
                                 const int32_t* n_clean, uint16_t* out, void* ws, int32_t* err_flag,
                                 cudaStream_t st, int* clear_extra, int* clear_range, int clear_count,
-                                bool pdl, bool* handled);
+                                bool pdl, bool bidir, bool* handled);
 
 // The tensor-core kernel (attention_tc.cu) where the shape fits it, else the
 // general mma.sync kernel above.  Either way the attention counters in the
@@ -522,11 +525,11 @@ cudaError_t launch_attention(const Plan& p, const isd_dims* d, const uint16_t* q
                              uint16_t* v_pool, const int32_t* page_table, const int32_t* kv_len,
                              const int32_t* n_clean, uint16_t* out, void* ws, int32_t* err_flag,
                              cudaStream_t st, int* clear_extra, int* clear_range, int clear_count,
-                             bool pdl) {
+                             bool pdl, bool bidir) {
     bool handled = false;
     const cudaError_t te = launch_attention_tc(p, d, q, k_new, v_new, k_pool, v_pool, page_table,
                                                kv_len, n_clean, out, ws, err_flag, st, clear_extra,
-                                               clear_range, clear_count, pdl, &handled);
+                                               clear_range, clear_count, pdl, bidir, &handled);
     if (handled || te != cudaSuccess) return te;
     cudaError_t me = cudaMemsetAsync(static_cast<char*>(ws) + p.off_attn_ticket, 0,
                                      (size_t)d->B * d->Hkv * p.attn_rgb * 4, st);
@@ -557,6 +560,7 @@ cudaError_t launch_attention(const Plan& p, const isd_dims* d, const uint16_t* q
     a.page_table = page_table;
     a.kv_len = kv_len;
     a.n_clean = n_clean;
+    a.bidir = bidir ? 1 : 0;
     a.out = reinterpret_cast<__nv_bfloat16*>(out);
     a.part = w + p.off_attn_part;
     a.part_stride = p.attn_part_stride;

@@ -84,7 +84,7 @@ cudaError_t launch_attention(const Plan& p, const isd_dims* d, const uint16_t* q
                              uint16_t* v_pool, const int32_t* page_table, const int32_t* kv_len,
                              const int32_t* n_clean, uint16_t* out, void* ws, int32_t* err_flag,
                              cudaStream_t st, int* clear_extra, int* clear_range, int clear_count,
-                             bool pdl);
+                             bool pdl, bool bidir);
 void set_last_error(const char* msg);
 }  // namespace isd
 
@@ -146,7 +146,7 @@ extern "C" isd_status isd_attention_noalloc(const isd_dims* d, const uint16_t* q
     cudaStream_t st = static_cast<cudaStream_t>(stream);
     // launch_attention clears the counters on the stream before the attention
     if (isd::launch_attention(p, d, q, k_new, v_new, k_pool, v_pool, page_table, kv_len, n_clean,
-                              out, ws, err_flag, st, nullptr, nullptr, 0, false) != cudaSuccess) {
+                              out, ws, err_flag, st, nullptr, nullptr, 0, false, false) != cudaSuccess) {
         isd::set_last_error("isd_attention_noalloc: launch failed");
         return ISD_ERR_CUDA;
     }

@@ -68,7 +68,8 @@ struct TcArgs {
     float scale_log2;
     const int32_t* page_table;
     const int32_t* kv_len;
-    const int32_t* n_clean;
+    const int32_t* n_clean;  // null: every one of the N first slots is active (c = N)
+    int bidir;          // 1: every row sees the whole block (block-causal mask)
     __nv_bfloat16* out;
     float* part;        // [gridDim.x][2][part_stride] partial results
     int part_stride;    // floats per partial: R maxima, R sums, R x 128 O values
@@ -83,12 +84,15 @@ ISD_DEVINL int tc_slot_pos(int s, int kv, int c, int N) {
     return kv + c + (s - N);
 }
 
-// Keys of request b (prefix and active block rows); 0 for a request that
-// cannot be served (bad n_clean, negative or over-capacity length).
+ISD_DEVINL int tc_clean(const TcArgs& a, int b) { return a.n_clean ? a.n_clean[b] : a.N; }
+
+// Keys of request b (prefix and active block rows: c clean slots, then the
+// Q - N slots after them); 0 for a request that cannot be served (bad
+// n_clean, negative or over-capacity length).
 ISD_DEVINL int tc_total_keys(const TcArgs& a, int b) {
-    const int kv = a.kv_len[b], c = a.n_clean[b];
+    const int kv = a.kv_len[b], c = tc_clean(a, b);
     if (c < 1 || c > a.N || kv < 0) return 0;
-    const long long t = (long long)kv + c + a.N - 1;
+    const long long t = (long long)kv + c + a.Q - a.N;
     if ((t + a.P - 1) / a.P > a.max_pages) return 0;
     return (int)t;
 }
@@ -110,9 +114,9 @@ __global__ void kv_append_kernel(TcArgs a, const __nv_bfloat16* k_new, const __n
             for (int i = threadIdx.x; i < clear_count; i += blockDim.x) clear_range[i] = 0;
         for (int i = threadIdx.x; i < 2 * kMaxSMs; i += blockDim.x) a.part_flag[i] = 0;
     }
-    const int kv = a.kv_len[b], c = a.n_clean[b];
+    const int kv = a.kv_len[b], c = tc_clean(a, b);
     const bool bad_c = (c < 1 || c > a.N);
-    const long long want = bad_c ? 0 : (long long)kv + c + a.N - 1;
+    const long long want = bad_c ? 0 : (long long)kv + c + a.Q - a.N;
     const bool over = kv < 0 || (want + a.P - 1) / a.P > a.max_pages;
     if (r == 0) {
         for (int i = threadIdx.x; i < a.Hkv; i += blockDim.x) a.ticket[b * a.Hkv + i] = 0;
@@ -129,7 +133,7 @@ __global__ void kv_append_kernel(TcArgs a, const __nv_bfloat16* k_new, const __n
         }
         return;
     }
-    if (r >= c + a.N - 1) return;  // block positions: c clean slots, then N - 1 MASK slots
+    if (r >= c + a.Q - a.N) return;  // block positions: c clean slots, then the Q - N after them
     const int t = kv + r;
     const int slot = r < c ? r : a.N + (r - c);
     const int page = a.page_table[(size_t)b * a.max_pages + t / a.P];
@@ -297,7 +301,7 @@ attention_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_const
     pdl_wait();
     for (int b = threadIdx.x; b < a.B; b += kThreads) {
         kvs[b] = a.kv_len[b];
-        cs[b] = a.n_clean[b];
+        cs[b] = tc_clean(a, b);
         tots[b] = tc_total_keys(a, b);
     }
     __syncthreads();
@@ -655,7 +659,7 @@ attention_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_const
                 // the group); read after the next group barrier
                 if (et < R) {
                     const int pos = et < a.rows ? tc_slot_pos(et / a.grp, kv, c, a.N) : -1;
-                    lim[et] = min(pos, total - 1);
+                    lim[et] = (a.bidir && pos >= 0) ? total - 1 : min(pos, total - 1);
                 }
     #pragma unroll
                 for (int r = 0; r < RC; ++r) {
@@ -1003,7 +1007,7 @@ cudaError_t launch_attention_tc(const Plan& p, const isd_dims* d, const uint16_t
                                 uint16_t* v_pool, const int32_t* page_table, const int32_t* kv_len,
                                 const int32_t* n_clean, uint16_t* out, void* ws, int32_t* err_flag,
                                 cudaStream_t st, int* clear_extra, int* clear_range, int clear_count,
-                                bool pdl, bool* handled) {
+                                bool pdl, bool bidir, bool* handled) {
     *handled = false;
     const int R = p.attn_tc_rows;
     if (R == 0) return cudaSuccess;
@@ -1058,6 +1062,7 @@ cudaError_t launch_attention_tc(const Plan& p, const isd_dims* d, const uint16_t
     a.page_table = page_table;
     a.kv_len = kv_len;
     a.n_clean = n_clean;
+    a.bidir = bidir ? 1 : 0;
     a.out = reinterpret_cast<__nv_bfloat16*>(out);
     a.part = reinterpret_cast<float*>(static_cast<char*>(ws) + p.off_attn_part);
     a.part_stride = p.attn_tc_part_stride;
@@ -1066,7 +1071,7 @@ cudaError_t launch_attention_tc(const Plan& p, const isd_dims* d, const uint16_t
     a.part_flag = reinterpret_cast<int*>(a.part + (size_t)kMaxSMs * 2 * a.part_stride);
     a.err_flag = err_flag;
     const int append_threads = (Hkv * 16 + 31) / 32 * 32;
-    cudaError_t e = launch_kernel(pdl, kv_append_kernel, dim3(d->B, 2 * d->N - 1),
+    cudaError_t e = launch_kernel(pdl, kv_append_kernel, dim3(d->B, Q),
                                   dim3(append_threads > 1024 ? 1024 : append_threads), 0, st, a,
                                   reinterpret_cast<const __nv_bfloat16*>(k_new),
                                   reinterpret_cast<const __nv_bfloat16*>(v_new),

@@ -36,7 +36,7 @@ cudaError_t launch_attention(const Plan& p, const isd_dims* d, const uint16_t* q
                              uint16_t* v_pool, const int32_t* page_table, const int32_t* kv_len,
                              const int32_t* n_clean, uint16_t* out, void* ws, int32_t* err_flag,
                              cudaStream_t st, int* clear_extra, int* clear_range, int clear_count,
-                             bool pdl);
+                             bool pdl, bool bidir);
 cudaError_t launch_lm_head(const uint16_t* hidden, const uint16_t* W, int Mh, int H, int V,
                            float* logits, float4* stats_part, void* tail_ws, int32_t* err_flag,
                            cudaStream_t st, bool pdl, bool counters_cleared);
@@ -48,11 +48,18 @@ cudaError_t launch_lora(const Plan& p, const isd_dims* d, const uint16_t* hidden
                         void* ws, cudaStream_t st, bool pdl);
 cudaError_t launch_row_stats(const Plan& p, const float* logits, int rows, int V,
                              isd_row_stat* out, void* ws, cudaStream_t st);
-cudaError_t launch_prepare_block(const isd_dims* d, const uint16_t* Eq, const uint16_t* Ek,
+cudaError_t launch_prepare_block(const isd_dims* d, int Q, const uint16_t* Eq, const uint16_t* Ek,
                                  const uint16_t* Ev, const int32_t* n_clean, const int32_t* clean_tok,
-                                 const int32_t* kv_len, int32_t* page_table, int32_t* pages_used,
-                                 int32_t* next_free, uint16_t* q, uint16_t* k_new, uint16_t* v_new,
-                                 int32_t* err_flag, cudaStream_t st, bool pdl);
+                                 bool mask_neg, const float* rope, int rope_len,
+                                 const int32_t* kv_len, int32_t* page_table,
+                                 int32_t* pages_used, int32_t* next_free, uint16_t* q,
+                                 uint16_t* k_new, uint16_t* v_new, int32_t* err_flag,
+                                 cudaStream_t st, bool pdl);
+cudaError_t launch_sdar_unmask(const isd_dims* d, float tau, bool sync, const float4* stats_part,
+                               int n_parts, const isd_row_stat* stats_in, isd_row_stat* stats_out,
+                               int32_t* block_tok, int32_t* steps, int32_t* kv_len,
+                               int32_t* unmasked, int32_t* out_tok, int32_t* block_steps,
+                               int* counters, int32_t* err_flag, cudaStream_t st, bool pdl);
 cudaError_t launch_accept(const Plan& p, const isd_dims* d, const float* logits,
                           const isd_row_stat* stats, const float* prev_logits,
                           const isd_row_stat* prev_stats, const int32_t* n_clean,
@@ -148,8 +155,10 @@ isd_status do_attention(const isd_dims* d, const Plan& p, const uint16_t* q,
                         const uint16_t* k_new, const uint16_t* v_new, uint16_t* k_pool,
                         uint16_t* v_pool, const int32_t* page_table, const int32_t* kv_len,
                         const int32_t* n_clean, uint16_t* out, void* ws, int32_t* err_flag,
-                        cudaStream_t st, bool in_step = false) {
-    if (!q || !k_new || !v_new || !k_pool || !v_pool || !page_table || !kv_len || !n_clean || !out)
+                        cudaStream_t st, bool in_step = false, bool bidir = false) {
+    // n_clean may be null only for a block-causal (SDAR) block, whose N slots are all active
+    if (!q || !k_new || !v_new || !k_pool || !v_pool || !page_table || !kv_len ||
+        (!n_clean && !bidir) || !out)
         return invalid("null attention pointer");
     ISD_TRY(check_attention_shape(d, p));
     // The launch clears the attention counters on the stream; inside the whole
@@ -163,7 +172,7 @@ isd_status do_attention(const isd_dims* d, const Plan& p, const uint16_t* q,
     }
     ISD_CUDA(isd::launch_attention(p, d, q, k_new, v_new, k_pool, v_pool, page_table, kv_len,
                                    n_clean, out, ws, err_flag, st, acc_ticket, lm_ticket,
-                                   in_step ? isd::kMaxSMs : 0, in_step && kStepPdl));
+                                   in_step ? isd::kMaxSMs : 0, in_step && kStepPdl, bidir));
     return ISD_OK;
 }
 
@@ -377,9 +386,10 @@ isd_status isd_prepare_block(const isd_dims* d, const uint16_t* Eq, const uint16
     ISD_TRY(plan_or_fail(d, &p));
     ISD_TRY(check_prepare(d, Eq, Ek, Ev, n_clean, clean_tok, kv_len, page_table, pages_used,
                           next_free_page, q, k_new, v_new));
-    ISD_CUDA(isd::launch_prepare_block(d, Eq, Ek, Ev, n_clean, clean_tok, kv_len, page_table,
-                                       pages_used, next_free_page, q, k_new, v_new, err_flag,
-                                       static_cast<cudaStream_t>(stream), false));
+    ISD_CUDA(isd::launch_prepare_block(d, p.Q, Eq, Ek, Ev, n_clean, clean_tok, false, nullptr, 0,
+                                       kv_len,
+                                       page_table, pages_used, next_free_page, q, k_new, v_new,
+                                       err_flag, static_cast<cudaStream_t>(stream), false));
     return ISD_OK;
 }
 
@@ -400,9 +410,10 @@ isd_status isd_loop(const isd_dims* d, int32_t n_steps, const isd_loop_args* a, 
     for (int s = 0; s < n_steps; ++s) {
         const int cur = s & 1, nxt = cur ^ 1;
         ISD_CUDA(isd::launch_prepare_block(
-            d, a->Eq, a->Ek, a->Ev, a->n_clean + (size_t)cur * B, a->clean_tok + (size_t)cur * B * N,
-            a->kv_len + (size_t)cur * B, a->page_table, a->pages_used, a->next_free_page, a->q,
-            a->k_new, a->v_new, err_flag, st, kStepPdl));
+            d, p.Q, a->Eq, a->Ek, a->Ev, a->n_clean + (size_t)cur * B,
+            a->clean_tok + (size_t)cur * B * N, false, nullptr, 0, a->kv_len + (size_t)cur * B,
+            a->page_table,
+            a->pages_used, a->next_free_page, a->q, a->k_new, a->v_new, err_flag, st, kStepPdl));
         ISD_TRY(step_impl(
             d, p, a->q, a->k_new, a->v_new, a->k_pool, a->v_pool, a->page_table,
             a->kv_len + (size_t)cur * B, a->n_clean + (size_t)cur * B,
@@ -413,6 +424,115 @@ isd_status isd_loop(const isd_dims* d, int32_t n_steps, const isd_loop_args* a, 
             a->out_tok_hist + (size_t)s * B * N, a->n_clean + (size_t)nxt * B,
             a->clean_tok + (size_t)nxt * B * N, a->kv_len + (size_t)nxt * B, nullptr, ws, ws_bytes,
             err_flag, stream));
+    }
+    return ISD_OK;
+}
+
+}  // extern "C"
+
+// ---------------------------------------------------------------------------
+// SDAR-style confidence-threshold block decoding (the batch-synchronous
+// comparison workload): a block of N query rows with a block-causal mask, the
+// same LM head, and the unmask decision kernel (sdar.cu).
+// ---------------------------------------------------------------------------
+static isd_status check_sdar(const isd_dims* d, Plan* p, void* ws, size_t ws_bytes, float tau) {
+    if (!isd::make_plan(d, p, d ? d->N : 0)) return invalid("dims");
+    ISD_TRY(check_ws(*p, ws, ws_bytes));
+    if (d->N > isd::kSdarMaxN) return unsupported("SDAR block size N must be <= 16");
+    if (d->lora_rank) return unsupported("the SDAR workload has no LoRA adapter (lora_rank must be 0)");
+    if (!(tau == tau)) return invalid("tau is NaN");
+    return ISD_OK;
+}
+
+static isd_status sdar_step_impl(const isd_dims* d, const Plan& p, float tau, int32_t sync,
+                                 const uint16_t* q, const uint16_t* k_new, const uint16_t* v_new,
+                                 uint16_t* k_pool, uint16_t* v_pool, const int32_t* page_table,
+                                 int32_t* kv_len, const uint16_t* W, uint16_t* hidden,
+                                 float* logits, isd_row_stat* row_stats, int32_t* block_tok,
+                                 int32_t* steps, int32_t* unmasked, int32_t* out_tok,
+                                 int32_t* block_steps, void* ws, int32_t* err_flag,
+                                 cudaStream_t st) {
+    if (!W || !logits || !block_tok || !steps || !unmasked || !out_tok || !block_steps)
+        return invalid("null SDAR step pointer");
+    ISD_TRY(check_attention_shape(d, p));
+    ISD_TRY(check_lm_shape(d, p, nullptr, nullptr));
+    uint16_t* h = hidden ? hidden
+                         : reinterpret_cast<uint16_t*>(static_cast<char*>(ws) + p.off_hidden);
+    // KV append + block-causal attention; the append also clears the LM
+    // head's counters and the unmask kernel's two counters
+    ISD_TRY(do_attention(d, p, q, k_new, v_new, k_pool, v_pool, page_table, kv_len, nullptr, h,
+                         ws, err_flag, st, true, true));
+    float4* part = reinterpret_cast<float4*>(static_cast<char*>(ws) + p.off_lm_stats);
+    ISD_CUDA(isd::launch_lm_head(h, W, p.M, p.H, d->V, logits, part,
+                                 static_cast<char*>(ws) + p.off_lm_tail, err_flag, st, kStepPdl,
+                                 true));
+    int* counters = reinterpret_cast<int*>(static_cast<char*>(ws) + p.off_acc_ticket);
+    ISD_CUDA(isd::launch_sdar_unmask(d, tau, sync != 0, part, isd::lm_head_stat_parts(p.M, p.H, d->V),
+                                     nullptr, row_stats, block_tok, steps, kv_len, unmasked,
+                                     out_tok, block_steps, counters, err_flag, st, kStepPdl));
+    return ISD_OK;
+}
+
+extern "C" {
+
+isd_status isd_sdar_step(const isd_dims* d, float tau, int32_t sync, const uint16_t* q,
+                         const uint16_t* k_new, const uint16_t* v_new, uint16_t* k_pool,
+                         uint16_t* v_pool, const int32_t* page_table, int32_t* kv_len,
+                         const uint16_t* W, uint16_t* hidden, float* logits,
+                         isd_row_stat* row_stats, int32_t* block_tok, int32_t* steps,
+                         int32_t* unmasked, int32_t* out_tok, int32_t* block_steps, void* ws,
+                         size_t ws_bytes, int32_t* err_flag, void* stream) {
+    Plan p;
+    ISD_TRY(check_sdar(d, &p, ws, ws_bytes, tau));
+    return sdar_step_impl(d, p, tau, sync, q, k_new, v_new, k_pool, v_pool, page_table, kv_len, W,
+                          hidden, logits, row_stats, block_tok, steps, unmasked, out_tok,
+                          block_steps, ws, err_flag, static_cast<cudaStream_t>(stream));
+}
+
+isd_status isd_sdar_unmask(const isd_dims* d, float tau, int32_t sync,
+                           const isd_row_stat* row_stats, int32_t* block_tok, int32_t* steps,
+                           int32_t* kv_len, int32_t* unmasked, int32_t* out_tok,
+                           int32_t* block_steps, void* ws, size_t ws_bytes, int32_t* err_flag,
+                           void* stream) {
+    Plan p;
+    ISD_TRY(check_sdar(d, &p, ws, ws_bytes, tau));
+    if (!row_stats || !block_tok || !steps || !kv_len || !unmasked || !out_tok || !block_steps)
+        return invalid("null SDAR unmask pointer");
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    int* counters = reinterpret_cast<int*>(static_cast<char*>(ws) + p.off_acc_ticket);
+    ISD_CUDA(cudaMemsetAsync(counters, 0, (size_t)d->B * 2 * 4 + 4, st));
+    ISD_CUDA(isd::launch_sdar_unmask(d, tau, sync != 0, nullptr, 0, row_stats, nullptr, block_tok,
+                                     steps, kv_len, unmasked, out_tok, block_steps, counters,
+                                     err_flag, st, false));
+    return ISD_OK;
+}
+
+isd_status isd_sdar_loop(const isd_dims* d, float tau, int32_t sync, int32_t n_steps,
+                         const isd_sdar_loop_args* a, void* ws, size_t ws_bytes,
+                         int32_t* err_flag, void* stream) {
+    Plan p;
+    if (!a) return invalid("null SDAR loop arguments");
+    ISD_TRY(check_sdar(d, &p, ws, ws_bytes, tau));
+    if (n_steps < 0) return invalid("n_steps must be >= 0");
+    ISD_TRY(check_prepare(d, a->Eq, a->Ek, a->Ev, a->block_tok, a->block_tok, a->kv_len,
+                          a->page_table, a->pages_used, a->next_free_page, a->q, a->k_new,
+                          a->v_new));
+    if (!a->unmasked_hist || !a->out_tok_hist || !a->block_steps_hist || !a->steps)
+        return invalid("null SDAR loop pointer");
+    if (a->rope && (a->rope_positions < 1 || d->D % 16))
+        return invalid("rope needs rope_positions >= 1 and D % 16 == 0");
+    const int B = d->B, N = d->N;
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    for (int s = 0; s < n_steps; ++s) {
+        ISD_CUDA(isd::launch_prepare_block(d, p.Q, a->Eq, a->Ek, a->Ev, nullptr, a->block_tok, true,
+                                           a->rope, a->rope_positions, a->kv_len, a->page_table, a->pages_used,
+                                           a->next_free_page, a->q, a->k_new, a->v_new, err_flag,
+                                           st, kStepPdl));
+        ISD_TRY(sdar_step_impl(d, p, tau, sync, a->q, a->k_new, a->v_new, a->k_pool, a->v_pool,
+                               a->page_table, a->kv_len, a->W, a->hidden, a->logits, a->row_stats,
+                               a->block_tok, a->steps, a->unmasked_hist + (size_t)s * B,
+                               a->out_tok_hist + (size_t)s * B * N,
+                               a->block_steps_hist + (size_t)s * B, ws, err_flag, st));
     }
     return ISD_OK;
 }

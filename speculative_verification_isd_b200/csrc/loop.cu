@@ -33,8 +33,11 @@ struct PrepArgs {
     const uint16_t* Eq;  // [V+1, Hq, D]
     const uint16_t* Ek;  // [V+1, Hkv, D]
     const uint16_t* Ev;
-    const int32_t* n_clean;
+    const int32_t* n_clean;    // null: the N first slots are all clean slots (c = N)
     const int32_t* clean_tok;
+    int mask_neg;              // 1: a negative token is an uncommitted position (MASK row)
+    const float2* rope;        // [rope_len][D/2] (cos, sin), or null: no rotation
+    int rope_len;
     const int32_t* kv_len;
     int32_t* page_table;
     int32_t* pages_used;
@@ -47,6 +50,48 @@ struct PrepArgs {
 
 constexpr int kPrepThreads = 256;
 
+// Rotary embedding of one 8-pair piece of a head vector: lo holds elements
+// 8j..8j+7 of the first half, hi the same elements of the second half (pairs
+// (i, i + D/2)); each product and sum is rounded separately (no contraction),
+// then the result is rounded once to bf16.
+ISD_DEVINL void rope_rotate8(const uint4& lo, const uint4& hi, const float2* cs, uint4& olo,
+                             uint4& ohi) {
+    const __nv_bfloat162* l2 = reinterpret_cast<const __nv_bfloat162*>(&lo);
+    const __nv_bfloat162* h2 = reinterpret_cast<const __nv_bfloat162*>(&hi);
+    __nv_bfloat162* ol = reinterpret_cast<__nv_bfloat162*>(&olo);
+    __nv_bfloat162* oh = reinterpret_cast<__nv_bfloat162*>(&ohi);
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+        const float2 x = __bfloat1622float2(l2[e]), y = __bfloat1622float2(h2[e]);
+        const float2 c0 = __ldg(cs + 2 * e), c1 = __ldg(cs + 2 * e + 1);
+        const float xl0 = __fsub_rn(__fmul_rn(x.x, c0.x), __fmul_rn(y.x, c0.y));
+        const float yh0 = __fadd_rn(__fmul_rn(y.x, c0.x), __fmul_rn(x.x, c0.y));
+        const float xl1 = __fsub_rn(__fmul_rn(x.y, c1.x), __fmul_rn(y.y, c1.y));
+        const float yh1 = __fadd_rn(__fmul_rn(y.y, c1.x), __fmul_rn(x.y, c1.y));
+        ol[e] = __floats2bfloat162_rn(xl0, xl1);
+        oh[e] = __floats2bfloat162_rn(yh0, yh1);
+    }
+}
+
+// One table row (id) of nh heads -> dst, rotated by position pos when cs
+// (that position's table row) is given, else copied.
+ISD_DEVINL void prep_rows(const uint16_t* table, int id, int nh, int D, uint16_t* dst_row,
+                          const float2* cs) {
+    const uint4* src = reinterpret_cast<const uint4*>(table + (size_t)id * nh * D);
+    uint4* dst = reinterpret_cast<uint4*>(dst_row);
+    if (!cs) {
+        for (int i = threadIdx.x; i < nh * D / 8; i += kPrepThreads) dst[i] = __ldg(src + i);
+        return;
+    }
+    const int halves = D / 16;  // 16-byte pieces in half a head vector
+    for (int i = threadIdx.x; i < nh * halves; i += kPrepThreads) {
+        const int h = i / halves, j = i - h * halves;
+        const uint4* sh = src + (size_t)h * (D / 8);
+        uint4* dh = dst + (size_t)h * (D / 8);
+        rope_rotate8(__ldg(sh + j), __ldg(sh + j + halves), cs + 8 * j, dh[j], dh[j + halves]);
+    }
+}
+
 // grid (Q, B): block slot s of request b copies its table rows (16 bytes per
 // thread); CTA (0, 0) also extends every request's page list, in request
 // order, from the bump allocator.
@@ -54,31 +99,24 @@ __global__ void __launch_bounds__(kPrepThreads) prepare_block_kernel(const __gri
     pdl_trigger();
     pdl_wait();  // the state was written by the previous step's accept
     const int s = blockIdx.x, b = blockIdx.y;
-    const int c = a.n_clean[b];
+    const int c = a.n_clean ? a.n_clean[b] : a.N;
     int id = a.V;  // the MASK row
     if (s < a.N && s < c && c <= a.N) {
         const int t = a.clean_tok[(size_t)b * a.N + s];
         if (t >= 0 && t < a.V) id = t;
-        else if (threadIdx.x == 0) raise_flag(a.err_flag, ISD_FLAG_TOKEN_OOB);
+        else if (!(a.mask_neg && t < 0) && threadIdx.x == 0) raise_flag(a.err_flag, ISD_FLAG_TOKEN_OOB);
     }
     const size_t row = (size_t)b * a.Q + s;
-    {
-        const int n16 = a.Hq * a.D / 8;
-        const uint4* src = reinterpret_cast<const uint4*>(a.Eq + (size_t)id * a.Hq * a.D);
-        uint4* dst = reinterpret_cast<uint4*>(a.q + row * a.Hq * a.D);
-        for (int i = threadIdx.x; i < n16; i += kPrepThreads) dst[i] = __ldg(src + i);
+    // rotary embedding (the block of N rows at kv_len .. kv_len+N-1 only)
+    const float2* cs = nullptr;
+    if (a.rope) {
+        const int pos = max(a.kv_len[b], 0) + s;
+        if (pos < a.rope_len) cs = a.rope + (size_t)pos * (a.D / 2);
+        else if (threadIdx.x == 0) raise_flag(a.err_flag, ISD_FLAG_CAPACITY);
     }
-    {
-        const int n16 = a.Hkv * a.D / 8;
-        const uint4* sk = reinterpret_cast<const uint4*>(a.Ek + (size_t)id * a.Hkv * a.D);
-        const uint4* sv = reinterpret_cast<const uint4*>(a.Ev + (size_t)id * a.Hkv * a.D);
-        uint4* dk = reinterpret_cast<uint4*>(a.k_new + row * a.Hkv * a.D);
-        uint4* dv = reinterpret_cast<uint4*>(a.v_new + row * a.Hkv * a.D);
-        for (int i = threadIdx.x; i < n16; i += kPrepThreads) {
-            dk[i] = __ldg(sk + i);
-            dv[i] = __ldg(sv + i);
-        }
-    }
+    prep_rows(a.Eq, id, a.Hq, a.D, a.q + row * a.Hq * a.D, cs);
+    prep_rows(a.Ek, id, a.Hkv, a.D, a.k_new + row * a.Hkv * a.D, cs);
+    prep_rows(a.Ev, id, a.Hkv, a.D, a.v_new + row * a.Hkv * a.D, nullptr);
     if (s != 0 || b != 0) return;
     // page bookkeeping: request r needs ceil((kv_len + Q) / P) pages (at most
     // the table's width); new pages are handed out in request order
@@ -132,15 +170,20 @@ __global__ void __launch_bounds__(kPrepThreads) prepare_block_kernel(const __gri
     if (threadIdx.x == 0) *a.next_free = min(s_base, a.num_pages);
 }
 
-cudaError_t launch_prepare_block(const isd_dims* d, const uint16_t* Eq, const uint16_t* Ek,
+// Q: block slots per request (2N - 1 for an ISD block; N for an SDAR block,
+// whose tokens come with n_clean null and mask_neg set, and whose q and k
+// rows may be rotated by position: rope [rope_len][D/2] (cos, sin) or null).
+cudaError_t launch_prepare_block(const isd_dims* d, int Q, const uint16_t* Eq, const uint16_t* Ek,
                                  const uint16_t* Ev, const int32_t* n_clean, const int32_t* clean_tok,
-                                 const int32_t* kv_len, int32_t* page_table, int32_t* pages_used,
-                                 int32_t* next_free, uint16_t* q, uint16_t* k_new, uint16_t* v_new,
-                                 int32_t* err_flag, cudaStream_t st, bool pdl) {
+                                 bool mask_neg, const float* rope, int rope_len,
+                                 const int32_t* kv_len, int32_t* page_table,
+                                 int32_t* pages_used, int32_t* next_free, uint16_t* q,
+                                 uint16_t* k_new, uint16_t* v_new, int32_t* err_flag,
+                                 cudaStream_t st, bool pdl) {
     PrepArgs a;
     a.B = d->B;
     a.N = d->N;
-    a.Q = 2 * d->N - 1;
+    a.Q = Q;
     a.Hq = d->Hq;
     a.Hkv = d->Hkv;
     a.D = d->D;
@@ -153,6 +196,9 @@ cudaError_t launch_prepare_block(const isd_dims* d, const uint16_t* Eq, const ui
     a.Ev = Ev;
     a.n_clean = n_clean;
     a.clean_tok = clean_tok;
+    a.mask_neg = mask_neg ? 1 : 0;
+    a.rope = reinterpret_cast<const float2*>(rope);
+    a.rope_len = rope_len;
     a.kv_len = kv_len;
     a.page_table = page_table;
     a.pages_used = pages_used;

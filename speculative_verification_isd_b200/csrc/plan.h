@@ -21,6 +21,8 @@ constexpr int kAcceptThreads = 256;
 constexpr int kAcceptChunk = 2048;
 // accept CTAs resident per SM (launch bounds: 64 registers a thread)
 constexpr int kAcceptMinBlocks = 4;
+// SDAR block size limit (one warp per block row in the unmask kernel)
+constexpr int kSdarMaxN = 16;
 // Persistent kernels (attention, LM head) run one CTA per SM of the current
 // device, at most kMaxSMs (a B200 has 148); the workspace is sized for
 // kMaxSMs, and the split heuristics below aim at a B200-sized grid.
@@ -71,14 +73,15 @@ inline size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
 // place the persistent kernels take their grid size from.
 int persistent_grid();
 
-// Returns false if the dims are invalid.
-inline bool make_plan(const isd_dims* d, Plan* p) {
+// Returns false if the dims are invalid.  block_q: query rows per request;
+// 0 means the ISD block of 2N - 1 slots (an SDAR block has N).
+inline bool make_plan(const isd_dims* d, Plan* p, int block_q = 0) {
     if (!d || d->B < 1 || d->N < 1 || d->Hq < 1 || d->Hkv < 1 || d->D < 1 || d->V < 1 ||
         d->page_size < 1 || d->num_pages < 1 || d->max_pages_per_req < 1 || d->lora_rank < 0 ||
         d->Hq % d->Hkv != 0 ||
         (d->proposal_mode != ISD_PROPOSE_ARGMAX && d->proposal_mode != ISD_PROPOSE_SAMPLE))
         return false;
-    p->Q = 2 * d->N - 1;
+    p->Q = block_q > 0 ? block_q : 2 * d->N - 1;
     p->H = d->Hq * d->D;
     p->M = d->B * p->Q;
     p->grp = d->Hq / d->Hkv;

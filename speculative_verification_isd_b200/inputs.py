@@ -268,6 +268,19 @@ def embed_block(tables: Dict[str, np.ndarray], clean_tok: np.ndarray, n_clean: n
     return tables["Eq"][ids], tables["Ek"][ids], tables["Ev"][ids]
 
 
+def rope_table(n_pos: int, D: int, base: float = 1.0e6) -> np.ndarray:
+    """Rotary-embedding table [n_pos, D/2, 2] float32: (cos, sin) of
+    pos * base^(-2i/D) for pair i, taken in float64 and rounded once.
+
+    Qwen3 rotates q and k by position with base 1e6; the table model of the
+    SDAR-style closed loop does the same, so the N rows of a block, which
+    carry the same MASK embedding, differ by position as a real model's do."""
+    i = np.arange(D // 2, dtype=np.float64)
+    inv = base ** (-2.0 * i / D)
+    ang = np.arange(n_pos, dtype=np.float64)[:, None] * inv[None, :]
+    return np.stack([np.cos(ang), np.sin(ang)], axis=-1).astype(np.float32)
+
+
 def workload_bytes(cfg: IsdConfig, kv_len: np.ndarray) -> Dict[str, float]:
     """Algorithmic HBM bytes of one step (used for roofline figures)."""
     kv = float(np.sum(kv_len.astype(np.float64))) * cfg.Hkv * cfg.D * 2 * 2
@@ -288,5 +301,6 @@ def ceil_div(a: int, b: int) -> int:
 __all__ = [
     "philox4x32_10", "step_uniforms", "f32_to_bf16_bits", "bf16_bits_to_f32", "IsdConfig",
     "CONFIGS", "prefix_lengths", "page_layout", "make_step_inputs", "random_logits",
-    "make_embedding_tables", "embed_block", "workload_bytes", "lm_head_flops", "ceil_div",
+    "make_embedding_tables", "embed_block", "rope_table", "workload_bytes", "lm_head_flops",
+    "ceil_div",
 ]

@@ -37,7 +37,8 @@ PROPOSE_SAMPLE = 1
 
 EXPORTED = ("isd_workspace_bytes", "isd_status_string", "isd_last_error", "isd_attention",
             "isd_lm_head", "isd_row_stats", "isd_accept", "isd_step", "isd_prepare_block",
-            "isd_loop", "isd_attention_noalloc")
+            "isd_loop", "isd_attention_noalloc", "isd_sdar_step", "isd_sdar_unmask",
+            "isd_sdar_loop")
 NOALLOC_SCRATCH_BYTES = 32 * 1024 * 1024  # ISD_NOALLOC_SCRATCH_BYTES in include/isd.h
 
 
@@ -73,6 +74,19 @@ class LoopArgs(ctypes.Structure):
     """isd_loop_args (include/isd.h): device pointers, in declaration order."""
     _fields_ = [(n, ctypes.c_void_p) for n in LOOP_FIELDS]
 
+
+SDAR_LOOP_FIELDS = ("Eq", "Ek", "Ev", "W", "k_pool", "v_pool", "page_table", "pages_used",
+                    "next_free_page", "kv_len", "block_tok", "steps", "logits", "row_stats", "q",
+                    "k_new", "v_new", "hidden", "unmasked_hist", "out_tok_hist",
+                    "block_steps_hist")
+
+
+class SdarLoopArgs(ctypes.Structure):
+    """isd_sdar_loop_args (include/isd.h): device pointers, then the optional
+    rotary table and its length, in declaration order."""
+    _fields_ = [(n, ctypes.c_void_p) for n in SDAR_LOOP_FIELDS] + [
+        ("rope", ctypes.c_void_p), ("rope_positions", ctypes.c_int32)]
+
 _vp = ctypes.c_void_p
 _sz = ctypes.c_size_t
 _i32 = ctypes.c_int32
@@ -100,6 +114,14 @@ _lib.isd_loop.argtypes = [_dims_p, _i32, ctypes.POINTER(LoopArgs), _vp, _sz, _vp
 _lib.isd_loop.restype = _i32
 _lib.isd_attention_noalloc.argtypes = [_dims_p] + [_vp] * 9 + [_vp, _vp]
 _lib.isd_attention_noalloc.restype = _i32
+_f32 = ctypes.c_float
+_lib.isd_sdar_step.argtypes = [_dims_p, _f32, _i32] + [_vp] * 17 + [_sz, _vp, _vp]
+_lib.isd_sdar_step.restype = _i32
+_lib.isd_sdar_unmask.argtypes = [_dims_p, _f32, _i32] + [_vp] * 8 + [_sz, _vp, _vp]
+_lib.isd_sdar_unmask.restype = _i32
+_lib.isd_sdar_loop.argtypes = [_dims_p, _f32, _i32, _i32, ctypes.POINTER(SdarLoopArgs), _vp, _sz,
+                               _vp, _vp]
+_lib.isd_sdar_loop.restype = _i32
 
 
 class IsdError(RuntimeError):
@@ -353,3 +375,83 @@ def row_stats_view(rs: torch.Tensor):
     f = r.view(torch.float32) if r.dtype == torch.int32 else r
     i = r if r.dtype == torch.int32 else r.view(torch.int32)
     return f[:, 0], f[:, 1], i[:, 2]
+
+
+# ---------------------------------------------------------------------------
+# SDAR-style confidence-threshold block decoding (blocks of N rows, Q = N)
+# ---------------------------------------------------------------------------
+def sdar_step(d: Dims, tau: float, sync: bool, q, k_new, v_new, k_pool, v_pool, page_table,
+              kv_len, W, logits, block_tok, steps, unmasked, out_tok, block_steps, ws,
+              hidden=None, row_stats=None, err_flag=None, stream=None):
+    """isd_sdar_step: block-causal attention over the block's N rows, LM head,
+    confidence-threshold unmask (state block_tok / steps / kv_len in place)."""
+    B, N = d.B, d.N
+    M = B * N
+    kvrow = d.page_size * d.Hkv * d.D
+    _check(_lib.isd_sdar_step(
+        ctypes.byref(d), float(tau), int(bool(sync)), _ptr(q, _BF16, M * d.Hq * d.D, "q"),
+        _ptr(k_new, _BF16, M * d.Hkv * d.D, "k_new"), _ptr(v_new, _BF16, M * d.Hkv * d.D, "v_new"),
+        _ptr(k_pool, _BF16, d.num_pages * kvrow, "k_pool"),
+        _ptr(v_pool, _BF16, d.num_pages * kvrow, "v_pool"),
+        _ptr(page_table, torch.int32, B * d.max_pages_per_req, "page_table"),
+        _ptr(kv_len, torch.int32, B, "kv_len"), _ptr(W, _BF16, d.V * d.H, "W"),
+        _ptr(hidden, _BF16, M * d.H, "hidden"), _ptr(logits, torch.float32, M * d.V, "logits"),
+        _ptr(row_stats, (torch.int32, torch.float32), M * ROW_STAT_FIELDS, "row_stats"),
+        _ptr(block_tok, torch.int32, B * N, "block_tok"), _ptr(steps, torch.int32, B, "steps"),
+        _ptr(unmasked, torch.int32, B, "unmasked"), _ptr(out_tok, torch.int32, B * N, "out_tok"),
+        _ptr(block_steps, torch.int32, B, "block_steps"),
+        _ptr(ws, torch.uint8, None, "ws"), ws.numel(),
+        _ptr(err_flag, torch.int32, 1, "err_flag"), _stream(stream)))
+
+
+def sdar_unmask(d: Dims, tau: float, sync: bool, row_stats, block_tok, steps, kv_len, unmasked,
+                out_tok, block_steps, ws, err_flag=None, stream=None):
+    """isd_sdar_unmask: the decision alone on given row statistics [B*N]."""
+    B, N = d.B, d.N
+    _check(_lib.isd_sdar_unmask(
+        ctypes.byref(d), float(tau), int(bool(sync)),
+        _ptr(row_stats, (torch.int32, torch.float32), B * N * ROW_STAT_FIELDS, "row_stats"),
+        _ptr(block_tok, torch.int32, B * N, "block_tok"), _ptr(steps, torch.int32, B, "steps"),
+        _ptr(kv_len, torch.int32, B, "kv_len"), _ptr(unmasked, torch.int32, B, "unmasked"),
+        _ptr(out_tok, torch.int32, B * N, "out_tok"),
+        _ptr(block_steps, torch.int32, B, "block_steps"),
+        _ptr(ws, torch.uint8, None, "ws"), ws.numel(),
+        _ptr(err_flag, torch.int32, 1, "err_flag"), _stream(stream)))
+
+
+def sdar_loop_args(d: Dims, n_steps: int, rope=None, **t) -> SdarLoopArgs:
+    """Checked isd_sdar_loop_args from tensors named as its fields; rope:
+    optional float32 [positions, D/2, 2] rotary table."""
+    B, N = d.B, d.N
+    M = B * N
+    kvrow = d.page_size * d.Hkv * d.D
+    want = dict(
+        Eq=(_BF16, (d.V + 1) * d.Hq * d.D), Ek=(_BF16, (d.V + 1) * d.Hkv * d.D),
+        Ev=(_BF16, (d.V + 1) * d.Hkv * d.D), W=(_BF16, d.V * d.H),
+        k_pool=(_BF16, d.num_pages * kvrow), v_pool=(_BF16, d.num_pages * kvrow),
+        page_table=(torch.int32, B * d.max_pages_per_req), pages_used=(torch.int32, B),
+        next_free_page=(torch.int32, 1), kv_len=(torch.int32, B), block_tok=(torch.int32, B * N),
+        steps=(torch.int32, B), logits=(torch.float32, M * d.V),
+        row_stats=((torch.int32, torch.float32), M * ROW_STAT_FIELDS),
+        q=(_BF16, M * d.Hq * d.D), k_new=(_BF16, M * d.Hkv * d.D), v_new=(_BF16, M * d.Hkv * d.D),
+        hidden=(_BF16, M * d.H), unmasked_hist=(torch.int32, n_steps * B),
+        out_tok_hist=(torch.int32, n_steps * B * N), block_steps_hist=(torch.int32, n_steps * B))
+    vals = {}
+    for n in SDAR_LOOP_FIELDS:
+        dt, numel = want[n]
+        vals[n] = _ptr(t.get(n), dt, numel, n)
+    if rope is not None:
+        if rope.dim() != 3 or rope.shape[1:] != (d.D // 2, 2):
+            raise ValueError(f"rope must be [positions, {d.D // 2}, 2]")
+        vals["rope"] = _ptr(rope, torch.float32, None, "rope")
+        vals["rope_positions"] = int(rope.shape[0])
+    return SdarLoopArgs(**vals)
+
+
+def sdar_loop(d: Dims, tau: float, sync: bool, n_steps: int, ws, err_flag=None, stream=None,
+              args: Optional[SdarLoopArgs] = None, **tensors):
+    """isd_sdar_loop: n_steps forwards of an SDAR-style stationary batch on the device."""
+    a = args if args is not None else sdar_loop_args(d, n_steps, **tensors)
+    _check(_lib.isd_sdar_loop(ctypes.byref(d), float(tau), int(bool(sync)), int(n_steps),
+                              ctypes.byref(a), _ptr(ws, torch.uint8, None, "ws"), ws.numel(),
+                              _ptr(err_flag, torch.int32, 1, "err_flag"), _stream(stream)))

@@ -364,4 +364,137 @@ def loop_stats(al: np.ndarray, N: int, start: int, stop: int, c_start=None) -> D
                 accept_rate_by_position=[float(a / max(t, 1)) for a, t in zip(acc_pos, tests_pos)])
 
 
-__all__ = ["DeviceWorkload", "LoopWorkload", "loop_stats", "request_slice"]
+class SdarLoopWorkload:
+    """A stationary batch of SDAR-style confidence-threshold block decoding
+    (isd_sdar_loop) on the synthetic table model of ``LoopWorkload`` (per-token
+    q/k/v tables with a MASK row, a random LM head, random prefixes), with q
+    and k rotated by position (rope=True): under the block's bidirectional
+    mask, rows that carry the same MASK embedding would otherwise be
+    identical and be committed all at once or one by one.  Blocks of N
+    positions; tau and sync are arguments of ``run``.  The state (kv_len,
+    block_tok, steps, page bookkeeping) is updated in place."""
+
+    FIELDS = ("Eq", "Ek", "Ev", "W", "k_pool", "v_pool", "page_table", "pages_used",
+              "next_free_page", "kv_len", "block_tok", "steps", "logits", "row_stats", "q",
+              "k_new", "v_new", "hidden")
+    STATE = ("page_table", "pages_used", "next_free_page", "kv_len", "block_tok", "steps")
+
+    def __init__(self, isd, cfg: I.IsdConfig, capacity_steps: int, seed: int = 0,
+                 w_std: Optional[float] = None, qkv_std: Optional[float] = None,
+                 kv_std: Optional[float] = None, rope: bool = True):
+        self.isd, self.cfg, self.seed = isd, cfg, seed
+        B, N, V, P = cfg.B, cfg.N, cfg.V, cfg.page_size
+        w_std = cfg.w_std if w_std is None else w_std
+        qkv_std = cfg.qkv_std if qkv_std is None else qkv_std
+        kv_std = cfg.kv_std if kv_std is None else kv_std
+        self.w_std, self.qkv_std, self.kv_std = w_std, qkv_std, kv_std
+        kv0 = I.prefix_lengths(cfg, seed)
+        pre = (kv0.astype(np.int64) + P - 1) // P
+        # a block advances kv_len by N at most once per forward
+        max_pages = int((kv0.max() + (capacity_steps + 1) * N + P - 1) // P + 1)
+        num_pages = int(pre.sum()) + B * max_pages
+        table = np.full((B, max_pages), -1, np.int32)
+        nxt = 0
+        for b in range(B):
+            table[b, : pre[b]] = np.arange(nxt, nxt + pre[b], dtype=np.int32)
+            nxt += int(pre[b])
+        self.kv0 = kv0
+        self.capacity_steps = capacity_steps
+        self.dims = isd.make_dims(B, N, cfg.Hq, cfg.Hkv, cfg.D, V, P, num_pages, max_pages)
+        gen = torch.Generator(device="cuda")
+        gen.manual_seed(seed)
+        self.Eq = _randn_bf16((V + 1, cfg.Hq, cfg.D), qkv_std, gen)
+        self.Ek = _randn_bf16((V + 1, cfg.Hkv, cfg.D), qkv_std, gen)
+        self.Ev = _randn_bf16((V + 1, cfg.Hkv, cfg.D), qkv_std, gen)
+        self.W = _randn_bf16((V, cfg.H), w_std, gen)
+        self.k_pool = _randn_bf16((num_pages, P, cfg.Hkv, cfg.D), kv_std, gen)
+        self.v_pool = _randn_bf16((num_pages, P, cfg.Hkv, cfg.D), kv_std, gen)
+        dev = lambda x: torch.from_numpy(np.ascontiguousarray(x)).cuda()
+        self.page_table = dev(table)
+        self.pages_used = dev(pre.astype(np.int32))
+        self.next_free_page = dev(np.array([nxt], np.int32))
+        self.kv_len = dev(kv0.astype(np.int32))
+        self.block_tok = dev(np.full((B, N), -1, np.int32))
+        self.steps = dev(np.zeros(B, np.int32))
+        M = B * N
+        self.logits = torch.zeros(M * V, dtype=torch.float32, device="cuda")
+        self.row_stats = torch.zeros(M * 4, dtype=torch.int32, device="cuda")
+        self.q = torch.empty(M * cfg.Hq * cfg.D, dtype=torch.bfloat16, device="cuda")
+        self.k_new = torch.empty(M * cfg.Hkv * cfg.D, dtype=torch.bfloat16, device="cuda")
+        self.v_new = torch.empty(M * cfg.Hkv * cfg.D, dtype=torch.bfloat16, device="cuda")
+        self.hidden = torch.empty(M * cfg.H, dtype=torch.bfloat16, device="cuda")
+        self.unmasked_hist = torch.zeros(capacity_steps, B, dtype=torch.int32, device="cuda")
+        self.out_tok_hist = torch.zeros(capacity_steps, B, N, dtype=torch.int32, device="cuda")
+        self.block_steps_hist = torch.zeros(capacity_steps, B, dtype=torch.int32, device="cuda")
+        # rotary table for every position the run can reach
+        self.rope = dev(I.rope_table(max_pages * P, cfg.D)) if rope else None
+        self.ws = isd.alloc_workspace(self.dims)
+        self.err = torch.zeros(1, dtype=torch.int32, device="cuda")
+        self.done = 0
+        self._initial = {f: getattr(self, f).clone() for f in self.STATE}
+
+    def reset(self):
+        """Back to the state before the first forward (stream-ordered copies)."""
+        for f in self.STATE:
+            getattr(self, f).copy_(self._initial[f])
+        self.done = 0
+
+    def args(self, start: int, n: int):
+        """Checked isd_sdar_loop arguments for forwards start .. start+n-1."""
+        if start + n > self.capacity_steps:
+            raise ValueError("loop steps must stay within capacity")
+        t = {f: getattr(self, f) for f in self.FIELDS}
+        t["unmasked_hist"] = self.unmasked_hist[start:start + n]
+        t["out_tok_hist"] = self.out_tok_hist[start:start + n]
+        t["block_steps_hist"] = self.block_steps_hist[start:start + n]
+        return self.isd.sdar_loop_args(self.dims, n, rope=self.rope, **t)
+
+    def run(self, n: int, tau: float, sync: bool, stream=None, args=None):
+        """Enqueue the next n forwards."""
+        a = args if args is not None else self.args(self.done, n)
+        self.isd.sdar_loop(self.dims, tau, sync, n, self.ws, err_flag=self.err, stream=stream,
+                           args=a)
+        self.done += n
+
+    def stats(self, start: int, stop: int) -> Dict[str, float]:
+        """Block statistics of forwards start .. stop-1 (see ``sdar_round_stats``)."""
+        h = self.block_steps_hist[start:stop].cpu().numpy()
+        return sdar_round_stats(h, self.cfg.N)
+
+
+def sdar_round_stats(block_steps_hist: np.ndarray, N: int) -> Dict[str, float]:
+    """Forwards per block from a decision history block_steps_hist [steps, B]
+    (S_b of a block that left the batch at that step, else 0).
+
+    S_b counts the denoising forwards request b's block needed on its own;
+    every block also takes one store pass.  Under batch sync all blocks of a
+    round leave at the same step, so every step with leavers closes a round
+    of max_b S_b + 1 forwards; tokens per forward of a request are then
+    N / (E[max S_b] + 1) against N / (E[S_b] + 1) without the sync."""
+    h = np.asarray(block_steps_hist, np.int64)
+    rows = h[(h > 0).any(axis=1)]
+    if rows.size == 0:
+        return dict(blocks=0, rounds=0, mean_S=float("nan"), mean_max_S=float("nan"),
+                    tpf_free=float("nan"), tpf_sync=float("nan"), pmf=[])
+    s_b = rows[rows > 0]
+    mean_s = float(s_b.mean())
+    mean_max = float(rows.max(axis=1).mean())
+    pmf = np.bincount(s_b, minlength=N + 1)[1:N + 1] / s_b.size
+    return dict(blocks=int(s_b.size), rounds=int(rows.shape[0]), mean_S=mean_s,
+                mean_max_S=mean_max, tpf_free=N / (mean_s + 1.0), tpf_sync=N / (mean_max + 1.0),
+                pmf=[float(x) for x in pmf])
+
+
+def expected_max_of(pmf, B: int) -> float:
+    """E[max of B independent draws] of S with P(S = s) = pmf[s-1], from the
+    distribution function: P(max <= s) = F(s)^B."""
+    F = np.cumsum(np.asarray(pmf, np.float64))
+    if F.size == 0 or F[-1] <= 0:
+        return float("nan")
+    F = np.minimum(F / F[-1], 1.0)
+    lower = np.concatenate([[0.0], F[:-1]])
+    return float(np.sum(np.arange(1, F.size + 1) * (F ** B - lower ** B)))
+
+
+__all__ = ["DeviceWorkload", "LoopWorkload", "SdarLoopWorkload", "expected_max_of",
+           "loop_stats", "request_slice", "sdar_round_stats"]

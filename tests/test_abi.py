@@ -112,5 +112,36 @@ def test_binding_prototypes_match_header(isd):
                 assert a in (ctypes.c_void_p, ctypes.c_char_p) or hasattr(a, "_type_"), (name, p)
             elif p.startswith("size_t"):
                 assert a is ctypes.c_size_t, (name, p)
+            elif p.startswith("float"):
+                assert a is ctypes.c_float, (name, p)
             else:
                 assert a is ctypes.c_int32, (name, p)
+
+
+def test_sdar_host_validation(isd):
+    """The SDAR-style calls reject bad dims and pointers on the host."""
+    lib = isd.library()
+    fake = ctypes.c_void_p(1 << 20)   # never dereferenced: validation fails first
+    d = isd.make_dims(2, 4, 4, 1, 128, 512, 16, 10, 4)
+    need = isd.workspace_bytes(d)
+    p16 = [fake] * 16
+    ok = lambda dd, tau, args: lib.isd_sdar_step(ctypes.byref(dd), tau, 1, *args, fake, need,
+                                                 None, None)
+    assert ok(d, float("nan"), p16) == isd.ISD_ERR_INVALID_ARG
+    assert ok(d, 0.5, [None] + p16[1:]) == isd.ISD_ERR_INVALID_ARG        # q
+    assert ok(d, 0.5, p16[:7] + [None] + p16[8:]) == isd.ISD_ERR_INVALID_ARG  # W
+    d_lora = isd.make_dims(2, 4, 4, 1, 128, 512, 16, 10, 4, lora_rank=32)
+    st = lib.isd_sdar_step(ctypes.byref(d_lora), 0.5, 1, *p16, fake,
+                           isd.workspace_bytes(d_lora), None, None)
+    assert st == isd.ISD_ERR_UNSUPPORTED_SHAPE
+    d_wide = isd.make_dims(2, 17, 4, 1, 128, 512, 16, 10, 8)
+    st = lib.isd_sdar_unmask(ctypes.byref(d_wide), 0.5, 1, *[fake] * 7, fake,
+                             isd.workspace_bytes(d_wide), None, None)
+    assert st == isd.ISD_ERR_UNSUPPORTED_SHAPE
+    st = lib.isd_sdar_unmask(ctypes.byref(d), 0.5, 1, None, *[fake] * 6, fake, need, None, None)
+    assert st == isd.ISD_ERR_INVALID_ARG
+    # workspace too small
+    st = lib.isd_sdar_unmask(ctypes.byref(d), 0.5, 1, *[fake] * 7, fake, 256, None, None)
+    assert st == isd.ISD_ERR_WORKSPACE
+    st = lib.isd_sdar_loop(ctypes.byref(d), 0.5, 1, 4, None, fake, need, None, None)
+    assert st == isd.ISD_ERR_INVALID_ARG

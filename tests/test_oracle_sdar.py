@@ -161,20 +161,24 @@ def test_unmask_threshold_limits():
 
 
 def _scripted_batch(sync):
-    """Three requests, blocks of N = 3, tau = 0.5.  Step 0: every confidence
-    is high, so every first block completes in one forward.  Steps 1 and 2:
-    request 0's confidences stay low (one position per forward), requests 1
-    and 2 stay high."""
+    """Three requests, blocks of N = 3, tau = 0.5, six forwards.  Forward 0:
+    every confidence is high, so every first block completes in one forward
+    (forward 1 is their store pass).  From forward 2 on, request 0's second
+    block has low confidences until forward 4 (one position per forward);
+    requests 1 and 2 stay high."""
     N, tau = 3, 0.5
     hi, lo = 0.9, 0.1
     conf = [[[hi] * 3, [hi] * 3, [hi] * 3],
+            [[hi] * 3, [hi] * 3, [hi] * 3],
             [[lo, 0.2, 0.3], [hi] * 3, [hi] * 3],
-            [[lo, 0.3, 0.2], [hi] * 3, [hi] * 3]]
+            [[lo, 0.3, 0.2], [hi] * 3, [hi] * 3],
+            [[hi] * 3, [hi] * 3, [hi] * 3],
+            [[hi] * 3, [hi] * 3, [hi] * 3]]
     tok = np.full((3, N), -1)
     steps = np.zeros(3, np.int64)
     kv = np.array([10, 20, 30])
     hist = []
-    for t in range(3):
+    for t in range(6):
         cand = np.full((3, N), 40 + t) + np.arange(3)[:, None] * 100
         r = S.unmask_batch(tok, steps, kv, np.float32(conf[t]), cand, tau, sync)
         hist.append(r)
@@ -183,38 +187,43 @@ def _scripted_batch(sync):
 
 
 def test_unmask_batch_free_and_sync():
-    """R7 on the scripted batch: without sync requests 1 and 2 move on every
-    forward; with sync they wait for request 0's slow second block."""
+    """R3, R7 on the scripted batch: a complete block leaves after its store
+    pass; without sync requests 1 and 2 move on by themselves, with sync they
+    wait for request 0's slow second block."""
     free = _scripted_batch(False)
     sync = _scripted_batch(True)
-    # step 0: every block completes at once, with or without sync
-    assert list(free[0]["block_steps"]) == [1, 1, 1]
-    assert list(sync[0]["block_steps"]) == [1, 1, 1]
-    assert list(sync[0]["kv_len"]) == [13, 23, 33]
-    # step 1: request 0 commits only its most confident position (2)
-    assert list(free[1]["unmasked"]) == [1, 3, 3]
-    assert list(free[1]["block_tok"][0]) == [-1, -1, 41]
-    assert list(free[1]["block_tok"][1]) == [-1, -1, -1]  # left: a fresh block
-    assert list(free[1]["block_steps"]) == [0, 1, 1]
-    assert list(sync[1]["block_steps"]) == [0, 0, 0]      # all wait for request 0
-    assert list(sync[1]["kv_len"]) == [13, 23, 33]
-    assert list(sync[1]["block_tok"][0]) == [-1, -1, 41]
-    # step 2 under sync: requests 1 and 2 idle (nothing to unmask, no step
-    # counted), request 0 commits position 1; the batch still waits
-    assert list(sync[2]["unmasked"]) == [1, 0, 0]
-    assert list(sync[2]["block_steps"]) == [0, 0, 0]
-    assert list(sync[2]["steps"]) == [2, 1, 1]
-    assert list(sync[2]["block_tok"][0]) == [-1, 42, 41]
-    # free: request 0 still open, 1 and 2 completed another block
-    assert list(free[2]["kv_len"]) == [13, 29, 39]
-    # the tokens a block leaves with are its candidates at commit time
-    assert list(free[1]["out_tok"][1]) == [141, 141, 141]
-    assert list(free[1]["out_tok"][0]) == [-1, -1, -1]
+    for h in (free, sync):
+        # forward 0 completes every block, forward 1 stores them and they leave
+        assert list(h[0]["unmasked"]) == [3, 3, 3] and list(h[0]["block_steps"]) == [0, 0, 0]
+        assert list(h[1]["unmasked"]) == [0, 0, 0] and list(h[1]["block_steps"]) == [1, 1, 1]
+        assert list(h[1]["kv_len"]) == [13, 23, 33]
+        assert list(h[1]["out_tok"][2]) == [240, 240, 240]
+        # forward 2: request 0 commits only its most confident position (2)
+        assert list(h[2]["unmasked"]) == [1, 3, 3]
+        assert list(h[2]["block_tok"][0]) == [-1, -1, 42]
+    # forward 3: requests 1 and 2 store; free they leave, synced they wait
+    assert list(free[3]["block_steps"]) == [0, 1, 1]
+    assert list(free[3]["out_tok"][1]) == [142, 142, 142]
+    assert list(free[3]["out_tok"][0]) == [-1, -1, -1]
+    assert list(sync[3]["block_steps"]) == [0, 0, 0]
+    assert list(sync[3]["unmasked"]) == [1, 0, 0]
+    assert list(sync[3]["steps"]) == [2, 1, 1]
+    assert list(sync[3]["block_tok"][0]) == [-1, 43, 42]
+    # forward 4 completes request 0's block (S = 3); forward 5 is its store
+    # pass: synced, the whole batch leaves together
+    assert list(sync[4]["block_steps"]) == [0, 0, 0]
+    assert list(sync[5]["block_steps"]) == [3, 1, 1]
+    assert list(sync[5]["kv_len"]) == [16, 26, 36]
+    assert list(sync[5]["out_tok"][0]) == [44, 43, 42]
+    # free: requests 1 and 2 completed another block in forward 4 and left in 5
+    assert list(free[5]["block_steps"]) == [3, 1, 1]
+    assert list(free[5]["kv_len"]) == [16, 29, 39]
 
 
 def test_sync_round_costs_the_slowest_block():
-    """Under sync the round length (forwards between two commits of the
-    batch) equals the largest S_b of that round, and round_stats reports it."""
+    """Under sync the round length (forwards between two departures of the
+    batch) is the largest S_b of that round plus the store pass, and
+    round_stats reports it."""
     rng = np.random.default_rng(4)
     B, N, tau = 5, 4, 0.6
     tok = np.full((B, N), -1)
@@ -229,14 +238,14 @@ def test_sync_round_costs_the_slowest_block():
         hist.append(r["block_steps"])
         if (r["block_steps"] > 0).any():
             assert (r["block_steps"] > 0).all()
-            assert t - last == r["block_steps"].max()
+            assert t - last == r["block_steps"].max() + 1
             last = t
     rs = S.round_stats(np.stack(hist), N)
     h = np.stack(hist)
     done = h[(h > 0).any(axis=1)]
     assert rs["rounds"] == done.shape[0] and rs["blocks"] == done.size
     assert rs["mean_max_S"] == pytest.approx(done.max(axis=1).mean())
-    assert rs["tpf_sync"] == pytest.approx(N / done.max(axis=1).mean())
+    assert rs["tpf_sync"] == pytest.approx(N / (done.max(axis=1).mean() + 1))
     assert rs["mean_max_S"] >= rs["mean_S"]
 
 
@@ -285,3 +294,81 @@ def test_sdar_step_tiny_closed_loop():
         tok, steps, kv = r["block_tok"], r["steps"], r["kv_len"]
     assert emitted >= B
     assert np.all(kv >= np.array([3, 9]) + N)
+
+
+def test_product_round_stats_match_the_oracle():
+    """The product-side statistics the benchmark reports (workload.py) agree
+    with the oracle's on synchronous and free-running decision histories."""
+    from speculative_verification_isd_b200.workload import expected_max_of, sdar_round_stats
+    rng = np.random.default_rng(8)
+    B, N, tau = 6, 4, 0.55
+    for sync in (True, False):
+        tok = np.full((B, N), -1)
+        steps = np.zeros(B, np.int64)
+        kv = np.zeros(B, np.int64)
+        hist = []
+        for t in range(300):
+            r = S.unmask_batch(tok, steps, kv, rng.random((B, N)).astype(np.float32),
+                               rng.integers(0, 9, (B, N)), tau, sync)
+            tok, steps, kv = r["block_tok"], r["steps"], r["kv_len"]
+            hist.append(r["block_steps"])
+        h = np.stack(hist)
+        mine = sdar_round_stats(h, N)
+        ref = S.round_stats(h, N)
+        assert mine["blocks"] == ref["blocks"]
+        assert mine["mean_S"] == pytest.approx(ref["mean_S"], rel=1e-12)
+        assert mine["tpf_free"] == pytest.approx(ref["tpf_free"], rel=1e-12)
+        if sync:
+            assert mine["rounds"] == ref["rounds"]
+            assert mine["mean_max_S"] == pytest.approx(ref["mean_max_S"], rel=1e-12)
+            assert mine["tpf_sync"] == pytest.approx(ref["tpf_sync"], rel=1e-12)
+        assert sum(mine["pmf"]) == pytest.approx(1.0)
+    for pmf in ([0.1, 0.4, 0.3, 0.2], [0.0, 1.0], [0.7, 0.2, 0.1, 0.0, 0.0]):
+        for Bb in (1, 3, 32):
+            assert expected_max_of(pmf, Bb) == pytest.approx(S.expected_max(np.array(pmf), Bb),
+                                                             rel=1e-12)
+
+
+def test_rope_rotation_layout_and_invariants():
+    """The stand-in's rotary embedding: rotate-half pairing, the frequency
+    ladder base^(-2i/D), identity at position 0, and the relative-position
+    property that makes it a rotary embedding."""
+    from speculative_verification_isd_b200.inputs import rope_table
+    D = 4
+    tab = rope_table(64, D, base=1.0e6)
+    # unit vectors: e_0 pairs with e_2 at frequency 1, e_1 with e_3 at 1e-3
+    p = 5
+    r0 = O.bf16_to_f64(S.rope_rotate(bf([1.0, 0, 0, 0]), tab[p]))
+    assert np.allclose(r0, [math.cos(p), 0, math.sin(p), 0], atol=2 ** -8)
+    r1 = O.bf16_to_f64(S.rope_rotate(bf([0, 1.0, 0, 0]), tab[p]))
+    assert np.allclose(r1, [0, math.cos(p * 1e-3), 0, math.sin(p * 1e-3)], atol=2 ** -8)
+    r2 = O.bf16_to_f64(S.rope_rotate(bf([0, 0, 1.0, 0]), tab[p]))
+    assert np.allclose(r2, [-math.sin(p), 0, math.cos(p), 0], atol=2 ** -8)
+    # position 0 is the identity, bit for bit
+    rng = np.random.default_rng(0)
+    D = 128
+    tab = rope_table(4096, D)
+    x = bf(rng.standard_normal((3, D)))
+    assert np.array_equal(S.rope_rotate(x, tab[0]), x)
+    # norms kept (to bf16 rounding); q(p).k(p') depends on p - p' only
+    q, k = bf(rng.standard_normal(D)), bf(rng.standard_normal(D))
+    nq = np.linalg.norm(O.bf16_to_f64(q))
+    for pos in (1, 77, 4000):
+        assert np.linalg.norm(O.bf16_to_f64(S.rope_rotate(q, tab[pos]))) == pytest.approx(nq, rel=1e-2)
+    dots = []
+    for p0 in (0, 100, 2500):
+        qa = O.bf16_to_f64(S.rope_rotate(q, tab[p0 + 37]))
+        ka = O.bf16_to_f64(S.rope_rotate(k, tab[p0]))
+        dots.append(float(qa @ ka))
+    scale = nq * np.linalg.norm(O.bf16_to_f64(k))
+    assert max(dots) - min(dots) <= 2e-2 * scale
+    # a block embedded with the table: committed tokens and MASK rows, rotated by position
+    V = 50
+    tables = dict(Eq=bf(rng.standard_normal((V + 1, 2, D))), Ek=bf(rng.standard_normal((V + 1, 1, D))),
+                  Ev=bf(rng.standard_normal((V + 1, 1, D))))
+    tok = np.array([[-1, 7, -1]])
+    qq, kk, vv = S.embed_block(tables, tok, V, np.array([10]), tab)
+    assert np.array_equal(qq[0, 1], S.rope_rotate(tables["Eq"][7], tab[11]))
+    assert np.array_equal(kk[0, 2], S.rope_rotate(tables["Ek"][V], tab[12]))
+    assert np.array_equal(vv[0, 0], tables["Ev"][V])
+    assert not np.array_equal(qq[0, 0], qq[0, 2])   # MASK rows differ by position
