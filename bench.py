@@ -47,6 +47,8 @@ def parse_args():
                     help="seconds of the sustained leg; 0 skips it")
     ap.add_argument("--loop-steps", type=int, default=400,
                     help="timed steps of the closed-loop leg (isd_loop); 0 skips it")
+    ap.add_argument("--sdar-only", action="store_true",
+                    help="run only the SDAR-style comparison leg and print its object")
     ap.add_argument("--sdar-steps", type=int, default=400,
                     help="timed forwards of the SDAR-style comparison leg (isd_sdar_loop), "
                          "per scheduling mode; 0 skips it")
@@ -456,6 +458,16 @@ def sdar_leg(isd, cfg, R, K, bus, seed):
     return out
 
 
+def gpu_bus_id():
+    """PCI bus id of the current GPU, for the clock sampler (None if unknown)."""
+    import torch
+    try:
+        pr = torch.cuda.get_device_properties(torch.cuda.current_device())
+        return "%08X:%02X:00.0" % (int(getattr(pr, "pci_domain_id", 0)), int(pr.pci_bus_id))
+    except Exception:
+        return None
+
+
 def config_dict(cfg, world):
     return {"workload": cfg.name, "B": cfg.B, "N": cfg.N, "Q": cfg.Q, "V": cfg.V,
             "hidden": cfg.H, "heads": f"{cfg.Hq}q/{cfg.Hkv}kv x {cfg.D}",
@@ -536,6 +548,12 @@ def main():
     from speculative_verification_isd_b200.workload import DeviceWorkload
     cfg = I.CONFIGS[args.config]
     hbm, tf_burst, tf_sus, peak_src = measured_peaks()
+    if args.sdar_only:
+        out = sdar_leg(isd, cfg, R, max(args.sdar_steps, 1), gpu_bus_id(), RK.rank_seed(0, rank))
+        if rank == 0:
+            print(json.dumps({"sdar_comparison": out, "n_gpus": world}), flush=True)
+        R.close()
+        return 0
     # weak scaling: every rank runs its own batch of B requests (requests are
     # independent), so there is no collective on the data path
     if args.accept_rate is not None:
@@ -555,12 +573,7 @@ def main():
     for k in range(W):
         run_step(k)
     torch.cuda.synchronize()
-    bus = None
-    try:
-        pr = torch.cuda.get_device_properties(torch.cuda.current_device())
-        bus = "%08X:%02X:00.0" % (int(getattr(pr, "pci_domain_id", 0)), int(pr.pci_bus_id))
-    except Exception:
-        bus = None
+    bus = gpu_bus_id()
     clocks = ClockSampler(bus)
     clocks.start()
     time.sleep(0.3)
