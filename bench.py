@@ -47,6 +47,11 @@ def parse_args():
                     help="seconds of the sustained leg; 0 skips it")
     ap.add_argument("--loop-steps", type=int, default=400,
                     help="timed steps of the closed-loop leg (isd_loop); 0 skips it")
+    ap.add_argument("--deep-steps", type=int, default=30,
+                    help="timed steps per stride of the full-depth leg (36 layers); 0 skips it")
+    ap.add_argument("--deep-layers", type=int, default=36)
+    ap.add_argument("--deep-only", action="store_true",
+                    help="run only the full-depth leg and print its object")
     ap.add_argument("--sdar-only", action="store_true",
                     help="run only the SDAR-style comparison leg and print its object")
     ap.add_argument("--sdar-steps", type=int, default=400,
@@ -458,6 +463,69 @@ def sdar_leg(isd, cfg, R, K, bus, seed):
     return out
 
 
+QWEN3_8B_INTER = 12288
+
+
+def deep_leg(isd, cfg, R, K, bus, seed, n_layers, tpf=None):
+    """Full-depth leg: the whole step through n_layers Qwen3-8B-shaped decoder
+    layers (embed, layers, final norm, LM head, accept), random weights, at
+    the ISD stride N (Q = 2N-1 queries per request, every request with c = N)
+    and at N = 1 (autoregressive decoding: one query per request) on the same
+    weights and caches.  Memory-bound decoding makes the two forwards cost
+    about the same, so the speed-up over AR is about TPF; tpf (the closed
+    loop's tokens per forward) turns the two step times into that speed-up."""
+    import numpy as np
+    import torch
+    from speculative_verification_isd_b200.workload import DeepWorkload
+    W = 3
+    dw = DeepWorkload(isd, cfg, n_layers, QWEN3_8B_INTER, seed=seed, max_q=cfg.Q)
+    dw.view(1)
+    stream = torch.cuda.current_stream()
+    out = {"workload": f"{cfg.name} full depth ({n_layers} layers)", "layers": n_layers,
+           "hidden": dw.H, "intermediate": QWEN3_8B_INTER,
+           "weights": "random, N(0, 1/fan_in); bf16", "gemm": "cuBLASLt bf16 (fp32 accumulate)"}
+    weight_bytes = dw.weight_bytes()
+    kv_bytes = n_layers * float(np.sum(dw.kv0.astype(np.float64))) * cfg.Hkv * cfg.D * 2 * 2
+    times = {}
+    for N in (cfg.N, 1):
+        v = dw.views[N]
+        for _ in range(W):
+            dw.step(N)
+        torch.cuda.synchronize()
+        clocks = ClockSampler(bus)
+        clocks.start()
+        time.sleep(0.2)
+        R.barrier()
+        torch.cuda.synchronize()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        for _ in range(K):
+            dw.step(N)
+        e1.record(stream)
+        torch.cuda.synchronize()
+        R.barrier()
+        clk = clocks.stop()
+        ms = R.max(e0.elapsed_time(e1)) / K
+        times[N] = ms
+        M = cfg.B * (2 * N - 1)
+        logits = float(M) * cfg.V * 4
+        byts = weight_bytes + kv_bytes + logits
+        out["isd" if N > 1 else "ar"] = {
+            "N": N, "queries_per_request": 2 * N - 1, "steps": K, "ms_per_step": ms,
+            "steps_per_s": R.world / (ms / 1e3), "algorithmic_bytes": byts,
+            "achieved_gbs": byts / (ms / 1e3) / 1e9, "err_flags": int(v["err"].item()),
+            "clocks": clk}
+    out["forward_time_ratio_isd_over_ar"] = times[cfg.N] / times[1]
+    if tpf is not None:
+        out["tpf_closed_loop"] = tpf
+        out["speedup_over_ar"] = tpf * times[1] / times[cfg.N]
+        out["isd_tokens_per_s"] = R.world * cfg.B * tpf / (times[cfg.N] / 1e3)
+        out["ar_tokens_per_s"] = R.world * cfg.B / (times[1] / 1e3)
+    del dw
+    torch.cuda.empty_cache()
+    return out
+
+
 def gpu_bus_id():
     """PCI bus id of the current GPU, for the clock sampler (None if unknown)."""
     import torch
@@ -548,6 +616,13 @@ def main():
     from speculative_verification_isd_b200.workload import DeviceWorkload
     cfg = I.CONFIGS[args.config]
     hbm, tf_burst, tf_sus, peak_src = measured_peaks()
+    if args.deep_only:
+        out = deep_leg(isd, cfg, R, max(args.deep_steps, 1), gpu_bus_id(), RK.rank_seed(0, rank),
+                       args.deep_layers)
+        if rank == 0:
+            print(json.dumps({"full_depth": out, "n_gpus": world}), flush=True)
+        R.close()
+        return 0
     if args.sdar_only:
         out = sdar_leg(isd, cfg, R, max(args.sdar_steps, 1), gpu_bus_id(), RK.rank_seed(0, rank))
         if rank == 0:
@@ -720,6 +795,10 @@ def main():
     sdar_line = None
     if args.sdar_steps > 0:
         sdar_line = sdar_leg(isd, cfg, R, args.sdar_steps, bus, RK.rank_seed(0, rank))
+    deep_line = None
+    if args.deep_steps > 0:
+        deep_line = deep_leg(isd, cfg, R, args.deep_steps, bus, RK.rank_seed(0, rank),
+                             args.deep_layers, loop_line["tpf"] if loop_line else None)
 
     # ---------------- roofline of the dominant kernel (LM head)
     lm_bytes = float(cfg.V) * cfg.H * 2 + float(cfg.M) * cfg.H * 2 + float(cfg.M) * cfg.V * 4
@@ -759,6 +838,8 @@ def main():
         line["closed_loop"] = loop_line
     if sdar_line is not None:
         line["sdar_comparison"] = sdar_line
+    if deep_line is not None:
+        line["full_depth"] = deep_line
     if lora_alpha is not None:
         # step time with the adapter / without it (the pages report about 1.12)
         line["lora_alpha"] = lora_alpha

@@ -416,6 +416,71 @@ isd_status isd_sdar_loop(const isd_dims* d, float tau, int32_t sync, int32_t n_s
                          const isd_sdar_loop_args* a, void* ws, size_t ws_bytes,
                          int32_t* err_flag, void* stream);
 
+/*
+ * ---------------------------------------------------------------------------
+ * isd_layers -- the full-depth forward over the ISD block: the decoder stack
+ * that the single-layer step stands in for.  I-DLM keeps the AR model's stack
+ * and serving path ([EXP §推理：复用 AR 推理栈]; its 8B model is built from
+ * Qwen3-8B); the layer internals are not in the pages and follow the base
+ * model (Qwen3) decoder layer, over all 2N-1 slots of the block at once:
+ *   x += O(attn(RoPE(qk_norm(QKV(rmsnorm_in(x))))))
+ *   x += down(silu(gate(h)) * up(h)),  h = rmsnorm_post(x)
+ * then, if final_norm is given, out = rmsnorm_final(x) (the LM head's input).
+ *  - attention: isd_attention's slot layout, strict-causal mask and paged
+ *    K/V append, with each layer's own pools (one page table for all);
+ *  - q and k are RMS-normalised per head (q_norm, k_norm over D) and rotated
+ *    by the slot's position (clean slot s: kv_len + s; MASK slot m:
+ *    kv_len + c + m) with rope [rope_positions, D/2, 2] fp32 (cos, sin),
+ *    rotate-half pairs (i, i + D/2); a position past the table raises
+ *    ISD_FLAG_CAPACITY (the last row is used);
+ *  - RMSNorm: x / sqrt(mean(x^2) + eps) * w, statistics in fp32;
+ *  - rounding to bf16 at every norm output, every GEMM output (the O and
+ *    down projections add the residual first), q / k after norm + rotation,
+ *    the attention output and silu(gate) * up; fp32 in between.  The four
+ *    projections run on cuBLASLt (bf16, fp32 accumulation).
+ * Shapes: H = Hq * D (multiple of 8), D in {64, 128}; x, out [B*(2N-1), H]
+ * bf16 (x is the residual stream, in/out); layers: a HOST array of n_layers
+ * isd_layer, each holding device pointers: in_norm, post_norm [H]; w_qkv
+ * [(Hq + 2 Hkv) D, H] (q rows, then k, then v); q_norm, k_norm [D]; w_o
+ * [H, Hq D]; w_gate_up [2 inter, H] (gate rows first); w_down [H, inter];
+ * k_pool, v_pool [num_pages, page_size, Hkv, D].
+ * Workspace: isd_layers_workspace_bytes(d, inter) bytes, 256-aligned (the
+ * first isd_workspace_bytes(d) of it serve the attention).  The first call
+ * for a new GEMM shape queries cuBLASLt's heuristic on the host; make it
+ * before any stream capture.  Errors as for isd_attention.
+ */
+typedef struct {
+    const uint16_t* in_norm;
+    const uint16_t* w_qkv;
+    const uint16_t* q_norm;
+    const uint16_t* k_norm;
+    const uint16_t* w_o;
+    const uint16_t* post_norm;
+    const uint16_t* w_gate_up;
+    const uint16_t* w_down;
+    uint16_t* k_pool;
+    uint16_t* v_pool;
+} isd_layer;
+
+size_t isd_layers_workspace_bytes(const isd_dims* d, int32_t inter);
+
+/*
+ * isd_embed_block -- the block's input embeddings for isd_layers: slot s of
+ * request b takes row E[t] of the embedding table E [V+1, H] bf16 (row V =
+ * MASK) for an active clean slot (s < n_clean[b]; t = clean_tok[b][s]), the
+ * MASK row for inactive clean slots and every MASK slot.  x [B*(2N-1), H].
+ * A token outside [0, V) raises ISD_FLAG_TOKEN_OOB (the MASK row is used).
+ */
+isd_status isd_embed_block(const isd_dims* d, const uint16_t* E, const int32_t* n_clean,
+                           const int32_t* clean_tok, uint16_t* x, int32_t* err_flag,
+                           void* stream);
+
+isd_status isd_layers(const isd_dims* d, int32_t n_layers, int32_t inter, float eps,
+                      const isd_layer* layers, const float* rope, int32_t rope_positions,
+                      const uint16_t* final_norm, uint16_t* x, uint16_t* out,
+                      const int32_t* page_table, const int32_t* kv_len, const int32_t* n_clean,
+                      void* ws, size_t ws_bytes, int32_t* err_flag, void* stream);
+
 #ifdef __cplusplus
 }
 #endif

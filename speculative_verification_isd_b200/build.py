@@ -18,6 +18,8 @@ NVCC_FLAGS = [
     "-shared", "-Xcompiler", "-fPIC", "-Xcompiler", "-fvisibility=default",
     "--expt-relaxed-constexpr",
 ]
+# cuBLASLt serves the full-depth forward's dense projections
+LINK_FLAGS = ["-lcublasLt", "-Xlinker", "-rpath=/usr/local/cuda/lib64"]
 
 
 def sources():
@@ -39,7 +41,8 @@ def build(verbose: bool = False, force: bool = False) -> str:
         lib_t = os.path.getmtime(LIB)
         if all(os.path.getmtime(d) <= lib_t for d in deps):
             return LIB
-    cmd = [_nvcc(), *NVCC_FLAGS, "-I", os.path.join(ROOT, "include"), "-o", LIB + ".tmp", *srcs]
+    cmd = [_nvcc(), *NVCC_FLAGS, "-I", os.path.join(ROOT, "include"), "-o", LIB + ".tmp", *srcs,
+           *LINK_FLAGS]
     if verbose:
         cmd.insert(1, "-Xptxas=-v")
     res = subprocess.run(cmd, capture_output=True, text=True)

@@ -55,6 +55,18 @@ cudaError_t launch_prepare_block(const isd_dims* d, int Q, const uint16_t* Eq, c
                                  int32_t* pages_used, int32_t* next_free, uint16_t* q,
                                  uint16_t* k_new, uint16_t* v_new, int32_t* err_flag,
                                  cudaStream_t st, bool pdl);
+cudaError_t gemm_bf16(int M, int Nout, int K, const void* X, const void* W, void* Y, bool acc,
+                      void* lt_ws, size_t lt_ws_bytes, cudaStream_t st);
+cudaError_t launch_rmsnorm(const void* x, const void* w, void* y, int M, int H, float eps,
+                           cudaStream_t st);
+cudaError_t launch_qk_norm_rope(const isd_dims* d, int Q, const void* qkv, const void* q_norm,
+                                const void* k_norm, const float* rope, int rope_len,
+                                const int32_t* kv_len, const int32_t* n_clean, float eps, void* q,
+                                void* k, void* v, int32_t* err_flag, cudaStream_t st);
+cudaError_t launch_silu_mul(const void* gu, void* act, int M, int I, cudaStream_t st);
+cudaError_t launch_embed_block(const isd_dims* d, int Q, const void* E, const int32_t* n_clean,
+                               const int32_t* clean_tok, void* x, int32_t* err_flag,
+                               cudaStream_t st);
 cudaError_t launch_sdar_unmask(const isd_dims* d, float tau, bool sync, const float4* stats_part,
                                int n_parts, const isd_row_stat* stats_in, isd_row_stat* stats_out,
                                int32_t* block_tok, int32_t* steps, int32_t* kv_len,
@@ -534,6 +546,121 @@ isd_status isd_sdar_loop(const isd_dims* d, float tau, int32_t sync, int32_t n_s
                                a->out_tok_hist + (size_t)s * B * N,
                                a->block_steps_hist + (size_t)s * B, ws, err_flag, st));
     }
+    return ISD_OK;
+}
+
+}  // extern "C"
+
+// ---------------------------------------------------------------------------
+// Full-depth forward (deep.cu): the decoder stack over the ISD block.  Its
+// workspace is the step's (for the attention) followed by the stack's
+// activations and the cuBLASLt workspace.
+// ---------------------------------------------------------------------------
+namespace {
+constexpr size_t kLtWorkspace = 32u << 20;
+
+struct DeepPlan {
+    size_t off_qkv, off_q, off_k, off_v, off_attn, off_h, off_gu, off_act, off_lt, total;
+};
+
+bool make_deep_plan(const isd_dims* d, const Plan& p, int inter, DeepPlan* dp) {
+    if (inter < 8 || inter % 8) return false;
+    const size_t M = (size_t)p.M, D = (size_t)d->D;
+    size_t off = isd::align_up(p.total, 256);
+    auto take = [&](size_t bytes) {
+        const size_t o = off;
+        off = isd::align_up(off + bytes, 256);
+        return o;
+    };
+    dp->off_qkv = take(M * (d->Hq + 2 * d->Hkv) * D * 2);
+    dp->off_q = take(M * d->Hq * D * 2);
+    dp->off_k = take(M * d->Hkv * D * 2);
+    dp->off_v = take(M * d->Hkv * D * 2);
+    dp->off_attn = take(M * p.H * 2);
+    dp->off_h = take(M * p.H * 2);
+    dp->off_gu = take(M * 2 * (size_t)inter * 2);
+    dp->off_act = take(M * (size_t)inter * 2);
+    dp->off_lt = take(kLtWorkspace);
+    dp->total = off;
+    return true;
+}
+}  // namespace
+
+extern "C" {
+
+isd_status isd_embed_block(const isd_dims* d, const uint16_t* E, const int32_t* n_clean,
+                           const int32_t* clean_tok, uint16_t* x, int32_t* err_flag,
+                           void* stream) {
+    Plan p;
+    ISD_TRY(plan_or_fail(d, &p));
+    if (!E || !n_clean || !clean_tok || !x) return invalid("null embed-block pointer");
+    if (p.H % 8) return unsupported("hidden size must be a multiple of 8");
+    ISD_CUDA(isd::launch_embed_block(d, p.Q, E, n_clean, clean_tok, x, err_flag,
+                                     static_cast<cudaStream_t>(stream)));
+    return ISD_OK;
+}
+
+size_t isd_layers_workspace_bytes(const isd_dims* d, int32_t inter) {
+    Plan p;
+    DeepPlan dp;
+    if (!isd::make_plan(d, &p) || !make_deep_plan(d, p, inter, &dp)) return 0;
+    return dp.total;
+}
+
+isd_status isd_layers(const isd_dims* d, int32_t n_layers, int32_t inter, float eps,
+                      const isd_layer* layers, const float* rope, int32_t rope_positions,
+                      const uint16_t* final_norm, uint16_t* x, uint16_t* out,
+                      const int32_t* page_table, const int32_t* kv_len, const int32_t* n_clean,
+                      void* ws, size_t ws_bytes, int32_t* err_flag, void* stream) {
+    Plan p;
+    DeepPlan dp;
+    ISD_TRY(plan_or_fail(d, &p));
+    if (!make_deep_plan(d, p, inter, &dp)) return invalid("intermediate size must be a multiple of 8");
+    if (!ws || ws_bytes < dp.total || (reinterpret_cast<uintptr_t>(ws) & 255)) {
+        snprintf(g_last_error, sizeof(g_last_error),
+                 "workspace: need %zu bytes (isd_layers_workspace_bytes), 256-aligned", dp.total);
+        return ISD_ERR_WORKSPACE;
+    }
+    if (n_layers < 0) return invalid("n_layers must be >= 0");
+    if (!layers && n_layers) return invalid("null layer array");
+    if (!x || !rope || !page_table || !kv_len || !n_clean || (final_norm && !out))
+        return invalid("null isd_layers pointer");
+    if (rope_positions < 1) return invalid("rope_positions must be >= 1");
+    if (p.H % 8) return unsupported("hidden size must be a multiple of 8");
+    ISD_TRY(check_attention_shape(d, p));
+    for (int l = 0; l < n_layers; ++l) {
+        const isd_layer& L = layers[l];
+        if (!L.in_norm || !L.w_qkv || !L.q_norm || !L.k_norm || !L.w_o || !L.post_norm ||
+            !L.w_gate_up || !L.w_down || !L.k_pool || !L.v_pool)
+            return invalid("null pointer in a layer");
+    }
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    char* w = static_cast<char*>(ws);
+    void* qkv = w + dp.off_qkv;
+    uint16_t* q = reinterpret_cast<uint16_t*>(w + dp.off_q);
+    uint16_t* k = reinterpret_cast<uint16_t*>(w + dp.off_k);
+    uint16_t* v = reinterpret_cast<uint16_t*>(w + dp.off_v);
+    uint16_t* attn = reinterpret_cast<uint16_t*>(w + dp.off_attn);
+    void* h = w + dp.off_h;
+    void* gu = w + dp.off_gu;
+    void* act = w + dp.off_act;
+    void* lt = w + dp.off_lt;
+    const int M = p.M, H = p.H, qkv_cols = (d->Hq + 2 * d->Hkv) * d->D;
+    for (int l = 0; l < n_layers; ++l) {
+        const isd_layer& L = layers[l];
+        ISD_CUDA(isd::launch_rmsnorm(x, L.in_norm, h, M, H, eps, st));
+        ISD_CUDA(isd::gemm_bf16(M, qkv_cols, H, h, L.w_qkv, qkv, false, lt, kLtWorkspace, st));
+        ISD_CUDA(isd::launch_qk_norm_rope(d, p.Q, qkv, L.q_norm, L.k_norm, rope, rope_positions,
+                                          kv_len, n_clean, eps, q, k, v, err_flag, st));
+        ISD_TRY(do_attention(d, p, q, k, v, L.k_pool, L.v_pool, page_table, kv_len, n_clean, attn,
+                             ws, err_flag, st));
+        ISD_CUDA(isd::gemm_bf16(M, H, H, attn, L.w_o, x, true, lt, kLtWorkspace, st));
+        ISD_CUDA(isd::launch_rmsnorm(x, L.post_norm, h, M, H, eps, st));
+        ISD_CUDA(isd::gemm_bf16(M, 2 * inter, H, h, L.w_gate_up, gu, false, lt, kLtWorkspace, st));
+        ISD_CUDA(isd::launch_silu_mul(gu, act, M, inter, st));
+        ISD_CUDA(isd::gemm_bf16(M, H, inter, act, L.w_down, x, true, lt, kLtWorkspace, st));
+    }
+    if (final_norm) ISD_CUDA(isd::launch_rmsnorm(x, final_norm, out, M, H, eps, st));
     return ISD_OK;
 }
 

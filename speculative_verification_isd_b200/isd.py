@@ -38,7 +38,7 @@ PROPOSE_SAMPLE = 1
 EXPORTED = ("isd_workspace_bytes", "isd_status_string", "isd_last_error", "isd_attention",
             "isd_lm_head", "isd_row_stats", "isd_accept", "isd_step", "isd_prepare_block",
             "isd_loop", "isd_attention_noalloc", "isd_sdar_step", "isd_sdar_unmask",
-            "isd_sdar_loop")
+            "isd_sdar_loop", "isd_layers_workspace_bytes", "isd_layers", "isd_embed_block")
 NOALLOC_SCRATCH_BYTES = 32 * 1024 * 1024  # ISD_NOALLOC_SCRATCH_BYTES in include/isd.h
 
 
@@ -122,6 +122,24 @@ _lib.isd_sdar_unmask.restype = _i32
 _lib.isd_sdar_loop.argtypes = [_dims_p, _f32, _i32, _i32, ctypes.POINTER(SdarLoopArgs), _vp, _sz,
                                _vp, _vp]
 _lib.isd_sdar_loop.restype = _i32
+
+
+LAYER_FIELDS = ("in_norm", "w_qkv", "q_norm", "k_norm", "w_o", "post_norm", "w_gate_up",
+                "w_down", "k_pool", "v_pool")
+
+
+class Layer(ctypes.Structure):
+    """isd_layer (include/isd.h): one decoder layer's device pointers."""
+    _fields_ = [(n, ctypes.c_void_p) for n in LAYER_FIELDS]
+
+
+_lib.isd_layers_workspace_bytes.argtypes = [_dims_p, _i32]
+_lib.isd_layers_workspace_bytes.restype = _sz
+_lib.isd_layers.argtypes = [_dims_p, _i32, _i32, _f32, ctypes.POINTER(Layer), _vp, _i32] + \
+    [_vp] * 6 + [_vp, _sz, _vp, _vp]
+_lib.isd_layers.restype = _i32
+_lib.isd_embed_block.argtypes = [_dims_p] + [_vp] * 6
+_lib.isd_embed_block.restype = _i32
 
 
 class IsdError(RuntimeError):
@@ -455,3 +473,58 @@ def sdar_loop(d: Dims, tau: float, sync: bool, n_steps: int, ws, err_flag=None, 
     _check(_lib.isd_sdar_loop(ctypes.byref(d), float(tau), int(bool(sync)), int(n_steps),
                               ctypes.byref(a), _ptr(ws, torch.uint8, None, "ws"), ws.numel(),
                               _ptr(err_flag, torch.int32, 1, "err_flag"), _stream(stream)))
+
+
+# ---------------------------------------------------------------------------
+# Full-depth forward over the ISD block
+# ---------------------------------------------------------------------------
+def layers_workspace_bytes(d: Dims, inter: int) -> int:
+    return int(_lib.isd_layers_workspace_bytes(ctypes.byref(d), int(inter)))
+
+
+def alloc_layers_workspace(d: Dims, inter: int, device="cuda") -> torch.Tensor:
+    n = layers_workspace_bytes(d, inter)
+    if n == 0:
+        raise IsdError(ISD_ERR_INVALID_ARG)
+    return torch.empty(n, dtype=torch.uint8, device=device)
+
+
+def layer_array(d: Dims, inter: int, layers) -> ctypes.Array:
+    """Checked isd_layer array from dicts of tensors named as its fields."""
+    H, D = d.Hq * d.D, d.D
+    kvrow = d.page_size * d.Hkv * D
+    want = dict(in_norm=H, w_qkv=(d.Hq + 2 * d.Hkv) * D * H, q_norm=D, k_norm=D, w_o=H * d.Hq * D,
+                post_norm=H, w_gate_up=2 * inter * H, w_down=H * inter,
+                k_pool=d.num_pages * kvrow, v_pool=d.num_pages * kvrow)
+    arr = (Layer * max(len(layers), 1))()
+    for i, L in enumerate(layers):
+        for n in LAYER_FIELDS:
+            setattr(arr[i], n, _ptr(L[n], _BF16, want[n], f"layer {i} {n}"))
+    return arr
+
+
+def layers(d: Dims, inter: int, eps: float, layer_arr, n_layers: int, rope, x, page_table,
+           kv_len, n_clean, ws, final_norm=None, out=None, err_flag=None, stream=None):
+    """isd_layers: n_layers decoder layers over the block (x in/out), then
+    the final RMSNorm into out when final_norm is given."""
+    M, H = d.M, d.Hq * d.D
+    if rope.dim() != 3 or rope.shape[1:] != (d.D // 2, 2):
+        raise ValueError(f"rope must be [positions, {d.D // 2}, 2]")
+    _check(_lib.isd_layers(
+        ctypes.byref(d), int(n_layers), int(inter), float(eps), layer_arr,
+        _ptr(rope, torch.float32, None, "rope"), int(rope.shape[0]),
+        _ptr(final_norm, _BF16, H, "final_norm"), _ptr(x, _BF16, M * H, "x"),
+        _ptr(out, _BF16, M * H, "out"),
+        _ptr(page_table, torch.int32, d.B * d.max_pages_per_req, "page_table"),
+        _ptr(kv_len, torch.int32, d.B, "kv_len"), _ptr(n_clean, torch.int32, d.B, "n_clean"),
+        _ptr(ws, torch.uint8, None, "ws"), ws.numel(),
+        _ptr(err_flag, torch.int32, 1, "err_flag"), _stream(stream)))
+
+
+def embed_block(d: Dims, E, n_clean, clean_tok, x, err_flag=None, stream=None):
+    """isd_embed_block: the block's input rows from the embedding table E [V+1, H]."""
+    H = d.Hq * d.D
+    _check(_lib.isd_embed_block(
+        ctypes.byref(d), _ptr(E, _BF16, (d.V + 1) * H, "E"), _ptr(n_clean, torch.int32, d.B, "n_clean"),
+        _ptr(clean_tok, torch.int32, d.B * d.N, "clean_tok"), _ptr(x, _BF16, d.M * H, "x"),
+        _ptr(err_flag, torch.int32, 1, "err_flag"), _stream(stream)))

@@ -496,5 +496,122 @@ def expected_max_of(pmf, B: int) -> float:
     return float(np.sum(np.arange(1, F.size + 1) * (F ** B - lower ** B)))
 
 
-__all__ = ["DeviceWorkload", "LoopWorkload", "SdarLoopWorkload", "expected_max_of",
-           "loop_stats", "request_slice", "sdar_round_stats"]
+class DeepWorkload:
+    """A full-depth synthetic model over the ISD block, resident on the GPU:
+    n_layers Qwen3-style decoder layers (hidden Hq*D, GQA Hkv heads,
+    intermediate ``inter``) with random weights, an embedding table with a
+    MASK row, the final norm and the LM head, one paged K/V pool per layer
+    holding random prefixes, and one batch state (kv_len, n_clean, clean
+    tokens).  ``views`` gives other strides N over the same weights and
+    pools (N = 1 is autoregressive decoding: one query per request).
+
+    Projections are drawn N(0, 1/K) for K inputs, so each keeps the scale of
+    its input; norm weights 1 + N(0, 0.1^2); embeddings N(0, 1)."""
+
+    def __init__(self, isd, cfg: I.IsdConfig, n_layers: int, inter: int, seed: int = 0,
+                 n_clean: str = "full", eps: float = 1e-6, max_q: Optional[int] = None):
+        self.isd, self.cfg, self.n_layers, self.inter, self.eps = isd, cfg, n_layers, inter, eps
+        B, N, V, P, D = cfg.B, cfg.N, cfg.V, cfg.page_size, cfg.D
+        H = cfg.Hq * D
+        self.H = H
+        kv0 = I.prefix_lengths(cfg, seed)
+        max_q = max_q or cfg.Q
+        need = (kv0.astype(np.int64) + max_q + P - 1) // P
+        max_pages = int(need.max())
+        num_pages = int(need.sum())
+        table = np.full((B, max_pages), -1, np.int32)
+        off = 0
+        for b in range(B):
+            table[b, : need[b]] = np.arange(off, off + need[b], dtype=np.int32)
+            off += int(need[b])
+        self.kv0 = kv0
+        self.num_pages, self.max_pages = num_pages, max_pages
+        gen = torch.Generator(device="cuda")
+        gen.manual_seed(seed)
+        rn = lambda shape, std: _randn_bf16(shape, std, gen)
+        ones = lambda n: (1.0 + 0.1 * torch.randn(n, device="cuda", generator=gen)).to(torch.bfloat16)
+        qkv_rows = (cfg.Hq + 2 * cfg.Hkv) * D
+        self.layers = []
+        for _ in range(n_layers):
+            self.layers.append(dict(
+                in_norm=ones(H), w_qkv=rn((qkv_rows, H), H ** -0.5), q_norm=ones(D), k_norm=ones(D),
+                w_o=rn((H, cfg.Hq * D), (cfg.Hq * D) ** -0.5), post_norm=ones(H),
+                w_gate_up=rn((2 * inter, H), H ** -0.5), w_down=rn((H, inter), inter ** -0.5),
+                k_pool=rn((num_pages, P, cfg.Hkv, D), 1.0), v_pool=rn((num_pages, P, cfg.Hkv, D), 1.0)))
+        self.E = rn((V + 1, H), 1.0)
+        self.final_norm = ones(H)
+        self.W = rn((V, H), cfg.w_std)
+        self.rope = torch.from_numpy(I.rope_table(max_pages * P, D)).cuda()
+        self.page_table = torch.from_numpy(table).cuda()
+        self.views = {}
+        self.view(N, n_clean, seed)
+
+    def view(self, N: int, n_clean: str = "full", seed: int = 0):
+        """Buffers and state for stride N (Q = 2N-1) over the shared weights."""
+        if N in self.views:
+            return self.views[N]
+        cfg, isd = self.cfg, self.isd
+        B, V, P, D = cfg.B, cfg.V, cfg.page_size, cfg.D
+        Q = 2 * N - 1
+        d = isd.make_dims(B, N, cfg.Hq, cfg.Hkv, D, V, P, self.num_pages, self.max_pages)
+        M = B * Q
+        rng = np.random.default_rng([seed, 41, N])
+        nc = np.full(B, N, np.int32) if n_clean == "full" else np.ones(B, np.int32)
+        dev = lambda a: torch.from_numpy(np.ascontiguousarray(a)).cuda()
+        v = dict(dims=d, Q=Q, M=M,
+                 kv_len=dev(self.kv0.astype(np.int32)), n_clean=dev(nc),
+                 clean_tok=dev(rng.integers(0, V, (B, N)).astype(np.int32)),
+                 x=torch.empty(M * self.H, dtype=torch.bfloat16, device="cuda"),
+                 out=torch.empty(M * self.H, dtype=torch.bfloat16, device="cuda"),
+                 logits=torch.zeros(M * V, dtype=torch.float32, device="cuda"),
+                 prev_logits=torch.zeros(M * V, dtype=torch.float32, device="cuda"),
+                 row_stats=torch.zeros(M * 4, dtype=torch.int32, device="cuda"),
+                 prev_row_stats=torch.zeros(M * 4, dtype=torch.int32, device="cuda"),
+                 uniforms=dev(I.step_uniforms(seed, 0, B, N)),
+                 accept_len=torch.zeros(B, dtype=torch.int32, device="cuda"),
+                 out_tok=torch.zeros(B * N, dtype=torch.int32, device="cuda"),
+                 next_n_clean=torch.zeros(B, dtype=torch.int32, device="cuda"),
+                 next_clean_tok=torch.zeros(B * N, dtype=torch.int32, device="cuda"),
+                 next_kv_len=torch.zeros(B, dtype=torch.int32, device="cuda"),
+                 ws=isd.alloc_layers_workspace(d, self.inter),
+                 err=torch.zeros(1, dtype=torch.int32, device="cuda"))
+        v["layer_arr"] = isd.layer_array(d, self.inter, self.layers)
+        self.views[N] = v
+        return v
+
+    def forward(self, N: int, n_layers: Optional[int] = None, stream=None, embed: bool = True):
+        """Embeddings (unless embed=False: x as it stands), the first n_layers
+        layers (all by default), the final norm into out."""
+        v, isd = self.views[N], self.isd
+        d = v["dims"]
+        if embed:
+            isd.embed_block(d, self.E, v["n_clean"], v["clean_tok"], v["x"], err_flag=v["err"],
+                            stream=stream)
+        n = self.n_layers if n_layers is None else n_layers
+        isd.layers(d, self.inter, self.eps, v["layer_arr"], n, self.rope, v["x"], self.page_table,
+                   v["kv_len"], v["n_clean"], v["ws"], final_norm=self.final_norm, out=v["out"],
+                   err_flag=v["err"], stream=stream)
+
+    def step(self, N: int, stream=None):
+        """One whole step at stride N: the forward, the LM head with row
+        statistics, the p/q accept against the previous logits buffer (the
+        state is not advanced: repeated steps replay the same block)."""
+        v, isd = self.views[N], self.isd
+        d = v["dims"]
+        self.forward(N, stream=stream)
+        isd.lm_head(d, v["out"], self.W, v["logits"], v["row_stats"], v["ws"], err_flag=v["err"],
+                    stream=stream)
+        isd.accept(d, v["logits"], v["row_stats"], v["prev_logits"], v["prev_row_stats"],
+                   v["n_clean"], v["clean_tok"], v["kv_len"], v["uniforms"], v["accept_len"],
+                   v["out_tok"], v["next_n_clean"], v["next_clean_tok"], v["next_kv_len"], v["ws"],
+                   err_flag=v["err"], stream=stream)
+
+    def weight_bytes(self) -> float:
+        """Bytes of weights one step streams: every layer's projections and
+        norms, the LM head (embedding rows read are negligible)."""
+        per = sum(t.numel() * 2 for k, t in self.layers[0].items() if k not in ("k_pool", "v_pool"))
+        return float(per * self.n_layers + self.W.numel() * 2)
+
+
+__all__ = ["DeepWorkload", "DeviceWorkload", "LoopWorkload", "SdarLoopWorkload",
+           "expected_max_of", "loop_stats", "request_slice", "sdar_round_stats"]
