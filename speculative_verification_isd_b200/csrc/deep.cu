@@ -25,6 +25,8 @@
 #include <cuda_bf16.h>
 #include <stdio.h>
 
+#include <mutex>
+
 #include "common.cuh"
 #include "launch.h"
 #include "plan.h"
@@ -208,6 +210,7 @@ constexpr int kMaxGemmPlans = 64;
 GemmPlan g_plans[kMaxGemmPlans];
 int g_nplans = 0;
 cublasLtHandle_t g_lt[64];
+std::mutex g_plan_mutex;  // the handle and plan caches are shared by all host threads
 
 cublasLtHandle_t lt_handle(int dev) {
     if (dev < 0 || dev >= 64) return nullptr;
@@ -216,12 +219,13 @@ cublasLtHandle_t lt_handle(int dev) {
 }
 
 const GemmPlan* gemm_plan(int dev, int M, int Nout, int K, bool acc, size_t ws) {
+    std::lock_guard<std::mutex> lock(g_plan_mutex);
     for (int i = 0; i < g_nplans; ++i) {
         const GemmPlan& p = g_plans[i];
         if (p.dev == dev && p.M == M && p.Nout == Nout && p.K == K && p.acc == (int)acc && p.ws == ws)
             return &p;
     }
-    if (g_nplans == kMaxGemmPlans) return nullptr;
+    if (g_nplans == kMaxGemmPlans) return nullptr;  // more shapes than the cache holds
     cublasLtHandle_t h = lt_handle(dev);
     if (!h) return nullptr;
     GemmPlan p{dev, M, Nout, K, (int)acc, ws};
@@ -255,11 +259,16 @@ cudaError_t gemm_bf16(int M, int Nout, int K, const void* X, const void* W, void
     cudaGetDevice(&dev);
     const GemmPlan* p = gemm_plan(dev, M, Nout, K, acc, lt_ws_bytes);
     if (!p) {
-        set_error_detail("cuBLASLt: no bf16 GEMM for this shape");
+        set_error_detail("cuBLASLt: no bf16 GEMM plan for this shape (no algorithm, or 64 shapes cached)");
         return cudaErrorNotSupported;
     }
+    cublasLtHandle_t h;
+    {
+        std::lock_guard<std::mutex> lock(g_plan_mutex);
+        h = g_lt[dev];
+    }
     const float alpha = 1.f, beta = acc ? 1.f : 0.f;
-    const cublasStatus_t s = cublasLtMatmul(lt_handle(dev), p->op, &alpha, W, p->a, X, p->b, &beta,
+    const cublasStatus_t s = cublasLtMatmul(h, p->op, &alpha, W, p->a, X, p->b, &beta,
                                             Y, p->c, Y, p->c, &p->algo, lt_ws, lt_ws_bytes, st);
     if (s != CUBLAS_STATUS_SUCCESS) {
         char msg[96];

@@ -145,3 +145,38 @@ def test_sdar_host_validation(isd):
     assert st == isd.ISD_ERR_WORKSPACE
     st = lib.isd_sdar_loop(ctypes.byref(d), 0.5, 1, 4, None, fake, need, None, None)
     assert st == isd.ISD_ERR_INVALID_ARG
+
+
+def test_full_depth_host_validation(isd):
+    """isd_layers / isd_embed_block reject bad sizes and pointers on the host."""
+    lib = isd.library()
+    fake = ctypes.c_void_p(1 << 20)   # never dereferenced: validation fails first
+    d = isd.make_dims(2, 4, 4, 2, 64, 500, 16, 10, 4)
+    assert isd.layers_workspace_bytes(d, 96) > isd.workspace_bytes(d)
+    assert isd.layers_workspace_bytes(d, 100) == 0          # intermediate not a multiple of 8
+    assert isd.layers_workspace_bytes(isd.make_dims(2, 0, 4, 2, 64, 500, 16, 10, 4), 96) == 0
+    need = isd.layers_workspace_bytes(d, 96)
+    arr = (isd.Layer * 1)()
+    for n in isd.LAYER_FIELDS:
+        setattr(arr[0], n, 1 << 20)
+    call = lambda **kw: lib.isd_layers(
+        ctypes.byref(kw.get("d", d)), kw.get("n", 1), kw.get("inter", 96), 1e-6,
+        kw.get("layers", arr), kw.get("rope", fake), kw.get("rope_n", 64), None,
+        kw.get("x", fake), None, fake, fake, fake, kw.get("ws", fake), kw.get("ws_bytes", need),
+        None, None)
+    assert call(inter=100) == isd.ISD_ERR_INVALID_ARG
+    assert call(ws_bytes=need - 256) == isd.ISD_ERR_WORKSPACE
+    assert call(x=None) == isd.ISD_ERR_INVALID_ARG
+    assert call(rope=None) == isd.ISD_ERR_INVALID_ARG
+    assert call(rope_n=0) == isd.ISD_ERR_INVALID_ARG
+    assert call(n=-1) == isd.ISD_ERR_INVALID_ARG
+    assert call(layers=None) == isd.ISD_ERR_INVALID_ARG
+    bad = (isd.Layer * 1)()
+    for n in isd.LAYER_FIELDS:
+        setattr(bad[0], n, 1 << 20)
+    bad[0].w_down = None
+    assert call(layers=bad) == isd.ISD_ERR_INVALID_ARG
+    d96 = isd.make_dims(2, 4, 4, 2, 96, 500, 16, 10, 4)     # head dim the attention lacks
+    assert call(d=d96, ws_bytes=isd.layers_workspace_bytes(d96, 96)) == isd.ISD_ERR_UNSUPPORTED_SHAPE
+    assert lib.isd_embed_block(ctypes.byref(d), None, fake, fake, fake, None, None) == \
+        isd.ISD_ERR_INVALID_ARG

@@ -336,3 +336,29 @@ def test_sdar_loop_captured_in_cuda_graph(isd):
                             w.logits)):
         assert torch.equal(a, b)
     del g
+
+
+@pytest.mark.parametrize("case", ["b1_sync", "n1_block", "tau_above_one", "tau_zero"])
+def test_sdar_loop_edge_cases(isd, case):
+    """Degenerate batches and thresholds, one forward per call against the
+    oracle: a batch of one; blocks of one position (every forward commits it,
+    so a block costs 2 forwards with its store pass); tau above every
+    confidence (S_b = N: one position per forward); tau = 0 (S_b = 1)."""
+    B, N, tau = 4, 4, 0.3
+    if case == "b1_sync":
+        B = 1
+    elif case == "n1_block":
+        N = 1
+    elif case == "tau_above_one":
+        tau = 1.5
+    elif case == "tau_zero":
+        tau = 0.0
+    cfg = I.IsdConfig("sdar_edge", B=B, N=N, Hq=8, Hkv=2, D=128, V=700, page_size=16,
+                      prefix_lo=0, prefix_hi=200, w_std=0.5, qkv_std=0.5, kv_std=1.0)
+    hist, _ = _loop_stepwise(isd, cfg, 24, tau, True, seed=11)
+    left = hist[hist > 0]
+    assert left.size > 0
+    if case == "n1_block" or case == "tau_zero":
+        assert np.all(left == 1)
+    if case == "tau_above_one":
+        assert np.all(left == N)
