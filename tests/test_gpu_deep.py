@@ -34,6 +34,9 @@ DEEP = {
                              prefix_lo=1, prefix_hi=300, w_std=0.5), 2, 512),
     "deep_d128": (I.IsdConfig("deep_d128", B=3, N=4, Hq=8, Hkv=2, D=128, V=1000, page_size=16,
                               prefix_lo=1, prefix_hi=300, w_std=0.5), 2, 1024),
+    # a wide MLP (intermediate 8192 against hidden 1024), one layer
+    "deep_wide": (I.IsdConfig("deep_wide", B=3, N=4, Hq=8, Hkv=2, D=128, V=1000, page_size=16,
+                              prefix_lo=1, prefix_hi=300, w_std=0.5), 1, 8192),
 }
 
 
