@@ -294,7 +294,7 @@ accept_kernel(const __grid_constant__ AcceptArgs a) {
     const bool fused = a.stats_part != nullptr;
     int* req_state = a.ticket + a.B;
     int* decided = a.ticket + 2 * a.B;
-    __shared__ int s_state, s_last, s_bad, s_b, s_ok;
+    __shared__ int s_last, s_bad, s_b, s_ok;
     __shared__ float s_ratio[16];
     __shared__ isd_row_stat s_stats[32];  // the decided request's merged rows (Q <= 31)
     __shared__ int picked[16];            // N <= 16 (checked on the host); written by thread 0
