@@ -751,38 +751,65 @@ def main():
     # A step's inputs travel in one pinned host buffer (one host-to-device
     # copy), its integer results come back in one (one device-to-host copy);
     # the caller waits for each step's result before issuing the next step.
+    # Inputs are double-buffered, as a serving loop would keep them: while
+    # step k runs, step k+1's inputs go up on a copy stream (every step's
+    # copy is inside the timed region; the first is not overlapped).
     in_dev, out_dev, layout = wl.pack_io()
-    host_in = torch.empty(in_dev.numel(), dtype=torch.uint8, pin_memory=True)
-    host_in.copy_(in_dev)
+    in_devs = [in_dev, in_dev.clone()]
+    host_ins = [torch.empty(in_dev.numel(), dtype=torch.uint8, pin_memory=True) for _ in range(2)]
+    for h in host_ins:
+        h.copy_(in_dev)
     u_off, u_nb = next((o, nb) for n, o, nb in layout if n == "uniforms")
-    host_u = host_in[u_off:u_off + u_nb].view(torch.float32)
+    host_us = [h[u_off:u_off + u_nb].view(torch.float32) for h in host_ins]
     u_steps = wl.uniforms_all.cpu().reshape(wl.uniforms_all.shape[0], -1)
     host_out = torch.empty(out_dev.numel(), dtype=torch.int32, pin_memory=True)
     h2d = in_dev.numel()
     d2h = host_out.numel() * 4
     KE = min(args.e2e_steps, K)
-    call = isd.StepCall(d, wl.q, wl.k_new, wl.v_new, wl.k_pool, wl.v_pool, wl.page_table,
-                        wl.kv_len, wl.n_clean, wl.clean_tok, wl.W, wl.prev_logits,
-                        wl.prev_row_stats, wl.uniforms, wl.logits, wl.row_stats, wl.accept_len,
-                        wl.out_tok, wl.next_n_clean, wl.next_clean_tok, wl.next_kv_len, wl.ws,
-                        hidden=wl.hidden, ratio=wl.ratio, lora_A=wl.lora_A, lora_B=wl.lora_B,
-                        err_flag=wl.err, stream=stream)
 
-    def e2e_step(k):
-        host_u.copy_(u_steps[k % u_steps.shape[0]])  # this step's uniforms
-        in_dev.copy_(host_in, non_blocking=True)
-        call()
-        host_out.copy_(out_dev, non_blocking=True)
-        stream.synchronize()  # the caller needs this step's result before the next one
+    def step_call(buf):
+        v = {n: buf[o:o + nb].view(getattr(wl, n).dtype).view(getattr(wl, n).shape)
+             for n, o, nb in layout}
+        return isd.StepCall(d, v["q"], v["k_new"], v["v_new"], wl.k_pool, wl.v_pool,
+                            v["page_table"], v["kv_len"], v["n_clean"], v["clean_tok"], wl.W,
+                            wl.prev_logits, wl.prev_row_stats, v["uniforms"], wl.logits,
+                            wl.row_stats, wl.accept_len, wl.out_tok, wl.next_n_clean,
+                            wl.next_clean_tok, wl.next_kv_len, wl.ws, hidden=wl.hidden,
+                            ratio=wl.ratio, lora_A=wl.lora_A, lora_B=wl.lora_B,
+                            err_flag=wl.err, stream=stream)
 
-    for k in range(max(3, W)):
-        e2e_step(k)
+    calls = [step_call(b) for b in in_devs]
+    copy_stream = torch.cuda.Stream()
+    uploaded = [torch.cuda.Event(), torch.cuda.Event()]
+    consumed = [torch.cuda.Event(), torch.cuda.Event()]
+    for ev in consumed:
+        ev.record(stream)
+
+    def upload(k, slot):
+        host_us[slot].copy_(u_steps[k % u_steps.shape[0]])  # step k's uniforms
+        with torch.cuda.stream(copy_stream):
+            copy_stream.wait_event(consumed[slot])  # the step that last read this buffer is done
+            in_devs[slot].copy_(host_ins[slot], non_blocking=True)
+            uploaded[slot].record(copy_stream)
+
+    def e2e_run(n):
+        upload(0, 0)
+        for k in range(n):
+            s_ = k & 1
+            stream.wait_event(uploaded[s_])
+            calls[s_]()
+            consumed[s_].record(stream)
+            host_out.copy_(out_dev, non_blocking=True)
+            if k + 1 < n:
+                upload(k + 1, s_ ^ 1)
+            stream.synchronize()  # the caller needs this step's result before the next one
+
+    e2e_run(max(3, W))
     R.barrier()
     torch.cuda.synchronize()
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     e0.record(stream)
-    for k in range(KE):
-        e2e_step(k)
+    e2e_run(KE)
     e1.record(stream)
     torch.cuda.synchronize()
     R.barrier()
@@ -828,7 +855,9 @@ def main():
                           "stage_ms": {"attention": t_attn, "lm_head_and_row_stats": t_lm,
                                        "accept": t_acc}},
         "e2e": {"value": e2e_value, "unit": "ISD steps/s", "h2d_bytes_per_step": int(h2d),
-                "d2h_bytes_per_step": int(d2h), "steps": KE, "warmup": max(3, W)},
+                "d2h_bytes_per_step": int(d2h), "steps": KE, "warmup": max(3, W),
+                "inputs": "double-buffered: step k+1's copy runs on a copy stream during step k",
+                "result_read_each_step": True},
         "sustained": sustained,
         # KV append, attention, LM head, accept (+ 3 LoRA kernels)
         "gpu_launches": K * (4 + (3 if cfg.lora_rank else 0)),

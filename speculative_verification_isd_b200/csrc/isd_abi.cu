@@ -167,7 +167,8 @@ isd_status do_attention(const isd_dims* d, const Plan& p, const uint16_t* q,
                         const uint16_t* k_new, const uint16_t* v_new, uint16_t* k_pool,
                         uint16_t* v_pool, const int32_t* page_table, const int32_t* kv_len,
                         const int32_t* n_clean, uint16_t* out, void* ws, int32_t* err_flag,
-                        cudaStream_t st, bool in_step = false, bool bidir = false) {
+                        cudaStream_t st, bool in_step = false, bool bidir = false,
+                        bool pdl = false) {
     // n_clean may be null only for a block-causal (SDAR) block, whose N slots are all active
     if (!q || !k_new || !v_new || !k_pool || !v_pool || !page_table || !kv_len ||
         (!n_clean && !bidir) || !out)
@@ -184,7 +185,8 @@ isd_status do_attention(const isd_dims* d, const Plan& p, const uint16_t* q,
     }
     ISD_CUDA(isd::launch_attention(p, d, q, k_new, v_new, k_pool, v_pool, page_table, kv_len,
                                    n_clean, out, ws, err_flag, st, acc_ticket, lm_ticket,
-                                   in_step ? isd::kMaxSMs : 0, in_step && kStepPdl, bidir));
+                                   in_step ? isd::kMaxSMs : 0, (in_step || pdl) && kStepPdl,
+                                   bidir));
     return ISD_OK;
 }
 
@@ -652,8 +654,9 @@ isd_status isd_layers(const isd_dims* d, int32_t n_layers, int32_t inter, float 
         ISD_CUDA(isd::gemm_bf16(M, qkv_cols, H, h, L.w_qkv, qkv, false, lt, kLtWorkspace, st));
         ISD_CUDA(isd::launch_qk_norm_rope(d, p.Q, qkv, L.q_norm, L.k_norm, rope, rope_positions,
                                           kv_len, n_clean, eps, q, k, v, err_flag, st));
+        // programmatic dependent launch: the attention's set-up overlaps the K/V append
         ISD_TRY(do_attention(d, p, q, k, v, L.k_pool, L.v_pool, page_table, kv_len, n_clean, attn,
-                             ws, err_flag, st));
+                             ws, err_flag, st, false, false, true));
         ISD_CUDA(isd::gemm_bf16(M, H, H, attn, L.w_o, x, true, lt, kLtWorkspace, st));
         ISD_CUDA(isd::launch_rmsnorm(x, L.post_norm, h, M, H, eps, st));
         ISD_CUDA(isd::gemm_bf16(M, 2 * inter, H, h, L.w_gate_up, gu, false, lt, kLtWorkspace, st));
