@@ -404,7 +404,7 @@ def closed_loop(isd, cfg, R, K, bus, seed):
 SDAR_TAU = 1.1e-5
 
 
-def sdar_leg(isd, cfg, R, K, bus, seed):
+def sdar_leg(isd, cfg, R, K, bus, seed, hbm=None):
     """SDAR-style block decoding on the same batch shape, in both scheduling
     modes: batch-synchronous (a round ends when every request's block is
     complete and stored, so it costs max_b S_b + 1 forwards) and free-running
@@ -425,6 +425,7 @@ def sdar_leg(isd, cfg, R, K, bus, seed):
                               qkv_std=LOOP_QKV_STD, kv_std=LOOP_KV_STD)
         sw.run(W, SDAR_TAU, sync)
         torch.cuda.synchronize()
+        kv_start = float(sw.kv_len.float().sum().item())
         args = sw.args(W, K)
         clocks = ClockSampler(bus)
         clocks.start()
@@ -441,11 +442,22 @@ def sdar_leg(isd, cfg, R, K, bus, seed):
         ms = R.max(e0.elapsed_time(e1))
         st = sdar_round_stats(sw.block_steps_hist[W:W + K].cpu().numpy(), cfg.N)
         tokens = R.sum(st["blocks"] * cfg.N)
+        # algorithmic bytes of one forward: the LM head's W and logits, the
+        # block's K/V prefix reads (the mean of the window's first and last
+        # prefix totals) and the block rows
+        kv_mean = 0.5 * (kv_start + float(sw.kv_len.float().sum().item()))
+        M = cfg.B * cfg.N
+        fwd_bytes = (float(cfg.V) * cfg.H * 2 + float(M) * cfg.V * 4
+                     + (kv_mean + M) * cfg.Hkv * cfg.D * 2 * 2 + float(M) * cfg.H * 2 * 2)
         mode = {"forwards": K, "ms_per_forward": ms / K, "forwards_per_s": K * R.world / (ms / 1e3),
                 "tokens_per_s": tokens / (ms / 1e3), "blocks": st["blocks"],
                 "mean_S": st["mean_S"], "S_pmf": st["pmf"],
                 "tokens_per_forward_per_request": st["blocks"] * cfg.N / (K * cfg.B),
+                "algorithmic_bytes_per_forward": fwd_bytes,
+                "achieved_gbs": fwd_bytes / (ms / K / 1e3) / 1e9,
                 "err_flags": int(sw.err.item()), "gpu_launches": 5 * K, "clocks": clk}
+        if hbm:
+            mode["frac_of_hbm"] = mode["achieved_gbs"] / hbm
         if sync:
             # forwards per block with the sync over those without it
             mode.update(rounds=st["rounds"], mean_max_S=st["mean_max_S"],
@@ -466,7 +478,7 @@ def sdar_leg(isd, cfg, R, K, bus, seed):
 QWEN3_8B_INTER = 12288
 
 
-def deep_leg(isd, cfg, R, K, bus, seed, n_layers, tpf=None):
+def deep_leg(isd, cfg, R, K, bus, seed, n_layers, tpf=None, hbm=None):
     """Full-depth leg: the whole step through n_layers Qwen3-8B-shaped decoder
     layers (embed, layers, final norm, LM head, accept), random weights, at
     the ISD stride N (Q = 2N-1 queries per request, every request with c = N)
@@ -515,6 +527,8 @@ def deep_leg(isd, cfg, R, K, bus, seed, n_layers, tpf=None):
             "steps_per_s": R.world / (ms / 1e3), "algorithmic_bytes": byts,
             "achieved_gbs": byts / (ms / 1e3) / 1e9, "err_flags": int(v["err"].item()),
             "clocks": clk}
+        if hbm:
+            out["isd" if N > 1 else "ar"]["frac_of_hbm"] = byts / (ms / 1e3) / 1e9 / hbm
     out["forward_time_ratio_isd_over_ar"] = times[cfg.N] / times[1]
     if tpf is not None:
         out["tpf_closed_loop"] = tpf
@@ -618,13 +632,14 @@ def main():
     hbm, tf_burst, tf_sus, peak_src = measured_peaks()
     if args.deep_only:
         out = deep_leg(isd, cfg, R, max(args.deep_steps, 1), gpu_bus_id(), RK.rank_seed(0, rank),
-                       args.deep_layers)
+                       args.deep_layers, hbm=hbm)
         if rank == 0:
             print(json.dumps({"full_depth": out, "n_gpus": world}), flush=True)
         R.close()
         return 0
     if args.sdar_only:
-        out = sdar_leg(isd, cfg, R, max(args.sdar_steps, 1), gpu_bus_id(), RK.rank_seed(0, rank))
+        out = sdar_leg(isd, cfg, R, max(args.sdar_steps, 1), gpu_bus_id(), RK.rank_seed(0, rank),
+                       hbm)
         if rank == 0:
             print(json.dumps({"sdar_comparison": out, "n_gpus": world}), flush=True)
         R.close()
@@ -821,11 +836,11 @@ def main():
         loop_line = closed_loop(isd, cfg, R, args.loop_steps, bus, RK.rank_seed(0, rank))
     sdar_line = None
     if args.sdar_steps > 0:
-        sdar_line = sdar_leg(isd, cfg, R, args.sdar_steps, bus, RK.rank_seed(0, rank))
+        sdar_line = sdar_leg(isd, cfg, R, args.sdar_steps, bus, RK.rank_seed(0, rank), hbm)
     deep_line = None
     if args.deep_steps > 0:
         deep_line = deep_leg(isd, cfg, R, args.deep_steps, bus, RK.rank_seed(0, rank),
-                             args.deep_layers, loop_line["tpf"] if loop_line else None)
+                             args.deep_layers, loop_line["tpf"] if loop_line else None, hbm)
 
     # ---------------- roofline of the dominant kernel (LM head)
     lm_bytes = float(cfg.V) * cfg.H * 2 + float(cfg.M) * cfg.H * 2 + float(cfg.M) * cfg.V * 4
