@@ -388,6 +388,8 @@ def closed_loop(isd, cfg, R, K, bus, seed):
            "accept_rate": st["accept_rate"],
            "accept_rate_by_position": st["accept_rate_by_position"],
            "tpf_restart_model_at_measured_rate": restart_model_tpf(st["accept_rate"], cfg.N),
+           # compute per output token against AR: TPF^2 / (queries per forward)
+           "compute_efficiency_tpf2_over_q": st["tpf"] ** 2 / cfg.Q,
            "model": {"w_std": LOOP_W_STD, "qkv_std": LOOP_QKV_STD, "kv_std": LOOP_KV_STD},
            "mean_kv_len": {"start": float(lw.kv0.mean()), "end": kv_end},
            "gpu_launches": 5 * K, "err_flags": int(lw.err.item()), "clocks": clk,
@@ -453,6 +455,8 @@ def sdar_leg(isd, cfg, R, K, bus, seed, hbm=None):
                 "tokens_per_s": tokens / (ms / 1e3), "blocks": st["blocks"],
                 "mean_S": st["mean_S"], "S_pmf": st["pmf"],
                 "tokens_per_forward_per_request": st["blocks"] * cfg.N / (K * cfg.B),
+                # TPF^2 / (queries per forward), N queries a forward
+                "compute_efficiency_tpf2_over_q": (st["blocks"] * cfg.N / (K * cfg.B)) ** 2 / cfg.N,
                 "algorithmic_bytes_per_forward": fwd_bytes,
                 "achieved_gbs": fwd_bytes / (ms / K / 1e3) / 1e9,
                 "err_flags": int(sw.err.item()), "gpu_launches": 5 * K, "clocks": clk}
