@@ -40,7 +40,9 @@ def parse_args():
     ap.add_argument("--config", default="qwen3_8b_b32_n4")
     ap.add_argument("--accept-rate", type=float, default=None,
                     help="constructed per-proposal acceptance (default: the config's)")
-    ap.add_argument("--e2e-steps", type=int, default=200)
+    ap.add_argument("--e2e-steps", type=int, default=2000,
+                    help="timed steps of the end-to-end leg (at most --steps; the same count "
+                         "keeps both legs in the same clock regime under the power cap)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-budget-s", type=float, default=20.0)
     ap.add_argument("--sustained-s", type=float, default=2.5,
@@ -826,12 +828,16 @@ def main():
     e2e_run(max(3, W))
     R.barrier()
     torch.cuda.synchronize()
+    clocks_e2e = ClockSampler(bus)
+    clocks_e2e.start()
+    time.sleep(0.2)
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     e0.record(stream)
     e2e_run(KE)
     e1.record(stream)
     torch.cuda.synchronize()
     R.barrier()
+    clk_e2e = clocks_e2e.stop()
     e2e_ms = R.max(e0.elapsed_time(e1))
     e2e_value = KE * world / (e2e_ms / 1e3)
 
@@ -876,7 +882,7 @@ def main():
         "e2e": {"value": e2e_value, "unit": "ISD steps/s", "h2d_bytes_per_step": int(h2d),
                 "d2h_bytes_per_step": int(d2h), "steps": KE, "warmup": max(3, W),
                 "inputs": "double-buffered: step k+1's copy runs on a copy stream during step k",
-                "result_read_each_step": True},
+                "result_read_each_step": True, "clocks": clk_e2e},
         "sustained": sustained,
         # KV append, attention, LM head, accept (+ 3 LoRA kernels)
         "gpu_launches": K * (4 + (3 if cfg.lora_rank else 0)),
