@@ -416,8 +416,10 @@ def sdar_leg(isd, cfg, R, K, bus, seed, hbm=None):
     then K timed ones of isd_sdar_loop (five kernels per forward).  Tokens
     count the blocks that left the batch in the timed window."""
     import torch
+    from speculative_verification_isd_b200 import inputs as I
     from speculative_verification_isd_b200.workload import (SdarLoopWorkload, expected_max_of,
                                                             sdar_round_stats)
+    I_prefix = I.prefix_lengths
     W = 16
     stream = torch.cuda.current_stream()
     out = {"workload": cfg.name + " SDAR-style blocks", "block": cfg.N, "queries_per_forward": cfg.N,
@@ -471,6 +473,26 @@ def sdar_leg(isd, cfg, R, K, bus, seed, hbm=None):
         out["sync" if sync else "free"] = mode
         del sw
         torch.cuda.empty_cache()
+    # the synchronised batch at smaller batch sizes (same model, the first B
+    # requests' prefixes): measured E[max S_b] and tokens per forward
+    by_batch = {}
+    for Bs in (4, 8, 16):
+        cb = dataclasses.replace(cfg, B=Bs, fixed_prefix=tuple(int(x) for x in
+                                                                I_prefix(cfg, seed)[:Bs]))
+        sw = SdarLoopWorkload(isd, cb, capacity_steps=W + K, seed=seed, w_std=LOOP_W_STD,
+                              qkv_std=LOOP_QKV_STD, kv_std=LOOP_KV_STD)
+        sw.run(W + K, SDAR_TAU, True)
+        torch.cuda.synchronize()
+        st = sdar_round_stats(sw.block_steps_hist[W:W + K].cpu().numpy(), cfg.N)
+        by_batch[str(Bs)] = {"mean_S": st["mean_S"], "mean_max_S": st["mean_max_S"],
+                             "rounds": st["rounds"],
+                             "tokens_per_forward_per_request": st["blocks"] * cfg.N / (K * Bs),
+                             "err_flags": int(sw.err.item())}
+        del sw
+        torch.cuda.empty_cache()
+    by_batch[str(cfg.B)] = {k: out["sync"][k] for k in ("mean_S", "mean_max_S", "rounds",
+                                                       "tokens_per_forward_per_request")}
+    out["sync_measured_by_batch"] = by_batch
     # E[max S_b] over a batch of B requests, from the free-running S pmf (the
     # distribution of one request's block on its own), and the tokens per
     # forward of a request that a synchronised batch of B would leave
