@@ -184,3 +184,18 @@ def test_deep_step_runs_lm_head_and_accept(isd):
     assert np.all(np.abs(z - ref) <= bound)
     al = v["accept_len"].cpu().numpy()
     assert np.all((al >= 1) & (al <= cfg.N))
+
+
+def test_short_rope_table_raises_flag(isd):
+    """Positions past the rotary table are reported (ISD_FLAG_CAPACITY) and
+    use its last row; nothing faults."""
+    from speculative_verification_isd_b200.workload import DeepWorkload
+    cfg, _, inter = DEEP["deep_d128"]
+    w = DeepWorkload(isd, cfg, 1, inter, seed=8)
+    v = w.views[cfg.N]
+    short = w.rope[:4].contiguous()
+    isd.embed_block(v["dims"], w.E, v["n_clean"], v["clean_tok"], v["x"], err_flag=v["err"])
+    isd.layers(v["dims"], w.inter, w.eps, v["layer_arr"], 1, short, v["x"], w.page_table,
+               v["kv_len"], v["n_clean"], v["ws"], err_flag=v["err"])
+    torch.cuda.synchronize()
+    assert int(v["err"].item()) & isd.FLAG_CAPACITY

@@ -362,3 +362,23 @@ def test_sdar_loop_edge_cases(isd, case):
         assert np.all(left == 1)
     if case == "tau_above_one":
         assert np.all(left == N)
+
+
+def test_sdar_bad_token_raises_flag(isd):
+    """A committed block token outside [0, V) is reported through the error
+    flag (the block row takes the MASK embedding); nothing faults."""
+    from speculative_verification_isd_b200.workload import SdarLoopWorkload
+    cfg = I.IsdConfig("sdar_flag", B=3, N=4, Hq=8, Hkv=2, D=128, V=700, page_size=16,
+                      prefix_lo=0, prefix_hi=100, w_std=0.5, qkv_std=0.5, kv_std=1.0)
+    w = SdarLoopWorkload(isd, cfg, capacity_steps=2, seed=1)
+    w.block_tok[1, 2] = cfg.V + 5
+    w.run(1, 0.3, True)
+    torch.cuda.synchronize()
+    assert int(w.err.item()) & isd.FLAG_TOKEN_OOB
+    # the row was built from the MASK embedding
+    q = bf16_host(w.q).reshape(cfg.B, cfg.N, cfg.Hq * cfg.D)
+    Eq = bf16_host(w.Eq).reshape(cfg.V + 1, cfg.Hq, cfg.D)
+    want, _, _ = S.embed_block({"Eq": Eq, "Ek": Eq[:, :cfg.Hkv], "Ev": Eq[:, :cfg.Hkv]},
+                               np.array([[-1] * cfg.N]), cfg.V, np.array([int(w.kv0[1]) + 0]),
+                               w.rope.cpu().numpy())
+    assert np.array_equal(q[1, 2], want[0, 2].reshape(-1))
