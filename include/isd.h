@@ -446,8 +446,11 @@ isd_status isd_sdar_loop(const isd_dims* d, float tau, int32_t sync, int32_t n_s
  * k_pool, v_pool [num_pages, page_size, Hkv, D].
  * Workspace: isd_layers_workspace_bytes(d, inter) bytes, 256-aligned (the
  * first isd_workspace_bytes(d) of it serve the attention).  The first call
- * for a new GEMM shape queries cuBLASLt's heuristic on the host; make it
- * before any stream capture.  Errors as for isd_attention.
+ * for a new projection shape queries cuBLASLt's heuristic and times its
+ * best candidates on the call's stream (this synchronises that stream once;
+ * the fastest is kept for the process); make it before any stream capture
+ * (under capture, the heuristic's first choice is used).  Errors as for
+ * isd_attention.
  */
 typedef struct {
     const uint16_t* in_norm;

@@ -196,7 +196,11 @@ cudaError_t launch_embed_block(const isd_dims* d, int Q, const void* E, const in
 // ---------------------------------------------------------------------------
 // cuBLASLt: Y[M, Nout] (+)= X[M, K] . W[Nout, K]^T, bf16 in/out, fp32 compute.
 // Column-major view: Y^T (Nout x M) = W (op T) x X^T.  Descriptors and the
-// heuristic's algorithm are cached per shape; the handle per device.
+// algorithm are cached per shape, the handle per device.  The algorithm: on
+// the first call for a shape (outside stream capture), the heuristic's best
+// few candidates are each timed on the call's own operands, writing into a
+// scratch output, and the fastest is kept; under capture, the heuristic's
+// first choice.
 // ---------------------------------------------------------------------------
 namespace {
 struct GemmPlan {
@@ -218,7 +222,41 @@ cublasLtHandle_t lt_handle(int dev) {
     return g_lt[dev];
 }
 
-const GemmPlan* gemm_plan(int dev, int M, int Nout, int K, bool acc, size_t ws) {
+constexpr int kTuneCandidates = 8;
+
+// Mean time of `reps` runs of one candidate (ms), or a negative value if it fails.
+float time_algo(cublasLtHandle_t h, const GemmPlan& p, const cublasLtMatmulAlgo_t& algo,
+                const void* X, const void* W, void* scratch, void* lt_ws, size_t ws,
+                cudaStream_t st) {
+    const float alpha = 1.f, beta = 0.f;
+    auto run = [&]() {
+        return cublasLtMatmul(h, p.op, &alpha, W, p.a, X, p.b, &beta, scratch, p.c, scratch, p.c,
+                              &algo, lt_ws, ws, st);
+    };
+    if (run() != CUBLAS_STATUS_SUCCESS) return -1.f;
+    cudaEvent_t e0, e1;
+    if (cudaEventCreate(&e0) != cudaSuccess) return -1.f;
+    if (cudaEventCreate(&e1) != cudaSuccess) {
+        cudaEventDestroy(e0);
+        return -1.f;
+    }
+    constexpr int reps = 3;
+    float ms = -1.f;
+    bool ok = cudaEventRecord(e0, st) == cudaSuccess;
+    for (int r = 0; ok && r < reps; ++r) ok = run() == CUBLAS_STATUS_SUCCESS;
+    if (ok && cudaEventRecord(e1, st) == cudaSuccess && cudaEventSynchronize(e1) == cudaSuccess &&
+        cudaEventElapsedTime(&ms, e0, e1) == cudaSuccess)
+        ms /= reps;
+    else
+        ms = -1.f;
+    cudaEventDestroy(e0);
+    cudaEventDestroy(e1);
+    return ms;
+}
+
+const GemmPlan* gemm_plan(int dev, int M, int Nout, int K, bool acc, size_t ws, const void* X,
+                          const void* W, void* scratch, size_t scratch_bytes, void* lt_ws,
+                          cudaStream_t stream) {
     std::lock_guard<std::mutex> lock(g_plan_mutex);
     for (int i = 0; i < g_nplans; ++i) {
         const GemmPlan& p = g_plans[i];
@@ -241,23 +279,42 @@ const GemmPlan* gemm_plan(int dev, int M, int Nout, int K, bool acc, size_t ws) 
     cublasLtMatmulPreferenceCreate(&pref);
     cublasLtMatmulPreferenceSetAttribute(pref, CUBLASLT_MATMUL_PREF_MAX_WORKSPACE_BYTES, &ws,
                                          sizeof(ws));
-    cublasLtMatmulHeuristicResult_t res;
+    cublasLtMatmulHeuristicResult_t res[kTuneCandidates];
     int n = 0;
-    const cublasStatus_t st =
-        cublasLtMatmulAlgoGetHeuristic(h, p.op, p.a, p.b, p.c, p.c, pref, 1, &res, &n);
+    const cublasStatus_t st = cublasLtMatmulAlgoGetHeuristic(h, p.op, p.a, p.b, p.c, p.c, pref,
+                                                             kTuneCandidates, res, &n);
     cublasLtMatmulPreferenceDestroy(pref);
     if (st != CUBLAS_STATUS_SUCCESS || n < 1) return nullptr;
-    p.algo = res.algo;
+    p.algo = res[0].algo;
+    cudaStreamCaptureStatus cap = cudaStreamCaptureStatusNone;
+    const bool capturing = cudaStreamIsCapturing(stream, &cap) != cudaSuccess ||
+                           cap != cudaStreamCaptureStatusNone;
+    if (n > 1 && !capturing && scratch && scratch_bytes >= (size_t)M * Nout * 2) {
+        float best = -1.f;
+        for (int i = 0; i < n; ++i) {
+            if (res[i].state != CUBLAS_STATUS_SUCCESS || res[i].workspaceSize > ws) continue;
+            const float t = time_algo(h, p, res[i].algo, X, W, scratch, lt_ws, ws, stream);
+            if (t > 0.f && (best < 0.f || t < best)) {
+                best = t;
+                p.algo = res[i].algo;
+            }
+        }
+        cudaGetLastError();  // a failed candidate leaves no sticky error
+    }
     g_plans[g_nplans] = p;
     return &g_plans[g_nplans++];
 }
 }  // namespace
 
+// scratch: scratch_bytes of device memory the first call for a shape may
+// overwrite while it times the candidates (not an operand of this call).
 cudaError_t gemm_bf16(int M, int Nout, int K, const void* X, const void* W, void* Y, bool acc,
-                      void* lt_ws, size_t lt_ws_bytes, cudaStream_t st) {
+                      void* lt_ws, size_t lt_ws_bytes, void* scratch, size_t scratch_bytes,
+                      cudaStream_t st) {
     int dev = 0;
     cudaGetDevice(&dev);
-    const GemmPlan* p = gemm_plan(dev, M, Nout, K, acc, lt_ws_bytes);
+    const GemmPlan* p = gemm_plan(dev, M, Nout, K, acc, lt_ws_bytes, X, W, scratch, scratch_bytes,
+                                  lt_ws, st);
     if (!p) {
         set_error_detail("cuBLASLt: no bf16 GEMM plan for this shape (no algorithm, or 64 shapes cached)");
         return cudaErrorNotSupported;

@@ -1,7 +1,9 @@
 // C-ABI entry points of libisd.so (declared in include/isd.h): host-side
 // validation, workspace checks and the launch sequence of one ISD step.  No
 // entry point allocates, synchronises or reads device data on the host, so a
-// whole step can be captured into a CUDA graph.
+// whole step can be captured into a CUDA graph.  One exception: the first
+// isd_layers call for a new projection shape times cuBLASLt's candidate
+// algorithms on its stream (outside stream capture only).
 #include <cuda_runtime.h>
 #include <stdint.h>
 #include <stdio.h>
@@ -56,7 +58,8 @@ cudaError_t launch_prepare_block(const isd_dims* d, int Q, const uint16_t* Eq, c
                                  uint16_t* k_new, uint16_t* v_new, int32_t* err_flag,
                                  cudaStream_t st, bool pdl);
 cudaError_t gemm_bf16(int M, int Nout, int K, const void* X, const void* W, void* Y, bool acc,
-                      void* lt_ws, size_t lt_ws_bytes, cudaStream_t st);
+                      void* lt_ws, size_t lt_ws_bytes, void* scratch, size_t scratch_bytes,
+                      cudaStream_t st);
 cudaError_t launch_rmsnorm(const void* x, const void* w, void* y, int M, int H, float eps,
                            cudaStream_t st);
 cudaError_t launch_qk_norm_rope(const isd_dims* d, int Q, const void* qkv, const void* q_norm,
@@ -648,20 +651,26 @@ isd_status isd_layers(const isd_dims* d, int32_t n_layers, int32_t inter, float 
     void* act = w + dp.off_act;
     void* lt = w + dp.off_lt;
     const int M = p.M, H = p.H, qkv_cols = (d->Hq + 2 * d->Hkv) * d->D;
+    // the gate/up buffer is free whenever a projection is first tuned (the
+    // gate/up projection itself writes it anyway)
+    const size_t gu_bytes = (size_t)M * 2 * inter * 2;
+    auto gemm = [&](int Nout, int K, const void* X, const void* Wt, void* Y, bool acc) {
+        return isd::gemm_bf16(M, Nout, K, X, Wt, Y, acc, lt, kLtWorkspace, gu, gu_bytes, st);
+    };
     for (int l = 0; l < n_layers; ++l) {
         const isd_layer& L = layers[l];
         ISD_CUDA(isd::launch_rmsnorm(x, L.in_norm, h, M, H, eps, st));
-        ISD_CUDA(isd::gemm_bf16(M, qkv_cols, H, h, L.w_qkv, qkv, false, lt, kLtWorkspace, st));
+        ISD_CUDA(gemm(qkv_cols, H, h, L.w_qkv, qkv, false));
         ISD_CUDA(isd::launch_qk_norm_rope(d, p.Q, qkv, L.q_norm, L.k_norm, rope, rope_positions,
                                           kv_len, n_clean, eps, q, k, v, err_flag, st));
         // programmatic dependent launch: the attention's set-up overlaps the K/V append
         ISD_TRY(do_attention(d, p, q, k, v, L.k_pool, L.v_pool, page_table, kv_len, n_clean, attn,
                              ws, err_flag, st, false, false, true));
-        ISD_CUDA(isd::gemm_bf16(M, H, H, attn, L.w_o, x, true, lt, kLtWorkspace, st));
+        ISD_CUDA(gemm(H, H, attn, L.w_o, x, true));
         ISD_CUDA(isd::launch_rmsnorm(x, L.post_norm, h, M, H, eps, st));
-        ISD_CUDA(isd::gemm_bf16(M, 2 * inter, H, h, L.w_gate_up, gu, false, lt, kLtWorkspace, st));
+        ISD_CUDA(gemm(2 * inter, H, h, L.w_gate_up, gu, false));
         ISD_CUDA(isd::launch_silu_mul(gu, act, M, inter, st));
-        ISD_CUDA(isd::gemm_bf16(M, H, inter, act, L.w_down, x, true, lt, kLtWorkspace, st));
+        ISD_CUDA(gemm(H, inter, act, L.w_down, x, true));
     }
     if (final_norm) ISD_CUDA(isd::launch_rmsnorm(x, final_norm, out, M, H, eps, st));
     return ISD_OK;
