@@ -154,15 +154,18 @@ def test_layers_ar_stride_one(isd):
     _check_stack(isd, w, 1, np.ones(cfg.B, np.int32))
 
 
-def test_layers_full_size_sampled(isd):
+@pytest.mark.parametrize("N", [4, 1])
+def test_layers_full_size_sampled(isd, N):
     """Two layers at the Qwen3-8B shapes (H 4096, 32/8 heads of 128,
-    intermediate 12288) over the B=32, N=4 block; the oracle recomputes three
-    requests (rows are independent in every GEMM, requests in the attention)."""
+    intermediate 12288) over the B=32 block at stride N (N = 1: AR decoding);
+    the oracle recomputes three requests (rows are independent in every GEMM,
+    requests in the attention)."""
     from speculative_verification_isd_b200.workload import DeepWorkload
     cfg = I.CONFIGS["qwen3_8b_b32_n4"]
     w = DeepWorkload(isd, cfg, 2, 12288, seed=5)
-    worst = _check_stack(isd, w, cfg.N, np.full(cfg.B, cfg.N), requests=[0, 15, 31])
-    record_parity(f"deep stack qwen3_8b_b32_n4 2 layers sampled (max rel err {worst:.2e})",
+    w.view(N)
+    worst = _check_stack(isd, w, N, np.full(cfg.B, N), requests=[0, 15, 31])
+    record_parity(f"deep stack qwen3_8b_b32 N={N} 2 layers sampled (max rel err {worst:.2e})",
                   dict(requests=3, near_threshold=0, mismatches=0))
 
 

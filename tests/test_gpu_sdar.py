@@ -135,7 +135,8 @@ def test_sdar_step_layers(isd, name, sync):
                        committed=int(r_g["unmasked"].sum())))
 
 
-def test_sdar_full_size_sampled(isd):
+@pytest.mark.parametrize("sync", [True, False])
+def test_sdar_full_size_sampled(isd, sync):
     """B=32, N=4 blocks at the Qwen3-8B shapes: whole-request attention for
     three requests, whole 256-row vocabulary tiles of the logits, all row
     statistics and the decisions."""
@@ -147,7 +148,7 @@ def test_sdar_full_size_sampled(isd):
     M = B * N
     tok0 = w.block_tok.cpu().numpy()
     kv0 = w.kv_len.cpu().numpy().astype(np.int64)
-    w.run(1, tau=0.02, sync=True)   # prepare + step (one forward of fresh blocks)
+    w.run(1, tau=0.02, sync=sync)   # prepare + step (one forward of fresh blocks)
     torch.cuda.synchronize()
     assert int(w.err.item()) == 0
     table = w.page_table.cpu().numpy().reshape(B, -1)
@@ -194,12 +195,12 @@ def test_sdar_full_size_sampled(isd):
     assert np.array_equal(m_g, m_h.astype(np.float32).astype(np.float64))
     assert np.all(np.abs(s_g - s_h) <= OP.NEAR * s_h)
     r = S.unmask_batch(tok0, np.zeros(B, np.int64), kv0, S.confidence(s_g).reshape(B, N),
-                       a_g.reshape(B, N), 0.02, True)
+                       a_g.reshape(B, N), 0.02, sync)
     assert np.array_equal(w.block_tok.cpu().numpy(), r["block_tok"])
     assert np.array_equal(w.unmasked_hist[0].cpu().numpy(), r["unmasked"])
     assert np.array_equal(w.block_steps_hist[0].cpu().numpy(), r["block_steps"])
     assert np.array_equal(w.kv_len.cpu().numpy(), r["kv_len"])
-    record_parity("SDAR step qwen3_8b_b32_n4 sampled",
+    record_parity(f"SDAR step qwen3_8b_b32_n4 sampled sync={sync}",
                   dict(requests=B, near_threshold=0, mismatches=0,
                        committed=int(r["unmasked"].sum())))
 
