@@ -338,9 +338,13 @@ isd_status isd_attention_noalloc(const isd_dims* d, const uint16_t* q, const uin
  * out_tok [B, N] (a block's tokens when it leaves the batch in this call,
  * else -1), block_steps [B] (its S_b, denoising forwards without the store
  * pass, then; else 0).
+ * Ownership: every pointer is the caller's device memory (the state buffers
+ * are read and written in place); nothing is allocated, nothing is read on
+ * the host, and the calls are capturable.
  * Errors: invalid pointers or dims -> ISD_ERR_INVALID_ARG; N > 16, lora_rank
  * != 0 or shapes the attention / LM head do not support ->
- * ISD_ERR_UNSUPPORTED_SHAPE.  On the device, a page id outside the pool
+ * ISD_ERR_UNSUPPORTED_SHAPE; a workspace too small or misaligned ->
+ * ISD_ERR_WORKSPACE.  On the device, a page id outside the pool
  * raises ISD_FLAG_PAGE_OOB, a block that does not fit the request's pages
  * ISD_FLAG_CAPACITY, a committed token outside [0, V) ISD_FLAG_TOKEN_OOB.
  * ---------------------------------------------------------------------------
@@ -449,8 +453,16 @@ isd_status isd_sdar_loop(const isd_dims* d, float tau, int32_t sync, int32_t n_s
  * for a new projection shape queries cuBLASLt's heuristic and times its
  * best candidates on the call's stream (this synchronises that stream once;
  * the fastest is kept for the process); make it before any stream capture
- * (under capture, the heuristic's first choice is used).  Errors as for
- * isd_attention.
+ * (under capture, the heuristic's first choice is used).
+ * Ownership: the layer array is the caller's host memory, read during the
+ * call only; every pointer in it and every other pointer is the caller's
+ * device memory; nothing is allocated.
+ * Errors: invalid dims, a null pointer, n_layers < 0, inter not a multiple
+ * of 8 or rope_positions < 1 -> ISD_ERR_INVALID_ARG; H not a multiple of 8
+ * or an attention shape isd_attention does not support ->
+ * ISD_ERR_UNSUPPORTED_SHAPE; a workspace below isd_layers_workspace_bytes or
+ * misaligned -> ISD_ERR_WORKSPACE; a cuBLASLt failure -> ISD_ERR_CUDA
+ * (isd_last_error() names it).
  */
 typedef struct {
     const uint16_t* in_norm;
@@ -473,6 +485,9 @@ size_t isd_layers_workspace_bytes(const isd_dims* d, int32_t inter);
  * MASK) for an active clean slot (s < n_clean[b]; t = clean_tok[b][s]), the
  * MASK row for inactive clean slots and every MASK slot.  x [B*(2N-1), H].
  * A token outside [0, V) raises ISD_FLAG_TOKEN_OOB (the MASK row is used).
+ * Ownership: caller's device memory throughout.  Errors: invalid dims or a
+ * null pointer -> ISD_ERR_INVALID_ARG; H not a multiple of 8 ->
+ * ISD_ERR_UNSUPPORTED_SHAPE.
  */
 isd_status isd_embed_block(const isd_dims* d, const uint16_t* E, const int32_t* n_clean,
                            const int32_t* clean_tok, uint16_t* x, int32_t* err_flag,
