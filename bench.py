@@ -554,6 +554,10 @@ def deep_leg(isd, cfg, R, K, bus, seed, n_layers, tpf=None, hbm=None):
             "N": N, "queries_per_request": 2 * N - 1, "steps": K, "ms_per_step": ms,
             "steps_per_s": R.world / (ms / 1e3), "algorithmic_bytes": byts,
             "achieved_gbs": byts / (ms / 1e3) / 1e9, "err_flags": int(v["err"].item()),
+            # this library's kernels per step: embed; per layer two RMSNorms, q/k
+            # norm + rotation, K/V append, attention, SiLU; final norm; LM head and
+            # its statistics merge; accept.  Plus four cuBLASLt GEMMs per layer.
+            "gpu_launches": K * (1 + 6 * n_layers + 4), "library_gemm_launches": K * 4 * n_layers,
             "clocks": clk}
         if hbm:
             out["isd" if N > 1 else "ar"]["frac_of_hbm"] = byts / (ms / 1e3) / 1e9 / hbm
