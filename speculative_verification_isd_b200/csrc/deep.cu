@@ -83,9 +83,10 @@ rmsnorm_kernel(const __nv_bfloat16* __restrict__ x, const __nv_bfloat16* __restr
 
 // Per head of one block row: q and k heads are RMS-normalised over D (weights
 // q_norm / k_norm), rotated by the slot's position (rotate-half pairs, table
-// rows (cos, sin)) and rounded once; v heads are copied.  One warp per head;
-// lane l holds elements e*32 + l (E = D/32 of them), whose rotation partner
-// is element (e + E/2)*32 + l.
+// rows (cos, sin)) and rounded once; v heads are copied.  A head takes
+// L = D/8 lanes (two heads per warp at D = 128, four at D = 64); lane j of a
+// head holds elements 4j..4j+3 and their rotation partners 4j+D/2..4j+D/2+3
+// (8-byte loads), so the rotation needs no exchange between lanes.
 template <int D>
 __global__ void __launch_bounds__(256)
 qk_norm_rope_kernel(const __nv_bfloat16* __restrict__ qkv, const __nv_bfloat16* __restrict__ q_norm,
@@ -94,8 +95,10 @@ qk_norm_rope_kernel(const __nv_bfloat16* __restrict__ qkv, const __nv_bfloat16* 
                     const int32_t* __restrict__ n_clean, int N, int Q, int Hq, int Hkv, float eps,
                     __nv_bfloat16* __restrict__ q_out, __nv_bfloat16* __restrict__ k_out,
                     __nv_bfloat16* __restrict__ v_out, int32_t* err_flag) {
-    constexpr int E = D / 32;
+    constexpr int L = D / 8;           // lanes per head (4 elements of each half each)
+    constexpr int HPW = 32 / L;        // heads per warp and pass
     const int row = blockIdx.x, warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int sub = lane / L, j = lane % L;
     const int b = row / Q, s = row - b * Q;
     const int kv = max(kv_len[b], 0), c = n_clean[b];
     int pos = s < N ? kv + s : kv + c + (s - N);
@@ -104,38 +107,65 @@ qk_norm_rope_kernel(const __nv_bfloat16* __restrict__ qkv, const __nv_bfloat16* 
         if (threadIdx.x == 0) raise_flag(err_flag, ISD_FLAG_CAPACITY);
         pos = rope_len - 1;
     }
-    const float2* cs = rope + (size_t)pos * (D / 2);
+    const float2* cs = rope + (size_t)pos * (D / 2) + 4 * j;
     const int heads = Hq + 2 * Hkv;
     const __nv_bfloat16* src = qkv + (size_t)row * heads * D;
-    for (int h = warp; h < heads; h += 8) {
-        float x[E];
-#pragma unroll
-        for (int e = 0; e < E; ++e) x[e] = __bfloat162float(src[h * D + e * 32 + lane]);
-        if (h >= Hq + Hkv) {
+    for (int h0 = warp * HPW; h0 < heads; h0 += 8 * HPW) {
+        const int h = h0 + sub;
+        const bool live = h < heads;
+        uint2 lo = make_uint2(0, 0), hi = make_uint2(0, 0);
+        if (live) {
+            lo = *reinterpret_cast<const uint2*>(src + h * D + 4 * j);
+            hi = *reinterpret_cast<const uint2*>(src + h * D + D / 2 + 4 * j);
+        }
+        if (live && h >= Hq + Hkv) {
             __nv_bfloat16* dst = v_out + ((size_t)row * Hkv + (h - Hq - Hkv)) * D;
-#pragma unroll
-            for (int e = 0; e < E; ++e) dst[e * 32 + lane] = __float2bfloat16_rn(x[e]);
-            continue;
+            *reinterpret_cast<uint2*>(dst + 4 * j) = lo;
+            *reinterpret_cast<uint2*>(dst + D / 2 + 4 * j) = hi;
         }
         const bool is_q = h < Hq;
-        const __nv_bfloat16* wn = is_q ? q_norm : k_norm;
+        const __nv_bfloat162* pl = reinterpret_cast<const __nv_bfloat162*>(&lo);
+        const __nv_bfloat162* ph = reinterpret_cast<const __nv_bfloat162*>(&hi);
+        float x[4], y[4];
+        {
+            const float2 a0 = __bfloat1622float2(pl[0]), a1 = __bfloat1622float2(pl[1]);
+            const float2 b0 = __bfloat1622float2(ph[0]), b1 = __bfloat1622float2(ph[1]);
+            x[0] = a0.x; x[1] = a0.y; x[2] = a1.x; x[3] = a1.y;
+            y[0] = b0.x; y[1] = b0.y; y[2] = b1.x; y[3] = b1.y;
+        }
         float ss = 0.f;
 #pragma unroll
-        for (int e = 0; e < E; ++e) ss = fmaf(x[e], x[e], ss);
+        for (int e = 0; e < 4; ++e) ss = fmaf(y[e], y[e], fmaf(x[e], x[e], ss));
+        // sum over the head's L lanes (an aligned group of the warp)
 #pragma unroll
-        for (int o = 16; o > 0; o >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, o);
+        for (int o = L / 2; o > 0; o >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, o);
+        if (!live || h >= Hq + Hkv) continue;
         const float r = __frsqrt_rn(ss / (float)D + eps);
+        const __nv_bfloat16* wn = is_q ? q_norm : k_norm;
+        const uint2 wl = __ldg(reinterpret_cast<const uint2*>(wn + 4 * j));
+        const uint2 wh = __ldg(reinterpret_cast<const uint2*>(wn + D / 2 + 4 * j));
+        const __nv_bfloat162* pwl = reinterpret_cast<const __nv_bfloat162*>(&wl);
+        const __nv_bfloat162* pwh = reinterpret_cast<const __nv_bfloat162*>(&wh);
+        const float2 w0 = __bfloat1622float2(pwl[0]), w1 = __bfloat1622float2(pwl[1]);
+        const float2 v0 = __bfloat1622float2(pwh[0]), v1 = __bfloat1622float2(pwh[1]);
+        const float wlo[4] = {w0.x, w0.y, w1.x, w1.y}, whi[4] = {v0.x, v0.y, v1.x, v1.y};
+        float olo[4], ohi[4];
 #pragma unroll
-        for (int e = 0; e < E; ++e) x[e] = x[e] * r * __bfloat162float(__ldg(wn + e * 32 + lane));
+        for (int e = 0; e < 4; ++e) {
+            const float2 t = __ldg(cs + e);
+            const float l = x[e] * r * wlo[e], u = y[e] * r * whi[e];
+            olo[e] = l * t.x - u * t.y;
+            ohi[e] = u * t.x + l * t.y;
+        }
         __nv_bfloat16* dst = is_q ? q_out + ((size_t)row * Hq + h) * D
                                   : k_out + ((size_t)row * Hkv + (h - Hq)) * D;
-#pragma unroll
-        for (int e = 0; e < E / 2; ++e) {
-            const float2 t = __ldg(cs + e * 32 + lane);
-            const float lo = x[e], hi = x[e + E / 2];
-            dst[e * 32 + lane] = __float2bfloat16_rn(lo * t.x - hi * t.y);
-            dst[(e + E / 2) * 32 + lane] = __float2bfloat16_rn(hi * t.x + lo * t.y);
-        }
+        uint2 ol, oh;
+        reinterpret_cast<__nv_bfloat162*>(&ol)[0] = __floats2bfloat162_rn(olo[0], olo[1]);
+        reinterpret_cast<__nv_bfloat162*>(&ol)[1] = __floats2bfloat162_rn(olo[2], olo[3]);
+        reinterpret_cast<__nv_bfloat162*>(&oh)[0] = __floats2bfloat162_rn(ohi[0], ohi[1]);
+        reinterpret_cast<__nv_bfloat162*>(&oh)[1] = __floats2bfloat162_rn(ohi[2], ohi[3]);
+        *reinterpret_cast<uint2*>(dst + 4 * j) = ol;
+        *reinterpret_cast<uint2*>(dst + D / 2 + 4 * j) = oh;
     }
 }
 
