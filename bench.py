@@ -547,6 +547,32 @@ def deep_leg(isd, cfg, R, K, bus, seed, n_layers, tpf=None, hbm=None):
         clk = clocks.stop()
         ms = R.max(e0.elapsed_time(e1)) / K
         times[N] = ms
+        # the same step captured once in a CUDA graph and replayed K times
+        # (the projections' algorithms were chosen in the eager steps)
+        graph = None
+        try:
+            g = torch.cuda.CUDAGraph()
+            gs = torch.cuda.Stream()
+            gs.wait_stream(stream)
+            with torch.cuda.stream(gs):
+                with torch.cuda.graph(g, stream=gs):
+                    dw.step(N, stream=gs)
+            torch.cuda.synchronize()
+            g.replay()
+            torch.cuda.synchronize()
+            R.barrier()
+            g0, g1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            g0.record(stream)
+            for _ in range(K):
+                g.replay()
+            g1.record(stream)
+            torch.cuda.synchronize()
+            R.barrier()
+            graph = {"ms_per_step": R.max(g0.elapsed_time(g1)) / K,
+                     "err_flags": int(v["err"].item())}
+            del g
+        except RuntimeError as e:  # capture unsupported in this process: report why
+            graph = {"unavailable": str(e).splitlines()[0][:200]}
         M = cfg.B * (2 * N - 1)
         logits = float(M) * cfg.V * 4
         byts = weight_bytes + kv_bytes + logits
@@ -558,10 +584,15 @@ def deep_leg(isd, cfg, R, K, bus, seed, n_layers, tpf=None, hbm=None):
             # norm + rotation, K/V append, attention, SiLU; final norm; LM head and
             # its statistics merge; accept.  Plus four cuBLASLt GEMMs per layer.
             "gpu_launches": K * (1 + 6 * n_layers + 4), "library_gemm_launches": K * 4 * n_layers,
-            "clocks": clk}
+            "clocks": clk, "cuda_graph": graph}
         if hbm:
             out["isd" if N > 1 else "ar"]["frac_of_hbm"] = byts / (ms / 1e3) / 1e9 / hbm
     out["forward_time_ratio_isd_over_ar"] = times[cfg.N] / times[1]
+    g_isd, g_ar = (out["isd"].get("cuda_graph") or {}), (out["ar"].get("cuda_graph") or {})
+    if "ms_per_step" in g_isd and "ms_per_step" in g_ar:
+        out["forward_time_ratio_isd_over_ar_graph"] = g_isd["ms_per_step"] / g_ar["ms_per_step"]
+        if tpf is not None:
+            out["speedup_over_ar_graph"] = tpf * g_ar["ms_per_step"] / g_isd["ms_per_step"]
     if tpf is not None:
         out["tpf_closed_loop"] = tpf
         out["speedup_over_ar"] = tpf * times[1] / times[cfg.N]
